@@ -1,0 +1,321 @@
+/*
+ * monarch_oracle.c -- plain float64 CPU oracle of the tiled MonarchRT attention
+ * forward pass.
+ *
+ * TEST INFRASTRUCTURE.  Only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg may load this code.  It shares nothing with the CUDA path:
+ * no header, no helper, no table.  It is deliberately slow and literal: one
+ * loop nest per step of the method, no blocking, no fusion.
+ *
+ * What it computes (sources: "MonarchRT: Efficient Attention for Real-Time
+ * Video Generation", the arXiv abstract; the Chinese explainer page
+ * "卡内基梅隆大学提出MonarchRT…", sections "Monarch矩阵：一种统一而强大的结构化近似工具"
+ * (Monarch matrices; Fig. 3, MonarchAttention's alternating optimisation of L
+ * and R from Q and K), "创新一：块对齐策略" (block alignment, N = f*h*w,
+ * (b1, b2) = (f*h, w)) and "创新二：平铺Monarch参数化" (tiled Monarch, Fig. 2);
+ * the VMonarch abstract for the entropy term of the L update).  The pages
+ * print no formula; the update rules below are the plainest reading of them:
+ *
+ *   Tokens n = u*b2 + v, u in [b1] (block row), v in [b2] (column).
+ *   M[(u,v),(u',v')] = L_v[u,u'] * R_{u',g(u)}[v,v'],   s = 1/sqrt(d),
+ *   where the tile g(u) is the g with floor(g*b1/t) <= u < floor((g+1)*b1/t).
+ *   M is the maximiser, over row-stochastic L and R, of
+ *       F(L,R) = sum_rows [ sum_cols M_ij * s*q_i.k_j + entropy(M_i,:) ],
+ *   the variational form of softmax, approached by alternating exact
+ *   maximisation over R and over L:
+ *     init      L_v[u,:] = 1/b1 (uniform)
+ *     R-step    for every u', tile g, column v, with weights w_u = L_v[u,u'],
+ *               u in T_g:  qbar = sum_u w_u q_(u,v) / sum_u w_u,
+ *               R_{u',g}[v,:] = softmax_v'( s*qbar.k_(u',v') ),
+ *               H = entropy of that row = lse - sum_v' R*logit,
+ *               Ktil = sum_v' R k_(u',v'),  Z = sum_v' R v_(u',v')
+ *     L-step    for every (u,v), g = g(u):
+ *               L_v[u,:] = softmax_u'( s*q_(u,v).Ktil[g,v,u'] + H[g,v,u'] )
+ *     output    y_(u,v) = sum_u' L_v[u,u'] Z[g(u),v,u']      (= M V)
+ *   One iteration is an R-step followed by an L-step.
+ *
+ * Every step for token column v and tile g reads only the query rows
+ * (u in T_g, v), all keys and all values, and writes only the outputs of
+ * those rows; the oracle therefore loops over independent (head, g, v)
+ * problems, which changes no arithmetic of any output.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_EINVAL 1
+#define ORACLE_ENOMEM 2
+
+/* first block row of tile g: floor(g*b1/t) */
+static int tile_first_row(int g, int b1, int tiles)
+{
+    return (int)(((int64_t)g * b1) / tiles);
+}
+
+/* Index maps of the method: u(n), v(n), the perfect shuffle P(n) = v*b1 + u,
+ * the tile boundaries and the tile of every block row. */
+int oracle_index_maps(int f, int h, int w, int b1, int b2, int tiles,
+                      int32_t *u_of_n, int32_t *v_of_n, int32_t *perm,
+                      int32_t *tile_lo, int32_t *tile_of_u)
+{
+    int64_t N = (int64_t)f * h * w;
+    if (f < 1 || h < 1 || w < 1 || b1 < 1 || b2 < 1 || (int64_t)b1 * b2 != N ||
+        tiles < 1 || tiles > b1)
+        return ORACLE_EINVAL;
+    for (int64_t n = 0; n < N; n++) {
+        int u = (int)(n / b2), v = (int)(n % b2);
+        u_of_n[n] = u;
+        v_of_n[n] = v;
+        perm[n] = v * b1 + u;
+    }
+    for (int g = 0; g <= tiles; g++)
+        tile_lo[g] = tile_first_row(g, b1, tiles);
+    for (int g = 0; g < tiles; g++)
+        for (int u = tile_lo[g]; u < tile_lo[g + 1]; u++)
+            tile_of_u[u] = g;
+    return ORACLE_OK;
+}
+
+static size_t workspace_doubles(int d, int b1, int b2, int tiles)
+{
+    int nq_max = (b1 + tiles - 1) / tiles + 1;
+    int mx = b1 > b2 ? b1 : b2;
+    return (size_t)nq_max * b1 + (size_t)b1 * b2 + 2 * (size_t)b1 * d + b1 + d + mx;
+}
+
+/*
+ * One (tile g, column c) problem of one head: runs `half_steps` alternating
+ * half-steps (R, L, R, L, ...) and writes y for the rows (u, c), u in T_g.
+ * q, k, v, y: one head, [N][d] row-major.
+ * L_out (optional) [b2][b1][b1]: L_c[u][u'] for u in T_g.
+ * R_out (optional) [b1][tiles][b2][b2]: R_{u',g}[c][:].
+ */
+static void solve_problem(const double *q, const double *k, const double *v, double *y,
+                          int d, int b1, int b2, int tiles, int g, int c, int half_steps,
+                          double *L_out, double *R_out, double *ws)
+{
+    const double s = 1.0 / sqrt((double)d);
+    const int u0 = tile_first_row(g, b1, tiles), u1 = tile_first_row(g + 1, b1, tiles);
+    const int nq = u1 - u0;
+    double *L = ws;                          /* [nq][b1]  L_c[u][u'], u in T_g */
+    double *R = L + (size_t)nq * b1;         /* [b1][b2]  R_{u',g}[c][:]       */
+    double *Kt = R + (size_t)b1 * b2;        /* [b1][d]   Ktil[g][c][u']       */
+    double *Z = Kt + (size_t)b1 * d;         /* [b1][d]   Z[g][c][u']          */
+    double *H = Z + (size_t)b1 * d;          /* [b1]      entropy of R row     */
+    double *qbar = H + b1;                   /* [d]                            */
+    double *logit = qbar + d;                /* [max(b1, b2)]                  */
+
+    for (size_t i = 0; i < (size_t)nq * b1; i++)
+        L[i] = 1.0 / b1;
+
+    for (int step = 0; step < half_steps; step++) {
+        if ((step & 1) == 0) {
+            /* R-step: every block u' of tile g, row c of R_{u',g} */
+            for (int up = 0; up < b1; up++) {
+                double wsum = 0.0;
+                for (int j = 0; j < d; j++)
+                    qbar[j] = 0.0;
+                for (int u = u0; u < u1; u++) {
+                    double wgt = L[(size_t)(u - u0) * b1 + up];
+                    const double *qr = q + ((int64_t)u * b2 + c) * d;
+                    wsum += wgt;
+                    for (int j = 0; j < d; j++)
+                        qbar[j] += wgt * qr[j];
+                }
+                /* a block that no row of the tile weighs does not enter F;
+                 * the oracle then takes qbar = 0 (a uniform R row) */
+                for (int j = 0; j < d; j++)
+                    qbar[j] = wsum > 0.0 ? qbar[j] / wsum : 0.0;
+
+                double mx = -INFINITY;
+                for (int vp = 0; vp < b2; vp++) {
+                    const double *kr = k + ((int64_t)up * b2 + vp) * d;
+                    double acc = 0.0;
+                    for (int j = 0; j < d; j++)
+                        acc += qbar[j] * kr[j];
+                    logit[vp] = s * acc;
+                    if (logit[vp] > mx)
+                        mx = logit[vp];
+                }
+                double sum = 0.0;
+                for (int vp = 0; vp < b2; vp++)
+                    sum += exp(logit[vp] - mx);
+                double lse = mx + log(sum);
+                double ent = lse;
+                for (int vp = 0; vp < b2; vp++) {
+                    double r = exp(logit[vp] - lse);
+                    R[(size_t)up * b2 + vp] = r;
+                    ent -= r * logit[vp];
+                }
+                H[up] = ent;
+                for (int j = 0; j < d; j++) {
+                    double kt = 0.0, z = 0.0;
+                    for (int vp = 0; vp < b2; vp++) {
+                        double r = R[(size_t)up * b2 + vp];
+                        kt += r * k[((int64_t)up * b2 + vp) * d + j];
+                        z += r * v[((int64_t)up * b2 + vp) * d + j];
+                    }
+                    Kt[(size_t)up * d + j] = kt;
+                    Z[(size_t)up * d + j] = z;
+                }
+            }
+        } else {
+            /* L-step: every query row u of tile g at column c */
+            for (int u = u0; u < u1; u++) {
+                const double *qr = q + ((int64_t)u * b2 + c) * d;
+                double mx = -INFINITY;
+                for (int up = 0; up < b1; up++) {
+                    double acc = 0.0;
+                    for (int j = 0; j < d; j++)
+                        acc += qr[j] * Kt[(size_t)up * d + j];
+                    logit[up] = s * acc + H[up];
+                    if (logit[up] > mx)
+                        mx = logit[up];
+                }
+                double sum = 0.0;
+                for (int up = 0; up < b1; up++)
+                    sum += exp(logit[up] - mx);
+                double lse = mx + log(sum);
+                for (int up = 0; up < b1; up++)
+                    L[(size_t)(u - u0) * b1 + up] = exp(logit[up] - lse);
+            }
+        }
+    }
+
+    /* output: y_(u,c) = sum_u' L_c[u,u'] Z[u'] */
+    for (int u = u0; u < u1; u++) {
+        double *yr = y + ((int64_t)u * b2 + c) * d;
+        for (int j = 0; j < d; j++) {
+            double acc = 0.0;
+            for (int up = 0; up < b1; up++)
+                acc += L[(size_t)(u - u0) * b1 + up] * Z[(size_t)up * d + j];
+            yr[j] = acc;
+        }
+    }
+
+    if (L_out)
+        for (int u = u0; u < u1; u++)
+            for (int up = 0; up < b1; up++)
+                L_out[((int64_t)c * b1 + u) * b1 + up] = L[(size_t)(u - u0) * b1 + up];
+    if (R_out)
+        for (int up = 0; up < b1; up++)
+            for (int vp = 0; vp < b2; vp++)
+                R_out[(((int64_t)up * tiles + g) * b2 + c) * b2 + vp] = R[(size_t)up * b2 + vp];
+}
+
+static int check_shape(int N, int d, int b1, int b2, int tiles, int half_steps)
+{
+    if (N < 1 || d < 1 || b1 < 1 || b2 < 1 || (int64_t)b1 * b2 != N || tiles < 1 ||
+        tiles > b1 || half_steps < 1)
+        return ORACLE_EINVAL;
+    return ORACLE_OK;
+}
+
+/*
+ * Full forward pass over BH heads.  q, k, v, y: [BH][N][d].  half_steps = 2*iters
+ * for the method; other counts stop after the matching half-step (the output
+ * then uses the latest L and the latest R).  L_out [BH][b2][b1][b1] and R_out
+ * [BH][b1][tiles][b2][b2] are optional.  nthreads <= 0 uses the OpenMP default.
+ */
+int oracle_monarch_attn(const double *q, const double *k, const double *v, double *y,
+                        int BH, int N, int d, int b1, int b2, int tiles, int half_steps,
+                        double *L_out, double *R_out, int nthreads)
+{
+    if (BH < 1 || check_shape(N, d, b1, b2, tiles, half_steps))
+        return ORACLE_EINVAL;
+    const int64_t nprob = (int64_t)BH * tiles * b2;
+    const size_t wsz = workspace_doubles(d, b1, b2, tiles);
+    int err = ORACLE_OK;
+#ifdef _OPENMP
+    if (nthreads <= 0)
+        nthreads = omp_get_max_threads();
+#pragma omp parallel num_threads(nthreads)
+#endif
+    {
+        double *ws = (double *)malloc(wsz * sizeof(double));
+        if (!ws) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            err = ORACLE_ENOMEM;
+        }
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+        for (int64_t p = 0; p < nprob; p++) {
+            if (!ws)
+                continue;
+            int bh = (int)(p / ((int64_t)tiles * b2));
+            int g = (int)((p / b2) % tiles);
+            int c = (int)(p % b2);
+            size_t off = (size_t)bh * N * d;
+            solve_problem(q + off, k + off, v + off, y + off, d, b1, b2, tiles, g, c,
+                          half_steps,
+                          L_out ? L_out + (size_t)bh * b2 * b1 * b1 : NULL,
+                          R_out ? R_out + (size_t)bh * b1 * tiles * b2 * b2 : NULL, ws);
+        }
+        free(ws);
+    }
+    return err;
+}
+
+/*
+ * Selected (head, tile, column) problems only: probs[3*i .. 3*i+2] = (bh, g, c).
+ * Writes the rows (u, c), u in T_g, of head bh in y [BH][N][d]; other rows are
+ * left untouched.  Used for sampled parity checks and for the timed CPU baseline.
+ */
+int oracle_monarch_problems(const double *q, const double *k, const double *v, double *y,
+                            int BH, int N, int d, int b1, int b2, int tiles, int half_steps,
+                            int nprob, const int32_t *probs, int nthreads)
+{
+    if (BH < 1 || nprob < 0 || check_shape(N, d, b1, b2, tiles, half_steps))
+        return ORACLE_EINVAL;
+    for (int i = 0; i < nprob; i++)
+        if (probs[3 * i] < 0 || probs[3 * i] >= BH || probs[3 * i + 1] < 0 ||
+            probs[3 * i + 1] >= tiles || probs[3 * i + 2] < 0 || probs[3 * i + 2] >= b2)
+            return ORACLE_EINVAL;
+    const size_t wsz = workspace_doubles(d, b1, b2, tiles);
+    int err = ORACLE_OK;
+#ifdef _OPENMP
+    if (nthreads <= 0)
+        nthreads = omp_get_max_threads();
+#pragma omp parallel num_threads(nthreads)
+#endif
+    {
+        double *ws = (double *)malloc(wsz * sizeof(double));
+        if (!ws) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            err = ORACLE_ENOMEM;
+        }
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+        for (int i = 0; i < nprob; i++) {
+            if (!ws)
+                continue;
+            int bh = probs[3 * i], g = probs[3 * i + 1], c = probs[3 * i + 2];
+            size_t off = (size_t)bh * N * d;
+            solve_problem(q + off, k + off, v + off, y + off, d, b1, b2, tiles, g, c,
+                          half_steps, NULL, NULL, ws);
+        }
+        free(ws);
+    }
+    return err;
+}
+
+/* Number of threads the OpenMP runtime would use (1 without OpenMP). */
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

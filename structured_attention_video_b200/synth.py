@@ -1,0 +1,270 @@
+"""Seeded synthetic video-attention inputs and the workload table.
+
+This module is shared by the CUDA path's tests and benchmark and by the CPU
+oracle's tests.  It holds shapes, random numbers and the synthetic data recipe
+only: nothing of the Monarch attention arithmetic lives here.
+
+Random numbers
+    A counter-based SplitMix64 stream (Steele, Lea and Flood, "Fast splittable
+    pseudorandom number generators", OOPSLA 2014; the 64-bit finaliser of
+    Vigna's public-domain splitmix64) feeds the Box-Muller transform (Box and
+    Muller, 1958).  Element i of a stream with key K is mix(K + (i + 1) * GAMMA),
+    so any element can be produced independently and in any order.
+
+Data recipe (MonarchRT, "Block alignment" and "Tiled Monarch" sections of the
+explainer page; the (f, h, w) video layout with N = f*h*w tokens)
+    * Tokens are ordered (frame, row, column) row-major: n = (fi*h + hi)*w + wi.
+    * A sinusoidal positional code p(fi, hi, wi) in R^d splits d into three axis
+      groups (f, h, w) of sizes g, g, d - 2g with g = floor(d/3) rounded down to
+      even; inside a group of n pairs, p[2j] = sin(omega_j * pos) and
+      p[2j+1] = cos(omega_j * pos) with omega_j = 10000^(-j/n).
+    * "tiny" workloads: Q, K, V = z + 1.0 * p with z ~ N(0, 1) i.i.d.
+    * "wan" workloads: Q, K = z + A * p with A = sqrt(6 / sqrt(d)) (a
+      same-position logit about 3 sigma above the noise at scale 1/sqrt(d)),
+      V = z / sqrt(d); then 8 planted query-key pairs per (b, h) in different
+      frames and more than 2 tokens apart in h and w, each receiving +beta*e on
+      the query and the key (e a random unit vector, beta = sqrt(4 * sqrt(d)),
+      a +4 sigma logit boost at scale 1/sqrt(d)).
+    * Values are generated in float64 and rounded once, round-to-nearest-even,
+      to the working dtype (float32 or bfloat16).  The rounded values are
+      exactly representable in float64, which is what the oracle consumes.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+GAMMA = np.uint64(0x9E3779B97F4A7C15)
+_M1 = np.uint64(0xBF58476D1CE4E5B9)
+_M2 = np.uint64(0x94D049BB133111EB)
+
+TENSOR_IDS = {"q": 1, "k": 2, "v": 3, "pairs": 4}
+
+
+# ----------------------------------------------------------------------------
+# workloads
+# ----------------------------------------------------------------------------
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    d: int
+    f: int
+    h: int
+    w: int
+    b1: int
+    b2: int
+    tiles: int
+    iters: int
+    dtype: str          # "f32" or "bf16"
+    seed: int
+    kind: str           # "tiny" or "wan"
+
+    @property
+    def N(self) -> int:
+        return self.f * self.h * self.w
+
+    def replace(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+    def monarch_flops(self) -> float:
+        """Algorithmic FLOPs of the forward pass (multiply-add = 2).
+
+        Per (b, h) and iteration: the R-step does 6*t*N*b2*d (logits plus the
+        two products with [V | K]); the L-step does 4*N*b1*d (logits plus the
+        product with Z); every iteration after the first re-aggregates the
+        queries with L (2*N*b1*d).
+        """
+        T, t, N = self.iters, self.tiles, self.N
+        per_head = (6 * t * N * self.b2 * self.d * T
+                    + 4 * N * self.b1 * self.d * T
+                    + 2 * N * self.b1 * self.d * (T - 1))
+        return float(self.B * self.H * per_head)
+
+    def dense_flops(self) -> float:
+        """FLOPs of exact softmax attention on the same shape (4*N^2*d per head)."""
+        return float(4 * self.B * self.H * self.N * self.N * self.d)
+
+    def io_bytes(self) -> int:
+        """Q, K, V read once and O written once, in the working dtype."""
+        es = 2 if self.dtype == "bf16" else 4
+        return 4 * self.B * self.H * self.N * self.d * es
+
+
+WORKLOADS = {
+    # tiny oracle case; b1 = 1 and b2 = 1 variants are derived in the tests
+    "tiny": Workload("tiny", 1, 2, 32, 3, 8, 8, 24, 8, 1, 1, "f32", 0, "tiny"),
+    # Wan-1.3B-shaped single chunk at 480p
+    "480p_chunk": Workload("480p_chunk", 1, 12, 128, 3, 30, 52, 90, 52, 1, 1, "bf16", 1, "wan"),
+    # Wan-1.3B full clip at 480p (tiles swept over 1, 2, 4, 8)
+    "480p_full": Workload("480p_full", 1, 12, 128, 21, 30, 52, 630, 52, 1, 1, "bf16", 2, "wan"),
+    # 720p clip: the headline throughput shape
+    "720p": Workload("720p", 1, 12, 128, 21, 45, 80, 945, 80, 4, 1, "bf16", 3, "wan"),
+    # Wan-14B-shaped stress case (iters swept over 1, 2, 5, 10)
+    "14b": Workload("14b", 2, 40, 128, 21, 30, 52, 630, 52, 2, 1, "bf16", 4, "wan"),
+}
+
+
+# ----------------------------------------------------------------------------
+# counter-based generator
+# ----------------------------------------------------------------------------
+def _mix64(z: np.ndarray) -> np.ndarray:
+    z = (z ^ (z >> np.uint64(30))) * _M1
+    z = (z ^ (z >> np.uint64(27))) * _M2
+    return z ^ (z >> np.uint64(31))
+
+
+def stream_key(seed: int, b: int, h: int, tensor: str, rank: int = 0) -> np.uint64:
+    """Key of the stream for (seed, rank, b, h, tensor): a SplitMix64 mix of the fields."""
+    with np.errstate(over="ignore"):
+        x = np.uint64(seed & 0xFFFFFFFF)
+        for field in (rank, b, h, TENSOR_IDS[tensor]):
+            x = _mix64(np.array([x + GAMMA * np.uint64(field + 1)], dtype=np.uint64))[0]
+    return x
+
+
+def uniform53(key: np.uint64, start: int, count: int) -> np.ndarray:
+    """Elements [start, start+count) of stream `key` as doubles in (0, 1]."""
+    with np.errstate(over="ignore"):
+        i = np.arange(start + 1, start + count + 1, dtype=np.uint64)
+        z = _mix64(key + i * GAMMA)
+    return ((z >> np.uint64(11)).astype(np.float64) + 1.0) * (1.0 / 9007199254740992.0)
+
+
+def normals(key: np.uint64, count: int) -> np.ndarray:
+    """`count` standard normals from stream `key` (Box-Muller on consecutive pairs)."""
+    m = (count + 1) // 2
+    u = uniform53(key, 0, 2 * m)
+    r = np.sqrt(-2.0 * np.log(u[0::2]))
+    th = (2.0 * math.pi) * u[1::2]
+    out = np.empty(2 * m, dtype=np.float64)
+    out[0::2] = r * np.cos(th)
+    out[1::2] = r * np.sin(th)
+    return out[:count]
+
+
+# ----------------------------------------------------------------------------
+# rounding to the working dtype
+# ----------------------------------------------------------------------------
+def round_to_dtype(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Round float64 values once, to nearest even, to float32 or bfloat16; return float64."""
+    if dtype == "f32":
+        return x.astype(np.float32).astype(np.float64)
+    if dtype != "bf16":
+        raise ValueError(dtype)
+    m, e = np.frexp(x)                     # x = m * 2^e, 0.5 <= |m| < 1
+    r = np.rint(m * 256.0)                 # 8 significant bits, ties to even
+    out = np.ldexp(r, e - 8)
+    small = np.abs(x) < 2.0 ** -126        # bf16 subnormal range: fixed spacing 2^-133
+    if small.any():
+        out[small] = np.rint(x[small] * 2.0 ** 133) * 2.0 ** -133
+    return out
+
+
+def to_device_bits(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Pack already-rounded float64 values into the dtype's storage (float32 or bf16 bits as uint16)."""
+    f = x.astype(np.float32)
+    if dtype == "f32":
+        return f
+    return (f.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+def from_device_bits(a: np.ndarray, dtype: str) -> np.ndarray:
+    """Exact float64 values of a float32 array or of bf16 bits stored as uint16."""
+    if dtype == "f32":
+        return a.astype(np.float64)
+    return (a.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+# ----------------------------------------------------------------------------
+# the recipe
+# ----------------------------------------------------------------------------
+def positional_code(f: int, h: int, w: int, d: int) -> np.ndarray:
+    """Sinusoidal code over (frame, row, column): shape [f*h*w, d], float64."""
+    g = (d // 3) & ~1
+    sizes = (g, g, d - 2 * g)
+    fi, hi, wi = np.meshgrid(np.arange(f), np.arange(h), np.arange(w), indexing="ij")
+    pos = (fi.reshape(-1), hi.reshape(-1), wi.reshape(-1))
+    cols = []
+    for size, p in zip(sizes, pos):
+        n = size // 2
+        j = np.arange(n, dtype=np.float64)
+        omega = 10000.0 ** (-j / max(n, 1))
+        ang = p[:, None].astype(np.float64) * omega[None, :]
+        blk = np.empty((p.shape[0], 2 * n), dtype=np.float64)
+        blk[:, 0::2] = np.sin(ang)
+        blk[:, 1::2] = np.cos(ang)
+        if size > 2 * n:                   # odd group size: pad with a zero column
+            blk = np.concatenate([blk, np.zeros((p.shape[0], size - 2 * n))], axis=1)
+        cols.append(blk)
+    return np.concatenate(cols, axis=1)
+
+
+def planted_pairs(wl: Workload, b: int, h: int, rank: int = 0, npairs: int = 8):
+    """The (query token, key token, unit direction) triples planted into one head."""
+    key = stream_key(wl.seed, b, h, "pairs", rank)
+    f, hh, ww, N = wl.f, wl.h, wl.w, wl.N
+    pairs = []
+    pos = 0
+    while len(pairs) < npairs and pos < 1 << 20:
+        u = uniform53(key, pos, 2)
+        pos += 2
+        i = min(int(u[0] * N), N - 1)
+        j = min(int(u[1] * N), N - 1)
+        fi, hi, wi = i // (hh * ww), (i // ww) % hh, i % ww
+        fj, hj, wj = j // (hh * ww), (j // ww) % hh, j % ww
+        if fi != fj and abs(hi - hj) > 2 and abs(wi - wj) > 2:
+            pairs.append((i, j))
+    dkey = stream_key(wl.seed, b, h, "pairs", rank + 7919)
+    dirs = normals(dkey, npairs * wl.d).reshape(npairs, wl.d)
+    dirs /= np.linalg.norm(dirs, axis=1, keepdims=True)
+    return [(i, j, dirs[t]) for t, (i, j) in enumerate(pairs)]
+
+
+def make_head(wl: Workload, b: int, h: int, rank: int = 0, pos_code: np.ndarray | None = None):
+    """Q, K, V of one (b, h) as float64 [N, d] arrays, already rounded to wl.dtype."""
+    N, d = wl.N, wl.d
+    p = positional_code(wl.f, wl.h, wl.w, d) if pos_code is None else pos_code
+    out = {}
+    for name in ("q", "k", "v"):
+        z = normals(stream_key(wl.seed, b, h, name, rank), N * d).reshape(N, d)
+        if wl.kind == "tiny":
+            x = z + p
+        elif name == "v":
+            x = z / math.sqrt(d)
+        else:
+            x = z + math.sqrt(6.0 / math.sqrt(d)) * p
+        out[name] = x
+    if wl.kind == "wan":
+        beta = math.sqrt(4.0 * math.sqrt(d))
+        for i, j, e in planted_pairs(wl, b, h, rank):
+            out["q"][i] += beta * e
+            out["k"][j] += beta * e
+    return {name: round_to_dtype(x, wl.dtype) for name, x in out.items()}
+
+
+def make_inputs(wl: Workload, rank: int = 0):
+    """Q, K, V for all heads as float64 arrays [B, H, N, d] (rounded to wl.dtype)."""
+    p = positional_code(wl.f, wl.h, wl.w, wl.d)
+    shape = (wl.B, wl.H, wl.N, wl.d)
+    q, k, v = (np.empty(shape) for _ in range(3))
+    for b in range(wl.B):
+        for h in range(wl.H):
+            x = make_head(wl, b, h, rank, p)
+            q[b, h], k[b, h], v[b, h] = x["q"], x["k"], x["v"]
+    return q, k, v
+
+
+def fill_device_bits(wl: Workload, q_out: np.ndarray, k_out: np.ndarray, v_out: np.ndarray,
+                     rank: int = 0) -> None:
+    """Write Q, K, V in storage format straight into caller arrays [B, H, N, d] (head by head)."""
+    p = positional_code(wl.f, wl.h, wl.w, wl.d)
+    for b in range(wl.B):
+        for h in range(wl.H):
+            x = make_head(wl, b, h, rank, p)
+            q_out[b, h] = to_device_bits(x["q"], wl.dtype)
+            k_out[b, h] = to_device_bits(x["k"], wl.dtype)
+            v_out[b, h] = to_device_bits(x["v"], wl.dtype)
