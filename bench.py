@@ -1,0 +1,417 @@
+#!/usr/bin/env python
+"""Benchmark of the tiled MonarchRT attention forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one forward pass (aggregated queries, R-step, L-step with the
+output) of the 720p Wan-shaped clip: B=1, H=12, d=128, f=21, h=45, w=80
+(N=75600 tokens), blocks (945, 80), 4 tiles, 1 iteration, bfloat16.  Inputs are
+seeded synthetic video tokens (positional code plus planted semantic pairs).
+With N > 1 (torchrun, one process per GPU) every rank runs its own clip (weak
+scaling, no data-path collective); the device time is the max over ranks.
+
+Prints ONE JSON line (rank 0).  `value` is dense-equivalent effective TFLOP/s
+(4*B*H*N^2*d per step over the device time, summed over ranks); `roofline`
+describes the dominant kernel, `path_roofline` the whole step against
+max(Monarch FLOPs / bf16 peak, Q/K/V/O bytes / HBM bandwidth).
+`--impl reference` times the float64 CPU oracle instead, on bounded samples.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from structured_attention_video_b200 import synth  # noqa: E402
+
+METRIC = "Monarch-attn fwd ms & effective TFLOP/s at 720p Wan shape; % of roofline"
+UNIT = "TFLOP/s (dense-equivalent effective)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            return json.load(fh), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(wl: synth.Workload, world: int) -> dict:
+    return {"workload": "%s Wan clip: B=%d H=%d d=%d f=%d h=%d w=%d (N=%d), blocks (%d,%d), "
+                        "tiles=%d, iters=%d" % (wl.name, wl.B, wl.H, wl.d, wl.f, wl.h, wl.w,
+                                                wl.N, wl.b1, wl.b2, wl.tiles, wl.iters),
+            "B": wl.B, "H": wl.H, "d": wl.d, "f": wl.f, "h": wl.h, "w": wl.w, "N": wl.N,
+            "b1": wl.b1, "b2": wl.b2, "tiles": wl.tiles, "iters": wl.iters,
+            "parallelism": "replicas x%d (independent clips per GPU)" % world,
+            "l2": "inputs (%.2f GB) larger than L2, and a %d MB buffer written between "
+                  "timed steps" % (3 * wl.B * wl.H * wl.N * wl.d * 2 / 1e9, L2_FLUSH_BYTES >> 20)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle samples (baseline and reference arm)
+# ---------------------------------------------------------------------------
+def sample_dense_flops(wl: synth.Workload, probs) -> float:
+    """Share of the dense-equivalent work that the sampled problems' output rows carry."""
+    rows = sum(((g + 1) * wl.b1) // wl.tiles - (g * wl.b1) // wl.tiles for _, g, _ in probs)
+    return 4.0 * rows * wl.N * wl.d
+
+
+class OracleSampler:
+    """Runs the float64 oracle on (head, tile, column) problems of one workload."""
+
+    def __init__(self, wl: synth.Workload, heads: int = 2):
+        from oracle import oracle
+        self.oracle = oracle
+        self.wl = wl
+        pos = synth.positional_code(wl.f, wl.h, wl.w, wl.d)
+        self.heads = list(range(min(heads, wl.B * wl.H)))
+        xs = [synth.make_head(wl, bh // wl.H, bh % wl.H, 0, pos) for bh in self.heads]
+        self.q = np.stack([x["q"] for x in xs])
+        self.k = np.stack([x["k"] for x in xs])
+        self.v = np.stack([x["v"] for x in xs])
+        self.cores = len(os.sched_getaffinity(0))
+
+    def problems(self, count: int, seed: int):
+        rng = np.random.default_rng(seed)
+        return [(int(rng.integers(len(self.heads))), int(rng.integers(self.wl.tiles)),
+                 int(rng.integers(self.wl.b2))) for _ in range(count)]
+
+    def run(self, probs) -> float:
+        wl = self.wl
+        t0 = time.perf_counter()
+        self.oracle.monarch_problems(self.q, self.k, self.v, wl.b1, wl.b2, wl.tiles, wl.iters,
+                                     probs, nthreads=self.cores)
+        return time.perf_counter() - t0
+
+
+def cpu_baseline(wl: synth.Workload, target_s: float) -> dict:
+    smp = OracleSampler(wl)
+    probe = smp.problems(smp.cores, seed=1)
+    t = smp.run(probe)
+    count = max(smp.cores, int(smp.cores * max(1.0, target_s / max(t, 1e-3))))
+    count = min(count, 4096)
+    probs = smp.problems(count, seed=2)
+    t = smp.run(probs)
+    value = sample_dense_flops(wl, probs) / t / 1e12
+    return {"value": value, "unit": UNIT, "cores": smp.cores, "kind": "oracle",
+            "seconds": t,
+            "sample": "%d (head, tile, column) problems of the %s workload (%.2f%% of one "
+                      "step's output rows), float64 C oracle with OpenMP" %
+                      (count, wl.name, 100.0 * sample_dense_flops(wl, probs) / wl.dense_flops())}
+
+
+def run_reference(args, wl: synth.Workload, world: int, rank: int):
+    if rank != 0:
+        return
+    smp = OracleSampler(wl)
+    per_step = smp.cores
+    times, flops = [], []
+    for step in range(args.warmup + args.steps):
+        probs = smp.problems(per_step, seed=100 + step)
+        t = smp.run(probs)
+        if step >= args.warmup:
+            times.append(t)
+            flops.append(sample_dense_flops(wl, probs))
+    value = sum(flops) / sum(times) / 1e12
+    sample = ("each step: %d (head, tile, column) problems of the %s workload (%.3f%% of its "
+              "output rows), float64 C oracle with OpenMP on %d cores" %
+              (per_step, wl.name, 100.0 * flops[0] / wl.dense_flops(), smp.cores))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(wl, 1),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": smp.cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.TemporaryFile(mode="w+")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait()
+        self.file.seek(0)
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.file.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        self.file.close()
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# kernel roofline bookkeeping
+# ---------------------------------------------------------------------------
+def kernel_roofline(name: str, ms_per_launch: float, wl: synth.Workload, peaks, peak_kind):
+    """Algorithmic work of one launch of kernel family `name` and its roofline fraction."""
+    BH, N, d, t = wl.B * wl.H, wl.N, wl.d, wl.tiles
+    es = 2 if wl.dtype == "bf16" else 4
+    if name.endswith("rstep_kernel"):
+        flops = 6.0 * t * N * wl.b2 * d * BH
+    elif name.endswith("lstep_kernel"):
+        flops = 4.0 * N * wl.b1 * d * BH
+    elif name == "qbar_weighted_kernel":
+        flops = 4.0 * N * wl.b1 * d * BH
+    else:
+        flops = None
+    tensor = name.startswith("tc_")
+    if flops is None:   # query aggregation: reads Q once
+        nbytes = BH * N * d * es
+        achieved = nbytes / (ms_per_launch * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_source": peak_kind + " hbm_gbs"}
+    achieved = flops / (ms_per_launch * 1e-3) / 1e12
+    if tensor:
+        peak = peaks["bf16_tflops"]
+        return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_source": peak_kind + " bf16_tflops (burst)"}
+    # SIMT float32 FMA: 148 SMs x 128 FP32 lanes x 2 FLOP x max SM clock
+    peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak,
+            "peak_source": "derived: 148 SMs x 128 FP32 FMA lanes x 2 x %s sm_max_mhz" % peak_kind}
+
+
+def kernel_traffic(name: str):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        rec = json.load(fh).get(name)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "structured_attention_video_b200", "csrc", rec["source"])
+    if not os.path.exists(src):
+        return None
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    return rec["dram_bytes_per_launch"] if digest == rec["source_sha256"] else None
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, wl: synth.Workload, world: int, rank: int, local: int):
+    import torch
+    import torch.distributed as dist
+    from structured_attention_video_b200 import _lib
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    shape = (wl.B, wl.H, wl.N, wl.d)
+    hq, hk, hv = (torch.empty(shape, dtype=torch.int16).pin_memory() for _ in range(3))
+    synth.fill_device_bits(wl, hq.numpy().view(np.uint16), hk.numpy().view(np.uint16),
+                           hv.numpy().view(np.uint16), rank)
+    q, k, v = (x.to(dev).view(torch.bfloat16) for x in (hq, hk, hv))
+    out = torch.empty_like(q)
+    hout = torch.empty(shape, dtype=torch.int16).pin_memory()
+    sargs = (wl.B, wl.H, wl.f, wl.h, wl.w, wl.d, wl.b1, wl.b2, wl.tiles, wl.iters)
+    ws_bytes = _lib.monarch_attn_workspace_bytes(*sargs, _lib.BF16)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    path = _lib.monarch_attn_path(*sargs, _lib.BF16)
+
+    def step():
+        _lib.check(_lib.monarch_attn_fwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                            out.data_ptr(), *sargs, _lib.BF16, ws.data_ptr(),
+                                            ws_bytes, sh), "monarch_attn_fwd_ws")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    _lib.check(_lib.monarch_last_device_status(sh), "device status after warm-up")
+    _lib.monarch_profile_collect()
+
+    props = torch.cuda.get_device_properties(dev)
+    clocks = ClockSampler("GPU-" + str(props.uuid))
+    clocks.start()
+    time.sleep(0.3)
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    _lib.monarch_profile_enable(1)
+    for a, b in events:
+        flush.zero_()
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    _lib.monarch_profile_enable(0)
+    clock_rec = clocks.stop()
+    prof = _lib.monarch_profile_collect()
+    _lib.check(_lib.monarch_last_device_status(sh), "device status after timed steps")
+    ms_total = sum(a.elapsed_time(b) for a, b in events)
+    ms_step = max_over_ranks(ms_total / args.steps)
+
+    # end to end through the host-buffer entry point: H2D inputs, forward, D2H output
+    e2e_times = []
+    for i in range(args.e2e_warmup + args.e2e_steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        _lib.check(_lib.monarch_attn_fwd_host(hq.data_ptr(), hk.data_ptr(), hv.data_ptr(),
+                                              hout.data_ptr(), *sargs, _lib.BF16, sh),
+                   "monarch_attn_fwd_host")
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.e2e_warmup:
+            e2e_times.append(a.elapsed_time(b))
+    e2e_ms = max_over_ranks(statistics.mean(e2e_times))
+
+    if rank != 0:
+        return
+    peaks, peak_kind = load_peaks()
+    dense = wl.dense_flops()
+    value = world * dense / (ms_step * 1e-3) / 1e12
+    kernels = {name: {"ms_per_launch": ms / n, "launches": n, "share": ms / max(1e-9, sum(
+        m for m, _ in prof.values()))} for name, (ms, n) in prof.items() if n > 0}
+    dominant = max(kernels, key=lambda kk: kernels[kk]["ms_per_launch"] * kernels[kk]["launches"])
+    roof = kernel_roofline(dominant, kernels[dominant]["ms_per_launch"], wl, peaks, peak_kind)
+    roof["kernel"] = dominant
+    traffic = kernel_traffic(dominant)
+    roof["traffic"] = traffic
+    roof["traffic_unit"] = "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"
+    flops = wl.monarch_flops()
+    io = wl.io_bytes()
+    roof_ms = max(flops / (peaks["bf16_tflops"] * 1e12), io / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    launches = sum(kk["launches"] for kk in kernels.values())
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(wl, world),
+        "monarch_tflops": world * flops / (ms_step * 1e-3) / 1e12,
+        "path_roofline": {"roofline_ms": roof_ms, "frac": roof_ms / ms_step,
+                          "flops_per_step": flops, "io_bytes_per_step": io,
+                          "peak_source": "%s bf16_tflops (burst) and hbm_gbs" % peak_kind},
+        "roofline": roof,
+        "kernels": kernels,
+        "kernel_path": "sm100 tensor-core" if path == 1 else "generic SIMT",
+        "gpu_launches": launches,
+        "e2e": {"value": world * dense / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": 3 * wl.B * wl.H * wl.N * wl.d * 2,
+                "d2h_bytes_per_step": wl.B * wl.H * wl.N * wl.d * 2,
+                "api": "monarch_attn_fwd_host (C ABI, pinned host buffers)"},
+        "clocks": clock_rec,
+        "gpu": props.name,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+    else:
+        line["cpu_baseline"] = None
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="720p", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-warmup", type=int, default=2)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        ap.error("--gpus %d but WORLD_SIZE=%d: launch N > 1 with torchrun" % (args.gpus, world))
+    wl = synth.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        run_reference(args, wl, world, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    try:
+        run_ours(args, wl, world, rank, local)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,199 @@
+/*
+ * monarch_attn.h -- C ABI of the tiled MonarchRT attention forward pass on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (sources: "MonarchRT: Efficient Attention for Real-Time Video
+ * Generation", abstract; the explainer page "卡内基梅隆大学提出MonarchRT…", sections
+ * "Monarch矩阵" with Fig. 3, "创新一：块对齐策略" and "创新二：平铺Monarch参数化" with
+ * Fig. 2; the VMonarch abstract for the entropy term).  The pages print no
+ * formulas; this library computes the following reading of them.
+ *
+ *   Video tokens n = (fi*h + hi)*w + wi, N = f*h*w, split as n = u*b2 + v with
+ *   block row u in [b1] and column v in [b2] (b1*b2 = N; the aligned choice is
+ *   (b1, b2) = (f*h, w)).  Attention softmax(Q K^T / sqrt(d)) is replaced by a
+ *   Monarch matrix M = P^T L P R: R has b1 diagonal blocks of b2 x b2, L has b2
+ *   diagonal blocks of b1 x b1, P is the perfect shuffle u*b2+v -> v*b1+u.  With
+ *   t tiles the block rows split into T_g = [floor(g*b1/t), floor((g+1)*b1/t))
+ *   and each tile g owns its own R:  M[(u,v),(u',v')] = L_v[u,u'] R_{u',g(u)}[v,v'].
+ *   L and R come from `iters` rounds of alternating maximisation of
+ *   sum_rows [<M_i, s q_i K^T> + entropy(M_i)], s = 1/sqrt(d), from uniform L:
+ *     R-step: R_{u',g}[v,:] = softmax_v'(s qbar.k_(u',v')), qbar the L-weighted
+ *             mean of the queries (u in T_g, v); it also yields the row entropy
+ *             H, Ktil = R K_u' and Z = R V_u';
+ *     L-step: L_v[u,:] = softmax_u'(s q_(u,v).Ktil[g,v,u'] + H[g,v,u']);
+ *   and the output is Y = M V, i.e. y_(u,v) = sum_u' L_v[u,u'] Z[g(u),v,u'].
+ *
+ * Tensor layout: Q, K, V and Y are contiguous [B][H][N][d] arrays (d
+ * innermost, token order as above) in the dtype given; Y has the dtype of the
+ * inputs.  All arithmetic after loading is float32 (bfloat16 operands of the
+ * tensor-core products, float32 accumulation and softmax).
+ *
+ * Conventions for every entry point:
+ *   - No call throws, aborts or traps; every call returns a monarch_status.
+ *   - Arguments are validated on the host before anything is enqueued; a call
+ *     that fails validation enqueues nothing and writes nothing.
+ *   - Device work is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream).  The caller keeps ownership of every buffer and
+ *     must keep it alive until that work has finished.
+ *   - The library keeps no global state other than a per-device cache of
+ *     kernel attributes and a device-side status word (see
+ *     monarch_last_device_status).
+ */
+#ifndef MONARCH_ATTN_H
+#define MONARCH_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MONARCH_API __attribute__((visibility("default")))
+#else
+#define MONARCH_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream, declared without the CUDA headers. */
+typedef struct CUstream_st *monarch_stream_t;
+
+typedef enum {
+    MONARCH_F32 = 0,  /* float32 inputs and output                                */
+    MONARCH_BF16 = 1  /* bfloat16 inputs and output (raw 16-bit storage)           */
+} monarch_dtype;
+
+typedef enum {
+    MONARCH_OK = 0,
+    MONARCH_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad dtype        */
+    MONARCH_ERR_SHAPE = 2,       /* b1*b2 != f*h*w, tiles outside [1, b1], iters < 1,
+                                    or a size too large for the index arithmetic     */
+    MONARCH_ERR_ALIGN = 3,       /* a pointer not 16-byte aligned                    */
+    MONARCH_ERR_UNSUPPORTED = 4, /* d not in {32, 64, 128}                           */
+    MONARCH_ERR_NO_MEMORY = 5,   /* workspace allocation failed, or ws_bytes too small */
+    MONARCH_ERR_CUDA = 6,        /* a CUDA runtime call or kernel launch failed      */
+    MONARCH_ERR_TIMEOUT = 7      /* a device-side bounded wait gave up (see below)   */
+} monarch_status;
+
+/*
+ * Forward pass with a library-managed workspace.
+ *   q, k, v   device pointers, [B][H][N][d] in `dtype`, N = f*h*w, read only.
+ *   out       device pointer, [B][H][N][d] in `dtype`, fully overwritten.
+ *   B, H      batch and heads (>= 1).     f, h, w  video latent grid (>= 1).
+ *   d         head dimension: 32, 64 or 128.
+ *   b1, b2    Monarch block sizes, b1*b2 = N (aligned choice: (f*h, w)).
+ *   tiles     tiles per block, 1 <= tiles <= b1.   iters  alternating rounds, >= 1.
+ * The workspace (monarch_attn_workspace_bytes) is taken with stream-ordered
+ * cudaMallocAsync on `stream` and released with cudaFreeAsync on it.
+ */
+MONARCH_API monarch_status monarch_attn_fwd(const void *q, const void *k, const void *v, void *out,
+                                int B, int H, int f, int h, int w, int d, int b1, int b2,
+                                int tiles, int iters, monarch_dtype dtype,
+                                monarch_stream_t stream);
+
+/*
+ * Workspace bytes that monarch_attn_fwd_ws needs for these arguments, or 0 if
+ * the arguments fail validation.  Pure host function; enqueues nothing.
+ * The workspace holds the aggregated queries, Ktil = R K and Z = R V for
+ * every (head, tile, column, block), the entropies H and, for iters > 1,
+ * the row log-sum-exp of the L-step.
+ */
+MONARCH_API size_t monarch_attn_workspace_bytes(int B, int H, int f, int h, int w, int d, int b1, int b2,
+                                    int tiles, int iters, monarch_dtype dtype);
+
+/*
+ * Forward pass with a caller-owned workspace: device memory of at least
+ * monarch_attn_workspace_bytes(...) bytes, 256-byte aligned.  Other arguments
+ * as monarch_attn_fwd.  Returns MONARCH_ERR_NO_MEMORY if ws_bytes is too small.
+ * The workspace contents need no initialisation and are garbage afterwards.
+ * Two calls that share a workspace must not overlap on the GPU.
+ */
+MONARCH_API monarch_status monarch_attn_fwd_ws(const void *q, const void *k, const void *v, void *out,
+                                   int B, int H, int f, int h, int w, int d, int b1, int b2,
+                                   int tiles, int iters, monarch_dtype dtype, void *workspace,
+                                   size_t ws_bytes, monarch_stream_t stream);
+
+/*
+ * Forward pass on HOST buffers: q, k, v, out are host pointers (pinned memory
+ * gives full PCIe bandwidth; pageable memory works but is slower).  Device
+ * copies of the inputs and output and the workspace are taken with
+ * cudaMallocAsync on `stream`; the call enqueues host-to-device copies, the
+ * forward pass and the device-to-host copy of `out`, then releases the device
+ * memory, all on `stream`.  `out` is valid once the stream has synchronised.
+ */
+MONARCH_API monarch_status monarch_attn_fwd_host(const void *q, const void *k, const void *v, void *out,
+                                     int B, int H, int f, int h, int w, int d, int b1, int b2,
+                                     int tiles, int iters, monarch_dtype dtype,
+                                     monarch_stream_t stream);
+
+/*
+ * Index maps of the method, on the host (int32, computed with the same
+ * inline functions the kernels use):
+ *   u_of_n[n] = n / b2, v_of_n[n] = n % b2, perm[n] = v*b1 + u   (each N entries),
+ *   tile_begin[g] = floor(g*b1/tiles) for g = 0..tiles        (tiles + 1 entries).
+ * Any output pointer may be NULL to skip it.
+ */
+MONARCH_API monarch_status monarch_index_maps(int f, int h, int w, int b1, int b2, int tiles,
+                                  int32_t *u_of_n, int32_t *v_of_n, int32_t *perm,
+                                  int32_t *tile_begin);
+
+/*
+ * The same maps computed by a kernel on the device into device buffers
+ * (sizes as above; NULL skips a map), enqueued on `stream`.
+ */
+MONARCH_API monarch_status monarch_index_maps_device(int f, int h, int w, int b1, int b2, int tiles,
+                                         int32_t *u_of_n, int32_t *v_of_n, int32_t *perm,
+                                         int32_t *tile_begin, monarch_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device-side status word of
+ * the current device.  Kernels that wait on barriers bound every wait; when one
+ * gives up it records MONARCH_ERR_TIMEOUT there and the kernel returns early
+ * (its output is then incomplete).  Returns MONARCH_OK if no wait gave up,
+ * MONARCH_ERR_CUDA if the synchronisation failed.
+ */
+MONARCH_API monarch_status monarch_last_device_status(monarch_stream_t stream);
+
+/*
+ * Test hook: the iteration limit of the device-side bounded waits (spins on an
+ * mbarrier).  0 restores the default.  Takes effect for launches enqueued after
+ * the call, on every device.  Returns the previous limit.
+ */
+MONARCH_API long long monarch_set_wait_limit(long long spins);
+
+/*
+ * Benchmark hook: per-kernel timing.  While enabled (on != 0), every kernel
+ * launch of the forward pass is bracketed by CUDA events recorded on its launch
+ * stream; the launches themselves are unchanged.  Disabling keeps the counters.
+ */
+MONARCH_API monarch_status monarch_profile_enable(int on);
+
+/*
+ * Waits for the recorded events, adds their durations to per-kernel counters
+ * and copies, for each kernel family k < max_kernels, the total milliseconds
+ * (ms[k]) and launch count (launches[k]) since the previous call, then resets
+ * the counters.  Either array may be NULL.  Returns the number of kernel
+ * families (the valid k), or -1 if waiting on an event failed.
+ */
+MONARCH_API int monarch_profile_collect(double *ms, long long *launches, int max_kernels);
+
+/* Name of kernel family k (static string), or NULL if k is out of range. */
+MONARCH_API const char *monarch_profile_kernel_name(int k);
+
+/* Static, NUL-terminated description of a status code. */
+MONARCH_API const char *monarch_status_string(monarch_status status);
+
+/*
+ * Which kernel family a call with these arguments dispatches to:
+ * 0 = generic SIMT kernels (any supported shape, float32 or bfloat16),
+ * 1 = sm_100a tensor-core kernels (bfloat16, d = 128, b2 <= 128, iters = 1),
+ * -1 = the arguments fail validation.  Pure host function.
+ */
+MONARCH_API int monarch_attn_path(int B, int H, int f, int h, int w, int d, int b1, int b2, int tiles,
+                      int iters, monarch_dtype dtype);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MONARCH_ATTN_H */

@@ -1,0 +1,69 @@
+"""Torch-facing entry points: argument checks and marshalling onto the C ABI.
+
+PyTorch supplies device memory (the output and the workspace, from its caching
+allocator) and the current stream; the forward pass itself runs entirely in
+the library's CUDA kernels.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+
+_DTYPES = {torch.float32: _lib.F32, torch.bfloat16: _lib.BF16}
+
+
+def _shape_args(q, f, h, w, b1, b2, tiles, iters):
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, N, d] tensors")
+    B, H, N, d = q.shape
+    if N != f * h * w:
+        raise ValueError("N = %d but f*h*w = %d" % (N, f * h * w))
+    return (B, H, f, h, w, d, b1, b2, tiles, iters)
+
+
+def _check_tensors(*ts):
+    dev = ts[0].device
+    for t in ts:
+        if not t.is_cuda or t.device != dev:
+            raise ValueError("all tensors must be on the same CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous [B, H, N, d]")
+        if t.dtype != ts[0].dtype or t.shape != ts[0].shape:
+            raise ValueError("q, k, v and out must share dtype and shape")
+    if ts[0].dtype not in _DTYPES:
+        raise ValueError("dtype must be float32 or bfloat16")
+
+
+def workspace_bytes(q, *, f, h, w, b1, b2, tiles=1, iters=1) -> int:
+    args = _shape_args(q, f, h, w, b1, b2, tiles, iters)
+    return _lib.monarch_attn_workspace_bytes(*args, _DTYPES[q.dtype])
+
+
+def kernel_path(q, *, f, h, w, b1, b2, tiles=1, iters=1) -> int:
+    """0 = generic SIMT kernels, 1 = sm_100a tensor-core kernels."""
+    args = _shape_args(q, f, h, w, b1, b2, tiles, iters)
+    return _lib.monarch_attn_path(*args, _DTYPES[q.dtype])
+
+
+def monarch_attention(q, k, v, *, f, h, w, b1, b2, tiles=1, iters=1, out=None, workspace=None):
+    """Y = M V with M the tiled Monarch approximation of softmax(Q K^T / sqrt(d))."""
+    if out is None:
+        out = torch.empty_like(q)
+    _check_tensors(q, k, v, out)
+    args = _shape_args(q, f, h, w, b1, b2, tiles, iters)
+    dt = _DTYPES[q.dtype]
+    need = _lib.monarch_attn_workspace_bytes(*args, dt)
+    if need == 0:
+        # validation failed: let the library report why
+        _lib.check(_lib.monarch_attn_fwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                            out.data_ptr(), *args, dt, 0, 0, 0),
+                   "monarch_attn_fwd_ws")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    _lib.check(_lib.monarch_attn_fwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                        *args, dt, workspace.data_ptr(),
+                                        workspace.numel() * workspace.element_size(), stream),
+               "monarch_attn_fwd_ws")
+    return out

@@ -1,0 +1,103 @@
+// monarch_common.cuh -- index arithmetic, problem description and the device
+// status word shared by the kernels of the Monarch attention library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/monarch_attn.h"
+
+namespace monarch {
+
+// Token n = u*b2 + v (block row u, column v); the Monarch permutation P sends
+// it to v*b1 + u (explainer page, "Monarch矩阵" section: a fixed permutation
+// between the two block-diagonal factors).
+__host__ __device__ __forceinline__ int block_row(int64_t n, int b2) { return (int)(n / b2); }
+__host__ __device__ __forceinline__ int block_col(int64_t n, int b2) { return (int)(n % b2); }
+__host__ __device__ __forceinline__ int64_t shuffle(int u, int v, int b1) {
+    return (int64_t)v * b1 + u;
+}
+
+// Tiled Monarch ("创新二：平铺Monarch参数化", Fig. 2): block rows split into t
+// contiguous tiles T_g = [floor(g*b1/t), floor((g+1)*b1/t)).
+__host__ __device__ __forceinline__ int tile_begin(int g, int b1, int tiles) {
+    return (int)(((int64_t)g * b1) / tiles);
+}
+__host__ __device__ __forceinline__ int tile_max_rows(int b1, int tiles) {
+    return (b1 + tiles - 1) / tiles;
+}
+
+// Everything a kernel needs to know about one call.
+struct Problem {
+    int B, H, BH;        // batch, heads, B*H
+    int N, d;            // tokens per head, head dim
+    int b1, b2, tiles;   // Monarch blocks and tiles
+    int iters;
+    float scale;         // 1/sqrt(d)
+};
+
+// Kernels that can give up a bounded wait receive a pointer to the device
+// status word of the library (one int per device, read and cleared by
+// monarch_last_device_status) and record MONARCH_ERR_TIMEOUT there.
+constexpr long long kDefaultWaitLimit = 1LL << 26;
+
+__device__ __forceinline__ void record_status(int *status, int code) {
+    atomicCAS(status, 0, code);
+}
+
+// Kernel families, for the optional per-kernel timing of monarch_profile_*.
+enum KernelId {
+    K_QBAR_MEAN = 0,      // S1, generic
+    K_RSTEP = 1,          // S2, generic
+    K_LSTEP = 2,          // S3, generic
+    K_QBAR_WEIGHTED = 3,  // S4, generic
+    K_TC_QBAR = 4,        // S1, tensor-core path
+    K_TC_RSTEP = 5,       // S2, tensor-core path
+    K_TC_LSTEP = 6,       // S3, tensor-core path
+    K_COUNT = 7
+};
+
+// Brackets one kernel launch with CUDA events while profiling is enabled.
+class ProfileScope {
+  public:
+    ProfileScope(KernelId id, cudaStream_t stream);
+    ~ProfileScope();
+
+  private:
+    KernelId id_;
+    cudaStream_t stream_;
+    void *start_ = nullptr;
+};
+
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+    return __bfloat162float(x);
+}
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Generic (SIMT) path: float32 intermediates.
+struct GenericWorkspace {
+    float *qbar;   // iters == 1: [BH][t][b2][d];  iters > 1: [BH][t][b2][b1][d]
+    float *ktil;   // [BH][t][b2][b1][d]   Ktil[g][v][u'] = sum_v' R_{u',g}[v,v'] k_(u',v')
+    float *z;      // [BH][t][b2][b1][d]   Z[g][v][u']    = sum_v' R_{u',g}[v,v'] v_(u',v')
+    float *hent;   // [BH][t][b2][b1]      entropy of R_{u',g}[v,:]
+    float *lse;    // [BH][N]              row log-sum-exp of the L-step (iters > 1)
+};
+
+size_t generic_workspace_bytes(const Problem &p, bool &overflow);
+GenericWorkspace generic_workspace_carve(const Problem &p, void *base);
+cudaError_t generic_forward(const Problem &p, monarch_dtype dtype, const void *q, const void *k,
+                            const void *v, void *out, const GenericWorkspace &ws,
+                            cudaStream_t stream);
+
+cudaError_t index_maps_device(int N, int b1, int b2, int tiles, int32_t *u_of_n,
+                              int32_t *v_of_n, int32_t *perm, int32_t *tile_lo,
+                              cudaStream_t stream);
+
+}  // namespace monarch

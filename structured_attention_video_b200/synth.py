@@ -9,7 +9,8 @@ Random numbers
     pseudorandom number generators", OOPSLA 2014; the 64-bit finaliser of
     Vigna's public-domain splitmix64) feeds the Box-Muller transform (Box and
     Muller, 1958).  Element i of a stream with key K is mix(K + (i + 1) * GAMMA),
-    so any element can be produced independently and in any order.
+    so any element can be produced independently and in any order.  The
+    streams and the bfloat16 rounding run in synth_gen.c (OpenMP).
 
 Data recipe (MonarchRT, "Block alignment" and "Tiled Monarch" sections of the
 explainer page; the (f, h, w) video layout with N = f*h*w tokens)
@@ -31,14 +32,15 @@ explainer page; the (f, h, w) video layout with N = f*h*w tokens)
 """
 from __future__ import annotations
 
+import ctypes
 import dataclasses
 import math
+import os
+import subprocess
 
 import numpy as np
 
-GAMMA = np.uint64(0x9E3779B97F4A7C15)
-_M1 = np.uint64(0xBF58476D1CE4E5B9)
-_M2 = np.uint64(0x94D049BB133111EB)
+GAMMA = 0x9E3779B97F4A7C15
 
 TENSOR_IDS = {"q": 1, "k": 2, "v": 3, "pairs": 4}
 
@@ -109,41 +111,64 @@ WORKLOADS = {
 
 
 # ----------------------------------------------------------------------------
-# counter-based generator
+# counter-based generator (synth_gen.c, built on first use with gcc + OpenMP)
 # ----------------------------------------------------------------------------
-def _mix64(z: np.ndarray) -> np.ndarray:
-    z = (z ^ (z >> np.uint64(30))) * _M1
-    z = (z ^ (z >> np.uint64(27))) * _M2
-    return z ^ (z >> np.uint64(31))
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_GEN_SRC = os.path.join(_HERE, "synth_gen.c")
+_GEN_LIB = os.path.join(_HERE, "_build", "libsynth.so")
+_gen = None
 
 
-def stream_key(seed: int, b: int, h: int, tensor: str, rank: int = 0) -> np.uint64:
+def build_generator(force: bool = False) -> str:
+    if force or not os.path.exists(_GEN_LIB) or \
+            os.path.getmtime(_GEN_LIB) < os.path.getmtime(_GEN_SRC):
+        os.makedirs(os.path.dirname(_GEN_LIB), exist_ok=True)
+        tmp = _GEN_LIB + ".tmp%d" % os.getpid()
+        subprocess.run(["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared", _GEN_SRC,
+                        "-o", tmp, "-lm"], check=True)
+        os.replace(tmp, _GEN_LIB)
+    return _GEN_LIB
+
+
+def _lib():
+    global _gen
+    if _gen is None:
+        lib = ctypes.CDLL(build_generator())
+        u64, i64 = ctypes.c_uint64, ctypes.c_int64
+        dp = ctypes.POINTER(ctypes.c_double)
+        lib.synth_mix64.argtypes = [u64]
+        lib.synth_mix64.restype = u64
+        lib.synth_uniform53.argtypes = [u64, i64, i64, dp]
+        lib.synth_normals.argtypes = [u64, i64, dp]
+        lib.synth_round_bf16.argtypes = [dp, i64, dp, ctypes.POINTER(ctypes.c_uint16)]
+        _gen = lib
+    return _gen
+
+
+def _dp(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def stream_key(seed: int, b: int, h: int, tensor: str, rank: int = 0) -> int:
     """Key of the stream for (seed, rank, b, h, tensor): a SplitMix64 mix of the fields."""
-    with np.errstate(over="ignore"):
-        x = np.uint64(seed & 0xFFFFFFFF)
-        for field in (rank, b, h, TENSOR_IDS[tensor]):
-            x = _mix64(np.array([x + GAMMA * np.uint64(field + 1)], dtype=np.uint64))[0]
+    x = seed & 0xFFFFFFFF
+    for field in (rank, b, h, TENSOR_IDS[tensor]):
+        x = _lib().synth_mix64((x + GAMMA * (field + 1)) & 0xFFFFFFFFFFFFFFFF)
     return x
 
 
-def uniform53(key: np.uint64, start: int, count: int) -> np.ndarray:
+def uniform53(key: int, start: int, count: int) -> np.ndarray:
     """Elements [start, start+count) of stream `key` as doubles in (0, 1]."""
-    with np.errstate(over="ignore"):
-        i = np.arange(start + 1, start + count + 1, dtype=np.uint64)
-        z = _mix64(key + i * GAMMA)
-    return ((z >> np.uint64(11)).astype(np.float64) + 1.0) * (1.0 / 9007199254740992.0)
+    out = np.empty(count, dtype=np.float64)
+    _lib().synth_uniform53(key, start, count, _dp(out))
+    return out
 
 
-def normals(key: np.uint64, count: int) -> np.ndarray:
+def normals(key: int, count: int) -> np.ndarray:
     """`count` standard normals from stream `key` (Box-Muller on consecutive pairs)."""
-    m = (count + 1) // 2
-    u = uniform53(key, 0, 2 * m)
-    r = np.sqrt(-2.0 * np.log(u[0::2]))
-    th = (2.0 * math.pi) * u[1::2]
-    out = np.empty(2 * m, dtype=np.float64)
-    out[0::2] = r * np.cos(th)
-    out[1::2] = r * np.sin(th)
-    return out[:count]
+    out = np.empty(count, dtype=np.float64)
+    _lib().synth_normals(key, count, _dp(out))
+    return out
 
 
 # ----------------------------------------------------------------------------
@@ -155,12 +180,9 @@ def round_to_dtype(x: np.ndarray, dtype: str) -> np.ndarray:
         return x.astype(np.float32).astype(np.float64)
     if dtype != "bf16":
         raise ValueError(dtype)
-    m, e = np.frexp(x)                     # x = m * 2^e, 0.5 <= |m| < 1
-    r = np.rint(m * 256.0)                 # 8 significant bits, ties to even
-    out = np.ldexp(r, e - 8)
-    small = np.abs(x) < 2.0 ** -126        # bf16 subnormal range: fixed spacing 2^-133
-    if small.any():
-        out[small] = np.rint(x[small] * 2.0 ** 133) * 2.0 ** -133
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty_like(x)
+    _lib().synth_round_bf16(_dp(x), x.size, _dp(out), None)
     return out
 
 

@@ -1,0 +1,224 @@
+"""CUDA path against the float64 oracle, element by element on seeded inputs.
+
+Tolerances: relative Frobenius error <= 1e-5 for float32 inputs and <= 1e-2 for
+bfloat16 inputs (float32 accumulation); index maps bit-exact.  Small shapes
+compare the whole output; the full-size shapes of the benchmark compare sampled
+(head, tile, column) problems, which the oracle computes one by one, plus
+properties that hold at any size (every output row is a convex combination of
+value rows)."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+from oracle import oracle  # noqa: E402
+from structured_attention_video_b200 import _lib, synth  # noqa: E402
+from structured_attention_video_b200.attention import kernel_path, monarch_attention  # noqa: E402
+
+from helpers import TOL, device_inputs, from_torch, rel_fro, sample_problems, sampled_error, to_torch  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+TINY = synth.WORKLOADS["tiny"]
+
+
+def dense_attention(q, k, v):
+    s = q @ np.swapaxes(k, -1, -2) / np.sqrt(q.shape[-1])
+    s -= s.max(-1, keepdims=True)
+    p = np.exp(s)
+    p /= p.sum(-1, keepdims=True)
+    return p @ v
+
+
+def run(wl, q, k, v, **kw):
+    args = dict(f=wl.f, h=wl.h, w=wl.w, b1=wl.b1, b2=wl.b2, tiles=wl.tiles, iters=wl.iters)
+    args.update(kw)
+    out = monarch_attention(q, k, v, **args)
+    torch.cuda.synchronize()
+    assert _lib.monarch_last_device_status(None) == 0
+    return out
+
+
+@pytest.fixture(scope="module")
+def tiny64():
+    return synth.make_inputs(TINY)
+
+
+# --------------------------------------------------------------------------
+# whole-output parity on small shapes (several tiles, ragged tails)
+# --------------------------------------------------------------------------
+SMALL = [(24, 8, 1, 1), (24, 8, 5, 1), (24, 8, 24, 1), (24, 8, 5, 2), (24, 8, 3, 3),
+         (1, 192, 1, 1), (192, 1, 1, 1), (192, 1, 7, 2), (3, 64, 2, 1), (8, 24, 3, 2),
+         (12, 16, 5, 1)]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("b1,b2,tiles,iters", SMALL)
+def test_tiny_whole_output(tiny64, dtype, b1, b2, tiles, iters):
+    q64, k64, v64 = (synth.round_to_dtype(x, dtype) for x in tiny64)
+    ref = oracle.monarch_attn(q64, k64, v64, b1, b2, tiles, iters)
+    q, k, v = (to_torch(x, dtype) for x in (q64, k64, v64))
+    out = run(TINY, q, k, v, b1=b1, b2=b2, tiles=tiles, iters=iters)
+    got = from_torch(out, dtype)
+    assert np.isfinite(got).all()
+    assert rel_fro(got, ref) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+def test_head_dims_and_odd_shapes_f32(d):
+    wl = TINY.replace(d=d, f=2, h=5, w=7, b1=10, b2=7, tiles=3, H=3)
+    q64, k64, v64 = synth.make_inputs(wl)
+    ref = oracle.monarch_attn(q64, k64, v64, wl.b1, wl.b2, wl.tiles, 2)
+    q, k, v = (to_torch(x, "f32") for x in (q64, k64, v64))
+    got = from_torch(run(wl, q, k, v, iters=2), "f32")
+    assert rel_fro(got, ref) <= TOL["f32"]
+
+
+def test_single_token_is_identity_on_v():
+    wl = TINY.replace(f=1, h=1, w=1, b1=1, b2=1, H=1)
+    q64, k64, v64 = synth.make_inputs(wl)
+    q, k, v = (to_torch(x, "f32") for x in (q64, k64, v64))
+    got = from_torch(run(wl, q, k, v), "f32")
+    assert np.array_equal(got, v64)
+
+
+def test_zero_queries_give_mean_of_v(tiny64):
+    _, k64, v64 = tiny64
+    q = torch.zeros(to_torch(k64, "f32").shape, device="cuda")
+    k, v = to_torch(k64, "f32"), to_torch(v64, "f32")
+    got = from_torch(run(TINY, q, k, v, tiles=5, iters=2), "f32")
+    assert np.abs(got - v64.mean(-2, keepdims=True)).max() < 1e-5
+
+
+def test_chunk_480p_whole_output():
+    wl = synth.WORKLOADS["480p_chunk"]
+    q, k, v = device_inputs(wl)
+    out = run(wl, q, k, v)
+    q64, k64, v64 = (from_torch(x, wl.dtype) for x in (q, k, v))
+    ref = oracle.monarch_attn(q64, k64, v64, wl.b1, wl.b2, wl.tiles, wl.iters)
+    assert rel_fro(from_torch(out, wl.dtype), ref) <= TOL[wl.dtype]
+
+
+def test_chunk_480p_one_block_is_exact_attention():
+    """b1 = 1: a single R block of N x N, i.e. softmax attention (checked on 2 heads)."""
+    wl = synth.WORKLOADS["480p_chunk"].replace(H=2, b1=1, b2=4680)
+    q, k, v = device_inputs(wl)
+    out = from_torch(run(wl, q, k, v), wl.dtype)
+    q64, k64, v64 = (from_torch(x, wl.dtype) for x in (q, k, v))
+    assert rel_fro(out, dense_attention(q64, k64, v64)) <= TOL[wl.dtype]
+
+
+# --------------------------------------------------------------------------
+# full-size shapes: sampled problems and size-independent properties
+# --------------------------------------------------------------------------
+def convex_hull_check(out, v):
+    """Every output row is a convex combination of value rows of its head."""
+    o = out.float()
+    vf = v.float()
+    lo = vf.amin(dim=2, keepdim=True)
+    hi = vf.amax(dim=2, keepdim=True)
+    slack = 1e-2 * (hi - lo) + 1e-6
+    assert torch.isfinite(o).all()
+    assert bool(((o >= lo - slack) & (o <= hi + slack)).all())
+
+
+@pytest.fixture(scope="module")
+def inputs_480p():
+    return device_inputs(synth.WORKLOADS["480p_full"])
+
+
+@pytest.mark.parametrize("tiles", [1, 2, 4, 8])
+def test_full_480p_tile_sweep(inputs_480p, tiles):
+    wl = synth.WORKLOADS["480p_full"].replace(tiles=tiles)
+    q, k, v = inputs_480p
+    out = run(wl, q, k, v)
+    convex_hull_check(out, v)
+    probs = sample_problems(wl, 12, seed=tiles)
+    assert sampled_error(wl, out, probs) <= TOL[wl.dtype]
+
+
+@pytest.fixture(scope="module")
+def inputs_720p():
+    return device_inputs(synth.WORKLOADS["720p"])
+
+
+def test_full_720p_headline(inputs_720p):
+    wl = synth.WORKLOADS["720p"]
+    q, k, v = inputs_720p
+    out = run(wl, q, k, v)
+    convex_hull_check(out, v)
+    probs = sample_problems(wl, 24, seed=720)
+    assert sampled_error(wl, out, probs) <= TOL[wl.dtype]
+
+
+def test_full_720p_deterministic(inputs_720p):
+    wl = synth.WORKLOADS["720p"]
+    q, k, v = inputs_720p
+    a = run(wl, q, k, v)
+    b = run(wl, q, k, v)
+    assert torch.equal(a, b)
+
+
+@pytest.fixture(scope="module")
+def inputs_14b():
+    return device_inputs(synth.WORKLOADS["14b"])
+
+
+@pytest.mark.parametrize("iters", [1, 2, 5, 10])
+def test_full_14b_iteration_sweep(inputs_14b, iters):
+    wl = synth.WORKLOADS["14b"].replace(iters=iters)
+    q, k, v = inputs_14b
+    out = run(wl, q, k, v)
+    convex_hull_check(out, v)
+    probs = sample_problems(wl, 8, seed=iters)
+    assert sampled_error(wl, out, probs) <= TOL[wl.dtype]
+
+
+# --------------------------------------------------------------------------
+# entry points and maps
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("f,h,w,b1,b2,tiles", [(3, 8, 8, 24, 8, 5), (3, 8, 8, 192, 1, 192),
+                                                (21, 45, 80, 945, 80, 4),
+                                                (21, 30, 52, 630, 52, 8)])
+def test_device_index_maps_bit_exact(f, h, w, b1, b2, tiles):
+    N = f * h * w
+    maps = [torch.full((N,), -1, dtype=torch.int32, device="cuda") for _ in range(3)]
+    tb = torch.full((tiles + 1,), -1, dtype=torch.int32, device="cuda")
+    st = _lib.monarch_index_maps_device(f, h, w, b1, b2, tiles, *(m.data_ptr() for m in maps),
+                                        tb.data_ptr(), None)
+    assert st == 0
+    torch.cuda.synchronize()
+    ref = oracle.index_maps(f, h, w, b1, b2, tiles)
+    for m, key in zip(maps, ("u_of_n", "v_of_n", "perm")):
+        assert np.array_equal(m.cpu().numpy(), ref[key])
+    assert np.array_equal(tb.cpu().numpy(), ref["tile_lo"])
+
+
+def test_entry_points_agree(tiny64):
+    """monarch_attn_fwd (library workspace), _ws and _host give identical bits."""
+    wl = TINY.replace(tiles=5, iters=2)
+    q64, k64, v64 = tiny64
+    q, k, v = (to_torch(x, "f32") for x in (q64, k64, v64))
+    ref = run(wl, q, k, v)
+    shape = (wl.B, wl.H, wl.f, wl.h, wl.w, wl.d, wl.b1, wl.b2, wl.tiles, wl.iters)
+    out = torch.empty_like(q)
+    assert _lib.monarch_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                 *shape, _lib.F32, None) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+    oh = torch.empty_like(qh).pin_memory()
+    assert _lib.monarch_attn_fwd_host(qh.data_ptr(), kh.data_ptr(), vh.data_ptr(), oh.data_ptr(),
+                                      *shape, _lib.F32, None) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(oh, ref.cpu())
+
+
+def test_device_entry_points_reject_bad_buffers(tiny64):
+    q = to_torch(tiny64[0], "f32")
+    shape = (1, 2, 3, 8, 8, 32, 24, 8, 1, 1)
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+    p = q.data_ptr()
+    assert _lib.monarch_attn_fwd_ws(p + 4, p, p, p, *shape, 0, ws.data_ptr(), 1 << 20, None) == 3
+    assert _lib.monarch_attn_fwd_ws(p, p, p, p, *shape, 0, ws.data_ptr(), 64, None) == 5
+    assert _lib.monarch_last_device_status(None) == 0
