@@ -72,7 +72,9 @@ typedef enum {
     MONARCH_ERR_UNSUPPORTED = 4, /* d not in {32, 64, 128}                           */
     MONARCH_ERR_NO_MEMORY = 5,   /* workspace allocation failed, or ws_bytes too small */
     MONARCH_ERR_CUDA = 6,        /* a CUDA runtime call or kernel launch failed      */
-    MONARCH_ERR_TIMEOUT = 7      /* a device-side bounded wait gave up (see below)   */
+    MONARCH_ERR_TIMEOUT = 7,     /* a device-side bounded wait gave up (see below)   */
+    MONARCH_ERR_SCRATCH_LIMIT = 8 /* needs more scratch than monarch_attn_fwd_noalloc's
+                                     static buffer (MONARCH_NOALLOC_SCRATCH_BYTES)    */
 } monarch_status;
 
 /*
@@ -90,6 +92,39 @@ MONARCH_API monarch_status monarch_attn_fwd(const void *q, const void *k, const 
                                 int B, int H, int f, int h, int w, int d, int b1, int b2,
                                 int tiles, int iters, monarch_dtype dtype,
                                 monarch_stream_t stream);
+
+/*
+ * Forward pass that allocates nothing.  (No counterpart in the MonarchRT
+ * pages: this is a deployment convenience of this library.)
+ *
+ * For callers that may not allocate device memory: code whose host framework
+ * owns every device allocation and forbids others, or loops where the implicit
+ * device synchronisation of cudaMalloc/cudaFree is not acceptable.  The call
+ * takes no workspace argument and calls no cudaMalloc, cudaFree, cudaMallocAsync
+ * or other allocating routine: its scratch space is one file-scope static
+ * device array of MONARCH_NOALLOC_SCRATCH_BYTES (64 MiB), which every GPU that
+ * loads the library's no-allocation module holds until the process exits.
+ *
+ * Arguments and layout as monarch_attn_fwd (q, k, v, out: caller-owned device
+ * buffers).  It runs the generic kernel family (any supported shape and dtype)
+ * with its float32 intermediates placed in the static array; problems whose
+ * scratch exceeds the array are rejected with MONARCH_ERR_SCRATCH_LIMIT before
+ * anything is enqueued.  The 480p chunk shape (B=1, H=12, d=128, N=4680) fits.
+ *
+ * The first call on each device looks up the array's device address with
+ * cudaGetSymbolAddress (with that device current); make that first call before
+ * any stream capture.  Every call on a device shares the one array, which keeps
+ * the contents of the last call; nothing in it needs to start at zero.  Calls
+ * that overlap on the GPU (different streams without ordering, or several host
+ * threads) race on the array and give wrong results: serialise them.
+ */
+#define MONARCH_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+MONARCH_API monarch_status monarch_attn_fwd_noalloc(const void *q, const void *k, const void *v,
+                                                    void *out, int B, int H, int f, int h,
+                                                    int w, int d, int b1, int b2, int tiles,
+                                                    int iters, monarch_dtype dtype,
+                                                    monarch_stream_t stream);
 
 /*
  * Workspace bytes that monarch_attn_fwd_ws needs for these arguments, or 0 if

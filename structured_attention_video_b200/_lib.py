@@ -22,7 +22,8 @@ _lib = ctypes.CDLL(LIB_PATH)
 F32, BF16 = 0, 1
 STATUS = {0: "MONARCH_OK", 1: "MONARCH_ERR_INVALID_ARG", 2: "MONARCH_ERR_SHAPE",
           3: "MONARCH_ERR_ALIGN", 4: "MONARCH_ERR_UNSUPPORTED", 5: "MONARCH_ERR_NO_MEMORY",
-          6: "MONARCH_ERR_CUDA", 7: "MONARCH_ERR_TIMEOUT"}
+          6: "MONARCH_ERR_CUDA", 7: "MONARCH_ERR_TIMEOUT", 8: "MONARCH_ERR_SCRATCH_LIMIT"}
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _vp, _i, _sz, _ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_longlong
 _ip = ctypes.POINTER(ctypes.c_int32)
@@ -33,6 +34,7 @@ SIGNATURES = {
     "monarch_attn_workspace_bytes": (_SHAPE + [_i], _sz),
     "monarch_attn_fwd_ws": ([_vp, _vp, _vp, _vp] + _SHAPE + [_i, _vp, _sz, _vp], _i),
     "monarch_attn_fwd_host": ([_vp, _vp, _vp, _vp] + _SHAPE + [_i, _vp], _i),
+    "monarch_attn_fwd_noalloc": ([_vp, _vp, _vp, _vp] + _SHAPE + [_i, _vp], _i),
     "monarch_index_maps": ([_i] * 6 + [_ip, _ip, _ip, _ip], _i),
     "monarch_index_maps_device": ([_i] * 6 + [_vp, _vp, _vp, _vp, _vp], _i),
     "monarch_last_device_status": ([_vp], _i),
@@ -81,6 +83,12 @@ def monarch_attn_fwd_ws(q, k, v, out, B, H, f, h, w, d, b1, b2, tiles, iters, dt
 def monarch_attn_fwd_host(q, k, v, out, B, H, f, h, w, d, b1, b2, tiles, iters, dtype, stream):
     return _lib.monarch_attn_fwd_host(q, k, v, out, B, H, f, h, w, d, b1, b2, tiles, iters,
                                       dtype, stream)
+
+
+def monarch_attn_fwd_noalloc(q, k, v, out, B, H, f, h, w, d, b1, b2, tiles, iters, dtype,
+                             stream):
+    return _lib.monarch_attn_fwd_noalloc(q, k, v, out, B, H, f, h, w, d, b1, b2, tiles, iters,
+                                         dtype, stream)
 
 
 def monarch_index_maps(f, h, w, b1, b2, tiles, u_of_n, v_of_n, perm, tile_begin):

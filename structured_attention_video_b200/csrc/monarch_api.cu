@@ -55,6 +55,8 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
+}  // namespace
+
 monarch_status validate_shape(int B, int H, int f, int h, int w, int d, int b1, int b2, int tiles,
                               int iters, monarch_dtype dtype, Problem *p) {
     if (B < 1 || H < 1 || f < 1 || h < 1 || w < 1 || d < 1 || b1 < 1 || b2 < 1)
@@ -84,6 +86,8 @@ monarch_status validate_shape(int B, int H, int f, int h, int w, int d, int b1, 
     p->scale = (float)(1.0 / sqrt((double)d));
     return MONARCH_OK;
 }
+
+namespace {
 
 int choose_path(const Problem &p, monarch_dtype dtype) {
     return sm100_supports(p, dtype) ? 1 : 0;
@@ -357,6 +361,8 @@ const char *monarch_status_string(monarch_status status) {
         case MONARCH_ERR_NO_MEMORY: return "workspace allocation failed or too small";
         case MONARCH_ERR_CUDA: return "CUDA error";
         case MONARCH_ERR_TIMEOUT: return "device-side wait timed out";
+        case MONARCH_ERR_SCRATCH_LIMIT:
+            return "problem needs more scratch than the no-allocation entry point's static buffer";
     }
     return "unknown status";
 }

@@ -81,6 +81,10 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
+// Host-side argument validation shared by the entry points; fills *p on success.
+monarch_status validate_shape(int B, int H, int f, int h, int w, int d, int b1, int b2, int tiles,
+                              int iters, monarch_dtype dtype, Problem *p);
+
 // Generic (SIMT) path: float32 intermediates.
 struct GenericWorkspace {
     float *qbar;   // iters == 1: [BH][t][b2][d];  iters > 1: [BH][t][b2][b1][d]
