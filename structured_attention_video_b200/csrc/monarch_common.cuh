@@ -40,7 +40,7 @@ struct Problem {
 // Kernels that can give up a bounded wait receive a pointer to the device
 // status word of the library (one int per device, read and cleared by
 // monarch_last_device_status) and record MONARCH_ERR_TIMEOUT there.
-constexpr long long kDefaultWaitLimit = 1LL << 26;
+constexpr long long kDefaultWaitLimit = 1LL << 22;
 
 __device__ __forceinline__ void record_status(int *status, int code) {
     atomicCAS(status, 0, code);

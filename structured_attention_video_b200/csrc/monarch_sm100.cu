@@ -1,18 +1,871 @@
-// monarch_sm100.cu -- sm_100a tensor-core kernels (tcgen05 / TMEM / TMA).
+// monarch_sm100.cu -- sm_100a tensor-core kernels of the Monarch attention
+// forward pass (bfloat16 inputs, d = 128, one alternating iteration).
+//
+// Steps (MonarchAttention as the MonarchRT pages describe it: explainer page,
+// "Monarch矩阵" section and Fig. 3; tiles from "创新二：平铺Monarch参数化", Fig. 2;
+// the entropy term after the VMonarch abstract's online entropy):
+//   S1 tc_qbar_kernel   qbar[g][v] = mean_{u in T_g} q_(u,v) -> bf16, rows
+//                       r = g*b2 + v of a [t*b2 padded to 128] x d tile stack
+//   S2 tc_rstep_kernel  per block u' and 128-row tile of qbar:
+//                         S = qbar K_u'^T                  (tcgen05, SMEM x SMEM)
+//                         R = rowsoftmax(s S), H = entropy (float32, per thread row)
+//                         [Z | Ktil] = R [V_u' | K_u']     (tcgen05, R from TMEM)
+//                       Z and Ktil leave through TMA stores whose 4-D tensor map
+//                       folds the Monarch permutation: row (g, v) of block u'
+//                       lands at [bh][g*b2+v][u'] (rows past t*b2 are clipped).
+//   S3 tc_lstep_kernel  per (bh, g, v) and pair of 128-query tiles: the queries
+//                       (u, v), u in T_g, come through a 3-D tensor map that
+//                       strides over b2 (P^T folded into the load); online
+//                       softmax over the b1 blocks with logits s q.Ktil + H,
+//                       O accumulated in TMEM, rows written back strided.
+// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM
+// owner, warps 4-7 and 8-11 the two softmax (L-step) or the softmax and
+// epilogue (R-step) warpgroups; warps 2-3 idle.  Every wait on another role is
+// a bounded mbarrier wait (tc_primitives.cuh): on time-out the kernel records
+// MONARCH_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
 #include "monarch_sm100.cuh"
+#include "tc_primitives.cuh"
+
+#include <mutex>
 
 namespace monarch {
+namespace {
 
-bool sm100_supports(const Problem &, monarch_dtype) { return false; }
+using namespace tc;
 
-size_t sm100_workspace_bytes(const Problem &, bool &overflow) {
-    overflow = false;
-    return 0;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kD = 128;                        // head dimension of this path
+constexpr uint32_t kPanel = 128 * 128;         // 128 rows x 64 bf16 (128 B), SW128
+constexpr uint32_t kTile = 2 * kPanel;         // 128 rows x 128 bf16
+constexpr int kMaxSmem = 232448;               // sm_100 opt-in dynamic shared memory
+constexpr long long kCleanupPolls = 1LL << 22;
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-cudaError_t sm100_forward(const Problem &, const void *, const void *, const void *, void *,
-                          void *, int *, long long, cudaStream_t) {
-    return cudaErrorNotSupported;
+// Warp-uniform bounded wait: all 32 lanes take the same decision.
+__device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, const WaitCtx &w) {
+    bool ok = wait_phase(bar, parity, w);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// =====================================================================
+// S1: aggregated queries
+// =====================================================================
+__global__ void __launch_bounds__(128) tc_qbar_kernel(const __nv_bfloat16 *__restrict__ q,
+                                                      __nv_bfloat16 *__restrict__ qbar, Problem p,
+                                                      int mpad) {
+    const int row_elems = p.b2 * kD;
+    const int nchunk = (row_elems / 8 + 127) / 128;
+    const int chunk = blockIdx.x % nchunk;
+    const int bhg = blockIdx.x / nchunk;
+    const int g = bhg % p.tiles, bh = bhg / p.tiles;
+    const int col = (chunk * 128 + threadIdx.x) * 8;
+    const int u0 = tile_begin(g, p.b1, p.tiles), u1 = tile_begin(g + 1, p.b1, p.tiles);
+    if (col < row_elems) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(q + (int64_t)bh * p.N * kD +
+                                                           (int64_t)u0 * row_elems + col);
+        const int64_t stride = row_elems / 8;
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++) acc[i] = 0.f;
+        int u = u0;
+        for (; u + 4 <= u1; u += 4) {
+            uint4 x[4];
+#pragma unroll
+            for (int k = 0; k < 4; k++) x[k] = __ldg(src + k * stride);
+            src += 4 * stride;
+#pragma unroll
+            for (int k = 0; k < 4; k++) {
+                const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&x[k]);
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    float2 f = __bfloat1622float2(h[i]);
+                    acc[2 * i] += f.x;
+                    acc[2 * i + 1] += f.y;
+                }
+            }
+        }
+        for (; u < u1; u++) {
+            uint4 x = __ldg(src);
+            src += stride;
+            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&x);
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                float2 f = __bfloat1622float2(h[i]);
+                acc[2 * i] += f.x;
+                acc[2 * i + 1] += f.y;
+            }
+        }
+        const float inv = 1.f / (float)(u1 - u0);
+        uint4 o;
+        uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+        for (int i = 0; i < 4; i++) ow[i] = pack_bf16(acc[2 * i] * inv, acc[2 * i + 1] * inv);
+        *reinterpret_cast<uint4 *>(qbar + ((int64_t)bh * mpad + (int64_t)g * p.b2) * kD + col) = o;
+    }
+    if (g == 0) {   // zero the padding rows [t*b2, mpad) of this head
+        const int64_t pad = (int64_t)(mpad - p.tiles * p.b2) * kD;
+        __nv_bfloat16 *base = qbar + ((int64_t)bh * mpad + (int64_t)p.tiles * p.b2) * kD;
+        for (int64_t e = col; e < pad; e += (int64_t)nchunk * 128 * 8)
+            *reinterpret_cast<uint4 *>(base + e) = make_uint4(0, 0, 0, 0);
+    }
+}
+
+// =====================================================================
+// S3: L-step with the output
+// =====================================================================
+namespace ls {
+constexpr uint32_t kQ = 0;               // query tiles 0, 1
+constexpr uint32_t kK = 2 * kTile;       // Ktil stages 0, 1
+constexpr uint32_t kZ = 4 * kTile;       // Z stages 0, 1
+constexpr uint32_t kH = 6 * kTile;       // H * log2(e) per stage: [2][128] floats
+constexpr uint32_t kBar = kH + 1024;
+constexpr uint32_t kSmem = kBar + 256 + 1024;
+}  // namespace ls
+
+struct LsArgs {
+    Problem p;
+    int nchunks;    // key chunks of 128 blocks
+    int npairs;     // pairs of 128-query tiles per (g, v)
+    float c_log2;   // (1/sqrt(d)) * log2(e)
+    const float *hent;
+    __nv_bfloat16 *out;
+    int *status;
+    long long limit;
+};
+
+__global__ void __launch_bounds__(384, 1)
+tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmZ, LsArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = align1024(smem_raw);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + ls::kBar);
+    uint64_t *q_full = bars + 0;
+    uint64_t *k_full = bars + 1;     // [2 stages]
+    uint64_t *z_full = bars + 3;     // [2 stages]
+    uint64_t *h_full = bars + 5;     // [2 stages], 32 arrivals
+    uint64_t *kv_empty = bars + 7;   // [2 stages]
+    uint64_t *s_full = bars + 9;     // [2 tiles]
+    uint64_t *p_full = bars + 11;    // [2 tiles], 128 arrivals
+    uint64_t *o_full = bars + 13;    // [2 tiles]
+    uint64_t *mma_done = bars + 15;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 17);
+
+    const Problem &p = a.p;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int unit = blockIdx.x;
+    const int pair = unit % a.npairs;
+    unit /= a.npairs;
+    const int v = unit % p.b2;
+    unit /= p.b2;
+    const int g = unit % p.tiles;
+    const int bh = unit / p.tiles;
+    const int u1 = tile_begin(g + 1, p.b1, p.tiles);
+    const int u_start = tile_begin(g, p.b1, p.tiles) + 256 * pair;
+    const int key_row0 = ((bh * p.tiles + g) * p.b2 + v) * p.b1;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < 2; s++) {
+            mbar_init(k_full + s, 1);
+            mbar_init(z_full + s, 1);
+            mbar_init(h_full + s, 32);
+            mbar_init(kv_empty + s, 1);
+            mbar_init(s_full + s, 1);
+            mbar_init(p_full + s, 128);
+            mbar_init(o_full + s, 1);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const WaitCtx w{a.limit, a.status, abort_flag};
+
+    if (warp == 0) {
+        // ---------------- producer: queries once, then Ktil / Z / H per chunk
+        if (lane == 0) {
+            mbar_expect_tx(q_full, 2 * kTile);
+            for (int t = 0; t < 2; t++)
+                for (int pn = 0; pn < 2; pn++)
+                    tma_load_3d(sm + ls::kQ + t * kTile + pn * kPanel, &tmQ, pn * 64, v,
+                                bh * p.b1 + u_start + t * 128, q_full);
+        }
+        int issued[2] = {0, 0};
+        for (int j = 0; j < a.nchunks; j++) {
+            const int st = j & 1;
+            if (j >= 2 && !wait_warp(kv_empty + st, ((j >> 1) - 1) & 1, w)) break;
+            if (lane == 0) {
+                mbar_expect_tx(k_full + st, kTile);
+                for (int pn = 0; pn < 2; pn++)
+                    tma_load_2d(sm + ls::kK + st * kTile + pn * kPanel, &tmK, pn * 64,
+                                key_row0 + j * 128, k_full + st);
+                mbar_expect_tx(z_full + st, kTile);
+                for (int pn = 0; pn < 2; pn++)
+                    tma_load_2d(sm + ls::kZ + st * kTile + pn * kPanel, &tmZ, pn * 64,
+                                key_row0 + j * 128, z_full + st);
+            }
+            issued[st]++;
+            float *hs = reinterpret_cast<float *>(sm + ls::kH) + st * 128;
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const int key = j * 128 + i * 32 + lane;
+                hs[i * 32 + lane] = key < p.b1 ? a.hent[key_row0 + key] * kLog2e : -INFINITY;
+            }
+            mbar_arrive(h_full + st);
+        }
+        if (lane == 0) {   // every issued copy lands before the CTA may exit
+            wait_phase_cleanup(q_full, 0, kCleanupPolls);
+            for (int s = 0; s < 2; s++)
+                if (issued[s] > 0) {
+                    wait_phase_cleanup(k_full + s, (issued[s] - 1) & 1, kCleanupPolls);
+                    wait_phase_cleanup(z_full + s, (issued[s] - 1) & 1, kCleanupPolls);
+                }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idS = idesc_bf16(128, 128, 0, 0);
+            const uint32_t idO = idesc_bf16(128, 128, 0, 1);
+            const uint32_t sQ = smem_u32(sm + ls::kQ), sK = smem_u32(sm + ls::kK),
+                           sZ = smem_u32(sm + ls::kZ);
+            bool ok = wait_phase(q_full, 0, w);
+            for (int j = 0; ok && j < a.nchunks; j++) {
+                const int st = j & 1;
+                const uint32_t ph = (j >> 1) & 1;
+                if (!wait_phase(k_full + st, ph, w)) break;
+                tc_fence_after();
+                for (int t = 0; t < 2 && ok; t++) {
+                    // S_t / P_t columns are free once PV_t of the previous chunk is done
+                    if (j > 0 && !wait_phase(o_full + t, (j - 1) & 1, w)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; kk++) {
+                        const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
+                        mma_ss(tmem + t * 128,
+                               smem_desc_sw128(sQ + t * kTile + off, 16, 1024),
+                               smem_desc_sw128(sK + st * kTile + off, 16, 1024), idS, kk > 0);
+                    }
+                    mma_commit(s_full + t);
+                }
+                if (!ok || !wait_phase(z_full + st, ph, w)) break;
+                for (int t = 0; t < 2 && ok; t++) {
+                    if (!wait_phase(p_full + t, j & 1, w)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; kk++)
+                        mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
+                               smem_desc_sw128(sZ + st * kTile + kk * 2048, kPanel, 1024), idO,
+                               (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(o_full + t);
+                }
+                if (!ok) break;
+                mma_commit(kv_empty + st);
+            }
+            mma_commit(mma_done);
+            wait_phase_cleanup(mma_done, 0, kCleanupPolls);
+        }
+    } else if (warp >= 4) {
+        // ---------------- softmax warpgroups: tile t = 0 (warps 4-7), 1 (warps 8-11)
+        const int t = (warp - 4) >> 2;
+        const int wq = warp & 3;
+        const int r = wq * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        const uint32_t tS = tmem + lane_off + t * 128;
+        const uint32_t tO = tmem + lane_off + 256 + t * 128;
+        float m_run = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        for (int j = 0; j < a.nchunks; j++) {
+            const int st = j & 1;
+            if (!wait_warp(s_full + t, j & 1, w) || !wait_warp(h_full + st, (j >> 1) & 1, w)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const float *hs = reinterpret_cast<const float *>(sm + ls::kH) + st * 128;
+            float x[128];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 4; c++) {
+                uint32_t raw[32];
+                tmem_ld32(tS + c * 32, raw);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; i++) {
+                    x[c * 32 + i] = fmaf(__uint_as_float(raw[i]), a.c_log2, hs[c * 32 + i]);
+                    mx = fmaxf(mx, x[c * 32 + i]);
+                }
+            }
+            // the running maximum moves only when it grows by more than 2^8: the
+            // probabilities stay below 256 and O is rescaled rarely
+            float alpha = 1.f;
+            bool rescale = false;
+            if (mx > m_run + 8.f) {
+                alpha = fast_exp2(m_run - mx);
+                m_run = mx;
+                rescale = true;
+            }
+            float sum = 0.f;
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; i++) {
+                    const float p0 = fast_exp2(x[h * 64 + 2 * i] - m_run);
+                    const float p1 = fast_exp2(x[h * 64 + 2 * i + 1] - m_run);
+                    sum += p0 + p1;
+                    pk[i] = pack_bf16(p0, p1);
+                }
+                tmem_st32(tS + h * 32, pk);
+            }
+            l_run = l_run * alpha + sum;
+            if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+                for (int c = 0; c < 4; c++) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + c * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st32(tO + c * 32, o);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(p_full + t);
+        }
+        if (ok && wait_warp(o_full + t, (a.nchunks - 1) & 1, w)) {
+            tc_fence_after();
+            // epilogue: O / l -> bf16 -> this warp's 32 rows of staging (inside the
+            // now idle query tile t, 16-byte chunks XOR-swizzled by row) -> 2 rows
+            // of 256 B per store instruction
+            const float inv_l = 1.f / l_run;
+            uint8_t *stg = sm + ls::kQ + t * kTile + wq * 32 * 256;
+#pragma unroll
+            for (int c = 0; c < 4; c++) {
+                uint32_t o[32];
+                tmem_ld32(tO + c * 32, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int qd = 0; qd < 4; qd++) {
+                    uint4 val;
+                    val.x = pack_bf16(__uint_as_float(o[8 * qd + 0]) * inv_l,
+                                      __uint_as_float(o[8 * qd + 1]) * inv_l);
+                    val.y = pack_bf16(__uint_as_float(o[8 * qd + 2]) * inv_l,
+                                      __uint_as_float(o[8 * qd + 3]) * inv_l);
+                    val.z = pack_bf16(__uint_as_float(o[8 * qd + 4]) * inv_l,
+                                      __uint_as_float(o[8 * qd + 5]) * inv_l);
+                    val.w = pack_bf16(__uint_as_float(o[8 * qd + 6]) * inv_l,
+                                      __uint_as_float(o[8 * qd + 7]) * inv_l);
+                    const int chunk = c * 4 + qd;
+                    *reinterpret_cast<uint4 *>(stg + lane * 256 + ((chunk ^ (lane & 15)) * 16)) = val;
+                }
+            }
+            __syncwarp();
+            const int row_base = u_start + t * 128 + wq * 32;
+#pragma unroll 4
+            for (int it = 0; it < 16; it++) {
+                const int rr = it * 2 + (lane >> 4), cidx = lane & 15;
+                const int u = row_base + rr;
+                const uint4 val =
+                    *reinterpret_cast<const uint4 *>(stg + rr * 256 + ((cidx ^ (rr & 15)) * 16));
+                if (u < u1)
+                    *reinterpret_cast<uint4 *>(
+                        a.out + ((int64_t)bh * p.N + (int64_t)u * p.b2 + v) * kD + cidx * 8) = val;
+            }
+        }
+        (void)r;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// =====================================================================
+// S2: R-step
+// =====================================================================
+struct RsArgs {
+    Problem p;
+    int nmt;             // 128-row tiles of qbar (t*b2 padded)
+    int mpad;            // nmt * 128
+    int bpc;             // blocks per CTA (flattened over heads and blocks)
+    float c_log2;
+    float *hent;
+    int *status;
+    long long limit;
+};
+
+template <int B2P>
+struct RsLayout {
+    static constexpr uint32_t kStage = 4 * B2P * 128;   // K and V: 2 panels each of B2P x 128 B
+    static constexpr uint32_t kVOff = 2 * B2P * 128;    // V inside a stage
+    static constexpr uint32_t kPanelKV = B2P * 128;
+    __host__ __device__ static uint32_t kv(int nmt) { return (uint32_t)nmt * kTile; }
+    __host__ __device__ static uint32_t stg(int nmt) { return kv(nmt) + 2 * kStage; }
+    __host__ __device__ static uint32_t bar(int nmt) { return stg(nmt) + 4 * 8192; }
+    __host__ __device__ static uint32_t smem(int nmt) { return bar(nmt) + 256 + 1024; }
+};
+
+template <int B2P>
+__global__ void __launch_bounds__(384, 1)
+tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmZs,
+                const __grid_constant__ CUtensorMap tmKs, RsArgs a) {
+    using L = RsLayout<B2P>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = align1024(smem_raw);
+    const int nmt = a.nmt;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::bar(nmt));
+    uint64_t *q_full = bars + 0;
+    uint64_t *q_empty = bars + 1;
+    uint64_t *kv_full = bars + 2;    // [2]
+    uint64_t *kv_empty = bars + 4;   // [2]
+    uint64_t *s_full = bars + 6;     // [2]
+    uint64_t *s_free = bars + 8;     // [2]
+    uint64_t *p_full = bars + 10;    // [2], 128 arrivals
+    uint64_t *o_full = bars + 12;    // [2]: Z part, Ktil part
+    uint64_t *o_empty = bars + 14;   // [2], 128 arrivals
+    uint64_t *mma_done = bars + 16;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 17);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 18);
+
+    const Problem &p = a.p;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int total = p.BH * p.b1;
+    const int first = blockIdx.x * a.bpc;
+    const int nblk = min(a.bpc, total - first);
+    const int nitems = nblk * nmt;
+    const int tb2 = p.tiles * p.b2;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int s = 0; s < 2; s++) {
+            mbar_init(kv_full + s, 1);
+            mbar_init(kv_empty + s, 1);
+            mbar_init(s_full + s, 1);
+            mbar_init(s_free + s, 1);
+            mbar_init(p_full + s, 128);
+            mbar_init(o_full + s, 1);
+            mbar_init(o_empty + s, 128);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const WaitCtx w{a.limit, a.status, abort_flag};
+
+    if (warp == 0) {
+        // ---------------- producer: qbar tiles per head, K and V per block
+        if (lane == 0) {
+            int heads = 0, cur = -1, issued[2] = {0, 0};
+            bool ok = true;
+            for (int ib = 0; ib < nblk && ok; ib++) {
+                const int fb = first + ib, bh = fb / p.b1, up = fb % p.b1;
+                if (bh != cur) {
+                    if (heads > 0 && !wait_phase(q_empty, (heads - 1) & 1, w)) break;
+                    mbar_expect_tx(q_full, nmt * kTile);
+                    for (int mt = 0; mt < nmt; mt++)
+                        for (int pn = 0; pn < 2; pn++)
+                            tma_load_2d(sm + mt * kTile + pn * kPanel, &tmQb, pn * 64,
+                                        bh * a.mpad + mt * 128, q_full);
+                    heads++;
+                    cur = bh;
+                }
+                const int st = ib & 1;
+                if (ib >= 2 && !wait_phase(kv_empty + st, ((ib >> 1) - 1) & 1, w)) break;
+                uint8_t *stage = sm + L::kv(nmt) + st * L::kStage;
+                mbar_expect_tx(kv_full + st, L::kStage);
+                const int row = bh * p.N + up * p.b2;
+                for (int pn = 0; pn < 2; pn++) {
+                    tma_load_2d(stage + pn * L::kPanelKV, &tmK, pn * 64, row, kv_full + st);
+                    tma_load_2d(stage + L::kVOff + pn * L::kPanelKV, &tmV, pn * 64, row,
+                                kv_full + st);
+                }
+                issued[st]++;
+            }
+            if (heads > 0) wait_phase_cleanup(q_full, (heads - 1) & 1, kCleanupPolls);
+            for (int s = 0; s < 2; s++)
+                if (issued[s] > 0)
+                    wait_phase_cleanup(kv_full + s, (issued[s] - 1) & 1, kCleanupPolls);
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t id1 = idesc_bf16(128, B2P, 0, 0);
+            const uint32_t id2 = idesc_bf16(128, 128, 0, 1);
+            const uint32_t sQ = smem_u32(sm), sKV = smem_u32(sm + L::kv(nmt));
+            int heads = 0;
+            bool ok = true;
+            // S = qbar_mt K_u'^T for item i into S buffer i & 1
+            auto gemm1 = [&](int i) -> bool {
+                const int ib = i / nmt, mt = i % nmt;
+                const int fb = first + ib, bh = fb / p.b1;
+                if (mt == 0) {
+                    if (ib == 0 || (fb - 1) / p.b1 != bh) {
+                        if (!wait_phase(q_full, heads & 1, w)) return false;
+                        heads++;
+                    }
+                    if (!wait_phase(kv_full + (ib & 1), (ib >> 1) & 1, w)) return false;
+                }
+                if (i >= 2 && !wait_phase(s_free + (i & 1), ((i >> 1) - 1) & 1, w)) return false;
+                tc_fence_after();
+                const uint32_t kb = sKV + (ib & 1) * L::kStage;
+#pragma unroll
+                for (int kk = 0; kk < 8; kk++) {
+                    const uint32_t qoff = mt * kTile + (kk >> 2) * kPanel + (kk & 3) * 32;
+                    const uint32_t koff = (kk >> 2) * L::kPanelKV + (kk & 3) * 32;
+                    mma_ss(tmem + (i & 1) * 128, smem_desc_sw128(sQ + qoff, 16, 1024),
+                           smem_desc_sw128(kb + koff, 16, 1024), id1, kk > 0);
+                }
+                mma_commit(s_full + (i & 1));
+                const bool head_ends = (ib == nblk - 1) || ((fb + 1) / p.b1 != bh);
+                if (mt == nmt - 1 && head_ends) mma_commit(q_empty);
+                return true;
+            };
+            if (nitems > 0) ok = gemm1(0);
+            for (int i = 0; ok && i < nitems; i++) {
+                if (i + 1 < nitems && !gemm1(i + 1)) break;
+                const int ib = i / nmt, mt = i % nmt;
+                if (!wait_phase(p_full + (i & 1), (i >> 1) & 1, w)) break;
+                tc_fence_after();
+                const uint32_t kb = sKV + (ib & 1) * L::kStage;
+                for (int part = 0; part < 2 && ok; part++) {   // 0: Z = R V, 1: Ktil = R K
+                    if (i > 0 && !wait_phase(o_empty + part, (i - 1) & 1, w)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t bbase = kb + (part == 0 ? L::kVOff : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < B2P / 16; kk++)
+                        mma_ts(tmem + 256 + part * 128, tmem + (i & 1) * 128 + kk * 8,
+                               smem_desc_sw128(bbase + kk * 2048, L::kPanelKV, 1024), id2,
+                               kk > 0 ? 1u : 0u);
+                    mma_commit(o_full + part);
+                }
+                if (!ok) break;
+                mma_commit(s_free + (i & 1));
+                if (mt == nmt - 1) mma_commit(kv_empty + (ib & 1));
+            }
+            mma_commit(mma_done);
+            wait_phase_cleanup(mma_done, 0, kCleanupPolls);
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ---------------- softmax: R rows, entropy, normalised P back to TMEM (bf16)
+        const int wq = warp & 3;
+        const int r = wq * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        for (int i = 0; i < nitems; i++) {
+            const int ib = i / nmt, mt = i % nmt;
+            const int fb = first + ib, bh = fb / p.b1, up = fb % p.b1;
+            if (!wait_warp(s_full + (i & 1), (i >> 1) & 1, w)) break;
+            tc_fence_after();
+            const uint32_t tS = tmem + lane_off + (i & 1) * 128;
+            float x[B2P];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < B2P / 16; c++) {
+                uint32_t raw[16];
+                tmem_ld16(tS + c * 16, raw);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 16; k++) {
+                    const int col = c * 16 + k;
+                    x[col] = col < p.b2 ? __uint_as_float(raw[k]) * a.c_log2 : -INFINITY;
+                    mx = fmaxf(mx, x[col]);
+                }
+            }
+            float l = 0.f, e = 0.f;
+#pragma unroll
+            for (int col = 0; col < B2P; col++) {
+                const float pr = fast_exp2(x[col] - mx);
+                l += pr;
+                e += col < p.b2 ? pr * x[col] : 0.f;
+                x[col] = pr;
+            }
+            const float inv = 1.f / l;
+            const int row = mt * 128 + r;
+            if (row < tb2)   // entropy of the row, natural log: ln2 * (log2 lse - E[x])
+                a.hent[((int64_t)bh * tb2 + row) * p.b1 + up] = kLn2 * (mx + log2f(l) - e * inv);
+#pragma unroll
+            for (int c = 0; c < B2P / 16; c++) {
+                uint32_t pk[8];
+#pragma unroll
+                for (int k = 0; k < 8; k++)
+                    pk[k] = pack_bf16(x[c * 16 + 2 * k] * inv, x[c * 16 + 2 * k + 1] * inv);
+                tmem_st8(tS + c * 8, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(p_full + (i & 1));
+        }
+    } else if (warp >= 8) {
+        // ---------------- epilogue: Z and Ktil rows -> bf16 -> staging -> TMA store
+        const int wq = warp & 3;
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        uint8_t *stg = sm + L::stg(nmt) + wq * 8192;   // 2 panels x 32 rows x 128 B
+        bool ok = true;
+        for (int i = 0; ok && i < nitems; i++) {
+            const int ib = i / nmt, mt = i % nmt;
+            const int fb = first + ib, bh = fb / p.b1, up = fb % p.b1;
+            for (int part = 0; part < 2; part++) {
+                if (!wait_warp(o_full + part, i & 1, w)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t pk[64];
+#pragma unroll
+                for (int c = 0; c < 4; c++) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_off + 256 + part * 128 + c * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int k = 0; k < 16; k++)
+                        pk[c * 16 + k] =
+                            pack_bf16(__uint_as_float(o[2 * k]), __uint_as_float(o[2 * k + 1]));
+                }
+                tc_fence_before();
+                mbar_arrive(o_empty + part);
+                // the previous store of this warp must have finished reading staging
+                if (lane == 0) tma_store_wait_read_all();
+                __syncwarp();
+#pragma unroll
+                for (int c = 0; c < 16; c++) {   // 16-byte chunk c of the 256-byte row
+                    const int pn = c >> 3, pos = (c & 7) ^ (lane & 7);
+                    *reinterpret_cast<uint4 *>(stg + pn * 4096 + lane * 128 + pos * 16) =
+                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    const CUtensorMap *map = part == 0 ? &tmZs : &tmKs;
+                    for (int pn = 0; pn < 2; pn++)
+                        tma_store_4d(map, stg + pn * 4096, pn * 64, up, mt * 128 + wq * 32, bh);
+                    tma_store_commit();
+                }
+            }
+        }
+        if (lane == 0) tma_store_wait_all();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// =====================================================================
+// host side
+// =====================================================================
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// bf16 tensor map, 128-byte swizzle; dims innermost first, strides in bytes for dims 1..rank-1
+bool make_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims,
+              const uint64_t *strides, const uint32_t *box) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base),
+              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int b2_padded(int b2) { return (b2 + 15) / 16 * 16; }
+int qbar_tiles(const Problem &p) { return (p.tiles * p.b2 + 127) / 128; }
+size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+uint32_t rstep_smem(int b2p, int nmt) {
+    switch (b2p) {
+#define MONARCH_RS_CASE(V) \
+    case V: return RsLayout<V>::smem(nmt);
+        MONARCH_RS_CASE(16) MONARCH_RS_CASE(32) MONARCH_RS_CASE(48) MONARCH_RS_CASE(64)
+        MONARCH_RS_CASE(80) MONARCH_RS_CASE(96) MONARCH_RS_CASE(112) MONARCH_RS_CASE(128)
+#undef MONARCH_RS_CASE
+    }
+    return 0xFFFFFFFFu;
+}
+
+struct TcWorkspace {
+    __nv_bfloat16 *qbar, *ktil, *z;
+    float *hent;
+};
+
+TcWorkspace carve(const Problem &p, void *base) {
+    const size_t mpad = (size_t)qbar_tiles(p) * 128;
+    const size_t kz = (size_t)p.BH * p.tiles * p.N * kD * 2;
+    char *c = (char *)base;
+    TcWorkspace ws;
+    ws.qbar = (__nv_bfloat16 *)c;
+    c += al256((size_t)p.BH * mpad * kD * 2);
+    ws.ktil = (__nv_bfloat16 *)c;
+    c += al256(kz);
+    ws.z = (__nv_bfloat16 *)c;
+    c += al256(kz);
+    ws.hent = (float *)c;
+    return ws;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, uint32_t bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <int B2P>
+cudaError_t launch_rstep(const CUtensorMap *maps, const RsArgs &a, int grid, cudaStream_t s) {
+    const uint32_t smem = RsLayout<B2P>::smem(a.nmt);
+    cudaError_t e = set_smem(tc_rstep_kernel<B2P>, smem);
+    if (e != cudaSuccess) return e;
+    tc_rstep_kernel<B2P><<<grid, 384, smem, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], a);
+    return cudaGetLastError();
+}
+
+int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+}  // namespace
+
+bool sm100_supports(const Problem &p, monarch_dtype dtype) {
+    if (dtype != MONARCH_BF16 || p.d != kD || p.iters != 1 || p.b2 > 128) return false;
+    if (rstep_smem(b2_padded(p.b2), qbar_tiles(p)) > (uint32_t)kMaxSmem) return false;
+    // TMA coordinates are 32-bit: every row index must fit
+    if ((int64_t)p.BH * p.tiles * p.N + 256 >= (1LL << 31)) return false;
+    if ((int64_t)p.BH * qbar_tiles(p) * 128 >= (1LL << 31)) return false;
+    if (encode_fn() == nullptr) return false;
+    return true;
+}
+
+size_t sm100_workspace_bytes(const Problem &p, bool &overflow) {
+    overflow = false;
+    const size_t mpad = (size_t)qbar_tiles(p) * 128;
+    const size_t kz = (size_t)p.BH * p.tiles * p.N * kD * 2;
+    return al256((size_t)p.BH * mpad * kD * 2) + 2 * al256(kz) +
+           al256((size_t)p.BH * p.tiles * p.N * 4);
+}
+
+cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const void *v,
+                          void *out, void *workspace, int *status, long long wait_limit,
+                          cudaStream_t stream) {
+    const TcWorkspace ws = carve(p, workspace);
+    const int nmt = qbar_tiles(p), mpad = nmt * 128, b2p = b2_padded(p.b2);
+    const float c_log2 = p.scale * kLog2e;
+
+    // S1
+    {
+        const int nchunk = (p.b2 * kD / 8 + 127) / 128;
+        ProfileScope scope(K_TC_QBAR, stream);
+        tc_qbar_kernel<<<p.BH * p.tiles * nchunk, 128, 0, stream>>>(
+            (const __nv_bfloat16 *)q, ws.qbar, p, mpad);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    // S2
+    {
+        CUtensorMap maps[5];
+        const uint64_t dq[2] = {(uint64_t)kD, (uint64_t)p.BH * mpad};
+        const uint64_t dkv[2] = {(uint64_t)kD, (uint64_t)p.BH * p.N};
+        const uint64_t s2[1] = {kD * 2};
+        const uint32_t bq[2] = {64, 128};
+        const uint32_t bkv[2] = {64, (uint32_t)b2p};
+        const uint64_t dst[4] = {(uint64_t)kD, (uint64_t)p.b1, (uint64_t)p.tiles * p.b2,
+                                 (uint64_t)p.BH};
+        const uint64_t sst[3] = {kD * 2, (uint64_t)p.b1 * kD * 2,
+                                 (uint64_t)p.tiles * p.b2 * p.b1 * kD * 2};
+        const uint32_t bst[4] = {64, 1, 32, 1};
+        if (!make_map(&maps[0], ws.qbar, 2, dq, s2, bq) || !make_map(&maps[1], k, 2, dkv, s2, bkv) ||
+            !make_map(&maps[2], v, 2, dkv, s2, bkv) || !make_map(&maps[3], ws.z, 4, dst, sst, bst) ||
+            !make_map(&maps[4], ws.ktil, 4, dst, sst, bst))
+            return cudaErrorInvalidValue;
+        const int total = p.BH * p.b1;
+        const int sms = sm_count();
+        const int bpc = (total + sms - 1) / sms;
+        const int grid = (total + bpc - 1) / bpc;
+        RsArgs a{p, nmt, mpad, bpc, c_log2, ws.hent, status, wait_limit};
+        ProfileScope scope(K_TC_RSTEP, stream);
+        cudaError_t e = cudaErrorInvalidValue;
+        switch (b2p) {
+            case 16: e = launch_rstep<16>(maps, a, grid, stream); break;
+            case 32: e = launch_rstep<32>(maps, a, grid, stream); break;
+            case 48: e = launch_rstep<48>(maps, a, grid, stream); break;
+            case 64: e = launch_rstep<64>(maps, a, grid, stream); break;
+            case 80: e = launch_rstep<80>(maps, a, grid, stream); break;
+            case 96: e = launch_rstep<96>(maps, a, grid, stream); break;
+            case 112: e = launch_rstep<112>(maps, a, grid, stream); break;
+            case 128: e = launch_rstep<128>(maps, a, grid, stream); break;
+        }
+        if (e != cudaSuccess) return e;
+    }
+    // S3
+    {
+        CUtensorMap maps[3];
+        const uint64_t dq[3] = {(uint64_t)kD, (uint64_t)p.b2, (uint64_t)p.BH * p.b1};
+        const uint64_t sq[2] = {kD * 2, (uint64_t)p.b2 * kD * 2};
+        const uint32_t bq[3] = {64, 1, 128};
+        const uint64_t dk[2] = {(uint64_t)kD, (uint64_t)p.BH * p.tiles * p.N};
+        const uint64_t sk[1] = {kD * 2};
+        const uint32_t bk[2] = {64, 128};
+        if (!make_map(&maps[0], q, 3, dq, sq, bq) || !make_map(&maps[1], ws.ktil, 2, dk, sk, bk) ||
+            !make_map(&maps[2], ws.z, 2, dk, sk, bk))
+            return cudaErrorInvalidValue;
+        const int nq_max = tile_max_rows(p.b1, p.tiles);
+        const int npairs = ((nq_max + 127) / 128 + 1) / 2;
+        LsArgs a{p, (p.b1 + 127) / 128, npairs, c_log2, ws.hent, (__nv_bfloat16 *)out, status,
+                 wait_limit};
+        cudaError_t e = set_smem(tc_lstep_kernel, ls::kSmem);
+        if (e != cudaSuccess) return e;
+        ProfileScope scope(K_TC_LSTEP, stream);
+        tc_lstep_kernel<<<p.BH * p.tiles * p.b2 * npairs, 384, ls::kSmem, stream>>>(
+            maps[0], maps[1], maps[2], a);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace monarch

@@ -145,6 +145,7 @@ def inputs_720p():
 def test_full_720p_headline(inputs_720p):
     wl = synth.WORKLOADS["720p"]
     q, k, v = inputs_720p
+    assert kernel_path(q, f=wl.f, h=wl.h, w=wl.w, b1=wl.b1, b2=wl.b2, tiles=wl.tiles) == 1
     out = run(wl, q, k, v)
     convex_hull_check(out, v)
     probs = sample_problems(wl, 24, seed=720)
@@ -222,3 +223,22 @@ def test_device_entry_points_reject_bad_buffers(tiny64):
     assert _lib.monarch_attn_fwd_ws(p + 4, p, p, p, *shape, 0, ws.data_ptr(), 1 << 20, None) == 3
     assert _lib.monarch_attn_fwd_ws(p, p, p, p, *shape, 0, ws.data_ptr(), 64, None) == 5
     assert _lib.monarch_last_device_status(None) == 0
+
+
+def test_tensor_core_path_survives_a_tiny_wait_limit():
+    """Bounded waits: with a limit of a few polls the kernels give up (status
+    MONARCH_ERR_TIMEOUT) or finish, but never hang, and the next call is correct."""
+    wl = synth.WORKLOADS["480p_chunk"].replace(H=4)
+    q, k, v = device_inputs(wl)
+    assert kernel_path(q, f=wl.f, h=wl.h, w=wl.w, b1=wl.b1, b2=wl.b2, tiles=wl.tiles) == 1
+    old = _lib.monarch_set_wait_limit(64)
+    try:
+        monarch_attention(q, k, v, f=wl.f, h=wl.h, w=wl.w, b1=wl.b1, b2=wl.b2, tiles=wl.tiles)
+        torch.cuda.synchronize()
+        assert _lib.monarch_last_device_status(None) in (0, 7)
+    finally:
+        _lib.monarch_set_wait_limit(old)
+    out = run(wl, q, k, v)
+    q64, k64, v64 = (from_torch(x, wl.dtype) for x in (q, k, v))
+    ref = oracle.monarch_attn(q64, k64, v64, wl.b1, wl.b2, wl.tiles, wl.iters)
+    assert rel_fro(from_torch(out, wl.dtype), ref) <= TOL[wl.dtype]
