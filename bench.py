@@ -327,7 +327,7 @@ def run_ours(args, wl: synth.Workload, world: int, rank: int, local: int):
         torch.cuda.synchronize()
         if i >= args.e2e_warmup:
             e2e_times.append(a.elapsed_time(b))
-    e2e_ms = max_over_ranks(statistics.mean(e2e_times))
+    e2e_ms = max_over_ranks(statistics.mean(e2e_times) if e2e_times else float("nan"))
 
     if rank != 0:
         return
@@ -377,14 +377,16 @@ def run_ours(args, wl: synth.Workload, world: int, rank: int, local: int):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="720p", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--e2e-warmup", type=int, default=2)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override H (smaller cases for ncu captures; not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -395,6 +397,8 @@ def main():
     if args.gpus != world:
         ap.error("--gpus %d but WORLD_SIZE=%d: launch N > 1 with torchrun" % (args.gpus, world))
     wl = synth.WORKLOADS[args.workload]
+    if args.heads > 0:
+        wl = wl.replace(H=args.heads)
 
     if args.impl == "reference":
         run_reference(args, wl, world, rank)

@@ -115,14 +115,16 @@ __global__ void __launch_bounds__(128) tc_qbar_kernel(const __nv_bfloat16 *__res
 }
 
 // =====================================================================
-// S3: L-step with the output
+// S3: L-step with the output (persistent: each CTA walks a strided list of
+// (bh, g, v, query-pair) problems; the next problem's queries load while the
+// current one finishes, and its first S MMAs overlap the current epilogue)
 // =====================================================================
 namespace ls {
-constexpr uint32_t kQ = 0;               // query tiles 0, 1
-constexpr uint32_t kK = 2 * kTile;       // Ktil stages 0, 1
-constexpr uint32_t kZ = 4 * kTile;       // Z stages 0, 1
-constexpr uint32_t kH = 6 * kTile;       // H * log2(e) per stage: [2][128] floats
-constexpr uint32_t kBar = kH + 1024;
+constexpr uint32_t kQ = 0;                 // query tiles 0, 1
+constexpr uint32_t kK = 2 * kTile;         // Ktil stages 0, 1
+constexpr uint32_t kZ = 4 * kTile;         // Z stages 0, 1
+constexpr uint32_t kH = 6 * kTile;         // H * log2(e) per chunk: 4 buffers of 128 floats
+constexpr uint32_t kBar = kH + 2048;
 constexpr uint32_t kSmem = kBar + 256 + 1024;
 }  // namespace ls
 
@@ -130,12 +132,32 @@ struct LsArgs {
     Problem p;
     int nchunks;    // key chunks of 128 blocks
     int npairs;     // pairs of 128-query tiles per (g, v)
+    int nprob;      // BH * t * b2 * npairs
     float c_log2;   // (1/sqrt(d)) * log2(e)
     const float *hent;
     __nv_bfloat16 *out;
     int *status;
     long long limit;
 };
+
+struct LsProblem {
+    int bh, g, v, u_start, u1, key_row0;
+};
+
+__device__ __forceinline__ LsProblem ls_problem(const LsArgs &a, int unit) {
+    const Problem &p = a.p;
+    LsProblem q;
+    const int pair = unit % a.npairs;
+    unit /= a.npairs;
+    q.v = unit % p.b2;
+    unit /= p.b2;
+    q.g = unit % p.tiles;
+    q.bh = unit / p.tiles;
+    q.u1 = tile_begin(q.g + 1, p.b1, p.tiles);
+    q.u_start = tile_begin(q.g, p.b1, p.tiles) + 256 * pair;
+    q.key_row0 = ((q.bh * p.tiles + q.g) * p.b2 + q.v) * p.b1;
+    return q;
+}
 
 __global__ void __launch_bounds__(384, 1)
 tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -144,41 +166,38 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     uint8_t *sm = align1024(smem_raw);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + ls::kBar);
     uint64_t *q_full = bars + 0;
-    uint64_t *k_full = bars + 1;     // [2 stages]
-    uint64_t *z_full = bars + 3;     // [2 stages]
-    uint64_t *h_full = bars + 5;     // [2 stages], 32 arrivals
-    uint64_t *kv_empty = bars + 7;   // [2 stages]
-    uint64_t *s_full = bars + 9;     // [2 tiles]
-    uint64_t *p_full = bars + 11;    // [2 tiles], 128 arrivals
-    uint64_t *o_full = bars + 13;    // [2 tiles]
-    uint64_t *mma_done = bars + 15;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 17);
+    uint64_t *q_empty = bars + 1;
+    uint64_t *k_full = bars + 2;     // [2 stages]
+    uint64_t *z_full = bars + 4;     // [2 stages]
+    uint64_t *k_empty = bars + 6;    // [2 stages]: both S MMAs of the chunk done
+    uint64_t *z_empty = bars + 8;    // [2 stages]: both PV MMAs of the chunk done
+    uint64_t *h_full = bars + 10;    // [4 buffers], 32 arrivals
+    uint64_t *s_full = bars + 14;    // [2 tiles]
+    uint64_t *p_full = bars + 16;    // [2 tiles], 128 arrivals
+    uint64_t *o_full = bars + 18;    // [2 tiles]
+    uint64_t *mma_done = bars + 20;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 21);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 22);
 
     const Problem &p = a.p;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int unit = blockIdx.x;
-    const int pair = unit % a.npairs;
-    unit /= a.npairs;
-    const int v = unit % p.b2;
-    unit /= p.b2;
-    const int g = unit % p.tiles;
-    const int bh = unit / p.tiles;
-    const int u1 = tile_begin(g + 1, p.b1, p.tiles);
-    const int u_start = tile_begin(g, p.b1, p.tiles) + 256 * pair;
-    const int key_row0 = ((bh * p.tiles + g) * p.b2 + v) * p.b1;
+    const int nmine = a.nprob > (int)blockIdx.x
+                          ? (a.nprob - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const int nch = a.nchunks;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
         for (int s = 0; s < 2; s++) {
             mbar_init(k_full + s, 1);
             mbar_init(z_full + s, 1);
-            mbar_init(h_full + s, 32);
-            mbar_init(kv_empty + s, 1);
+            mbar_init(k_empty + s, 1);
+            mbar_init(z_empty + s, 1);
             mbar_init(s_full + s, 1);
             mbar_init(p_full + s, 128);
             mbar_init(o_full + s, 1);
         }
+        for (int s = 0; s < 4; s++) mbar_init(h_full + s, 32);
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -191,90 +210,130 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const WaitCtx w{a.limit, a.status, abort_flag};
 
     if (warp == 0) {
-        // ---------------- producer: queries once, then Ktil / Z / H per chunk
-        if (lane == 0) {
-            mbar_expect_tx(q_full, 2 * kTile);
-            for (int t = 0; t < 2; t++)
-                for (int pn = 0; pn < 2; pn++)
-                    tma_load_3d(sm + ls::kQ + t * kTile + pn * kPanel, &tmQ, pn * 64, v,
-                                bh * p.b1 + u_start + t * 128, q_full);
-        }
-        int issued[2] = {0, 0};
-        for (int j = 0; j < a.nchunks; j++) {
-            const int st = j & 1;
-            if (j >= 2 && !wait_warp(kv_empty + st, ((j >> 1) - 1) & 1, w)) break;
+        // ---------------- producer: queries per problem; per chunk Ktil and H as
+        // soon as the S MMAs of two chunks back are done, Z once their PV MMAs are.
+        // H has four buffers: when S1 of chunk jc-2 completes, both softmax
+        // warpgroups have finished chunk jc-3, so buffer jc & 3 (last read for
+        // chunk jc-4) is free.
+        int issued[2] = {0, 0}, issued_z[2] = {0, 0}, qloads = 0;
+        bool ok = true;
+        for (int pi = 0; ok && pi < nmine; pi++) {
+            const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
+            if (pi > 0 && !wait_warp(q_empty, (pi - 1) & 1, w)) break;
             if (lane == 0) {
-                mbar_expect_tx(k_full + st, kTile);
-                for (int pn = 0; pn < 2; pn++)
-                    tma_load_2d(sm + ls::kK + st * kTile + pn * kPanel, &tmK, pn * 64,
-                                key_row0 + j * 128, k_full + st);
-                mbar_expect_tx(z_full + st, kTile);
-                for (int pn = 0; pn < 2; pn++)
-                    tma_load_2d(sm + ls::kZ + st * kTile + pn * kPanel, &tmZ, pn * 64,
-                                key_row0 + j * 128, z_full + st);
+                mbar_expect_tx(q_full, 2 * kTile);
+                for (int t = 0; t < 2; t++)
+                    for (int pn = 0; pn < 2; pn++)
+                        tma_load_3d(sm + ls::kQ + t * kTile + pn * kPanel, &tmQ, pn * 64, pr.v,
+                                    pr.bh * p.b1 + pr.u_start + t * 128, q_full);
             }
-            issued[st]++;
-            float *hs = reinterpret_cast<float *>(sm + ls::kH) + st * 128;
+            qloads++;
+            for (int j = 0; j < nch; j++) {
+                const int jc = pi * nch + j, st = jc & 1;
+                if (jc >= 2 && !wait_warp(k_empty + st, ((jc >> 1) - 1) & 1, w)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    mbar_expect_tx(k_full + st, kTile);
+                    for (int pn = 0; pn < 2; pn++)
+                        tma_load_2d(sm + ls::kK + st * kTile + pn * kPanel, &tmK, pn * 64,
+                                    pr.key_row0 + j * 128, k_full + st);
+                    // a TMA load takes several chunk periods under load: start moving
+                    // the chunk two stages further into L2 now (rows past this
+                    // problem belong to the next problem of the row range or lie out
+                    // of bounds; either is harmless for a prefetch)
+                    for (int pn = 0; pn < 2; pn++) {
+                        tma_prefetch_2d(&tmK, pn * 64, pr.key_row0 + (j + 2) * 128);
+                        tma_prefetch_2d(&tmZ, pn * 64, pr.key_row0 + (j + 2) * 128);
+                    }
+                }
+                issued[st]++;
+                float *hs = reinterpret_cast<float *>(sm + ls::kH) + (jc & 3) * 128;
 #pragma unroll
-            for (int i = 0; i < 4; i++) {
-                const int key = j * 128 + i * 32 + lane;
-                hs[i * 32 + lane] = key < p.b1 ? a.hent[key_row0 + key] * kLog2e : -INFINITY;
+                for (int i = 0; i < 4; i++) {
+                    const int key = j * 128 + i * 32 + lane;
+                    hs[i * 32 + lane] =
+                        key < p.b1 ? a.hent[pr.key_row0 + key] * kLog2e : -INFINITY;
+                }
+                mbar_arrive(h_full + (jc & 3));
+                if (jc >= 2 && !wait_warp(z_empty + st, ((jc >> 1) - 1) & 1, w)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    mbar_expect_tx(z_full + st, kTile);
+                    for (int pn = 0; pn < 2; pn++)
+                        tma_load_2d(sm + ls::kZ + st * kTile + pn * kPanel, &tmZ, pn * 64,
+                                    pr.key_row0 + j * 128, z_full + st);
+                }
+                issued_z[st]++;
             }
-            mbar_arrive(h_full + st);
         }
         if (lane == 0) {   // every issued copy lands before the CTA may exit
-            wait_phase_cleanup(q_full, 0, kCleanupPolls);
-            for (int s = 0; s < 2; s++)
-                if (issued[s] > 0) {
-                    wait_phase_cleanup(k_full + s, (issued[s] - 1) & 1, kCleanupPolls);
-                    wait_phase_cleanup(z_full + s, (issued[s] - 1) & 1, kCleanupPolls);
-                }
+            if (qloads > 0) wait_phase_cleanup(q_full, (qloads - 1) & 1, kCleanupPolls);
+            for (int s = 0; s < 2; s++) {
+                if (issued[s] > 0) wait_phase_cleanup(k_full + s, (issued[s] - 1) & 1, kCleanupPolls);
+                if (issued_z[s] > 0)
+                    wait_phase_cleanup(z_full + s, (issued_z[s] - 1) & 1, kCleanupPolls);
+            }
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer
+        // ---------------- MMA issuer.  Per chunk: PV0, then S0 of the next chunk,
+        // PV1, S1 of the next chunk, so that a tile's chain never waits on the
+        // other tile's softmax.  Descriptors are precomputed bases plus
+        // compile-time K-step offsets, keeping the single issuing thread lean.
         if (lane == 0) {
-            const uint32_t idS = idesc_bf16(128, 128, 0, 0);
-            const uint32_t idO = idesc_bf16(128, 128, 0, 1);
-            const uint32_t sQ = smem_u32(sm + ls::kQ), sK = smem_u32(sm + ls::kK),
-                           sZ = smem_u32(sm + ls::kZ);
-            bool ok = wait_phase(q_full, 0, w);
-            for (int j = 0; ok && j < a.nchunks; j++) {
-                const int st = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
-                if (!wait_phase(k_full + st, ph, w)) break;
+            constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
+            constexpr uint32_t idO = idesc_bf16(128, 128, 0, 1);
+            const uint64_t dQ = smem_desc_sw128(smem_u32(sm + ls::kQ), 16, 1024);
+            const uint64_t dK = smem_desc_sw128(smem_u32(sm + ls::kK), 16, 1024);
+            const uint64_t dZ = smem_desc_sw128(smem_u32(sm + ls::kZ), kPanel, 1024);
+            const int total = nmine * nch;
+            bool ok = true;
+            // S_t for global chunk index jc (waits for the chunk's Ktil and, if the
+            // chunk opens a problem, for its queries)
+            auto issue_s = [&](int t, int jc) -> bool {
+                const int st = jc & 1;
+                if (t == 0 && jc % nch == 0 && !spin_phase(q_full, (jc / nch) & 1, w)) return false;
+                if (t == 0 && !spin_phase(k_full + st, (jc >> 1) & 1, w)) return false;
                 tc_fence_after();
-                for (int t = 0; t < 2 && ok; t++) {
-                    // S_t / P_t columns are free once PV_t of the previous chunk is done
-                    if (j > 0 && !wait_phase(o_full + t, (j - 1) & 1, w)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
+                const uint64_t a0 = desc_plus(dQ, t * kTile), b0 = desc_plus(dK, st * kTile);
 #pragma unroll
-                    for (int kk = 0; kk < 8; kk++) {
-                        const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-                        mma_ss(tmem + t * 128,
-                               smem_desc_sw128(sQ + t * kTile + off, 16, 1024),
-                               smem_desc_sw128(sK + st * kTile + off, 16, 1024), idS, kk > 0);
-                    }
-                    mma_commit(s_full + t);
+                for (int kk = 0; kk < 8; kk++) {
+                    const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
+                    mma_ss(tmem + t * 128, desc_plus(a0, off), desc_plus(b0, off), idS, kk > 0);
                 }
-                if (!ok || !wait_phase(z_full + st, ph, w)) break;
-                for (int t = 0; t < 2 && ok; t++) {
-                    if (!wait_phase(p_full + t, j & 1, w)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
+                mma_commit(s_full + t);
+                if (t == 1) mma_commit(k_empty + st);
+                if (t == 1 && jc % nch == nch - 1) mma_commit(q_empty);   // queries no longer read
+                return true;
+            };
+            auto issue_pv = [&](int t, int jc) -> bool {
+                const int st = jc & 1;
+                if (t == 0 && !spin_phase(z_full + st, (jc >> 1) & 1, w)) return false;
+                if (!spin_phase(p_full + t, jc & 1, w)) return false;
+                tc_fence_after();
+                const uint64_t b0 = desc_plus(dZ, st * kTile);
+                const uint32_t acc0 = (jc % nch) > 0 ? 1u : 0u;
 #pragma unroll
-                    for (int kk = 0; kk < 8; kk++)
-                        mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
-                               smem_desc_sw128(sZ + st * kTile + kk * 2048, kPanel, 1024), idO,
-                               (j > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(o_full + t);
+                for (int kk = 0; kk < 8; kk++)
+                    mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, desc_plus(b0, kk * 2048),
+                           idO, kk > 0 ? 1u : acc0);
+                mma_commit(o_full + t);
+                if (t == 1) mma_commit(z_empty + st);
+                return true;
+            };
+            // S_t of the next chunk overwrites the columns that PV_t reads as P:
+            // tcgen05 MMAs issued by one thread execute in issue order, so it is
+            // issued right behind PV_t without waiting; its commit (s_full) also
+            // covers PV_t, which orders the softmax's rescale of O_t after PV_t.
+            if (total > 0) ok = issue_s(0, 0) && issue_s(1, 0);
+            for (int jc = 0; ok && jc < total; jc++) {
+                for (int t = 0; t < 2 && ok; t++) {
+                    ok = issue_pv(t, jc);
+                    if (ok && jc + 1 < total) ok = issue_s(t, jc + 1);
                 }
-                if (!ok) break;
-                mma_commit(kv_empty + st);
             }
             mma_commit(mma_done);
             wait_phase_cleanup(mma_done, 0, kCleanupPolls);
@@ -283,112 +342,107 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // ---------------- softmax warpgroups: tile t = 0 (warps 4-7), 1 (warps 8-11)
         const int t = (warp - 4) >> 2;
         const int wq = warp & 3;
-        const int r = wq * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
         const uint32_t tS = tmem + lane_off + t * 128;
         const uint32_t tO = tmem + lane_off + 256 + t * 128;
-        float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
-        for (int j = 0; j < a.nchunks; j++) {
-            const int st = j & 1;
-            if (!wait_warp(s_full + t, j & 1, w) || !wait_warp(h_full + st, (j >> 1) & 1, w)) {
+        for (int pi = 0; ok && pi < nmine; pi++) {
+            const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
+            float m_run = -INFINITY, l_run = 0.f;
+            for (int j = 0; j < nch; j++) {
+                const int jc = pi * nch + j;
+                if (!wait_warp(s_full + t, jc & 1, w) ||
+                    !wait_warp(h_full + (jc & 3), (jc >> 2) & 1, w)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                float x[128];
+#pragma unroll
+                for (int c = 0; c < 4; c++) tmem_ld32f(tS + c * 32, &x[c * 32]);
+                tmem_wait_ld();
+                // x = s * c_log2 + H * log2(e), two columns per packed FMA
+                const uint64_t *hs = reinterpret_cast<const uint64_t *>(sm + ls::kH + (jc & 3) * 512);
+                const uint64_t c2 = f2_pack(a.c_log2, a.c_log2);
+                uint64_t xp[64];
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int i = 0; i < 64; i++) {
+                    xp[i] = f2_fma(f2_pack(x[2 * i], x[2 * i + 1]), c2, hs[i]);
+                    float lo, hi;
+                    f2_unpack(xp[i], lo, hi);
+                    mx4[i & 3] = fmax3(mx4[i & 3], lo, hi);
+                }
+                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+                // the running maximum moves only when it grows by more than 2^8: the
+                // probabilities stay below 256 and O is rescaled rarely
+                float alpha = 1.f;
+                bool rescale = false;
+                if (mx > m_run + 8.f) {
+                    alpha = fast_exp2(m_run - mx);
+                    m_run = mx;
+                    rescale = true;
+                }
+                const uint64_t nm2 = f2_pack(-m_run, -m_run);
+                uint64_t sum2[4] = {0, 0, 0, 0};
+#pragma unroll
+                for (int h = 0; h < 2; h++) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int i = 0; i < 32; i++) {
+                        float lo, hi;
+                        f2_unpack(f2_add(xp[h * 32 + i], nm2), lo, hi);
+                        const float p0 = fast_exp2(lo), p1 = fast_exp2(hi);
+                        sum2[i & 3] = f2_add(sum2[i & 3], f2_pack(p0, p1));
+                        pk[i] = pack_bf16(p0, p1);
+                    }
+                    tmem_st32(tS + h * 32, pk);
+                }
+                float s0, s1;
+                f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), s0, s1);
+                l_run = l_run * alpha + (s0 + s1);
+                if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+                    float o[128];
+#pragma unroll
+                    for (int c = 0; c < 4; c++) tmem_ld32f(tO + c * 32, &o[c * 32]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 128; i++) o[i] *= alpha;
+#pragma unroll
+                    for (int c = 0; c < 4; c++) tmem_st32f(tO + c * 32, &o[c * 32]);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(p_full + t);
+            }
+            if (!ok || !wait_warp(o_full + t, (pi * nch + nch - 1) & 1, w)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const float *hs = reinterpret_cast<const float *>(sm + ls::kH) + st * 128;
-            float x[128];
-            float mx = -INFINITY;
+            // epilogue: each thread writes its own output row, O / l in bf16,
+            // as sixteen 16-byte stores (the L2 merges the row's sectors)
+            float o[128];
 #pragma unroll
-            for (int c = 0; c < 4; c++) {
-                uint32_t raw[32];
-                tmem_ld32(tS + c * 32, raw);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; i++) {
-                    x[c * 32 + i] = fmaf(__uint_as_float(raw[i]), a.c_log2, hs[c * 32 + i]);
-                    mx = fmaxf(mx, x[c * 32 + i]);
-                }
-            }
-            // the running maximum moves only when it grows by more than 2^8: the
-            // probabilities stay below 256 and O is rescaled rarely
-            float alpha = 1.f;
-            bool rescale = false;
-            if (mx > m_run + 8.f) {
-                alpha = fast_exp2(m_run - mx);
-                m_run = mx;
-                rescale = true;
-            }
-            float sum = 0.f;
-#pragma unroll
-            for (int h = 0; h < 2; h++) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int i = 0; i < 32; i++) {
-                    const float p0 = fast_exp2(x[h * 64 + 2 * i] - m_run);
-                    const float p1 = fast_exp2(x[h * 64 + 2 * i + 1] - m_run);
-                    sum += p0 + p1;
-                    pk[i] = pack_bf16(p0, p1);
-                }
-                tmem_st32(tS + h * 32, pk);
-            }
-            l_run = l_run * alpha + sum;
-            if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-                for (int c = 0; c < 4; c++) {
-                    uint32_t o[32];
-                    tmem_ld32(tO + c * 32, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    tmem_st32(tO + c * 32, o);
-                }
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(p_full + t);
-        }
-        if (ok && wait_warp(o_full + t, (a.nchunks - 1) & 1, w)) {
-            tc_fence_after();
-            // epilogue: O / l -> bf16 -> this warp's 32 rows of staging (inside the
-            // now idle query tile t, 16-byte chunks XOR-swizzled by row) -> 2 rows
-            // of 256 B per store instruction
+            for (int c = 0; c < 4; c++) tmem_ld32f(tO + c * 32, &o[c * 32]);
+            tmem_wait_ld();
             const float inv_l = 1.f / l_run;
-            uint8_t *stg = sm + ls::kQ + t * kTile + wq * 32 * 256;
+            const int u = pr.u_start + t * 128 + wq * 32 + lane;
+            if (u < pr.u1) {
+                uint4 *dst = reinterpret_cast<uint4 *>(
+                    a.out + ((int64_t)pr.bh * p.N + (int64_t)u * p.b2 + pr.v) * kD);
 #pragma unroll
-            for (int c = 0; c < 4; c++) {
-                uint32_t o[32];
-                tmem_ld32(tO + c * 32, o);
-                tmem_wait_ld();
-#pragma unroll
-                for (int qd = 0; qd < 4; qd++) {
+                for (int ch = 0; ch < 16; ch++) {
+                    const float *src = &o[ch * 8];
                     uint4 val;
-                    val.x = pack_bf16(__uint_as_float(o[8 * qd + 0]) * inv_l,
-                                      __uint_as_float(o[8 * qd + 1]) * inv_l);
-                    val.y = pack_bf16(__uint_as_float(o[8 * qd + 2]) * inv_l,
-                                      __uint_as_float(o[8 * qd + 3]) * inv_l);
-                    val.z = pack_bf16(__uint_as_float(o[8 * qd + 4]) * inv_l,
-                                      __uint_as_float(o[8 * qd + 5]) * inv_l);
-                    val.w = pack_bf16(__uint_as_float(o[8 * qd + 6]) * inv_l,
-                                      __uint_as_float(o[8 * qd + 7]) * inv_l);
-                    const int chunk = c * 4 + qd;
-                    *reinterpret_cast<uint4 *>(stg + lane * 256 + ((chunk ^ (lane & 15)) * 16)) = val;
+                    val.x = pack_bf16(src[0] * inv_l, src[1] * inv_l);
+                    val.y = pack_bf16(src[2] * inv_l, src[3] * inv_l);
+                    val.z = pack_bf16(src[4] * inv_l, src[5] * inv_l);
+                    val.w = pack_bf16(src[6] * inv_l, src[7] * inv_l);
+                    dst[ch] = val;
                 }
             }
-            __syncwarp();
-            const int row_base = u_start + t * 128 + wq * 32;
-#pragma unroll 4
-            for (int it = 0; it < 16; it++) {
-                const int rr = it * 2 + (lane >> 4), cidx = lane & 15;
-                const int u = row_base + rr;
-                const uint4 val =
-                    *reinterpret_cast<const uint4 *>(stg + rr * 256 + ((cidx ^ (rr & 15)) * 16));
-                if (u < u1)
-                    *reinterpret_cast<uint4 *>(
-                        a.out + ((int64_t)bh * p.N + (int64_t)u * p.b2 + v) * kD + cidx * 8) = val;
-            }
         }
-        (void)r;
     }
     tc_fence_before();
     __syncthreads();
@@ -514,9 +568,11 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
     } else if (warp == 1) {
         // ---------------- MMA issuer
         if (lane == 0) {
-            const uint32_t id1 = idesc_bf16(128, B2P, 0, 0);
-            const uint32_t id2 = idesc_bf16(128, 128, 0, 1);
-            const uint32_t sQ = smem_u32(sm), sKV = smem_u32(sm + L::kv(nmt));
+            constexpr uint32_t id1 = idesc_bf16(128, B2P, 0, 0);
+            constexpr uint32_t id2 = idesc_bf16(128, 128, 0, 1);
+            const uint64_t dQ = smem_desc_sw128(smem_u32(sm), 16, 1024);
+            const uint64_t dK = smem_desc_sw128(smem_u32(sm + L::kv(nmt)), 16, 1024);
+            const uint64_t dV = smem_desc_sw128(smem_u32(sm + L::kv(nmt)), L::kPanelKV, 1024);
             int heads = 0;
             bool ok = true;
             // S = qbar_mt K_u'^T for item i into S buffer i & 1
@@ -532,14 +588,13 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 }
                 if (i >= 2 && !wait_phase(s_free + (i & 1), ((i >> 1) - 1) & 1, w)) return false;
                 tc_fence_after();
-                const uint32_t kb = sKV + (ib & 1) * L::kStage;
+                const uint64_t a0 = desc_plus(dQ, mt * kTile);
+                const uint64_t b0 = desc_plus(dK, (ib & 1) * L::kStage);
 #pragma unroll
-                for (int kk = 0; kk < 8; kk++) {
-                    const uint32_t qoff = mt * kTile + (kk >> 2) * kPanel + (kk & 3) * 32;
-                    const uint32_t koff = (kk >> 2) * L::kPanelKV + (kk & 3) * 32;
-                    mma_ss(tmem + (i & 1) * 128, smem_desc_sw128(sQ + qoff, 16, 1024),
-                           smem_desc_sw128(kb + koff, 16, 1024), id1, kk > 0);
-                }
+                for (int kk = 0; kk < 8; kk++)
+                    mma_ss(tmem + (i & 1) * 128,
+                           desc_plus(a0, (kk >> 2) * kPanel + (kk & 3) * 32),
+                           desc_plus(b0, (kk >> 2) * L::kPanelKV + (kk & 3) * 32), id1, kk > 0);
                 mma_commit(s_full + (i & 1));
                 const bool head_ends = (ib == nblk - 1) || ((fb + 1) / p.b1 != bh);
                 if (mt == nmt - 1 && head_ends) mma_commit(q_empty);
@@ -551,22 +606,22 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 const int ib = i / nmt, mt = i % nmt;
                 if (!wait_phase(p_full + (i & 1), (i >> 1) & 1, w)) break;
                 tc_fence_after();
-                const uint32_t kb = sKV + (ib & 1) * L::kStage;
-                for (int part = 0; part < 2 && ok; part++) {   // 0: Z = R V, 1: Ktil = R K
-                    if (i > 0 && !wait_phase(o_empty + part, (i - 1) & 1, w)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t bbase = kb + (part == 0 ? L::kVOff : 0u);
+                const uint32_t pa = tmem + (i & 1) * 128;
+                // 0: Z = R V, 1: Ktil = R K
+                const uint64_t bz = desc_plus(dV, (ib & 1) * L::kStage + L::kVOff);
+                const uint64_t bk = desc_plus(dV, (ib & 1) * L::kStage);
+                if (i > 0 && !wait_phase(o_empty + 0, (i - 1) & 1, w)) break;
+                tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < B2P / 16; kk++)
-                        mma_ts(tmem + 256 + part * 128, tmem + (i & 1) * 128 + kk * 8,
-                               smem_desc_sw128(bbase + kk * 2048, L::kPanelKV, 1024), id2,
-                               kk > 0 ? 1u : 0u);
-                    mma_commit(o_full + part);
-                }
-                if (!ok) break;
+                for (int kk = 0; kk < B2P / 16; kk++)
+                    mma_ts(tmem + 256, pa + kk * 8, desc_plus(bz, kk * 2048), id2, kk > 0 ? 1u : 0u);
+                mma_commit(o_full + 0);
+                if (i > 0 && !wait_phase(o_empty + 1, (i - 1) & 1, w)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < B2P / 16; kk++)
+                    mma_ts(tmem + 384, pa + kk * 8, desc_plus(bk, kk * 2048), id2, kk > 0 ? 1u : 0u);
+                mma_commit(o_full + 1);
                 mma_commit(s_free + (i & 1));
                 if (mt == nmt - 1) mma_commit(kv_empty + (ib & 1));
             }
@@ -855,13 +910,14 @@ cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const 
             return cudaErrorInvalidValue;
         const int nq_max = tile_max_rows(p.b1, p.tiles);
         const int npairs = ((nq_max + 127) / 128 + 1) / 2;
-        LsArgs a{p, (p.b1 + 127) / 128, npairs, c_log2, ws.hent, (__nv_bfloat16 *)out, status,
-                 wait_limit};
+        const int nprob = p.BH * p.tiles * p.b2 * npairs;
+        LsArgs a{p, (p.b1 + 127) / 128, npairs, nprob, c_log2, ws.hent, (__nv_bfloat16 *)out,
+                 status, wait_limit};
         cudaError_t e = set_smem(tc_lstep_kernel, ls::kSmem);
         if (e != cudaSuccess) return e;
+        const int grid = nprob < sm_count() ? nprob : sm_count();
         ProfileScope scope(K_TC_LSTEP, stream);
-        tc_lstep_kernel<<<p.BH * p.tiles * p.b2 * npairs, 384, ls::kSmem, stream>>>(
-            maps[0], maps[1], maps[2], a);
+        tc_lstep_kernel<<<grid, 384, ls::kSmem, stream>>>(maps[0], maps[1], maps[2], a);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
