@@ -34,12 +34,12 @@ namespace {
 using namespace tc;
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kD = 128;                        // head dimension of this path
 constexpr uint32_t kPanel = 128 * 128;         // 128 rows x 64 bf16 (128 B), SW128
 constexpr uint32_t kTile = 2 * kPanel;         // 128 rows x 128 bf16
 constexpr int kMaxSmem = 232448;               // sm_100 opt-in dynamic shared memory
 constexpr long long kCleanupPolls = 1LL << 22;
+constexpr int kPrefetch = 4;                   // L-step: chunks of Ktil / Z prefetched to L2 ahead
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -133,6 +133,7 @@ struct LsArgs {
     int nchunks;    // key chunks of 128 blocks
     int npairs;     // pairs of 128-query tiles per (g, v)
     int nprob;      // BH * t * b2 * npairs
+    int hstride;    // row length of the entropy array
     float c_log2;   // (1/sqrt(d)) * log2(e)
     const float *hent;
     __nv_bfloat16 *out;
@@ -141,7 +142,7 @@ struct LsArgs {
 };
 
 struct LsProblem {
-    int bh, g, v, u_start, u1, key_row0;
+    int bh, g, v, u_start, u1, key_row0, h_row0;
 };
 
 __device__ __forceinline__ LsProblem ls_problem(const LsArgs &a, int unit) {
@@ -156,6 +157,7 @@ __device__ __forceinline__ LsProblem ls_problem(const LsArgs &a, int unit) {
     q.u1 = tile_begin(q.g + 1, p.b1, p.tiles);
     q.u_start = tile_begin(q.g, p.b1, p.tiles) + 256 * pair;
     q.key_row0 = ((q.bh * p.tiles + q.g) * p.b2 + q.v) * p.b1;
+    q.h_row0 = ((q.bh * p.tiles + q.g) * p.b2 + q.v) * a.hstride;
     return q;
 }
 
@@ -171,7 +173,7 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     uint64_t *z_full = bars + 4;     // [2 stages]
     uint64_t *k_empty = bars + 6;    // [2 stages]: both S MMAs of the chunk done
     uint64_t *z_empty = bars + 8;    // [2 stages]: both PV MMAs of the chunk done
-    uint64_t *h_full = bars + 10;    // [4 buffers], 32 arrivals
+    uint64_t *h_full = bars + 10;    // [4 buffers]: bulk copy of the chunk's entropies
     uint64_t *s_full = bars + 14;    // [2 tiles]
     uint64_t *p_full = bars + 16;    // [2 tiles], 128 arrivals
     uint64_t *o_full = bars + 18;    // [2 tiles]
@@ -197,7 +199,7 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             mbar_init(p_full + s, 128);
             mbar_init(o_full + s, 1);
         }
-        for (int s = 0; s < 4; s++) mbar_init(h_full + s, 32);
+        for (int s = 0; s < 4; s++) mbar_init(h_full + s, 1);
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -215,7 +217,7 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // H has four buffers: when S1 of chunk jc-2 completes, both softmax
         // warpgroups have finished chunk jc-3, so buffer jc & 3 (last read for
         // chunk jc-4) is free.
-        int issued[2] = {0, 0}, issued_z[2] = {0, 0}, qloads = 0;
+        int issued[2] = {0, 0}, issued_z[2] = {0, 0}, qloads = 0, issued_h = 0;
         bool ok = true;
         for (int pi = 0; ok && pi < nmine; pi++) {
             const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
@@ -239,24 +241,34 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     for (int pn = 0; pn < 2; pn++)
                         tma_load_2d(sm + ls::kK + st * kTile + pn * kPanel, &tmK, pn * 64,
                                     pr.key_row0 + j * 128, k_full + st);
-                    // a TMA load takes several chunk periods under load: start moving
-                    // the chunk two stages further into L2 now (rows past this
-                    // problem belong to the next problem of the row range or lie out
-                    // of bounds; either is harmless for a prefetch)
-                    for (int pn = 0; pn < 2; pn++) {
-                        tma_prefetch_2d(&tmK, pn * 64, pr.key_row0 + (j + 2) * 128);
-                        tma_prefetch_2d(&tmZ, pn * 64, pr.key_row0 + (j + 2) * 128);
+                    // Only two chunks fit in shared memory, fewer than the memory
+                    // latency needs: move the chunk kPrefetch steps ahead (possibly of
+                    // this CTA's next problem) into L2 now, and at the start of a
+                    // problem the next problem's queries.
+                    const int ahead = j + kPrefetch, pa = pi + ahead / nch;
+                    if (pa < nmine) {
+                        const LsProblem pn2 = ls_problem(a, blockIdx.x + pa * gridDim.x);
+                        const int row = pn2.key_row0 + (ahead % nch) * 128;
+                        for (int pn = 0; pn < 2; pn++) {
+                            tma_prefetch_2d(&tmK, pn * 64, row);
+                            tma_prefetch_2d(&tmZ, pn * 64, row);
+                        }
+                        if (j == 0 && pi + 1 < nmine) {
+                            const LsProblem nq = ls_problem(a, blockIdx.x + (pi + 1) * gridDim.x);
+                            for (int t = 0; t < 2; t++)
+                                for (int pn = 0; pn < 2; pn++)
+                                    tma_prefetch_3d(&tmQ, pn * 64, nq.v,
+                                                    nq.bh * p.b1 + nq.u_start + t * 128);
+                        }
                     }
                 }
                 issued[st]++;
-                float *hs = reinterpret_cast<float *>(sm + ls::kH) + (jc & 3) * 128;
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    const int key = j * 128 + i * 32 + lane;
-                    hs[i * 32 + lane] =
-                        key < p.b1 ? a.hent[pr.key_row0 + key] * kLog2e : -INFINITY;
+                if (lane == 0) {   // the chunk's entropies (log2 units, -inf past b1)
+                    mbar_expect_tx(h_full + (jc & 3), 512);
+                    bulk_load(sm + ls::kH + (jc & 3) * 512, a.hent + pr.h_row0 + j * 128, 512,
+                              h_full + (jc & 3));
                 }
-                mbar_arrive(h_full + (jc & 3));
+                issued_h++;
                 if (jc >= 2 && !wait_warp(z_empty + st, ((jc >> 1) - 1) & 1, w)) {
                     ok = false;
                     break;
@@ -276,6 +288,11 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 if (issued[s] > 0) wait_phase_cleanup(k_full + s, (issued[s] - 1) & 1, kCleanupPolls);
                 if (issued_z[s] > 0)
                     wait_phase_cleanup(z_full + s, (issued_z[s] - 1) & 1, kCleanupPolls);
+            }
+            for (int hb = 0; hb < 4; hb++) {   // the last copy into each entropy buffer
+                if (issued_h <= hb) continue;
+                const int last = hb + ((issued_h - 1 - hb) / 4) * 4;
+                wait_phase_cleanup(h_full + hb, (last >> 2) & 1, kCleanupPolls);
             }
         }
     } else if (warp == 1) {
@@ -361,17 +378,32 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
                 for (int c = 0; c < 4; c++) tmem_ld32f(tS + c * 32, &x[c * 32]);
                 tmem_wait_ld();
-                // x = s * c_log2 + H * log2(e), two columns per packed FMA
+                // x = s * c_log2 + H / ln2 (the entropy arrives in log2 units)
                 const uint64_t *hs = reinterpret_cast<const uint64_t *>(sm + ls::kH + (jc & 3) * 512);
                 const uint64_t c2 = f2_pack(a.c_log2, a.c_log2);
                 uint64_t xp[64];
                 float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                const int nvalid = p.b1 - j * 128;   // keys of this chunk inside the row
+                if (nvalid >= 128) {
 #pragma unroll
-                for (int i = 0; i < 64; i++) {
-                    xp[i] = f2_fma(f2_pack(x[2 * i], x[2 * i + 1]), c2, hs[i]);
-                    float lo, hi;
-                    f2_unpack(xp[i], lo, hi);
-                    mx4[i & 3] = fmax3(mx4[i & 3], lo, hi);
+                    for (int i = 0; i < 64; i++) {
+                        xp[i] = f2_fma(f2_pack(x[2 * i], x[2 * i + 1]), c2, hs[i]);
+                        float lo, hi;
+                        f2_unpack(xp[i], lo, hi);
+                        mx4[i & 3] = fmax3(mx4[i & 3], lo, hi);
+                    }
+                } else {
+                    // the ragged last chunk: S and the entropy copy run past the row
+                    // (into the next row or the workspace slack), so mask by selection
+#pragma unroll
+                    for (int i = 0; i < 64; i++) {
+                        float lo, hi;
+                        f2_unpack(f2_fma(f2_pack(x[2 * i], x[2 * i + 1]), c2, hs[i]), lo, hi);
+                        lo = 2 * i < nvalid ? lo : -INFINITY;
+                        hi = 2 * i + 1 < nvalid ? hi : -INFINITY;
+                        xp[i] = f2_pack(lo, hi);
+                        mx4[i & 3] = fmax3(mx4[i & 3], lo, hi);
+                    }
                 }
                 const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
                 // the running maximum moves only when it grows by more than 2^8: the
@@ -460,6 +492,7 @@ struct RsArgs {
     int nmt;             // 128-row tiles of qbar (t*b2 padded)
     int mpad;            // nmt * 128
     int bpc;             // blocks per CTA (flattened over heads and blocks)
+    int hstride;         // row length of the entropy array (b1 rounded up to 4)
     float c_log2;
     float *hent;
     int *status;
@@ -663,8 +696,9 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
             }
             const float inv = 1.f / l;
             const int row = mt * 128 + r;
-            if (row < tb2)   // entropy of the row, natural log: ln2 * (log2 lse - E[x])
-                a.hent[((int64_t)bh * tb2 + row) * p.b1 + up] = kLn2 * (mx + log2f(l) - e * inv);
+            // entropy of the row in log2 units (the L-step works in base 2):
+            // log2(sum 2^x) - E_R[x] = H / ln 2
+            if (row < tb2) a.hent[((int64_t)bh * tb2 + row) * a.hstride + up] = mx + log2f(l) - e * inv;
 #pragma unroll
             for (int c = 0; c < B2P / 16; c++) {
                 uint32_t pk[8];
@@ -769,6 +803,9 @@ bool make_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims,
 }
 
 int b2_padded(int b2) { return (b2 + 15) / 16 * 16; }
+// entropy rows start on 16-byte boundaries (bulk copies); the L-step's copy of
+// the last chunk of a row runs up to 512 bytes past it, hence the tail slack
+int h_stride(const Problem &p) { return (p.b1 + 3) / 4 * 4; }
 int qbar_tiles(const Problem &p) { return (p.tiles * p.b2 + 127) / 128; }
 size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -832,6 +869,7 @@ bool sm100_supports(const Problem &p, monarch_dtype dtype) {
     // TMA coordinates are 32-bit: every row index must fit
     if ((int64_t)p.BH * p.tiles * p.N + 256 >= (1LL << 31)) return false;
     if ((int64_t)p.BH * qbar_tiles(p) * 128 >= (1LL << 31)) return false;
+    if ((int64_t)p.BH * p.tiles * p.b2 * h_stride(p) + 128 >= (1LL << 31)) return false;
     if (encode_fn() == nullptr) return false;
     return true;
 }
@@ -840,8 +878,9 @@ size_t sm100_workspace_bytes(const Problem &p, bool &overflow) {
     overflow = false;
     const size_t mpad = (size_t)qbar_tiles(p) * 128;
     const size_t kz = (size_t)p.BH * p.tiles * p.N * kD * 2;
+    const size_t hrows = (size_t)p.BH * p.tiles * p.b2;
     return al256((size_t)p.BH * mpad * kD * 2) + 2 * al256(kz) +
-           al256((size_t)p.BH * p.tiles * p.N * 4);
+           al256(hrows * h_stride(p) * 4 + 512);
 }
 
 cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const void *v,
@@ -881,7 +920,7 @@ cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const 
         const int sms = sm_count();
         const int bpc = (total + sms - 1) / sms;
         const int grid = (total + bpc - 1) / bpc;
-        RsArgs a{p, nmt, mpad, bpc, c_log2, ws.hent, status, wait_limit};
+        RsArgs a{p, nmt, mpad, bpc, h_stride(p), c_log2, ws.hent, status, wait_limit};
         ProfileScope scope(K_TC_RSTEP, stream);
         cudaError_t e = cudaErrorInvalidValue;
         switch (b2p) {
@@ -911,7 +950,8 @@ cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const 
         const int nq_max = tile_max_rows(p.b1, p.tiles);
         const int npairs = ((nq_max + 127) / 128 + 1) / 2;
         const int nprob = p.BH * p.tiles * p.b2 * npairs;
-        LsArgs a{p, (p.b1 + 127) / 128, npairs, nprob, c_log2, ws.hent, (__nv_bfloat16 *)out,
+        LsArgs a{p, (p.b1 + 127) / 128, npairs, nprob, h_stride(p), c_log2, ws.hent,
+                 (__nv_bfloat16 *)out,
                  status, wait_limit};
         cudaError_t e = set_smem(tc_lstep_kernel, ls::kSmem);
         if (e != cudaSuccess) return e;
