@@ -245,11 +245,35 @@ def kernel_traffic(name: str):
 
 
 # ---------------------------------------------------------------------------
+# ranks (one process per GPU; every rank runs its own clip, no data-path collective)
+# ---------------------------------------------------------------------------
+def rank_barrier(world: int) -> None:
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's time: every rank must call this, in the same order."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, dense_flops_per_clip: float, ms_step: float) -> float:
+    """Whole-job dense-equivalent TFLOP/s: every rank processed one clip per step."""
+    return world * dense_flops_per_clip / (ms_step * 1e-3) / 1e12
+
+
+# ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 def run_ours(args, wl: synth.Workload, world: int, rank: int, local: int):
     import torch
-    import torch.distributed as dist
     from structured_attention_video_b200 import _lib
 
     torch.cuda.set_device(local)
@@ -274,17 +298,6 @@ def run_ours(args, wl: synth.Workload, world: int, rank: int, local: int):
                                             out.data_ptr(), *sargs, _lib.BF16, ws.data_ptr(),
                                             ws_bytes, sh), "monarch_attn_fwd_ws")
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     for _ in range(args.warmup):
         flush.zero_()
         step()
@@ -298,7 +311,7 @@ def run_ours(args, wl: synth.Workload, world: int, rank: int, local: int):
     time.sleep(0.3)
     events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
-    barrier()
+    rank_barrier(world)
     torch.cuda.synchronize()
     _lib.monarch_profile_enable(1)
     for a, b in events:
@@ -307,17 +320,17 @@ def run_ours(args, wl: synth.Workload, world: int, rank: int, local: int):
         step()
         b.record(stream)
     torch.cuda.synchronize()
-    barrier()
+    rank_barrier(world)
     _lib.monarch_profile_enable(0)
     clock_rec = clocks.stop()
     prof = _lib.monarch_profile_collect()
     _lib.check(_lib.monarch_last_device_status(sh), "device status after timed steps")
     ms_total = sum(a.elapsed_time(b) for a, b in events)
-    ms_step = max_over_ranks(ms_total / args.steps)
+    ms_step = max_over_ranks(ms_total / args.steps, world, dev)
 
     # end to end through the host-buffer entry point: H2D inputs, forward, D2H output
     e2e_times = []
-    for i in range(args.e2e_warmup + args.e2e_steps):
+    for i in range(args.e2e_warmup + args.e2e_steps if args.e2e_steps > 0 else 0):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         _lib.check(_lib.monarch_attn_fwd_host(hq.data_ptr(), hk.data_ptr(), hv.data_ptr(),
@@ -327,13 +340,13 @@ def run_ours(args, wl: synth.Workload, world: int, rank: int, local: int):
         torch.cuda.synchronize()
         if i >= args.e2e_warmup:
             e2e_times.append(a.elapsed_time(b))
-    e2e_ms = max_over_ranks(statistics.mean(e2e_times) if e2e_times else float("nan"))
+    e2e_ms = max_over_ranks(statistics.mean(e2e_times), world, dev) if e2e_times else None
 
     if rank != 0:
         return
     peaks, peak_kind = load_peaks()
     dense = wl.dense_flops()
-    value = world * dense / (ms_step * 1e-3) / 1e12
+    value = job_throughput(world, dense, ms_step)
     kernels = {name: {"ms_per_launch": ms / n, "launches": n, "share": ms / max(1e-9, sum(
         m for m, _ in prof.values()))} for name, (ms, n) in prof.items() if n > 0}
     dominant = max(kernels, key=lambda kk: kernels[kk]["ms_per_launch"] * kernels[kk]["launches"])
@@ -359,11 +372,12 @@ def run_ours(args, wl: synth.Workload, world: int, rank: int, local: int):
         "kernels": kernels,
         "kernel_path": "sm100 tensor-core" if path == 1 else "generic SIMT",
         "gpu_launches": launches,
-        "e2e": {"value": world * dense / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
-                "ms_per_step": e2e_ms,
-                "h2d_bytes_per_step": 3 * wl.B * wl.H * wl.N * wl.d * 2,
-                "d2h_bytes_per_step": wl.B * wl.H * wl.N * wl.d * 2,
-                "api": "monarch_attn_fwd_host (C ABI, pinned host buffers)"},
+        "e2e": None if e2e_ms is None else {
+            "value": job_throughput(world, dense, e2e_ms), "unit": UNIT,
+            "ms_per_step": e2e_ms,
+            "h2d_bytes_per_step": 3 * wl.B * wl.H * wl.N * wl.d * 2,
+            "d2h_bytes_per_step": wl.B * wl.H * wl.N * wl.d * 2,
+            "api": "monarch_attn_fwd_host (C ABI, pinned host buffers)"},
         "clocks": clock_rec,
         "gpu": props.name,
     }
