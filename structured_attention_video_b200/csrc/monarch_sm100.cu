@@ -18,9 +18,10 @@
 //                       strides over b2 (P^T folded into the load); online
 //                       softmax over the b1 blocks with logits s q.Ktil + H,
 //                       O accumulated in TMEM, rows written back strided.
-// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM
-// owner, warps 4-7 and 8-11 the two softmax (L-step) or the softmax and
-// epilogue (R-step) warpgroups; warps 2-3 idle.  Every wait on another role is
+// Warp roles (384 threads): warp 0 TMA producer (in the L-step: queries, Ktil
+// and entropies; warp 2 produces Z), warp 1 MMA issuer and TMEM owner, warps
+// 4-7 and 8-11 the two softmax (L-step) or the softmax and epilogue (R-step)
+// warpgroups; the remaining warps idle.  Every wait on another role is
 // a bounded mbarrier wait (tc_primitives.cuh): on time-out the kernel records
 // MONARCH_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
 #include "monarch_sm100.cuh"
@@ -120,12 +121,17 @@ __global__ void __launch_bounds__(128) tc_qbar_kernel(const __nv_bfloat16 *__res
 // current one finishes, and its first S MMAs overlap the current epilogue)
 // =====================================================================
 namespace ls {
-constexpr uint32_t kQ = 0;                 // query tiles 0, 1
-constexpr uint32_t kK = 2 * kTile;         // Ktil stages 0, 1
-constexpr uint32_t kZ = 4 * kTile;         // Z stages 0, 1
-constexpr uint32_t kH = 6 * kTile;         // H * log2(e) per chunk: 4 buffers of 128 floats
+// Ktil and Z stages in shared memory (a third Ktil stage measured slower: it
+// leaves the L1 cache almost no room)
+constexpr int kKStages = 2;
+constexpr uint32_t kQ = 0;                          // query tiles 0, 1
+constexpr uint32_t kK = 2 * kTile;                  // Ktil stages
+constexpr uint32_t kZ = kK + kKStages * kTile;      // Z stages 0, 1
+constexpr uint32_t kH = kZ + 2 * kTile;             // entropies: 4 buffers of 128 floats
 constexpr uint32_t kBar = kH + 2048;
-constexpr uint32_t kSmem = kBar + 256 + 1024;
+constexpr uint32_t kSmem = kBar + 256;              // the base is 1024-aligned (checked)
+static_assert(kSmem <= (uint32_t)kMaxSmem, "L-step shared memory");
+static_assert(kKStages >= 2 && kKStages <= 3, "the four entropy buffers cover at most three Ktil stages");
 }  // namespace ls
 
 struct LsArgs {
@@ -164,22 +170,28 @@ __device__ __forceinline__ LsProblem ls_problem(const LsArgs &a, int unit) {
 __global__ void __launch_bounds__(384, 1)
 tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmZ, LsArgs a) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = align1024(smem_raw);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // the SW128 operand tiles need a 1024-byte aligned base; the layout leaves no
+    // room to align by hand, so a misaligned base is reported, not worked around
+    if ((smem_u32(smem_raw) & 1023u) != 0) {
+        if (threadIdx.x == 0) record_status(a.status, MONARCH_ERR_CUDA);
+        return;
+    }
+    uint8_t *sm = smem_raw;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + ls::kBar);
     uint64_t *q_full = bars + 0;
     uint64_t *q_empty = bars + 1;
-    uint64_t *k_full = bars + 2;     // [2 stages]
-    uint64_t *z_full = bars + 4;     // [2 stages]
-    uint64_t *k_empty = bars + 6;    // [2 stages]: both S MMAs of the chunk done
-    uint64_t *z_empty = bars + 8;    // [2 stages]: both PV MMAs of the chunk done
-    uint64_t *h_full = bars + 10;    // [4 buffers]: bulk copy of the chunk's entropies
-    uint64_t *s_full = bars + 14;    // [2 tiles]
-    uint64_t *p_full = bars + 16;    // [2 tiles], 128 arrivals
-    uint64_t *o_full = bars + 18;    // [2 tiles]
-    uint64_t *mma_done = bars + 20;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 21);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 22);
+    uint64_t *k_full = bars + 2;     // [3 stages]
+    uint64_t *k_empty = bars + 5;    // [3 stages]: both S MMAs of the chunk done
+    uint64_t *z_full = bars + 8;     // [2 stages]
+    uint64_t *z_empty = bars + 10;   // [2 stages]: both PV MMAs of the chunk done
+    uint64_t *h_full = bars + 12;    // [4 buffers]: bulk copy of the chunk's entropies
+    uint64_t *s_full = bars + 16;    // [2 tiles]
+    uint64_t *p_full = bars + 18;    // [2 tiles], one arrival per softmax warp
+    uint64_t *o_full = bars + 20;    // [2 tiles]
+    uint64_t *mma_done = bars + 22;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 23);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 24);
 
     const Problem &p = a.p;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -190,13 +202,15 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
         mbar_init(q_empty, 1);
-        for (int s = 0; s < 2; s++) {
+        for (int s = 0; s < ls::kKStages; s++) {
             mbar_init(k_full + s, 1);
-            mbar_init(z_full + s, 1);
             mbar_init(k_empty + s, 1);
+        }
+        for (int s = 0; s < 2; s++) {
+            mbar_init(z_full + s, 1);
             mbar_init(z_empty + s, 1);
             mbar_init(s_full + s, 1);
-            mbar_init(p_full + s, 128);
+            mbar_init(p_full + s, 4);   // one arrival per softmax warp
             mbar_init(o_full + s, 1);
         }
         for (int s = 0; s < 4; s++) mbar_init(h_full + s, 1);
@@ -214,10 +228,11 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     if (warp == 0) {
         // ---------------- producer: queries per problem; per chunk Ktil and H as
         // soon as the S MMAs of two chunks back are done, Z once their PV MMAs are.
-        // H has four buffers: when S1 of chunk jc-2 completes, both softmax
-        // warpgroups have finished chunk jc-3, so buffer jc & 3 (last read for
-        // chunk jc-4) is free.
-        int issued[2] = {0, 0}, issued_z[2] = {0, 0}, qloads = 0, issued_h = 0;
+        // H has four buffers: S1 of chunk jc - kKStages (whose completion frees
+        // the Ktil stage of chunk jc) is issued only after both softmax
+        // warpgroups have finished chunk jc - kKStages - 1, so buffer jc & 3
+        // (last read for chunk jc - 4) is free for kKStages <= 3.
+        int issued[ls::kKStages] = {}, qloads = 0, issued_h = 0;
         bool ok = true;
         for (int pi = 0; ok && pi < nmine; pi++) {
             const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
@@ -231,16 +246,17 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             }
             qloads++;
             for (int j = 0; j < nch; j++) {
-                const int jc = pi * nch + j, st = jc & 1;
-                if (jc >= 2 && !wait_warp(k_empty + st, ((jc >> 1) - 1) & 1, w)) {
+                const int jc = pi * nch + j, sk = jc % ls::kKStages;
+                if (jc >= ls::kKStages &&
+                    !wait_warp(k_empty + sk, ((jc / ls::kKStages) - 1) & 1, w)) {
                     ok = false;
                     break;
                 }
                 if (lane == 0) {
-                    mbar_expect_tx(k_full + st, kTile);
+                    mbar_expect_tx(k_full + sk, kTile);
                     for (int pn = 0; pn < 2; pn++)
-                        tma_load_2d(sm + ls::kK + st * kTile + pn * kPanel, &tmK, pn * 64,
-                                    pr.key_row0 + j * 128, k_full + st);
+                        tma_load_2d(sm + ls::kK + sk * kTile + pn * kPanel, &tmK, pn * 64,
+                                    pr.key_row0 + j * 128, k_full + sk);
                     // Only two chunks fit in shared memory, fewer than the memory
                     // latency needs: move the chunk kPrefetch steps ahead (possibly of
                     // this CTA's next problem) into L2 now, and at the start of a
@@ -262,13 +278,34 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                         }
                     }
                 }
-                issued[st]++;
+                issued[sk]++;
                 if (lane == 0) {   // the chunk's entropies (log2 units, -inf past b1)
                     mbar_expect_tx(h_full + (jc & 3), 512);
                     bulk_load(sm + ls::kH + (jc & 3) * 512, a.hent + pr.h_row0 + j * 128, 512,
                               h_full + (jc & 3));
                 }
                 issued_h++;
+            }
+        }
+        if (lane == 0) {   // every issued copy lands before the CTA may exit
+            if (qloads > 0) wait_phase_cleanup(q_full, (qloads - 1) & 1, kCleanupPolls);
+            for (int s = 0; s < ls::kKStages; s++)
+                if (issued[s] > 0) wait_phase_cleanup(k_full + s, (issued[s] - 1) & 1, kCleanupPolls);
+            for (int hb = 0; hb < 4; hb++) {   // the last copy into each entropy buffer
+                if (issued_h <= hb) continue;
+                const int last = hb + ((issued_h - 1 - hb) / 4) * 4;
+                wait_phase_cleanup(h_full + hb, (last >> 2) & 1, kCleanupPolls);
+            }
+        }
+    } else if (warp == 2) {
+        // ---------------- Z producer: its own warp, so that a Ktil load never
+        // queues behind the wait for a Z stage (released one PV later than Ktil)
+        int issued_z[2] = {0, 0};
+        bool ok = true;
+        for (int pi = 0; ok && pi < nmine; pi++) {
+            const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
+            for (int j = 0; j < nch; j++) {
+                const int jc = pi * nch + j, st = jc & 1;
                 if (jc >= 2 && !wait_warp(z_empty + st, ((jc >> 1) - 1) & 1, w)) {
                     ok = false;
                     break;
@@ -282,25 +319,17 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 issued_z[st]++;
             }
         }
-        if (lane == 0) {   // every issued copy lands before the CTA may exit
-            if (qloads > 0) wait_phase_cleanup(q_full, (qloads - 1) & 1, kCleanupPolls);
-            for (int s = 0; s < 2; s++) {
-                if (issued[s] > 0) wait_phase_cleanup(k_full + s, (issued[s] - 1) & 1, kCleanupPolls);
+        if (lane == 0)
+            for (int s = 0; s < 2; s++)
                 if (issued_z[s] > 0)
                     wait_phase_cleanup(z_full + s, (issued_z[s] - 1) & 1, kCleanupPolls);
-            }
-            for (int hb = 0; hb < 4; hb++) {   // the last copy into each entropy buffer
-                if (issued_h <= hb) continue;
-                const int last = hb + ((issued_h - 1 - hb) / 4) * 4;
-                wait_phase_cleanup(h_full + hb, (last >> 2) & 1, kCleanupPolls);
-            }
-        }
     } else if (warp == 1) {
         // ---------------- MMA issuer.  Per chunk: PV0, then S0 of the next chunk,
         // PV1, S1 of the next chunk, so that a tile's chain never waits on the
         // other tile's softmax.  Descriptors are precomputed bases plus
-        // compile-time K-step offsets, keeping the single issuing thread lean.
-        if (lane == 0) {
+        // compile-time K-step offsets.  The whole warp runs this loop and one
+        // elected lane issues each MMA (see mma_ss_warp).
+        {
             constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t idO = idesc_bf16(128, 128, 0, 1);
             const uint64_t dQ = smem_desc_sw128(smem_u32(sm + ls::kQ), 16, 1024);
@@ -311,34 +340,34 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             // S_t for global chunk index jc (waits for the chunk's Ktil and, if the
             // chunk opens a problem, for its queries)
             auto issue_s = [&](int t, int jc) -> bool {
-                const int st = jc & 1;
-                if (t == 0 && jc % nch == 0 && !spin_phase(q_full, (jc / nch) & 1, w)) return false;
-                if (t == 0 && !spin_phase(k_full + st, (jc >> 1) & 1, w)) return false;
+                const int sk = jc % ls::kKStages;
+                if (t == 0 && jc % nch == 0 && !spin_warp(q_full, (jc / nch) & 1, w)) return false;
+                if (t == 0 && !spin_warp(k_full + sk, (jc / ls::kKStages) & 1, w)) return false;
                 tc_fence_after();
-                const uint64_t a0 = desc_plus(dQ, t * kTile), b0 = desc_plus(dK, st * kTile);
+                const uint64_t a0 = desc_plus(dQ, t * kTile), b0 = desc_plus(dK, sk * kTile);
 #pragma unroll
                 for (int kk = 0; kk < 8; kk++) {
                     const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-                    mma_ss(tmem + t * 128, desc_plus(a0, off), desc_plus(b0, off), idS, kk > 0);
+                    mma_ss_warp(tmem + t * 128, desc_plus(a0, off), desc_plus(b0, off), idS, kk > 0);
                 }
-                mma_commit(s_full + t);
-                if (t == 1) mma_commit(k_empty + st);
-                if (t == 1 && jc % nch == nch - 1) mma_commit(q_empty);   // queries no longer read
+                mma_commit_warp(s_full + t);
+                if (t == 1) mma_commit_warp(k_empty + sk);
+                if (t == 1 && jc % nch == nch - 1) mma_commit_warp(q_empty);   // queries no longer read
                 return true;
             };
             auto issue_pv = [&](int t, int jc) -> bool {
                 const int st = jc & 1;
-                if (t == 0 && !spin_phase(z_full + st, (jc >> 1) & 1, w)) return false;
-                if (!spin_phase(p_full + t, jc & 1, w)) return false;
+                if (t == 0 && !spin_warp(z_full + st, (jc >> 1) & 1, w)) return false;
+                if (!spin_warp(p_full + t, jc & 1, w)) return false;
                 tc_fence_after();
                 const uint64_t b0 = desc_plus(dZ, st * kTile);
                 const uint32_t acc0 = (jc % nch) > 0 ? 1u : 0u;
 #pragma unroll
                 for (int kk = 0; kk < 8; kk++)
-                    mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, desc_plus(b0, kk * 2048),
+                    mma_ts_warp(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, desc_plus(b0, kk * 2048),
                            idO, kk > 0 ? 1u : acc0);
-                mma_commit(o_full + t);
-                if (t == 1) mma_commit(z_empty + st);
+                mma_commit_warp(o_full + t);
+                if (t == 1) mma_commit_warp(z_empty + st);
                 return true;
             };
             // S_t of the next chunk overwrites the columns that PV_t reads as P:
@@ -352,7 +381,7 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     if (ok && jc + 1 < total) ok = issue_s(t, jc + 1);
                 }
             }
-            mma_commit(mma_done);
+            mma_commit_warp(mma_done);
             wait_phase_cleanup(mma_done, 0, kCleanupPolls);
         }
     } else if (warp >= 4) {
@@ -445,7 +474,7 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(p_full + t);
+                mbar_arrive_warp(p_full + t);
             }
             if (!ok || !wait_warp(o_full + t, (pi * nch + nch - 1) & 1, w)) {
                 ok = false;
@@ -526,9 +555,9 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
     uint64_t *kv_empty = bars + 4;   // [2]
     uint64_t *s_full = bars + 6;     // [2]
     uint64_t *s_free = bars + 8;     // [2]
-    uint64_t *p_full = bars + 10;    // [2], 128 arrivals
+    uint64_t *p_full = bars + 10;    // [2], one arrival per softmax warp
     uint64_t *o_full = bars + 12;    // [2]: Z part, Ktil part
-    uint64_t *o_empty = bars + 14;   // [2], 128 arrivals
+    uint64_t *o_empty = bars + 14;   // [2], one arrival per epilogue warp
     uint64_t *mma_done = bars + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 17);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 18);
@@ -549,9 +578,9 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
             mbar_init(kv_empty + s, 1);
             mbar_init(s_full + s, 1);
             mbar_init(s_free + s, 1);
-            mbar_init(p_full + s, 128);
+            mbar_init(p_full + s, 4);   // one arrival per softmax warp
             mbar_init(o_full + s, 1);
-            mbar_init(o_empty + s, 128);
+            mbar_init(o_empty + s, 4);   // one arrival per epilogue warp
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -599,8 +628,9 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                     wait_phase_cleanup(kv_full + s, (issued[s] - 1) & 1, kCleanupPolls);
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer
-        if (lane == 0) {
+        // ---------------- MMA issuer: the whole warp runs the loop, one elected
+        // lane issues each MMA (see mma_ss_warp)
+        {
             constexpr uint32_t id1 = idesc_bf16(128, B2P, 0, 0);
             constexpr uint32_t id2 = idesc_bf16(128, 128, 0, 1);
             const uint64_t dQ = smem_desc_sw128(smem_u32(sm), 16, 1024);
@@ -614,51 +644,51 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 const int fb = first + ib, bh = fb / p.b1;
                 if (mt == 0) {
                     if (ib == 0 || (fb - 1) / p.b1 != bh) {
-                        if (!wait_phase(q_full, heads & 1, w)) return false;
+                        if (!wait_warp(q_full, heads & 1, w)) return false;
                         heads++;
                     }
-                    if (!wait_phase(kv_full + (ib & 1), (ib >> 1) & 1, w)) return false;
+                    if (!wait_warp(kv_full + (ib & 1), (ib >> 1) & 1, w)) return false;
                 }
-                if (i >= 2 && !wait_phase(s_free + (i & 1), ((i >> 1) - 1) & 1, w)) return false;
+                if (i >= 2 && !wait_warp(s_free + (i & 1), ((i >> 1) - 1) & 1, w)) return false;
                 tc_fence_after();
                 const uint64_t a0 = desc_plus(dQ, mt * kTile);
                 const uint64_t b0 = desc_plus(dK, (ib & 1) * L::kStage);
 #pragma unroll
                 for (int kk = 0; kk < 8; kk++)
-                    mma_ss(tmem + (i & 1) * 128,
+                    mma_ss_warp(tmem + (i & 1) * 128,
                            desc_plus(a0, (kk >> 2) * kPanel + (kk & 3) * 32),
                            desc_plus(b0, (kk >> 2) * L::kPanelKV + (kk & 3) * 32), id1, kk > 0);
-                mma_commit(s_full + (i & 1));
+                mma_commit_warp(s_full + (i & 1));
                 const bool head_ends = (ib == nblk - 1) || ((fb + 1) / p.b1 != bh);
-                if (mt == nmt - 1 && head_ends) mma_commit(q_empty);
+                if (mt == nmt - 1 && head_ends) mma_commit_warp(q_empty);
                 return true;
             };
             if (nitems > 0) ok = gemm1(0);
             for (int i = 0; ok && i < nitems; i++) {
                 if (i + 1 < nitems && !gemm1(i + 1)) break;
                 const int ib = i / nmt, mt = i % nmt;
-                if (!wait_phase(p_full + (i & 1), (i >> 1) & 1, w)) break;
+                if (!wait_warp(p_full + (i & 1), (i >> 1) & 1, w)) break;
                 tc_fence_after();
                 const uint32_t pa = tmem + (i & 1) * 128;
                 // 0: Z = R V, 1: Ktil = R K
                 const uint64_t bz = desc_plus(dV, (ib & 1) * L::kStage + L::kVOff);
                 const uint64_t bk = desc_plus(dV, (ib & 1) * L::kStage);
-                if (i > 0 && !wait_phase(o_empty + 0, (i - 1) & 1, w)) break;
+                if (i > 0 && !wait_warp(o_empty + 0, (i - 1) & 1, w)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < B2P / 16; kk++)
-                    mma_ts(tmem + 256, pa + kk * 8, desc_plus(bz, kk * 2048), id2, kk > 0 ? 1u : 0u);
-                mma_commit(o_full + 0);
-                if (i > 0 && !wait_phase(o_empty + 1, (i - 1) & 1, w)) break;
+                    mma_ts_warp(tmem + 256, pa + kk * 8, desc_plus(bz, kk * 2048), id2, kk > 0 ? 1u : 0u);
+                mma_commit_warp(o_full + 0);
+                if (i > 0 && !wait_warp(o_empty + 1, (i - 1) & 1, w)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < B2P / 16; kk++)
-                    mma_ts(tmem + 384, pa + kk * 8, desc_plus(bk, kk * 2048), id2, kk > 0 ? 1u : 0u);
-                mma_commit(o_full + 1);
-                mma_commit(s_free + (i & 1));
-                if (mt == nmt - 1) mma_commit(kv_empty + (ib & 1));
+                    mma_ts_warp(tmem + 384, pa + kk * 8, desc_plus(bk, kk * 2048), id2, kk > 0 ? 1u : 0u);
+                mma_commit_warp(o_full + 1);
+                mma_commit_warp(s_free + (i & 1));
+                if (mt == nmt - 1) mma_commit_warp(kv_empty + (ib & 1));
             }
-            mma_commit(mma_done);
+            mma_commit_warp(mma_done);
             wait_phase_cleanup(mma_done, 0, kCleanupPolls);
         }
     } else if (warp >= 4 && warp < 8) {
@@ -709,7 +739,7 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(p_full + (i & 1));
+            mbar_arrive_warp(p_full + (i & 1));
         }
     } else if (warp >= 8) {
         // ---------------- epilogue: Z and Ktil rows -> bf16 -> staging -> TMA store
@@ -738,7 +768,7 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                             pack_bf16(__uint_as_float(o[2 * k]), __uint_as_float(o[2 * k + 1]));
                 }
                 tc_fence_before();
-                mbar_arrive(o_empty + part);
+                mbar_arrive_warp(o_empty + part);
                 // the previous store of this warp must have finished reading staging
                 if (lane == 0) tma_store_wait_read_all();
                 __syncwarp();

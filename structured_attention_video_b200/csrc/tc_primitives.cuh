@@ -53,6 +53,15 @@ struct WaitCtx {
     volatile int *abort;
 };
 
+// One arrival for the whole (converged) warp, on barriers that count warps:
+// the lanes synchronise first, so lane 0's arrival (a release) also orders the
+// other lanes' earlier writes, and the barrier takes one shared-memory atomic
+// per warp instead of 32.
+__device__ __forceinline__ void mbar_arrive_warp(uint64_t *bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 // Waits for the phase with `parity` of `bar` to complete.  Returns false when
 // the CTA is aborting or after `limit` polls (then it records
 // MONARCH_ERR_TIMEOUT and raises the abort flag).  Never traps, never spins
@@ -188,6 +197,37 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
     asm volatile(
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+// Warp-collective forms of the three calls above: every lane of a converged
+// warp executes them with the same (warp-uniform) operands and elect.sync
+// picks the lane that issues.  Keeping the issuing warp convergent lets the
+// operands live in uniform registers; an MMA issued from a one-lane divergent
+// branch costs several times more issue slots, which the softmax warps sharing
+// the SM sub-partition then take away (measured: 209 instead of 97 clocks per
+// M128 N128 K16 MMA next to FMA-bound warps, against 64 on a quiet SM).
+__device__ __forceinline__ void mma_ss_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit_warp(uint64_t *bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
             smem_u32(bar))
         : "memory");
 }
@@ -359,6 +399,12 @@ __device__ __forceinline__ bool spin_phase(uint64_t *bar, uint32_t parity, const
             }
         }
     }
+}
+
+// spin_phase for a whole warp: every lane polls, and the warp takes one decision.
+__device__ __forceinline__ bool spin_warp(uint64_t *bar, uint32_t parity, const WaitCtx &w) {
+    const bool ok = spin_phase(bar, parity, w);
+    return __all_sync(0xffffffffu, ok);
 }
 
 // ---------------------------------------------------------------- math
