@@ -326,60 +326,72 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     } else if (warp == 1) {
         // ---------------- MMA issuer.  Per chunk: PV0, then S0 of the next chunk,
         // PV1, S1 of the next chunk, so that a tile's chain never waits on the
-        // other tile's softmax.  Descriptors are precomputed bases plus
-        // compile-time K-step offsets.  The whole warp runs this loop and one
-        // elected lane issues each MMA (see mma_ss_warp).
+        // other tile's softmax.  The whole warp runs this loop; every group of
+        // eight MMAs goes out from one elect.sync region with descriptors
+        // computed once here (mma_group_ss), and the chunk loop is unrolled by
+        // the stage parity so that they stay in registers.
+        static_assert(ls::kKStages == 2, "the MMA loop unrolls over two stages");
         {
             constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t idO = idesc_bf16(128, 128, 0, 1);
             const uint64_t dQ = smem_desc_sw128(smem_u32(sm + ls::kQ), 16, 1024);
             const uint64_t dK = smem_desc_sw128(smem_u32(sm + ls::kK), 16, 1024);
             const uint64_t dZ = smem_desc_sw128(smem_u32(sm + ls::kZ), kPanel, 1024);
+            uint64_t aq0[8], aq1[8], bk0[8], bk1[8], bz0[8], bz1[8];
+#pragma unroll
+            for (int kk = 0; kk < 8; kk++) {
+                const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
+                aq0[kk] = desc_plus(dQ, off);
+                aq1[kk] = desc_plus(dQ, kTile + off);
+                bk0[kk] = desc_plus(dK, off);
+                bk1[kk] = desc_plus(dK, kTile + off);
+                bz0[kk] = desc_plus(dZ, kk * 2048);
+                bz1[kk] = desc_plus(dZ, kTile + kk * 2048);
+            }
             const int total = nmine * nch;
             bool ok = true;
             // S_t for global chunk index jc (waits for the chunk's Ktil and, if the
             // chunk opens a problem, for its queries)
-            auto issue_s = [&](int t, int jc) -> bool {
-                const int sk = jc % ls::kKStages;
+            auto issue_s = [&](int t, int jc, const uint64_t(&aq)[8], const uint64_t(&bk)[8]) -> bool {
+                const int sk = jc & 1;
                 if (t == 0 && jc % nch == 0 && !spin_warp(q_full, (jc / nch) & 1, w)) return false;
-                if (t == 0 && !spin_warp(k_full + sk, (jc / ls::kKStages) & 1, w)) return false;
+                if (t == 0 && !spin_warp(k_full + sk, (jc >> 1) & 1, w)) return false;
                 tc_fence_after();
-                const uint64_t a0 = desc_plus(dQ, t * kTile), b0 = desc_plus(dK, sk * kTile);
-#pragma unroll
-                for (int kk = 0; kk < 8; kk++) {
-                    const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-                    mma_ss_warp(tmem + t * 128, desc_plus(a0, off), desc_plus(b0, off), idS, kk > 0);
-                }
+                mma_group_ss(tmem + t * 128, aq, bk, idS, 0u, 8u);
                 mma_commit_warp(s_full + t);
                 if (t == 1) mma_commit_warp(k_empty + sk);
                 if (t == 1 && jc % nch == nch - 1) mma_commit_warp(q_empty);   // queries no longer read
                 return true;
             };
-            auto issue_pv = [&](int t, int jc) -> bool {
+            auto issue_pv = [&](int t, int jc, const uint64_t(&bz)[8]) -> bool {
                 const int st = jc & 1;
                 if (t == 0 && !spin_warp(z_full + st, (jc >> 1) & 1, w)) return false;
                 if (!spin_warp(p_full + t, jc & 1, w)) return false;
                 tc_fence_after();
-                const uint64_t b0 = desc_plus(dZ, st * kTile);
-                const uint32_t acc0 = (jc % nch) > 0 ? 1u : 0u;
-#pragma unroll
-                for (int kk = 0; kk < 8; kk++)
-                    mma_ts_warp(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, desc_plus(b0, kk * 2048),
-                           idO, kk > 0 ? 1u : acc0);
+                mma_group_ts(tmem + 256 + t * 128, tmem + t * 128, bz, idO,
+                             (jc % nch) > 0 ? 1u : 0u, 8u);
                 mma_commit_warp(o_full + t);
                 if (t == 1) mma_commit_warp(z_empty + st);
+                return true;
+            };
+            // one chunk: PV_t of chunk jc (Z stage jc & 1), then S_t of chunk jc + 1
+            // (Ktil stage (jc + 1) & 1)
+            auto chunk = [&](int jc, const uint64_t(&bz)[8], const uint64_t(&bkn)[8]) -> bool {
+                const bool more = jc + 1 < total;
+                if (!issue_pv(0, jc, bz)) return false;
+                if (more && !issue_s(0, jc + 1, aq0, bkn)) return false;
+                if (!issue_pv(1, jc, bz)) return false;
+                if (more && !issue_s(1, jc + 1, aq1, bkn)) return false;
                 return true;
             };
             // S_t of the next chunk overwrites the columns that PV_t reads as P:
             // tcgen05 MMAs issued by one thread execute in issue order, so it is
             // issued right behind PV_t without waiting; its commit (s_full) also
             // covers PV_t, which orders the softmax's rescale of O_t after PV_t.
-            if (total > 0) ok = issue_s(0, 0) && issue_s(1, 0);
-            for (int jc = 0; ok && jc < total; jc++) {
-                for (int t = 0; t < 2 && ok; t++) {
-                    ok = issue_pv(t, jc);
-                    if (ok && jc + 1 < total) ok = issue_s(t, jc + 1);
-                }
+            if (total > 0) ok = issue_s(0, 0, aq0, bk0) && issue_s(1, 0, aq1, bk0);
+            for (int jc = 0; ok && jc < total; jc += 2) {
+                ok = chunk(jc, bz0, bk1);
+                if (ok && jc + 1 < total) ok = chunk(jc + 1, bz1, bk0);
             }
             mma_commit_warp(mma_done);
             wait_phase_cleanup(mma_done, 0, kCleanupPolls);
