@@ -73,13 +73,15 @@ __global__ void __launch_bounds__(128) tc_qbar_kernel(const __nv_bfloat16 *__res
 #pragma unroll
         for (int i = 0; i < 8; i++) acc[i] = 0.f;
         int u = u0;
-        for (; u + 4 <= u1; u += 4) {
-            uint4 x[4];
+        // eight independent 16-byte loads in flight per thread: the grid has only
+        // B*H*t*ceil(b2*d/1024) blocks, too few warps to cover the memory latency
+        for (; u + 8 <= u1; u += 8) {
+            uint4 x[8];
 #pragma unroll
-            for (int k = 0; k < 4; k++) x[k] = __ldg(src + k * stride);
-            src += 4 * stride;
+            for (int k = 0; k < 8; k++) x[k] = __ldg(src + k * stride);
+            src += 8 * stride;
 #pragma unroll
-            for (int k = 0; k < 4; k++) {
+            for (int k = 0; k < 8; k++) {
                 const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&x[k]);
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
