@@ -40,7 +40,6 @@ constexpr uint32_t kPanel = 128 * 128;         // 128 rows x 64 bf16 (128 B), SW
 constexpr uint32_t kTile = 2 * kPanel;         // 128 rows x 128 bf16
 constexpr int kMaxSmem = 232448;               // sm_100 opt-in dynamic shared memory
 constexpr long long kCleanupPolls = 1LL << 22;
-constexpr int kPrefetch = 4;                   // L-step: chunks of Ktil / Z prefetched to L2 ahead
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -181,19 +180,19 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     uint8_t *sm = smem_raw;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + ls::kBar);
-    uint64_t *q_full = bars + 0;
-    uint64_t *q_empty = bars + 1;
-    uint64_t *k_full = bars + 2;     // [3 stages]
-    uint64_t *k_empty = bars + 5;    // [3 stages]: both S MMAs of the chunk done
-    uint64_t *z_full = bars + 8;     // [2 stages]
-    uint64_t *z_empty = bars + 10;   // [2 stages]: both PV MMAs of the chunk done
-    uint64_t *h_full = bars + 12;    // [4 buffers]: bulk copy of the chunk's entropies
-    uint64_t *s_full = bars + 16;    // [2 tiles]
-    uint64_t *p_full = bars + 18;    // [2 tiles], one arrival per softmax warp
-    uint64_t *o_full = bars + 20;    // [2 tiles]
-    uint64_t *mma_done = bars + 22;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 23);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 24);
+    uint64_t *q_full = bars + 0;     // [2 tiles]
+    uint64_t *q_empty = bars + 2;    // [2 tiles]: the tile's last S MMA of a problem done
+    uint64_t *k_full = bars + 4;     // [3 stages]
+    uint64_t *k_empty = bars + 7;    // [3 stages]: both S MMAs of the chunk done
+    uint64_t *z_full = bars + 10;    // [2 stages]
+    uint64_t *z_empty = bars + 12;   // [2 stages]: both PV MMAs of the chunk done
+    uint64_t *h_full = bars + 14;    // [4 buffers]: bulk copy of the chunk's entropies
+    uint64_t *s_full = bars + 18;    // [2 tiles]
+    uint64_t *p_full = bars + 20;    // [2 tiles], one arrival per softmax warp
+    uint64_t *o_full = bars + 22;    // [2 tiles]
+    uint64_t *mma_done = bars + 24;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 25);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 26);
 
     const Problem &p = a.p;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -202,8 +201,10 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int nch = a.nchunks;
 
     if (threadIdx.x == 0) {
-        mbar_init(q_full, 1);
-        mbar_init(q_empty, 1);
+        for (int t = 0; t < 2; t++) {
+            mbar_init(q_full + t, 1);
+            mbar_init(q_empty + t, 1);
+        }
         for (int s = 0; s < ls::kKStages; s++) {
             mbar_init(k_full + s, 1);
             mbar_init(k_empty + s, 1);
@@ -238,14 +239,21 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         bool ok = true;
         for (int pi = 0; ok && pi < nmine; pi++) {
             const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
-            if (pi > 0 && !wait_warp(q_empty, (pi - 1) & 1, w)) break;
-            if (lane == 0) {
-                mbar_expect_tx(q_full, 2 * kTile);
-                for (int t = 0; t < 2; t++)
+            // each query tile reloads as soon as its own last S MMA of the
+            // previous problem is done (tile 0 one PV + S earlier than tile 1)
+            for (int t = 0; ok && t < 2; t++) {
+                if (pi > 0 && !wait_warp(q_empty + t, (pi - 1) & 1, w)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    mbar_expect_tx(q_full + t, kTile);
                     for (int pn = 0; pn < 2; pn++)
                         tma_load_3d(sm + ls::kQ + t * kTile + pn * kPanel, &tmQ, pn * 64, pr.v,
-                                    pr.bh * p.b1 + pr.u_start + t * 128, q_full);
+                                    pr.bh * p.b1 + pr.u_start + t * 128, q_full + t);
+                }
             }
+            if (!ok) break;
             qloads++;
             for (int j = 0; j < nch; j++) {
                 const int jc = pi * nch + j, sk = jc % ls::kKStages;
@@ -259,29 +267,9 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     for (int pn = 0; pn < 2; pn++)
                         tma_load_2d(sm + ls::kK + sk * kTile + pn * kPanel, &tmK, pn * 64,
                                     pr.key_row0 + j * 128, k_full + sk);
-                    // Only two chunks fit in shared memory, fewer than the memory
-                    // latency needs: move the chunk kPrefetch steps ahead (possibly of
-                    // this CTA's next problem) into L2 now, and at the start of a
-                    // problem the next problem's queries.
-                    const int ahead = j + kPrefetch, pa = pi + ahead / nch;
-                    if (pa < nmine) {
-                        const LsProblem pn2 = ls_problem(a, blockIdx.x + pa * gridDim.x);
-                        const int row = pn2.key_row0 + (ahead % nch) * 128;
-                        for (int pn = 0; pn < 2; pn++) {
-                            tma_prefetch_2d(&tmK, pn * 64, row);
-                            tma_prefetch_2d(&tmZ, pn * 64, row);
-                        }
-                        if (j == 0 && pi + 1 < nmine) {
-                            const LsProblem nq = ls_problem(a, blockIdx.x + (pi + 1) * gridDim.x);
-                            for (int t = 0; t < 2; t++)
-                                for (int pn = 0; pn < 2; pn++)
-                                    tma_prefetch_3d(&tmQ, pn * 64, nq.v,
-                                                    nq.bh * p.b1 + nq.u_start + t * 128);
-                        }
-                    }
                 }
                 issued[sk]++;
-                if (lane == 0) {   // the chunk's entropies (log2 units, -inf past b1)
+                if (lane == 0) {   // the chunk's entropies (log2 units; keys past b1 are masked later)
                     mbar_expect_tx(h_full + (jc & 3), 512);
                     bulk_load(sm + ls::kH + (jc & 3) * 512, a.hent + pr.h_row0 + j * 128, 512,
                               h_full + (jc & 3));
@@ -290,7 +278,8 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             }
         }
         if (lane == 0) {   // every issued copy lands before the CTA may exit
-            if (qloads > 0) wait_phase_cleanup(q_full, (qloads - 1) & 1, kCleanupPolls);
+            for (int t = 0; t < 2; t++)
+                if (qloads > 0) wait_phase_cleanup(q_full + t, (qloads - 1) & 1, kCleanupPolls);
             for (int s = 0; s < ls::kKStages; s++)
                 if (issued[s] > 0) wait_phase_cleanup(k_full + s, (issued[s] - 1) & 1, kCleanupPolls);
             for (int hb = 0; hb < 4; hb++) {   // the last copy into each entropy buffer
@@ -356,13 +345,13 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             // chunk opens a problem, for its queries)
             auto issue_s = [&](int t, int jc, const uint64_t(&aq)[8], const uint64_t(&bk)[8]) -> bool {
                 const int sk = jc & 1;
-                if (t == 0 && jc % nch == 0 && !spin_warp(q_full, (jc / nch) & 1, w)) return false;
+                if (jc % nch == 0 && !spin_warp(q_full + t, (jc / nch) & 1, w)) return false;
                 if (t == 0 && !spin_warp(k_full + sk, (jc >> 1) & 1, w)) return false;
                 tc_fence_after();
                 mma_group_ss(tmem + t * 128, aq, bk, idS, 0u, 8u);
                 mma_commit_warp(s_full + t);
                 if (t == 1) mma_commit_warp(k_empty + sk);
-                if (t == 1 && jc % nch == nch - 1) mma_commit_warp(q_empty);   // queries no longer read
+                if (jc % nch == nch - 1) mma_commit_warp(q_empty + t);   // tile t no longer read
                 return true;
             };
             auto issue_pv = [&](int t, int jc, const uint64_t(&bz)[8]) -> bool {
