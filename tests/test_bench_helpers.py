@@ -1,0 +1,93 @@
+"""bench.py's host-side bookkeeping, on the CPU: rooflines, the traffic record
+and the workload description.  The GPU timing itself is covered by running
+bench.py on a B200."""
+import hashlib
+import json
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from structured_attention_video_b200 import synth  # noqa: E402
+
+PEAKS = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0,
+         "sm_max_mhz": 1965.0}
+
+
+def test_lstep_roofline_uses_the_algorithmic_flops_and_the_sustained_peak():
+    wl = synth.WORKLOADS["720p"]
+    flops = 4.0 * wl.N * wl.b1 * wl.d * wl.B * wl.H
+    r = bench.kernel_roofline("tc_lstep_kernel", 1.0, wl, PEAKS, "measured")
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["achieved"] == pytest.approx(flops / 1e-3 / 1e12)
+    assert r["peak"] == 1400.0
+    assert r["frac"] == pytest.approx(r["achieved"] / 1400.0)
+    assert r["frac_of_burst"] == pytest.approx(r["achieved"] / 1600.0)
+
+
+def test_rstep_roofline_counts_every_tile():
+    wl = synth.WORKLOADS["720p"]
+    r = bench.kernel_roofline("tc_rstep_kernel", 2.0, wl, PEAKS, "measured")
+    flops = 6.0 * wl.tiles * wl.N * wl.b2 * wl.d * wl.B * wl.H
+    assert r["achieved"] == pytest.approx(flops / 2e-3 / 1e12)
+
+
+def test_query_aggregation_is_bandwidth_bound():
+    wl = synth.WORKLOADS["720p"]
+    r = bench.kernel_roofline("tc_qbar_kernel", 0.05, wl, PEAKS, "measured")
+    nbytes = wl.B * wl.H * wl.N * wl.d * 2
+    assert r["bound"] == "hbm"
+    assert r["achieved"] == pytest.approx(nbytes / 0.05e-3 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / 6000.0)
+
+
+def test_generic_kernels_report_against_the_alu_peak():
+    wl = synth.WORKLOADS["480p_chunk"]
+    r = bench.kernel_roofline("lstep_kernel", 1.0, wl, PEAKS, "measured")
+    assert r["bound"] == "alu"
+    assert r["peak"] == pytest.approx(148 * 128 * 2 * 1965.0e6 / 1e12)
+
+
+def _fake_tree(tmp_path, source_text, recorded_text):
+    csrc = tmp_path / "structured_attention_video_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_text(source_text)
+    (tmp_path / "profiles").mkdir()
+    rec = {"tc_lstep_kernel": {"source": "k.cu",
+                               "source_sha256": hashlib.sha256(recorded_text.encode()).hexdigest(),
+                               "dram_bytes_per_launch": 123.0}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+
+
+def test_traffic_is_reported_for_the_source_it_was_measured_on(tmp_path, monkeypatch):
+    _fake_tree(tmp_path, "kernel v1", "kernel v1")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.kernel_traffic("tc_lstep_kernel") == 123.0
+    assert bench.kernel_traffic("tc_rstep_kernel") is None
+
+
+def test_traffic_is_null_once_the_kernel_changed(tmp_path, monkeypatch):
+    _fake_tree(tmp_path, "kernel v2", "kernel v1")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.kernel_traffic("tc_lstep_kernel") is None
+
+
+def test_committed_traffic_record_names_existing_sources():
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as fh:
+        rec = json.load(fh)
+    for name, entry in rec.items():
+        assert os.path.exists(os.path.join(ROOT, "structured_attention_video_b200", "csrc",
+                                           entry["source"])), name
+        assert entry["dram_bytes_per_launch"] > 0
+
+
+def test_workload_config_names_the_shape_and_the_l2_policy():
+    wl = synth.WORKLOADS["720p"]
+    cfg = bench.workload_config(wl, 2)
+    assert cfg["N"] == 75600 and cfg["b1"] == 945 and cfg["b2"] == 80 and cfg["tiles"] == 4
+    assert "720p" in cfg["workload"] and "x2" in cfg["parallelism"]
+    assert "L2" in cfg["l2"]
