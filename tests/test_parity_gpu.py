@@ -90,6 +90,32 @@ def test_zero_queries_give_mean_of_v(tiny64):
     assert np.abs(got - v64.mean(-2, keepdims=True)).max() < 1e-5
 
 
+# tensor-core kernels at the edges of their dispatch range (bf16, d = 128, one
+# iteration), whole output against the oracle
+TC_EDGES = [
+    # f, h, w, b1, b2, tiles
+    (1, 64, 1, 64, 1, 2),        # b2 = 1: every R block is 1 x 1
+    (1, 1, 128, 1, 128, 1),      # b1 = 1: a single L block (exact attention); b2 padded to 128
+    (2, 3, 100, 6, 100, 2),      # b2 padded to 112, two 128-row qbar tiles
+    (3, 4, 16, 12, 16, 12),      # one query row per tile (t = b1)
+    (2, 100, 7, 200, 7, 3),      # b2 padded to 16; ragged last key chunk (200 = 128 + 72)
+    (5, 60, 48, 300, 48, 5),     # 60 rows per tile: the second query tile of a pair is empty
+    (10, 100, 16, 1000, 16, 1),  # 1000 query rows per tile: four pairs of query tiles
+]
+
+
+@pytest.mark.parametrize("f,h,w,b1,b2,tiles", TC_EDGES)
+def test_tensor_core_edge_shapes(f, h, w, b1, b2, tiles):
+    wl = TINY.replace(H=2, d=128, f=f, h=h, w=w, b1=b1, b2=b2, tiles=tiles, iters=1)
+    q64, k64, v64 = (synth.round_to_dtype(x, "bf16") for x in synth.make_inputs(wl))
+    q, k, v = (to_torch(x, "bf16") for x in (q64, k64, v64))
+    assert kernel_path(q, f=f, h=h, w=w, b1=b1, b2=b2, tiles=tiles) == 1
+    ref = oracle.monarch_attn(q64, k64, v64, b1, b2, tiles, 1)
+    got = from_torch(run(wl, q, k, v), "bf16")
+    assert np.isfinite(got).all()
+    assert rel_fro(got, ref) <= TOL["bf16"]
+
+
 def test_chunk_480p_whole_output():
     wl = synth.WORKLOADS["480p_chunk"]
     q, k, v = device_inputs(wl)
