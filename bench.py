@@ -411,6 +411,11 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and "OMP_NUM_THREADS" not in os.environ:
+        # each rank generates its own clip on the host with OpenMP: share the cores
+        # (set before torch loads the OpenMP runtime, which reads it once)
+        per_node = int(os.environ.get("LOCAL_WORLD_SIZE", str(world)))
+        os.environ["OMP_NUM_THREADS"] = str(max(1, len(os.sched_getaffinity(0)) // per_node))
     if args.gpus != world:
         ap.error("--gpus %d but WORLD_SIZE=%d: launch N > 1 with torchrun" % (args.gpus, world))
     wl = synth.WORKLOADS[args.workload]
