@@ -14,6 +14,8 @@ Prints ONE JSON line (rank 0).  `value` is dense-equivalent effective TFLOP/s
 (4*B*H*N^2*d per step over the device time, summed over ranks); `roofline`
 describes the dominant kernel, `path_roofline` the whole step against
 max(Monarch FLOPs / bf16 peak, Q/K/V/O bytes / HBM bandwidth).
+`also_480p` adds the device time of the 480p full clip (B=1 H=12 N=32760, blocks
+(630,52), 1 tile) at N=1, beside the line (not a bench line of its own).
 `--impl reference` times the float64 CPU oracle instead, on bounded samples.
 """
 from __future__ import annotations
@@ -272,6 +274,55 @@ def job_throughput(world: int, dense_flops_per_clip: float, ms_step: float) -> f
     return world * dense_flops_per_clip / (ms_step * 1e-3) / 1e12
 
 
+def secondary_workload(wl: synth.Workload, steps: int, warmup: int, flush, stream) -> dict:
+    """Device time of one more Wan-shaped clip (480p), reported beside the bench line.
+
+    Same timing rules as the main measurement (CUDA events on the launch stream,
+    L2 flushed between steps); runs on one GPU only and never fails the bench."""
+    import torch
+    from structured_attention_video_b200 import _lib
+    try:
+        dev = flush.device
+        shape = (wl.B, wl.H, wl.N, wl.d)
+        hq, hk, hv = (torch.empty(shape, dtype=torch.int16) for _ in range(3))
+        synth.fill_device_bits(wl, hq.numpy().view(np.uint16), hk.numpy().view(np.uint16),
+                               hv.numpy().view(np.uint16), 0)
+        q, k, v = (x.to(dev).view(torch.bfloat16) for x in (hq, hk, hv))
+        out = torch.empty_like(q)
+        sargs = (wl.B, wl.H, wl.f, wl.h, wl.w, wl.d, wl.b1, wl.b2, wl.tiles, wl.iters)
+        ws_bytes = _lib.monarch_attn_workspace_bytes(*sargs, _lib.BF16)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        sh = stream.cuda_stream
+
+        def step():
+            _lib.check(_lib.monarch_attn_fwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                out.data_ptr(), *sargs, _lib.BF16, ws.data_ptr(),
+                                                ws_bytes, sh), "monarch_attn_fwd_ws")
+
+        for _ in range(warmup):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
+        total = 0.0
+        for _ in range(steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            step()
+            b.record(stream)
+            torch.cuda.synchronize()
+            total += a.elapsed_time(b)
+        _lib.check(_lib.monarch_last_device_status(sh), "device status (secondary workload)")
+        ms = total / steps
+        return {"workload": workload_config(wl, 1)["workload"], "ms_per_step": ms,
+                "value": job_throughput(1, wl.dense_flops(), ms), "unit": UNIT,
+                "monarch_tflops": wl.monarch_flops() / (ms * 1e-3) / 1e12,
+                "kernel_path": "sm100 tensor-core" if _lib.monarch_attn_path(*sargs, _lib.BF16) == 1
+                else "generic SIMT", "steps": steps, "warmup": warmup}
+    except Exception as exc:   # reported, never fatal to the bench line
+        return {"workload": wl.name, "error": str(exc)}
+
+
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
@@ -384,6 +435,9 @@ def run_ours(args, wl: synth.Workload, world: int, rank: int, local: int):
         "clocks": clock_rec,
         "gpu": props.name,
     }
+    if world == 1 and args.secondary_steps > 0 and args.workload == "720p" and args.heads == 0:
+        line["also_480p"] = secondary_workload(synth.WORKLOADS["480p_full"], args.secondary_steps,
+                                               3, flush, stream)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
     else:
@@ -402,6 +456,8 @@ def main():
     ap.add_argument("--e2e-warmup", type=int, default=2)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--secondary-steps", type=int, default=50,
+                    help="timed steps of the 480p full clip reported beside the line (0: skip)")
     ap.add_argument("--heads", type=int, default=0,
                     help="override H (smaller cases for ncu captures; not a bench line)")
     args = ap.parse_args()
