@@ -111,9 +111,11 @@ MONARCH_API monarch_status monarch_attn_fwd(const void *q, const void *k, const 
  * scratch exceeds the array are rejected with MONARCH_ERR_SCRATCH_LIMIT before
  * anything is enqueued.  The 480p chunk shape (B=1, H=12, d=128, N=4680) fits.
  *
- * The first call on each device looks up the array's device address with
- * cudaGetSymbolAddress (with that device current); make that first call before
- * any stream capture.  Every call on a device shares the one array, which keeps
+ * The first call in each CUDA context (normally the primary context of each
+ * device) looks up the array's device address with cudaGetSymbolAddress, with
+ * that context current, and caches it under the context's id, so a context that
+ * was reset or replaced gets a fresh lookup; make that first call before any
+ * stream capture.  Every call on a device shares the one array, which keeps
  * the contents of the last call; nothing in it needs to start at zero.  Calls
  * that overlap on the GPU (different streams without ordering, or several host
  * threads) race on the array and give wrong results: serialise them.
@@ -195,6 +197,19 @@ MONARCH_API monarch_status monarch_last_device_status(monarch_stream_t stream);
  * the call, on every device.  Returns the previous limit.
  */
 MONARCH_API long long monarch_set_wait_limit(long long spins);
+
+/*
+ * Test hook: fault injection for the bounded waits.  While on (on != 0), the
+ * MMA-issuing warp of every tensor-core kernel launched afterwards first waits
+ * on a barrier that nothing ever completes.  The wait gives up after the wait
+ * limit, records MONARCH_ERR_TIMEOUT in the status word and the kernel takes
+ * its abort path: every other role stops waiting, the kernel waits for its own
+ * copies and tensor-core work in flight, frees its tensor memory and returns,
+ * leaving the output incomplete.  Nothing faults, traps or hangs.  Affects
+ * launches enqueued after the call, on every device.  Returns the previous
+ * setting.  (No counterpart in the pages: a test facility of this library.)
+ */
+MONARCH_API int monarch_debug_inject_stall(int on);
 
 /*
  * Benchmark hook: per-kernel timing.  While enabled (on != 0), every kernel

@@ -39,6 +39,7 @@ SIGNATURES = {
     "monarch_index_maps_device": ([_i] * 6 + [_vp, _vp, _vp, _vp, _vp], _i),
     "monarch_last_device_status": ([_vp], _i),
     "monarch_set_wait_limit": ([_ll], _ll),
+    "monarch_debug_inject_stall": ([_i], _i),
     "monarch_status_string": ([_i], ctypes.c_char_p),
     "monarch_attn_path": (_SHAPE + [_i], _i),
     "monarch_profile_enable": ([_i], _i),
@@ -109,6 +110,10 @@ def monarch_last_device_status(stream):
 
 def monarch_set_wait_limit(spins):
     return _lib.monarch_set_wait_limit(spins)
+
+
+def monarch_debug_inject_stall(on):
+    return _lib.monarch_debug_inject_stall(1 if on else 0)
 
 
 def monarch_status_string(status):

@@ -4,6 +4,8 @@
 #include "monarch_common.cuh"
 #include "monarch_sm100.cuh"
 
+#include <cuda.h>
+
 #include <atomic>
 #include <map>
 #include <math.h>
@@ -18,21 +20,28 @@ __device__ int g_device_status = 0;
 namespace {
 
 std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
+std::atomic<int> g_inject_stall{0};
 std::mutex g_dev_mutex;
 constexpr int kMaxDevices = 64;
-int *g_status_ptr[kMaxDevices] = {nullptr};
 bool g_pool_configured[kMaxDevices] = {false};
+SymbolAddressCache g_status_cache;
 
+// The status word of the current context (see SymbolAddressCache).
 int *status_word_on_current_device() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    std::lock_guard<std::mutex> lock(g_dev_mutex);
-    if (!g_status_ptr[dev]) {
-        void *ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_device_status) != cudaSuccess) return nullptr;
-        g_status_ptr[dev] = (int *)ptr;
-    }
-    return g_status_ptr[dev];
+    void *ptr = nullptr;
+    return g_status_cache.lookup(g_device_status, &ptr) == cudaSuccess ? (int *)ptr : nullptr;
+}
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+template <typename Fn> Fn driver_fn(const char *name) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<Fn>(ptr);
 }
 
 // Stream-ordered allocations of the entry points that allocate come from the
@@ -52,6 +61,24 @@ void configure_pool_once() {
 }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+
+bool current_context_id(unsigned long long *id) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+        get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    });
+    if (!get_current || !get_id) return false;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+namespace {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
@@ -105,7 +132,8 @@ monarch_status run_forward(const Problem &p, monarch_dtype dtype, const void *q,
     if (path == 1) {
         int *status = status_word_on_current_device();
         if (!status) return MONARCH_ERR_CUDA;
-        e = sm100_forward(p, q, k, v, out, ws, status, g_wait_limit.load(), stream);
+        e = sm100_forward(p, q, k, v, out, ws, status, g_wait_limit.load(),
+                          g_inject_stall.load(), stream);
     } else {
         e = generic_forward(p, dtype, q, k, v, out, generic_workspace_carve(p, ws), stream);
     }
@@ -303,6 +331,8 @@ monarch_status monarch_last_device_status(monarch_stream_t stream) {
 long long monarch_set_wait_limit(long long spins) {
     return g_wait_limit.exchange(spins > 0 ? spins : kDefaultWaitLimit);
 }
+
+int monarch_debug_inject_stall(int on) { return g_inject_stall.exchange(on != 0 ? 1 : 0); }
 
 monarch_status monarch_profile_enable(int on) {
     g_prof_on.store(on != 0);

@@ -6,6 +6,10 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <utility>
+#include <vector>
+
 #include "../../include/monarch_attn.h"
 
 namespace monarch {
@@ -68,6 +72,48 @@ class ProfileScope {
     KernelId id_;
     cudaStream_t stream_;
     void *start_ = nullptr;
+};
+
+// Device addresses of module-scope __device__ variables are valid only in the
+// CUDA context that loaded the module: a cache of such an address must be keyed
+// by the context, not by the device ordinal (a primary context that was reset,
+// or a context the caller created and made current, loads the module again at
+// another address).  current_context_id() gives the id of the context current
+// on the calling thread (CUDA never reuses an id within a process).
+bool current_context_id(unsigned long long *id);
+
+// The device address of one module-scope symbol, looked up with
+// cudaGetSymbolAddress once per context (with that context current) and cached
+// under the context id.  lookup() must run in the translation unit that
+// defines the symbol.  Nothing here allocates device memory.
+class SymbolAddressCache {
+  public:
+    template <typename T> cudaError_t lookup(const T &symbol, void **out) {
+        unsigned long long ctx = 0;
+        bool have_ctx = current_context_id(&ctx);
+        if (have_ctx) {
+            std::lock_guard<std::mutex> lock(mu_);
+            for (const auto &e : entries_)
+                if (e.first == ctx) {
+                    *out = e.second;
+                    return cudaSuccess;
+                }
+        }
+        void *ptr = nullptr;
+        cudaError_t err = cudaGetSymbolAddress(&ptr, symbol);   // creates the context if needed
+        if (err != cudaSuccess) return err;
+        if (!have_ctx) have_ctx = current_context_id(&ctx);
+        if (have_ctx) {
+            std::lock_guard<std::mutex> lock(mu_);
+            entries_.emplace_back(ctx, ptr);
+        }
+        *out = ptr;
+        return cudaSuccess;
+    }
+
+  private:
+    std::mutex mu_;
+    std::vector<std::pair<unsigned long long, void *>> entries_;
 };
 
 template <typename T> __device__ __forceinline__ float to_f32(T x);

@@ -3,8 +3,6 @@
 // static device array below; nothing here allocates.
 #include "monarch_common.cuh"
 
-#include <mutex>
-
 namespace monarch {
 namespace {
 
@@ -12,27 +10,13 @@ namespace {
 // every device that loads this module, kept until the process exits.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[MONARCH_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void *g_scratch_ptr[kMaxDevices] = {nullptr};
+SymbolAddressCache g_scratch_cache;
 
 // In host code g_noalloc_scratch names a host-side stand-in, not device
 // memory: the kernels must receive the device address, looked up once per
-// device (with that device current) and cached.
+// CUDA context (with that context current) and cached under its id.
 cudaError_t scratch_on_current_device(void **out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_ptr[dev]) {
-        void *ptr = nullptr;
-        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = ptr;
-    }
-    *out = g_scratch_ptr[dev];
-    return cudaSuccess;
+    return g_scratch_cache.lookup(g_noalloc_scratch, out);
 }
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }

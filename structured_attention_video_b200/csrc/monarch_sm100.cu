@@ -118,21 +118,32 @@ __global__ void __launch_bounds__(128) tc_qbar_kernel(const __nv_bfloat16 *__res
 
 // =====================================================================
 // S3: L-step with the output (persistent: each CTA walks a strided list of
-// (bh, g, v, query-pair) problems; the next problem's queries load while the
-// current one finishes, and its first S MMAs overlap the current epilogue)
+// (bh, g, v, query-pair) problems, two 128-query tiles per problem)
+//
+// 16 warps.  Warps 0-3 and 4-7: the softmax warpgroups of query tiles 0 and 1
+// (one query row per thread); warps 8-11: the epilogue warpgroup (O / l to
+// bfloat16 rows of Y, off the softmax warps' chain); warp 12: the TMA producer
+// of the queries, Ktil and the entropies; warp 13: the MMA issuer; warp 14:
+// the producer of Z; warp 15 idles.  setmaxnreg moves registers from the
+// producer and epilogue warpgroups to the softmax warpgroups.
+// Tensor memory: S_0 | S_1 | O_0 | O_1 (128 columns each); P_t overwrites the
+// first 64 columns of S_t as packed bfloat16 pairs.
 // =====================================================================
 namespace ls {
-// Ktil and Z stages in shared memory (a third Ktil stage measured slower: it
-// leaves the L1 cache almost no room)
-constexpr int kKStages = 2;
+constexpr int kThreads = 512;
+constexpr int kSoftmaxRegs = 184, kEpilogueRegs = 88, kProducerRegs = 56;
+static_assert(2 * kSoftmaxRegs + kEpilogueRegs + kProducerRegs == 4 * (65536 / kThreads),
+              "the warpgroups' registers must add up to the launch's 128 per thread");
+// one pair of every kPolyEvery takes its exponentials on the FMA pipe (0: none)
+constexpr int kPolyEvery = 4;
 constexpr uint32_t kQ = 0;                          // query tiles 0, 1
-constexpr uint32_t kK = 2 * kTile;                  // Ktil stages
-constexpr uint32_t kZ = kK + kKStages * kTile;      // Z stages 0, 1
+constexpr uint32_t kK = 2 * kTile;                  // Ktil stages 0, 1
+constexpr uint32_t kZ = kK + 2 * kTile;             // Z stages 0, 1
 constexpr uint32_t kH = kZ + 2 * kTile;             // entropies: 4 buffers of 128 floats
-constexpr uint32_t kBar = kH + 2048;
-constexpr uint32_t kSmem = kBar + 256;              // the base is 1024-aligned (checked)
+constexpr uint32_t kL = kH + 2048;                  // row sums [problem parity][tile][128]
+constexpr uint32_t kBar = kL + 2048;
+constexpr uint32_t kSmem = kBar + 512;              // the base is 1024-aligned (checked)
 static_assert(kSmem <= (uint32_t)kMaxSmem, "L-step shared memory");
-static_assert(kKStages >= 2 && kKStages <= 3, "the four entropy buffers cover at most three Ktil stages");
 }  // namespace ls
 
 struct LsArgs {
@@ -146,6 +157,7 @@ struct LsArgs {
     __nv_bfloat16 *out;
     int *status;
     long long limit;
+    int stall;      // test hook: the MMA warp first waits on a barrier nothing completes
 };
 
 struct LsProblem {
@@ -168,7 +180,7 @@ __device__ __forceinline__ LsProblem ls_problem(const LsArgs &a, int unit) {
     return q;
 }
 
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(ls::kThreads, 1)
 tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmZ, LsArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -182,17 +194,21 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + ls::kBar);
     uint64_t *q_full = bars + 0;     // [2 tiles]
     uint64_t *q_empty = bars + 2;    // [2 tiles]: the tile's last S MMA of a problem done
-    uint64_t *k_full = bars + 4;     // [3 stages]
-    uint64_t *k_empty = bars + 7;    // [3 stages]: both S MMAs of the chunk done
-    uint64_t *z_full = bars + 10;    // [2 stages]
-    uint64_t *z_empty = bars + 12;   // [2 stages]: both PV MMAs of the chunk done
-    uint64_t *h_full = bars + 14;    // [4 buffers]: bulk copy of the chunk's entropies
-    uint64_t *s_full = bars + 18;    // [2 tiles]
-    uint64_t *p_full = bars + 20;    // [2 tiles], one arrival per softmax warp
-    uint64_t *o_full = bars + 22;    // [2 tiles]
-    uint64_t *mma_done = bars + 24;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 25);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 26);
+    uint64_t *k_full = bars + 4;     // [2 stages]
+    uint64_t *k_empty = bars + 6;    // [2 stages]: both S MMAs of the chunk done
+    uint64_t *z_full = bars + 8;     // [2 stages]
+    uint64_t *z_empty = bars + 10;   // [2 stages]: both PV MMAs of the chunk done
+    uint64_t *h_full = bars + 12;    // [4 buffers]: bulk copy of the chunk's entropies
+    uint64_t *s_full = bars + 16;    // [2 tiles]
+    uint64_t *p_full = bars + 18;    // [2 tiles], one arrival per softmax warp
+    uint64_t *o_full = bars + 20;    // [2 tiles]: the last PV MMA of a problem done
+    uint64_t *o_free = bars + 22;    // [2 tiles], one arrival per epilogue warp: O_t read
+    uint64_t *l_full = bars + 24;    // [2 tiles], one arrival per softmax warp: row sums written
+    uint64_t *mma_done = bars + 26;
+    uint64_t *stall_bar = bars + 27;   // never completed (fault-injection hook)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 28);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 29);
+    float *lsum = reinterpret_cast<float *>(sm + ls::kL);   // [2][2][128]
 
     const Problem &p = a.p;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -204,199 +220,218 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int t = 0; t < 2; t++) {
             mbar_init(q_full + t, 1);
             mbar_init(q_empty + t, 1);
-        }
-        for (int s = 0; s < ls::kKStages; s++) {
-            mbar_init(k_full + s, 1);
-            mbar_init(k_empty + s, 1);
-        }
-        for (int s = 0; s < 2; s++) {
-            mbar_init(z_full + s, 1);
-            mbar_init(z_empty + s, 1);
-            mbar_init(s_full + s, 1);
-            mbar_init(p_full + s, 4);   // one arrival per softmax warp
-            mbar_init(o_full + s, 1);
+            mbar_init(k_full + t, 1);
+            mbar_init(k_empty + t, 1);
+            mbar_init(z_full + t, 1);
+            mbar_init(z_empty + t, 1);
+            mbar_init(s_full + t, 1);
+            mbar_init(p_full + t, 4);   // one arrival per softmax warp
+            mbar_init(o_full + t, 1);
+            mbar_init(o_free + t, 4);   // one arrival per epilogue warp
+            mbar_init(l_full + t, 4);   // one arrival per softmax warp
         }
         for (int s = 0; s < 4; s++) mbar_init(h_full + s, 1);
         mbar_init(mma_done, 1);
+        mbar_init(stall_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 1) tmem_alloc(tmem_slot, 512);
+    if (warp == 13) tmem_alloc(tmem_slot, 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const WaitCtx w{a.limit, a.status, abort_flag};
 
-    if (warp == 0) {
-        // ---------------- producer: queries per problem; per chunk Ktil and H as
-        // soon as the S MMAs of two chunks back are done, Z once their PV MMAs are.
-        // H has four buffers: S1 of chunk jc - kKStages (whose completion frees
-        // the Ktil stage of chunk jc) is issued only after both softmax
-        // warpgroups have finished chunk jc - kKStages - 1, so buffer jc & 3
-        // (last read for chunk jc - 4) is free for kKStages <= 3.
-        int issued[ls::kKStages] = {}, qloads = 0, issued_h = 0;
-        bool ok = true;
-        for (int pi = 0; ok && pi < nmine; pi++) {
-            const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
-            // each query tile reloads as soon as its own last S MMA of the
-            // previous problem is done (tile 0 one PV + S earlier than tile 1)
-            for (int t = 0; ok && t < 2; t++) {
-                if (pi > 0 && !wait_warp(q_empty + t, (pi - 1) & 1, w)) {
-                    ok = false;
-                    break;
+    if (warp >= 12) {
+        regs_dec<ls::kProducerRegs>();
+        if (warp == 12) {
+            // ---------------- producer: queries per problem; per chunk Ktil and H as
+            // soon as the S MMAs of two chunks back are done.  H has four buffers:
+            // S_1 of chunk jc - 2 (whose completion frees the Ktil stage of chunk jc)
+            // is issued only after both softmax warpgroups finished chunk jc - 3,
+            // so buffer jc & 3 (last read for chunk jc - 4) is free.
+            int issued[2] = {0, 0}, qloads = 0, issued_h = 0;
+            bool ok = true;
+            for (int pi = 0; ok && pi < nmine; pi++) {
+                const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
+                // each query tile reloads as soon as its own last S MMA of the
+                // previous problem is done
+                for (int t = 0; ok && t < 2; t++) {
+                    if (pi > 0 && !wait_warp(q_empty + t, (pi - 1) & 1, w)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        mbar_expect_tx(q_full + t, kTile);
+                        for (int pn = 0; pn < 2; pn++)
+                            tma_load_3d(sm + ls::kQ + t * kTile + pn * kPanel, &tmQ, pn * 64, pr.v,
+                                        pr.bh * p.b1 + pr.u_start + t * 128, q_full + t);
+                    }
                 }
-                if (lane == 0) {
-                    mbar_expect_tx(q_full + t, kTile);
-                    for (int pn = 0; pn < 2; pn++)
-                        tma_load_3d(sm + ls::kQ + t * kTile + pn * kPanel, &tmQ, pn * 64, pr.v,
-                                    pr.bh * p.b1 + pr.u_start + t * 128, q_full + t);
+                if (!ok) break;
+                qloads++;
+                for (int j = 0; j < nch; j++) {
+                    const int jc = pi * nch + j, sk = jc & 1;
+                    if (jc >= 2 && !wait_warp(k_empty + sk, ((jc >> 1) - 1) & 1, w)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        mbar_expect_tx(k_full + sk, kTile);
+                        for (int pn = 0; pn < 2; pn++)
+                            tma_load_2d(sm + ls::kK + sk * kTile + pn * kPanel, &tmK, pn * 64,
+                                        pr.key_row0 + j * 128, k_full + sk);
+                        // the chunk's entropies (log2 units; keys past b1 are masked later)
+                        mbar_expect_tx(h_full + (jc & 3), 512);
+                        bulk_load(sm + ls::kH + (jc & 3) * 512, a.hent + pr.h_row0 + j * 128, 512,
+                                  h_full + (jc & 3));
+                    }
+                    issued[sk]++;
+                    issued_h++;
                 }
             }
-            if (!ok) break;
-            qloads++;
-            for (int j = 0; j < nch; j++) {
-                const int jc = pi * nch + j, sk = jc % ls::kKStages;
-                if (jc >= ls::kKStages &&
-                    !wait_warp(k_empty + sk, ((jc / ls::kKStages) - 1) & 1, w)) {
-                    ok = false;
-                    break;
+            if (lane == 0) {   // every issued copy lands before the CTA may exit
+                for (int t = 0; t < 2; t++)
+                    if (qloads > 0) wait_phase_cleanup(q_full + t, (qloads - 1) & 1, kCleanupPolls);
+                for (int s = 0; s < 2; s++)
+                    if (issued[s] > 0) wait_phase_cleanup(k_full + s, (issued[s] - 1) & 1, kCleanupPolls);
+                for (int hb = 0; hb < 4; hb++) {   // the last copy into each entropy buffer
+                    if (issued_h <= hb) continue;
+                    const int last = hb + ((issued_h - 1 - hb) / 4) * 4;
+                    wait_phase_cleanup(h_full + hb, (last >> 2) & 1, kCleanupPolls);
                 }
-                if (lane == 0) {
-                    mbar_expect_tx(k_full + sk, kTile);
-                    for (int pn = 0; pn < 2; pn++)
-                        tma_load_2d(sm + ls::kK + sk * kTile + pn * kPanel, &tmK, pn * 64,
-                                    pr.key_row0 + j * 128, k_full + sk);
-                }
-                issued[sk]++;
-                if (lane == 0) {   // the chunk's entropies (log2 units; keys past b1 are masked later)
-                    mbar_expect_tx(h_full + (jc & 3), 512);
-                    bulk_load(sm + ls::kH + (jc & 3) * 512, a.hent + pr.h_row0 + j * 128, 512,
-                              h_full + (jc & 3));
-                }
-                issued_h++;
             }
-        }
-        if (lane == 0) {   // every issued copy lands before the CTA may exit
-            for (int t = 0; t < 2; t++)
-                if (qloads > 0) wait_phase_cleanup(q_full + t, (qloads - 1) & 1, kCleanupPolls);
-            for (int s = 0; s < ls::kKStages; s++)
-                if (issued[s] > 0) wait_phase_cleanup(k_full + s, (issued[s] - 1) & 1, kCleanupPolls);
-            for (int hb = 0; hb < 4; hb++) {   // the last copy into each entropy buffer
-                if (issued_h <= hb) continue;
-                const int last = hb + ((issued_h - 1 - hb) / 4) * 4;
-                wait_phase_cleanup(h_full + hb, (last >> 2) & 1, kCleanupPolls);
-            }
-        }
-    } else if (warp == 2) {
-        // ---------------- Z producer: its own warp, so that a Ktil load never
-        // queues behind the wait for a Z stage (released one PV later than Ktil)
-        int issued_z[2] = {0, 0};
-        bool ok = true;
-        for (int pi = 0; ok && pi < nmine; pi++) {
-            const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
-            for (int j = 0; j < nch; j++) {
-                const int jc = pi * nch + j, st = jc & 1;
-                if (jc >= 2 && !wait_warp(z_empty + st, ((jc >> 1) - 1) & 1, w)) {
-                    ok = false;
-                    break;
+        } else if (warp == 14) {
+            // ---------------- Z producer: its own warp, so that a Ktil load never
+            // queues behind the wait for a Z stage (released one PV later than Ktil)
+            int issued_z[2] = {0, 0};
+            bool ok = true;
+            for (int pi = 0; ok && pi < nmine; pi++) {
+                const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
+                for (int j = 0; j < nch; j++) {
+                    const int jc = pi * nch + j, st = jc & 1;
+                    if (jc >= 2 && !wait_warp(z_empty + st, ((jc >> 1) - 1) & 1, w)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        mbar_expect_tx(z_full + st, kTile);
+                        for (int pn = 0; pn < 2; pn++)
+                            tma_load_2d(sm + ls::kZ + st * kTile + pn * kPanel, &tmZ, pn * 64,
+                                        pr.key_row0 + j * 128, z_full + st);
+                    }
+                    issued_z[st]++;
                 }
-                if (lane == 0) {
-                    mbar_expect_tx(z_full + st, kTile);
-                    for (int pn = 0; pn < 2; pn++)
-                        tma_load_2d(sm + ls::kZ + st * kTile + pn * kPanel, &tmZ, pn * 64,
-                                    pr.key_row0 + j * 128, z_full + st);
-                }
-                issued_z[st]++;
             }
-        }
-        if (lane == 0)
-            for (int s = 0; s < 2; s++)
-                if (issued_z[s] > 0)
-                    wait_phase_cleanup(z_full + s, (issued_z[s] - 1) & 1, kCleanupPolls);
-    } else if (warp == 1) {
-        // ---------------- MMA issuer.  Per chunk: PV0, then S0 of the next chunk,
-        // PV1, S1 of the next chunk, so that a tile's chain never waits on the
-        // other tile's softmax.  The whole warp runs this loop; every group of
-        // eight MMAs goes out from one elect.sync region with descriptors
-        // computed once here (mma_group_ss), and the chunk loop is unrolled by
-        // the stage parity so that they stay in registers.
-        static_assert(ls::kKStages == 2, "the MMA loop unrolls over two stages");
-        {
+            if (lane == 0)
+                for (int s = 0; s < 2; s++)
+                    if (issued_z[s] > 0)
+                        wait_phase_cleanup(z_full + s, (issued_z[s] - 1) & 1, kCleanupPolls);
+        } else if (warp == 13) {
+            // ---------------- MMA issuer.  Order: S_0 and S_1 of the first chunk, then
+            // per chunk PV_0, S_0 of the next chunk, PV_1, S_1 of the next chunk, so
+            // that a tile's chain never waits on the other tile's softmax.  S_t of
+            // the next chunk overwrites the columns that PV_t reads as P: tcgen05
+            // MMAs issued by one thread execute in issue order, so it follows PV_t
+            // without a wait, and its commit (s_full) also covers PV_t, which orders
+            // the softmax's rescale of O_t after PV_t.
             constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t idO = idesc_bf16(128, 128, 0, 1);
             const uint64_t dQ = smem_desc_sw128(smem_u32(sm + ls::kQ), 16, 1024);
             const uint64_t dK = smem_desc_sw128(smem_u32(sm + ls::kK), 16, 1024);
             const uint64_t dZ = smem_desc_sw128(smem_u32(sm + ls::kZ), kPanel, 1024);
-            uint64_t aq0[8], aq1[8], bk0[8], bk1[8], bz0[8], bz1[8];
-#pragma unroll
-            for (int kk = 0; kk < 8; kk++) {
-                const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-                aq0[kk] = desc_plus(dQ, off);
-                aq1[kk] = desc_plus(dQ, kTile + off);
-                bk0[kk] = desc_plus(dK, off);
-                bk1[kk] = desc_plus(dK, kTile + off);
-                bz0[kk] = desc_plus(dZ, kk * 2048);
-                bz1[kk] = desc_plus(dZ, kTile + kk * 2048);
-            }
+            constexpr uint32_t kTileDesc = kTile >> 4;
             const int total = nmine * nch;
-            bool ok = true;
-            // S_t for global chunk index jc (waits for the chunk's Ktil and, if the
-            // chunk opens a problem, for its queries)
-            auto issue_s = [&](int t, int jc, const uint64_t(&aq)[8], const uint64_t(&bk)[8]) -> bool {
+            // fault injection: a wait that can only give up (bounded, then abort)
+            bool ok = !a.stall || spin_warp(stall_bar, 0, w);
+            auto issue_s = [&](int t, int jc) -> bool {
                 const int sk = jc & 1;
                 if (jc % nch == 0 && !spin_warp(q_full + t, (jc / nch) & 1, w)) return false;
                 if (t == 0 && !spin_warp(k_full + sk, (jc >> 1) & 1, w)) return false;
                 tc_fence_after();
-                mma_group_ss(tmem + t * 128, aq, bk, idS, 0u, 8u);
+                mma8_ss_k128(tmem + t * 128, dQ + t * kTileDesc, dK + sk * kTileDesc, idS, 0u);
                 mma_commit_warp(s_full + t);
                 if (t == 1) mma_commit_warp(k_empty + sk);
                 if (jc % nch == nch - 1) mma_commit_warp(q_empty + t);   // tile t no longer read
                 return true;
             };
-            auto issue_pv = [&](int t, int jc, const uint64_t(&bz)[8]) -> bool {
-                const int st = jc & 1;
+            auto issue_pv = [&](int t, int jc) -> bool {
+                const int st = jc & 1, j = jc % nch;
                 if (t == 0 && !spin_warp(z_full + st, (jc >> 1) & 1, w)) return false;
                 if (!spin_warp(p_full + t, jc & 1, w)) return false;
+                // the first PV of a problem overwrites O_t: the epilogue of the
+                // previous problem must have read it
+                if (j == 0 && jc >= nch && !spin_warp(o_free + t, ((jc / nch) - 1) & 1, w))
+                    return false;
                 tc_fence_after();
-                mma_group_ts(tmem + 256 + t * 128, tmem + t * 128, bz, idO,
-                             (jc % nch) > 0 ? 1u : 0u, 8u);
-                mma_commit_warp(o_full + t);
+                mma8_ts_mn128(tmem + 256 + t * 128, tmem + t * 128, dZ + st * kTileDesc, idO,
+                              j > 0 ? 1u : 0u);
                 if (t == 1) mma_commit_warp(z_empty + st);
+                if (j == nch - 1) mma_commit_warp(o_full + t);
                 return true;
             };
-            // one chunk: PV_t of chunk jc (Z stage jc & 1), then S_t of chunk jc + 1
-            // (Ktil stage (jc + 1) & 1)
-            auto chunk = [&](int jc, const uint64_t(&bz)[8], const uint64_t(&bkn)[8]) -> bool {
+            if (ok && total > 0) ok = issue_s(0, 0) && issue_s(1, 0);
+            for (int jc = 0; ok && jc < total; jc++) {
                 const bool more = jc + 1 < total;
-                if (!issue_pv(0, jc, bz)) return false;
-                if (more && !issue_s(0, jc + 1, aq0, bkn)) return false;
-                if (!issue_pv(1, jc, bz)) return false;
-                if (more && !issue_s(1, jc + 1, aq1, bkn)) return false;
-                return true;
-            };
-            // S_t of the next chunk overwrites the columns that PV_t reads as P:
-            // tcgen05 MMAs issued by one thread execute in issue order, so it is
-            // issued right behind PV_t without waiting; its commit (s_full) also
-            // covers PV_t, which orders the softmax's rescale of O_t after PV_t.
-            if (total > 0) ok = issue_s(0, 0, aq0, bk0) && issue_s(1, 0, aq1, bk0);
-            for (int jc = 0; ok && jc < total; jc += 2) {
-                ok = chunk(jc, bz0, bk1);
-                if (ok && jc + 1 < total) ok = chunk(jc + 1, bz1, bk0);
+                ok = issue_pv(0, jc) && (!more || issue_s(0, jc + 1)) && issue_pv(1, jc) &&
+                     (!more || issue_s(1, jc + 1));
             }
             mma_commit_warp(mma_done);
             wait_phase_cleanup(mma_done, 0, kCleanupPolls);
         }
-    } else if (warp >= 4) {
-        // ---------------- softmax warpgroups: tile t = 0 (warps 4-7), 1 (warps 8-11)
-        const int t = (warp - 4) >> 2;
+    } else if (warp >= 8) {
+        // ---------------- epilogue warpgroup: per problem and tile, O_t / l to
+        // bfloat16; each thread writes its own output row as sixteen 16-byte stores
+        regs_dec<ls::kEpilogueRegs>();
+        const int wq = warp & 3;
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        bool ok = true;
+        for (int pi = 0; ok && pi < nmine; pi++) {
+            const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
+            for (int t = 0; t < 2; t++) {
+                if (!wait_warp(o_full + t, pi & 1, w) || !wait_warp(l_full + t, pi & 1, w)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float inv_l = 1.f / lsum[((pi & 1) * 2 + t) * 128 + wq * 32 + lane];
+                const int u = pr.u_start + t * 128 + wq * 32 + lane;
+                uint4 *dst = reinterpret_cast<uint4 *>(
+                    a.out + ((int64_t)pr.bh * p.N + (int64_t)u * p.b2 + pr.v) * kD);
+#pragma unroll
+                for (int c = 0; c < 4; c++) {   // 32 columns at a time
+                    float o[32];
+                    tmem_ld32f(tmem + lane_off + 256 + t * 128 + c * 32, o);
+                    tmem_wait_ld();
+                    if (c == 3) {   // all of O_t is in registers: the next PV may start
+                        tc_fence_before();
+                        mbar_arrive_warp(o_free + t);
+                    }
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int k = 0; k < 16; k++)
+                        pk[k] = pack_bf16(o[2 * k] * inv_l, o[2 * k + 1] * inv_l);
+                    if (u < pr.u1) {
+#pragma unroll
+                        for (int ch = 0; ch < 4; ch++)
+                            dst[c * 4 + ch] = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2],
+                                                         pk[4 * ch + 3]);
+                    }
+                }
+            }
+        }
+    } else {
+        // ---------------- softmax warpgroups: tile t = 0 (warps 0-3), 1 (warps 4-7)
+        regs_inc<ls::kSoftmaxRegs>();
+        const int t = warp >> 2;
         const int wq = warp & 3;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
         const uint32_t tS = tmem + lane_off + t * 128;
         const uint32_t tO = tmem + lane_off + 256 + t * 128;
+        const uint64_t c2 = f2_pack(a.c_log2, a.c_log2);
         bool ok = true;
         for (int pi = 0; ok && pi < nmine; pi++) {
-            const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
             float m_run = -INFINITY, l_run = 0.f;
             for (int j = 0; j < nch; j++) {
                 const int jc = pi * nch + j;
@@ -410,13 +445,14 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
                 for (int c = 0; c < 4; c++) tmem_ld32f(tS + c * 32, &x[c * 32]);
                 tmem_wait_ld();
-                // x = s * c_log2 + H / ln2 (the entropy arrives in log2 units)
+                // logits in log2 units: x * s * log2(e) + H / ln 2 (the entropy
+                // arrives in log2 units)
                 const uint64_t *hs = reinterpret_cast<const uint64_t *>(sm + ls::kH + (jc & 3) * 512);
-                const uint64_t c2 = f2_pack(a.c_log2, a.c_log2);
                 uint64_t xp[64];
                 float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
                 const int nvalid = p.b1 - j * 128;   // keys of this chunk inside the row
-                if (nvalid >= 128) {
+                const bool full = nvalid >= 128;
+                if (full) {
 #pragma unroll
                     for (int i = 0; i < 64; i++) {
                         xp[i] = f2_fma(f2_pack(x[2 * i], x[2 * i + 1]), c2, hs[i]);
@@ -454,10 +490,18 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     uint32_t pk[32];
 #pragma unroll
                     for (int i = 0; i < 32; i++) {
-                        float lo, hi;
-                        f2_unpack(f2_add(xp[h * 32 + i], nm2), lo, hi);
-                        const float p0 = fast_exp2(lo), p1 = fast_exp2(hi);
-                        sum2[i & 3] = f2_add(sum2[i & 3], f2_pack(p0, p1));
+                        const uint64_t d2 = f2_add(xp[h * 32 + i], nm2);
+                        uint64_t e2;
+                        if (ls::kPolyEvery > 0 && (i % ls::kPolyEvery) == ls::kPolyEvery - 1 && full) {
+                            e2 = exp2_poly_x2(d2);
+                        } else {
+                            float lo, hi;
+                            f2_unpack(d2, lo, hi);
+                            e2 = f2_pack(fast_exp2(lo), fast_exp2(hi));
+                        }
+                        sum2[i & 3] = f2_add(sum2[i & 3], e2);
+                        float p0, p1;
+                        f2_unpack(e2, p0, p1);
                         pk[i] = pack_bf16(p0, p1);
                     }
                     tmem_st32(tS + h * 32, pk);
@@ -466,51 +510,33 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), s0, s1);
                 l_run = l_run * alpha + (s0 + s1);
                 if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-                    float o[128];
+                    // O_t is complete up to the previous chunk (the commit of this
+                    // chunk's S covers the previous PV); scale it in four slices
 #pragma unroll
-                    for (int c = 0; c < 4; c++) tmem_ld32f(tO + c * 32, &o[c * 32]);
-                    tmem_wait_ld();
+                    for (int c = 0; c < 4; c++) {
+                        float o[32];
+                        tmem_ld32f(tO + c * 32, o);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 128; i++) o[i] *= alpha;
-#pragma unroll
-                    for (int c = 0; c < 4; c++) tmem_st32f(tO + c * 32, &o[c * 32]);
+                        for (int i = 0; i < 32; i++) o[i] *= alpha;
+                        tmem_st32f(tO + c * 32, o);
+                    }
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive_warp(p_full + t);
             }
-            if (!ok || !wait_warp(o_full + t, (pi * nch + nch - 1) & 1, w)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            // epilogue: each thread writes its own output row, O / l in bf16,
-            // as sixteen 16-byte stores (the L2 merges the row's sectors)
-            float o[128];
-#pragma unroll
-            for (int c = 0; c < 4; c++) tmem_ld32f(tO + c * 32, &o[c * 32]);
-            tmem_wait_ld();
-            const float inv_l = 1.f / l_run;
-            const int u = pr.u_start + t * 128 + wq * 32 + lane;
-            if (u < pr.u1) {
-                uint4 *dst = reinterpret_cast<uint4 *>(
-                    a.out + ((int64_t)pr.bh * p.N + (int64_t)u * p.b2 + pr.v) * kD);
-#pragma unroll
-                for (int ch = 0; ch < 16; ch++) {
-                    const float *src = &o[ch * 8];
-                    uint4 val;
-                    val.x = pack_bf16(src[0] * inv_l, src[1] * inv_l);
-                    val.y = pack_bf16(src[2] * inv_l, src[3] * inv_l);
-                    val.z = pack_bf16(src[4] * inv_l, src[5] * inv_l);
-                    val.w = pack_bf16(src[6] * inv_l, src[7] * inv_l);
-                    dst[ch] = val;
-                }
-            }
+            if (!ok) break;
+            // the row sums for the epilogue; slot pi & 1 is rewritten two problems
+            // later, when the epilogue has released O_t (o_free) of this problem,
+            // which the first PV of the problem after next waits for
+            lsum[((pi & 1) * 2 + t) * 128 + wq * 32 + lane] = l_run;
+            mbar_arrive_warp(l_full + t);
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == 13) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -529,6 +555,7 @@ struct RsArgs {
     float *hent;
     int *status;
     long long limit;
+    int stall;           // test hook: the MMA warp first waits on a barrier nothing completes
 };
 
 template <int B2P>
@@ -564,6 +591,7 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
     uint64_t *mma_done = bars + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 17);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 18);
+    uint64_t *stall_bar = bars + 19;   // never completed (fault-injection hook)
 
     const Problem &p = a.p;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -586,6 +614,7 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
             mbar_init(o_empty + s, 4);   // one arrival per epilogue warp
         }
         mbar_init(mma_done, 1);
+        mbar_init(stall_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -640,7 +669,8 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
             const uint64_t dK = smem_desc_sw128(smem_u32(sm + L::kv(nmt)), 16, 1024);
             const uint64_t dV = smem_desc_sw128(smem_u32(sm + L::kv(nmt)), L::kPanelKV, 1024);
             int heads = 0;
-            bool ok = true;
+            // fault injection: a wait that can only give up (bounded, then abort)
+            bool ok = !a.stall || spin_warp(stall_bar, 0, w);
             // S = qbar_mt K_u'^T for item i into S buffer i & 1
             auto gemm1 = [&](int i) -> bool {
                 const int ib = i / nmt, mt = i % nmt;
@@ -666,7 +696,7 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 if (mt == nmt - 1 && head_ends) mma_commit_warp(q_empty);
                 return true;
             };
-            if (nitems > 0) ok = gemm1(0);
+            if (ok && nitems > 0) ok = gemm1(0);
             for (int i = 0; ok && i < nitems; i++) {
                 if (i + 1 < nitems && !gemm1(i + 1)) break;
                 const int ib = i / nmt, mt = i % nmt;
@@ -918,7 +948,7 @@ size_t sm100_workspace_bytes(const Problem &p, bool &overflow) {
 
 cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const void *v,
                           void *out, void *workspace, int *status, long long wait_limit,
-                          cudaStream_t stream) {
+                          int stall, cudaStream_t stream) {
     const TcWorkspace ws = carve(p, workspace);
     const int nmt = qbar_tiles(p), mpad = nmt * 128, b2p = b2_padded(p.b2);
     const float c_log2 = p.scale * kLog2e;
@@ -953,7 +983,7 @@ cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const 
         const int sms = sm_count();
         const int bpc = (total + sms - 1) / sms;
         const int grid = (total + bpc - 1) / bpc;
-        RsArgs a{p, nmt, mpad, bpc, h_stride(p), c_log2, ws.hent, status, wait_limit};
+        RsArgs a{p, nmt, mpad, bpc, h_stride(p), c_log2, ws.hent, status, wait_limit, stall};
         ProfileScope scope(K_TC_RSTEP, stream);
         cudaError_t e = cudaErrorInvalidValue;
         switch (b2p) {
@@ -985,12 +1015,12 @@ cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const 
         const int nprob = p.BH * p.tiles * p.b2 * npairs;
         LsArgs a{p, (p.b1 + 127) / 128, npairs, nprob, h_stride(p), c_log2, ws.hent,
                  (__nv_bfloat16 *)out,
-                 status, wait_limit};
+                 status, wait_limit, stall};
         cudaError_t e = set_smem(tc_lstep_kernel, ls::kSmem);
         if (e != cudaSuccess) return e;
         const int grid = nprob < sm_count() ? nprob : sm_count();
         ProfileScope scope(K_TC_LSTEP, stream);
-        tc_lstep_kernel<<<grid, 384, ls::kSmem, stream>>>(maps[0], maps[1], maps[2], a);
+        tc_lstep_kernel<<<grid, ls::kThreads, ls::kSmem, stream>>>(maps[0], maps[1], maps[2], a);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

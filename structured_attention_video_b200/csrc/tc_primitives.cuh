@@ -287,6 +287,76 @@ __device__ __forceinline__ void mma_group_ts(uint32_t d_tmem, uint32_t a_tmem,
         : "memory");
 }
 
+// Eight K-steps (K = 128) of D (+)= A B^T with both operands 128-deep, K-major,
+// 128-byte swizzled tiles of two 64-column panels (16 KB apart): K-step k starts
+// (k & 3) * 32 bytes into panel k >> 2, i.e. the base descriptors plus
+// (k >> 2) * 1024 + (k & 3) * 2 in 16-byte units.  The warp stays convergent;
+// elect.sync picks the issuing lane, and the seven offset descriptors are formed
+// inside the asm block, so the issuing warp needs no registers for them.
+__device__ __forceinline__ void mma8_ss_k128(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                             uint32_t idesc, uint32_t acc0) {
+    asm volatile(
+        "{\n\t.reg .pred e, p0;\n\t"
+        ".reg .b64 a1, a2, a3, a4, a5, a6, a7, b1, b2, b3, b4, b5, b6, b7;\n\t"
+        "add.s64 a1, %1, 2;\n\tadd.s64 a2, %1, 4;\n\tadd.s64 a3, %1, 6;\n\t"
+        "add.s64 a4, %1, 1024;\n\tadd.s64 a5, %1, 1026;\n\tadd.s64 a6, %1, 1028;\n\t"
+        "add.s64 a7, %1, 1030;\n\t"
+        "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
+        "add.s64 b4, %2, 1024;\n\tadd.s64 b5, %2, 1026;\n\tadd.s64 b6, %2, 1028;\n\t"
+        "add.s64 b7, %2, 1030;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.and.b32 p0, %4, 0, e;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a4, b4, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a5, b5, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a6, b6, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a7, b7, %3, 1;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc0)
+        : "memory");
+}
+// Eight K-steps (K = 128) of D (+)= A B with A in tensor memory (bfloat16 pairs,
+// K-step k at columns a_tmem + 8k) and B an MN-major 128-byte swizzled tile
+// whose K-step k starts 16 rows = 2048 bytes further (descriptor + 128k).
+__device__ __forceinline__ void mma8_ts_mn128(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                              uint32_t idesc, uint32_t acc0) {
+    asm volatile(
+        "{\n\t.reg .pred e, p0;\n\t"
+        ".reg .b32 a1, a2, a3, a4, a5, a6, a7;\n\t"
+        ".reg .b64 b1, b2, b3, b4, b5, b6, b7;\n\t"
+        "add.u32 a1, %1, 8;\n\tadd.u32 a2, %1, 16;\n\tadd.u32 a3, %1, 24;\n\t"
+        "add.u32 a4, %1, 32;\n\tadd.u32 a5, %1, 40;\n\tadd.u32 a6, %1, 48;\n\t"
+        "add.u32 a7, %1, 56;\n\t"
+        "add.s64 b1, %2, 128;\n\tadd.s64 b2, %2, 256;\n\tadd.s64 b3, %2, 384;\n\t"
+        "add.s64 b4, %2, 512;\n\tadd.s64 b5, %2, 640;\n\tadd.s64 b6, %2, 768;\n\t"
+        "add.s64 b7, %2, 896;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.and.b32 p0, %4, 0, e;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a4], b4, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a5], b5, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a6], b6, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a7], b7, %3, 1;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc0)
+        : "memory");
+}
+
+// Warpgroup register reallocation (all four warps of a warpgroup execute the
+// same call): dec returns registers to the CTA's pool, inc waits until the pool
+// can give the warp N registers per thread.  The pool is what the block was
+// launched with, so the warpgroups' final counts must sum to at most that.
+template <int N> __device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N> __device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Warp-collective loads/stores of 32 lanes x N consecutive 32-bit columns:
 // lane i of the warp reads/writes TMEM lane (32*(warp%4) + i).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -463,6 +533,42 @@ __device__ __forceinline__ bool spin_warp(uint64_t *bar, uint32_t parity, const 
 }
 
 // ---------------------------------------------------------------- math
+// 2^d for a packed pair of float32 values d <= 0 (finite), on the FMA and
+// integer pipes instead of the MUFU.  Range reduction after Cody and Waite:
+// d = j + f with j = floor(d) (the round-down addition of 1.5 * 2^23 leaves j in
+// the low mantissa bits) and f in [0, 1); 2^f is the degree-3 polynomial that
+// minimises the maximum relative error on [0, 1) (Remez exchange; 7.5e-5 in
+// float32), and 2^j enters by adding j << 23 to the polynomial's bit pattern.
+// j is clamped to -126: the polynomial lies in [0.99992, 2), so the exponent
+// field of the result never goes below zero, and results below 2^-126 come out
+// as values of at most 2^-125 (zero after the bfloat16 rounding of P would be
+// no more accurate: such terms vanish next to the row maximum's 2^0).
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t d) {
+    const uint64_t magic = f2_pack(12582912.f, 12582912.f);
+    const uint64_t neg_magic = f2_pack(-12582912.f, -12582912.f);
+    const uint64_t neg_one = f2_pack(-1.f, -1.f);
+    uint64_t t, jf, f, p;
+    asm("add.rm.f32x2 %0, %1, %2;" : "=l"(t) : "l"(d), "l"(magic));   // magic + floor(d)
+    jf = f2_add(t, neg_magic);                                        // floor(d), exact
+    f = f2_fma(jf, neg_one, d);                                       // d - floor(d)
+    p = f2_fma(f, f2_pack(0.07802452147006989f, 0.07802452147006989f),
+               f2_pack(0.22606715559959412f, 0.22606715559959412f));
+    p = f2_fma(p, f, f2_pack(0.6958335638046265f, 0.6958335638046265f));
+    p = f2_fma(p, f, f2_pack(0.9999251961708069f, 0.9999251961708069f));
+    uint32_t tlo, thi, plo, phi;
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(tlo), "=r"(thi) : "l"(t));
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(plo), "=r"(phi) : "l"(p));
+    const int lo_min = 0x4B400000 - 126;
+    tlo = (uint32_t)max((int)tlo, lo_min);
+    thi = (uint32_t)max((int)thi, lo_min);
+    // (magic + j) << 23 == j << 23 (mod 2^32): the magic's set bits shift out
+    plo = tlo * 8388608u + plo;
+    phi = thi * 8388608u + phi;
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(plo), "r"(phi));
+    return r;
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

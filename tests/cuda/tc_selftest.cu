@@ -114,6 +114,21 @@ __global__ void wait_kernel(int *status, long long limit, int *result) {
     if (threadIdx.x == 0) result[0] = ok ? 1 : 0;
 }
 
+// exp2_poly_x2 on n values (pairs of consecutive entries), next to the MUFU ex2.
+__global__ void exp2_kernel(const float *x, float *poly, float *mufu, int n) {
+    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (i + 1 >= n + 1) return;
+    const float a = x[i], b = i + 1 < n ? x[i + 1] : 0.f;
+    float lo, hi;
+    f2_unpack(exp2_poly_x2(f2_pack(a, b)), lo, hi);
+    poly[i] = lo;
+    mufu[i] = fast_exp2(a);
+    if (i + 1 < n) {
+        poly[i + 1] = hi;
+        mufu[i + 1] = fast_exp2(b);
+    }
+}
+
 typedef CUresult (*EncodeFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                              const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                              const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -161,5 +176,11 @@ extern "C" __attribute__((visibility("default"))) int selftest_gemm(const void *
 extern "C" __attribute__((visibility("default"))) int selftest_wait(int *status, long long limit,
                                                                   int *result) {
     wait_kernel<<<1, 32>>>(status, limit, result);
+    return (int)cudaDeviceSynchronize();
+}
+
+extern "C" __attribute__((visibility("default"))) int selftest_exp2(const float *x, float *poly,
+                                                                  float *mufu, int n) {
+    exp2_kernel<<<(n / 2 + 128) / 128, 128>>>(x, poly, mufu, n);
     return (int)cudaDeviceSynchronize();
 }

@@ -18,15 +18,51 @@ PEAKS = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400
          "sm_max_mhz": 1965.0}
 
 
-def test_lstep_roofline_uses_the_algorithmic_flops_and_the_sustained_peak():
+def test_lstep_roofline_uses_the_algorithmic_flops_and_the_burst_peak():
+    """The timed region is short and runs at boost clock: the burst GEMM figure is
+    the peak; the sustained (power-capped) figure is only a side field."""
     wl = synth.WORKLOADS["720p"]
     flops = 4.0 * wl.N * wl.b1 * wl.d * wl.B * wl.H
     r = bench.kernel_roofline("tc_lstep_kernel", 1.0, wl, PEAKS, "measured")
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert r["achieved"] == pytest.approx(flops / 1e-3 / 1e12)
-    assert r["peak"] == 1400.0
-    assert r["frac"] == pytest.approx(r["achieved"] / 1400.0)
-    assert r["frac_of_burst"] == pytest.approx(r["achieved"] / 1600.0)
+    assert r["peak"] == 1600.0
+    assert r["frac"] == pytest.approx(r["achieved"] / 1600.0)
+    assert r["frac_of_sustained"] == pytest.approx(r["achieved"] / 1400.0)
+    assert "burst" in r["peak_source"]
+
+
+def test_clock_scaling_lowers_the_peak_to_the_run_clock():
+    wl = synth.WORKLOADS["720p"]
+    r = bench.kernel_roofline("tc_lstep_kernel", 1.0, wl, PEAKS, "measured")
+    bench.clock_scaled(r, {"sm_mhz": 1965.0 / 2}, PEAKS)
+    assert r["frac_at_run_clock"] == pytest.approx(2 * r["frac"])
+    r2 = bench.kernel_roofline("tc_lstep_kernel", 1.0, wl, PEAKS, "measured")
+    bench.clock_scaled(r2, {"sm_mhz": 1965.0}, PEAKS)
+    assert r2["frac_at_run_clock"] == pytest.approx(r2["frac"])
+
+
+def test_step_stats_percentiles():
+    st = bench.step_stats([float(x) for x in range(1, 101)])
+    assert st["median"] == pytest.approx(50.5)
+    assert st["p10"] == pytest.approx(10.9)
+    assert st["p90"] == pytest.approx(90.1)
+    assert st["min"] == 1.0 and st["max"] == 100.0
+
+
+def test_sampled_rel_err_compares_the_problem_rows():
+    import numpy as np
+    wl = synth.WORKLOADS["tiny"].replace(tiles=3)
+    rng = np.random.default_rng(0)
+    ref = {0: rng.standard_normal((wl.N, wl.d)), 1: rng.standard_normal((wl.N, wl.d))}
+    probs = [(0, 0, 0), (1, 2, 7)]
+    exact = bench.sampled_rel_err(wl, probs, ref, lambda bh, rows: ref[bh][rows])
+    assert exact["value"] == 0.0
+    assert exact["rows"] == sum(len(bench.problem_rows(wl, g, c)) for _, g, c in probs)
+    off = bench.sampled_rel_err(wl, probs, ref, lambda bh, rows: 1.01 * ref[bh][rows])
+    assert off["value"] == pytest.approx(0.01)
+    # the rows of a problem are the tile's block rows at its column
+    assert list(bench.problem_rows(wl, 1, 2)) == [u * wl.b2 + 2 for u in range(8, 16)]
 
 
 def test_rstep_roofline_counts_every_tile():

@@ -251,6 +251,31 @@ def test_device_entry_points_reject_bad_buffers(tiny64):
     assert _lib.monarch_last_device_status(None) == 0
 
 
+def test_injected_stall_times_out_and_the_next_call_is_correct():
+    """Fault injection on the host: with the stall hook on, each tensor-core kernel's
+    MMA warp waits on a barrier that nothing completes.  The bounded wait must give
+    up, so the status is MONARCH_ERR_TIMEOUT for certain; the kernels then take
+    their abort path (the other roles stop, in-flight copies and MMAs drain, tensor
+    memory is freed) and the following call on the same context is correct."""
+    wl = synth.WORKLOADS["480p_chunk"].replace(H=4)
+    q, k, v = device_inputs(wl)
+    assert kernel_path(q, f=wl.f, h=wl.h, w=wl.w, b1=wl.b1, b2=wl.b2, tiles=wl.tiles) == 1
+    old_limit = _lib.monarch_set_wait_limit(1 << 12)
+    old_stall = _lib.monarch_debug_inject_stall(1)
+    try:
+        monarch_attention(q, k, v, f=wl.f, h=wl.h, w=wl.w, b1=wl.b1, b2=wl.b2, tiles=wl.tiles)
+        torch.cuda.synchronize()
+        assert _lib.monarch_last_device_status(None) == 7
+    finally:
+        _lib.monarch_debug_inject_stall(old_stall)
+        _lib.monarch_set_wait_limit(old_limit)
+    assert _lib.monarch_last_device_status(None) == 0   # the word was read and cleared
+    out = run(wl, q, k, v)
+    q64, k64, v64 = (from_torch(x, wl.dtype) for x in (q, k, v))
+    ref = oracle.monarch_attn(q64, k64, v64, wl.b1, wl.b2, wl.tiles, wl.iters)
+    assert rel_fro(from_torch(out, wl.dtype), ref) <= TOL[wl.dtype]
+
+
 def test_tensor_core_path_survives_a_tiny_wait_limit():
     """Bounded waits: with a limit of a few polls the kernels give up (status
     MONARCH_ERR_TIMEOUT) or finish, but never hang, and the next call is correct."""

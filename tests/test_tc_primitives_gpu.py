@@ -30,6 +30,7 @@ def lib():
     vp = ctypes.c_void_p
     so.selftest_gemm.argtypes = [vp, vp, ctypes.c_int, vp, vp, vp]
     so.selftest_wait.argtypes = [vp, ctypes.c_longlong, vp]
+    so.selftest_exp2.argtypes = [vp, vp, vp, ctypes.c_int]
     return so
 
 
@@ -57,3 +58,27 @@ def test_bounded_wait_gives_up(lib):
     assert int(res.item()) == 0          # the wait returned "not completed"
     assert int(st.item()) == 7           # MONARCH_ERR_TIMEOUT recorded
     assert torch.ones(4, device="cuda").sum().item() == 4   # the context is still usable
+
+
+def test_polynomial_exp2_within_its_error_bound(lib):
+    """exp2_poly_x2 (Cody-Waite reduction, degree-3 minimax on [0, 1)) against 2^d in
+    float64: relative error <= 1e-4 (the fit's 7.5e-5 plus float32 rounding) down to
+    2^-125; below that a non-negative value of at most 2^-125 (at 2^-126 the result's
+    exponent field reaches zero and precision drops); and it agrees
+    with the MUFU exponential it replaces to the same bound."""
+    d = torch.cat([torch.linspace(-130.0, 0.0, 200001, dtype=torch.float64),
+                   torch.tensor([0.0, -1e-7, -0.5, -1.0, -126.0, -126.5, -127.0, -1e4,
+                                 -3e38], dtype=torch.float64)]).float()
+    n = d.numel()
+    x = d.cuda()
+    poly = torch.empty(n, device="cuda")
+    mufu = torch.empty(n, device="cuda")
+    assert lib.selftest_exp2(x.data_ptr(), poly.data_ptr(), mufu.data_ptr(), n) == 0
+    ref = torch.exp2(d.double())
+    got = poly.cpu().double()
+    normal = ref >= 2.0 ** -125
+    rel = ((got[normal] - ref[normal]).abs() / ref[normal]).max().item()
+    assert rel <= 1e-4
+    assert bool((got[~normal] >= 0).all()) and bool((got[~normal] <= 2.0 ** -125).all())
+    m = mufu.cpu().double()
+    assert ((got[normal] - m[normal]).abs() / m[normal]).max().item() <= 1.2e-4

@@ -64,6 +64,60 @@ def test_two_calls_in_a_row_match_the_workspace_entry_point(name, dtype, kw):
     assert not torch.equal(runs[0][3], runs[1][3])
 
 
+class DefaultPoolWatch:
+    """The current device's default CUDA memory pool through the driver API: the
+    pool that stream-ordered allocations (cudaMallocAsync) draw from."""
+    RESERVED_CURRENT, USED_CURRENT, USED_HIGH = 5, 7, 8
+
+    def __init__(self):
+        import ctypes
+        self.ct = ctypes
+        self.cu = ctypes.CDLL("libcuda.so.1")
+        dev = ctypes.c_int()
+        assert self.cu.cuDeviceGet(ctypes.byref(dev), torch.cuda.current_device()) == 0
+        self.pool = ctypes.c_void_p()
+        assert self.cu.cuDeviceGetDefaultMemPool(ctypes.byref(self.pool), dev) == 0
+
+    def get(self, attr):
+        v = self.ct.c_uint64()
+        assert self.cu.cuMemPoolGetAttribute(self.pool, attr, self.ct.byref(v)) == 0
+        return v.value
+
+    def reset_high(self):
+        zero = self.ct.c_uint64(0)
+        assert self.cu.cuMemPoolSetAttribute(self.pool, self.USED_HIGH, self.ct.byref(zero)) == 0
+
+
+def test_a_call_allocates_nothing():
+    """The defining property: after a first call (which looks up the static array's
+    address for this context), a call changes neither torch's allocator counters,
+    nor the device's free memory, nor the default memory pool's usage, not even
+    transiently (the pool's high-water mark stays at its current usage)."""
+    wl = synth.WORKLOADS["480p_chunk"].replace(H=2)
+    args = shape_args(wl)
+    q64, k64, v64 = synth.make_inputs(wl)
+    q, k, v = (to_torch(x, "bf16") for x in (q64, k64, v64))
+    out = torch.empty_like(q)
+    call = lambda: _lib.check(_lib.monarch_attn_fwd_noalloc(   # noqa: E731
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), *args, _lib.BF16, None),
+        "fwd_noalloc")
+    call()
+    torch.cuda.synchronize()
+    pool = DefaultPoolWatch()
+    pool.reset_high()
+    before = (torch.cuda.memory_allocated(), torch.cuda.memory_reserved(),
+              torch.cuda.mem_get_info()[0], pool.get(pool.USED_CURRENT),
+              pool.get(pool.RESERVED_CURRENT))
+    call()
+    torch.cuda.synchronize()
+    after = (torch.cuda.memory_allocated(), torch.cuda.memory_reserved(),
+             torch.cuda.mem_get_info()[0], pool.get(pool.USED_CURRENT),
+             pool.get(pool.RESERVED_CURRENT))
+    assert after == before
+    assert pool.get(pool.USED_HIGH) == pool.get(pool.USED_CURRENT)
+    assert _lib.monarch_last_device_status(None) == 0
+
+
 def test_rejects_problems_beyond_the_static_scratch():
     wl = synth.WORKLOADS["720p"]
     args = shape_args(wl)
