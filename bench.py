@@ -53,13 +53,15 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def workload_config(wl: synth.Workload, world: int) -> dict:
+def workload_config(wl: synth.Workload, world: int, shard: bool = False) -> dict:
+    par = ("units x%d (one clip's (head, tile) units split across GPUs, disjoint output rows)"
+           % world if shard else "replicas x%d (independent clips per GPU)" % world)
     return {"workload": "%s Wan clip: B=%d H=%d d=%d f=%d h=%d w=%d (N=%d), blocks (%d,%d), "
                         "tiles=%d, iters=%d" % (wl.name, wl.B, wl.H, wl.d, wl.f, wl.h, wl.w,
                                                 wl.N, wl.b1, wl.b2, wl.tiles, wl.iters),
             "B": wl.B, "H": wl.H, "d": wl.d, "f": wl.f, "h": wl.h, "w": wl.w, "N": wl.N,
             "b1": wl.b1, "b2": wl.b2, "tiles": wl.tiles, "iters": wl.iters,
-            "parallelism": "replicas x%d (independent clips per GPU)" % world,
+            "parallelism": par,
             "l2": "inputs (%.2f GB) larger than L2, and a %d MB buffer written between "
                   "timed steps" % (3 * wl.B * wl.H * wl.N * wl.d * 2 / 1e9, L2_FLUSH_BYTES >> 20)}
 
@@ -324,6 +326,18 @@ def max_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
+def unit_partition(total_units: int, world: int, rank: int):
+    """Rank's contiguous, balanced share [begin, end) of one clip's (head, tile) units."""
+    return (total_units * rank) // world, (total_units * (rank + 1)) // world
+
+
+def unit_rows(wl: synth.Workload, unit: int):
+    """(head, token rows) that one (head, tile) unit writes: rows (u, v), u in tile g."""
+    bh, g = divmod(unit, wl.tiles)
+    u = np.arange((g * wl.b1) // wl.tiles, ((g + 1) * wl.b1) // wl.tiles)
+    return bh, (u[:, None] * wl.b2 + np.arange(wl.b2)[None, :]).ravel()
+
+
 def job_throughput(world: int, dense_flops_per_clip: float, ms_step: float) -> float:
     """Whole-job dense-equivalent TFLOP/s: every rank processed one clip per step."""
     return world * dense_flops_per_clip / (ms_step * 1e-3) / 1e12
@@ -499,8 +513,11 @@ def run_ours(args, wl: synth.Workload, world: int, rank: int, local: int):
     dev = torch.device("cuda", local)
     shape = (wl.B, wl.H, wl.N, wl.d)
     hq, hk, hv = (torch.empty(shape, dtype=torch.int16).pin_memory() for _ in range(3))
+    # replicas: every rank its own clip; shard: every rank the same clip, its own units
+    shard = args.shard
     synth.fill_device_bits(wl, hq.numpy().view(np.uint16), hk.numpy().view(np.uint16),
-                           hv.numpy().view(np.uint16), rank)
+                           hv.numpy().view(np.uint16), 0 if shard else rank)
+    units = unit_partition(wl.B * wl.H * wl.tiles, world, rank) if shard else None
     q, k, v = (x.to(dev).view(torch.bfloat16) for x in (hq, hk, hv))
     out = torch.empty_like(q)
     hout = torch.empty(shape, dtype=torch.int16).pin_memory()
@@ -513,9 +530,15 @@ def run_ours(args, wl: synth.Workload, world: int, rank: int, local: int):
     path = _lib.monarch_attn_path(*sargs, _lib.BF16)
 
     def step():
-        _lib.check(_lib.monarch_attn_fwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                            out.data_ptr(), *sargs, _lib.BF16, ws.data_ptr(),
-                                            ws_bytes, sh), "monarch_attn_fwd_ws")
+        if shard:
+            _lib.check(_lib.monarch_attn_fwd_units_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                      out.data_ptr(), *sargs, _lib.BF16, *units,
+                                                      ws.data_ptr(), ws_bytes, sh),
+                       "monarch_attn_fwd_units_ws")
+        else:
+            _lib.check(_lib.monarch_attn_fwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                out.data_ptr(), *sargs, _lib.BF16, ws.data_ptr(),
+                                                ws_bytes, sh), "monarch_attn_fwd_ws")
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -549,14 +572,30 @@ def run_ours(args, wl: synth.Workload, world: int, rank: int, local: int):
     # percentiles of the per-step times, each the max over ranks (same order on every rank)
     stats = {k: max_over_ranks(v, world, dev) for k, v in step_stats(step_ms).items()}
 
-    # end to end through the host-buffer entry point: H2D inputs, forward, D2H output
+    # end to end through the C ABI with host buffers: H2D inputs, forward, D2H output.
+    # Replicas: monarch_attn_fwd_host.  Shard: pinned copies of the clip in, the
+    # rank's units through monarch_attn_fwd_units_ws, the rank's heads out.
     e2e_times = []
+    es = 2
+    head_bytes = wl.N * wl.d * es
+    if shard:
+        hb, he = units[0] // wl.tiles, (units[1] + wl.tiles - 1) // wl.tiles
+        h2d_bytes, d2h_bytes = 3 * wl.B * wl.H * head_bytes, (he - hb) * head_bytes
+    else:
+        h2d_bytes, d2h_bytes = 3 * wl.B * wl.H * head_bytes, wl.B * wl.H * head_bytes
     for i in range(args.e2e_warmup + args.e2e_steps if args.e2e_steps > 0 else 0):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        _lib.check(_lib.monarch_attn_fwd_host(hq.data_ptr(), hk.data_ptr(), hv.data_ptr(),
-                                              hout.data_ptr(), *sargs, _lib.BF16, sh),
-                   "monarch_attn_fwd_host")
+        if shard:
+            for dst, src in ((q, hq), (k, hk), (v, hv)):
+                dst.view(torch.int16).copy_(src, non_blocking=True)
+            step()
+            hout.view(wl.B * wl.H, -1)[hb:he].copy_(
+                out.view(torch.int16).view(wl.B * wl.H, -1)[hb:he], non_blocking=True)
+        else:
+            _lib.check(_lib.monarch_attn_fwd_host(hq.data_ptr(), hk.data_ptr(), hv.data_ptr(),
+                                                  hout.data_ptr(), *sargs, _lib.BF16, sh),
+                       "monarch_attn_fwd_host")
         b.record(stream)
         torch.cuda.synchronize()
         if i >= args.e2e_warmup:
@@ -567,7 +606,8 @@ def run_ours(args, wl: synth.Workload, world: int, rank: int, local: int):
         return
     peaks, peak_kind = load_peaks()
     dense = wl.dense_flops()
-    value = job_throughput(world, dense, ms_step)
+    clips = 1 if shard else world   # clips the whole job processes per step
+    value = job_throughput(clips, dense, ms_step)
     kernels = {name: {"ms_per_launch": ms / n, "launches": n, "share": ms / max(1e-9, sum(
         m for m, _ in prof.values()))} for name, (ms, n) in prof.items() if n > 0}
     dominant = max(kernels, key=lambda kk: kernels[kk]["ms_per_launch"] * kernels[kk]["launches"])
@@ -584,10 +624,10 @@ def run_ours(args, wl: synth.Workload, world: int, rank: int, local: int):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(wl, world),
+        "scaling": "strong" if shard else "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": workload_config(wl, world, shard),
         "ms_stats": stats,
-        "monarch_tflops": world * flops / (ms_step * 1e-3) / 1e12,
+        "monarch_tflops": clips * flops / (ms_step * 1e-3) / 1e12,
         "path_roofline": {"roofline_ms": roof_ms, "frac": roof_ms / ms_step,
                           "flops_per_step": flops, "io_bytes_per_step": io,
                           "peak_source": "%s bf16_tflops (burst) and hbm_gbs" % peak_kind,
@@ -599,14 +639,17 @@ def run_ours(args, wl: synth.Workload, world: int, rank: int, local: int):
         "kernel_path": "sm100 tensor-core" if path == 1 else "generic SIMT",
         "gpu_launches": launches,
         "e2e": None if e2e_ms is None else {
-            "value": job_throughput(world, dense, e2e_ms), "unit": UNIT,
+            "value": job_throughput(clips, dense, e2e_ms), "unit": UNIT,
             "ms_per_step": e2e_ms,
-            "h2d_bytes_per_step": 3 * wl.B * wl.H * wl.N * wl.d * 2,
-            "d2h_bytes_per_step": wl.B * wl.H * wl.N * wl.d * 2,
-            "api": "monarch_attn_fwd_host (C ABI, pinned host buffers)"},
+            "h2d_bytes_per_step": h2d_bytes,
+            "d2h_bytes_per_step": d2h_bytes,
+            "api": ("monarch_attn_fwd_units_ws with pinned host copies (rank's heads out)"
+                    if shard else "monarch_attn_fwd_host (C ABI, pinned host buffers)")},
         "clocks": clock_rec,
         "gpu": props.name,
     }
+    if shard:
+        line["units"] = {"rank0": list(units), "total": wl.B * wl.H * wl.tiles}
     if world == 1 and args.secondary_steps > 0 and args.workload == "720p" and args.heads == 0:
         line["also_480p"] = secondary_workload(synth.WORKLOADS["480p_full"], args.secondary_steps,
                                                3, flush, stream)
@@ -637,6 +680,9 @@ def main():
                     help="timed steps of the 480p full clip reported beside the line (0: skip)")
     ap.add_argument("--heads", type=int, default=0,
                     help="override H (smaller cases for ncu captures; not a bench line)")
+    ap.add_argument("--shard", action="store_true",
+                    help="N > 1: split ONE clip's (head, tile) units across the ranks "
+                         "(strong scaling) instead of one clip per rank")
     ap.add_argument("--sweep", action="store_true",
                     help="error-vs-cost sweeps (tiles on 480p, iterations on Wan-14B) instead "
                          "of the bench line; one GPU")

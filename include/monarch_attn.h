@@ -151,6 +151,28 @@ MONARCH_API monarch_status monarch_attn_fwd_ws(const void *q, const void *k, con
                                    size_t ws_bytes, monarch_stream_t stream);
 
 /*
+ * Forward pass over a contiguous range of (batch, head, tile) units, for
+ * splitting one call's work across GPUs or streams.  Unit index
+ * ((b*H + h)*tiles + g), 0 <= unit_begin <= unit_end <= B*H*tiles.  A unit
+ * is independent of every other one from the aggregated query to its output
+ * (the method's tiles each own their R factor; explainer page, "创新二：平铺
+ * Monarch参数化"), so the union of calls over a partition of the units gives
+ * exactly the output of one full call, bit for bit.  Writes only the output
+ * rows of those units, i.e. rows (u, v) with u in tile g, every v, of head
+ * (b, h); every other row of out is left untouched.  q, k, v must hold the
+ * whole clip.  Workspace and other arguments as monarch_attn_fwd_ws (the
+ * workspace size does not depend on the range; the tensor-core path computes
+ * the R-step of every tile of the heads that the range touches).
+ * Returns MONARCH_ERR_SHAPE for a range outside [0, B*H*tiles].
+ */
+MONARCH_API monarch_status monarch_attn_fwd_units_ws(const void *q, const void *k, const void *v,
+                                                     void *out, int B, int H, int f, int h, int w,
+                                                     int d, int b1, int b2, int tiles, int iters,
+                                                     monarch_dtype dtype, int unit_begin,
+                                                     int unit_end, void *workspace,
+                                                     size_t ws_bytes, monarch_stream_t stream);
+
+/*
  * Forward pass on HOST buffers: q, k, v, out are host pointers (pinned memory
  * gives full PCIe bandwidth; pageable memory works but is slower).  Device
  * copies of the inputs and output and the workspace are taken with

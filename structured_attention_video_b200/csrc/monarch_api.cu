@@ -93,6 +93,7 @@ monarch_status validate_shape(int B, int H, int f, int h, int w, int d, int b1, 
     if (N > (1LL << 30) || (int64_t)b1 * b2 != N) return MONARCH_ERR_SHAPE;
     if (tiles < 1 || tiles > b1 || iters < 1 || iters > 1000) return MONARCH_ERR_SHAPE;
     if ((int64_t)B * H > (1LL << 24)) return MONARCH_ERR_SHAPE;
+    if ((int64_t)B * H * tiles >= (1LL << 31)) return MONARCH_ERR_SHAPE;   // unit indices
     if (d != 32 && d != 64 && d != 128) return MONARCH_ERR_UNSUPPORTED;
     // every grid of the generic kernels must fit in 2^31 - 1 blocks
     const int64_t BHt = (int64_t)B * H * tiles;
@@ -111,6 +112,8 @@ monarch_status validate_shape(int B, int H, int f, int h, int w, int d, int b1, 
     p->tiles = tiles;
     p->iters = iters;
     p->scale = (float)(1.0 / sqrt((double)d));
+    p->unit_begin = 0;
+    p->unit_end = B * H * tiles;
     return MONARCH_OK;
 }
 
@@ -225,6 +228,29 @@ monarch_status monarch_attn_fwd_ws(const void *q, const void *k, const void *v, 
     const size_t need = workspace_bytes_for(p, dtype, choose_path(p, dtype), overflow);
     if (overflow) return MONARCH_ERR_SHAPE;
     if (ws_bytes < need) return MONARCH_ERR_NO_MEMORY;
+    return run_forward(p, dtype, q, k, v, out, workspace, (cudaStream_t)stream);
+}
+
+monarch_status monarch_attn_fwd_units_ws(const void *q, const void *k, const void *v, void *out,
+                                         int B, int H, int f, int h, int w, int d, int b1, int b2,
+                                         int tiles, int iters, monarch_dtype dtype, int unit_begin,
+                                         int unit_end, void *workspace, size_t ws_bytes,
+                                         monarch_stream_t stream) {
+    if (!q || !k || !v || !out || !workspace) return MONARCH_ERR_INVALID_ARG;
+    Problem p;
+    monarch_status st = validate_shape(B, H, f, h, w, d, b1, b2, tiles, iters, dtype, &p);
+    if (st != MONARCH_OK) return st;
+    if (unit_begin < 0 || unit_end > p.unit_end || unit_begin > unit_end) return MONARCH_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        ((uintptr_t)workspace & 255u))
+        return MONARCH_ERR_ALIGN;
+    bool overflow = false;
+    const size_t need = workspace_bytes_for(p, dtype, choose_path(p, dtype), overflow);
+    if (overflow) return MONARCH_ERR_SHAPE;
+    if (ws_bytes < need) return MONARCH_ERR_NO_MEMORY;
+    if (unit_begin == unit_end) return MONARCH_OK;   // nothing to compute
+    p.unit_begin = unit_begin;
+    p.unit_end = unit_end;
     return run_forward(p, dtype, q, k, v, out, workspace, (cudaStream_t)stream);
 }
 

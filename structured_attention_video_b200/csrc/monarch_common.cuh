@@ -39,6 +39,12 @@ struct Problem {
     int b1, b2, tiles;   // Monarch blocks and tiles
     int iters;
     float scale;         // 1/sqrt(d)
+    // the (head, tile) units this call computes, unit = (b*H + h)*tiles + g:
+    // [unit_begin, unit_end); every unit is independent from the aggregated
+    // query to its output rows (all of them by default)
+    int unit_begin, unit_end;
+    __host__ __device__ int head_begin() const { return unit_begin / tiles; }
+    __host__ __device__ int head_end() const { return (unit_end + tiles - 1) / tiles; }
 };
 
 // Kernels that can give up a bounded wait receive a pointer to the device

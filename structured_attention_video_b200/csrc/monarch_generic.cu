@@ -42,9 +42,11 @@ __device__ __forceinline__ float warp_sum(float x) {
 template <typename T>
 __global__ void qbar_mean_kernel(const T *__restrict__ q, float *__restrict__ qbar, Problem p) {
     const int64_t row_elems = (int64_t)p.b2 * p.d;
-    const int64_t total = (int64_t)p.BH * p.tiles * row_elems;
-    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-         idx += (int64_t)gridDim.x * blockDim.x) {
+    // the (head, tile) units of the call: unit = bh * tiles + g
+    const int64_t total = (int64_t)p.unit_end * row_elems;
+    for (int64_t idx = (int64_t)p.unit_begin * row_elems + (int64_t)blockIdx.x * blockDim.x +
+                       threadIdx.x;
+         idx < total; idx += (int64_t)gridDim.x * blockDim.x) {
         const int64_t bhg = idx / row_elems, col = idx % row_elems;
         const int g = (int)(bhg % p.tiles), bh = (int)(bhg / p.tiles);
         const int u0 = tile_begin(g, p.b1, p.tiles), u1 = tile_begin(g + 1, p.b1, p.tiles);
@@ -69,7 +71,7 @@ rstep_kernel(const T *__restrict__ k, const T *__restrict__ v, const float *__re
     float *sv = sk + KC * DS;     // [KC][DS]
 
     const int nvg = (p.b2 + GW - 1) / GW;
-    int64_t bid = blockIdx.x;
+    int64_t bid = blockIdx.x + (int64_t)p.unit_begin * p.b1 * nvg;   // from the first unit
     const int vg = (int)(bid % nvg);
     bid /= nvg;
     const int up = (int)(bid % p.b1);
@@ -157,7 +159,7 @@ lstep_kernel(const T *__restrict__ q, const float *__restrict__ ktil, const floa
     float *sh = sz + KC * DS;     // [KC]
 
     const int nug = (tile_max_rows(p.b1, p.tiles) + GW - 1) / GW;
-    int64_t bid = blockIdx.x;
+    int64_t bid = blockIdx.x + (int64_t)p.unit_begin * p.b2 * nug;   // from the first unit
     const int ug = (int)(bid % nug);
     bid /= nug;
     const int vcol = (int)(bid % p.b2);
@@ -235,7 +237,7 @@ qbar_weighted_kernel(const T *__restrict__ q, const float *__restrict__ ktil,
     float *sl = sq + KC * DS;     // [KC]
 
     const int nupg = (p.b1 + GW - 1) / GW;
-    int64_t bid = blockIdx.x;
+    int64_t bid = blockIdx.x + (int64_t)p.unit_begin * p.b2 * nupg;   // from the first unit
     const int upg = (int)(bid % nupg);
     bid /= nupg;
     const int vcol = (int)(bid % p.b2);
@@ -318,16 +320,16 @@ cudaError_t run_generic(const Problem &p, const T *q, const T *k, const T *v, T 
     const size_t smem_r = (GW * D + 2 * KC * (D + 1)) * sizeof(float);
     const size_t smem_l = (GW * D + 2 * KC * (D + 1) + KC) * sizeof(float);
     const size_t smem_w = (GW * D + KC * (D + 1) + KC) * sizeof(float);
-    const int64_t nmean = (int64_t)p.BH * p.tiles * p.b2 * p.d;
+    const int64_t units = p.unit_end - p.unit_begin;
+    const int64_t nmean = units * p.b2 * p.d;
     const int mean_blocks = (int)((nmean + 255) / 256 < 148 * 64 ? (nmean + 255) / 256 : 148 * 64);
     {
         ProfileScope scope(K_QBAR_MEAN, stream);
         qbar_mean_kernel<T><<<mean_blocks, 256, 0, stream>>>(q, ws.qbar, p);
     }
-    const unsigned r_blocks = (unsigned)((int64_t)p.BH * p.tiles * p.b1 * ((p.b2 + GW - 1) / GW));
-    const unsigned l_blocks = (unsigned)((int64_t)p.BH * p.tiles * p.b2 *
-                                         ((tile_max_rows(p.b1, p.tiles) + GW - 1) / GW));
-    const unsigned w_blocks = (unsigned)((int64_t)p.BH * p.tiles * p.b2 * ((p.b1 + GW - 1) / GW));
+    const unsigned r_blocks = (unsigned)(units * p.b1 * ((p.b2 + GW - 1) / GW));
+    const unsigned l_blocks = (unsigned)(units * p.b2 * ((tile_max_rows(p.b1, p.tiles) + GW - 1) / GW));
+    const unsigned w_blocks = (unsigned)(units * p.b2 * ((p.b1 + GW - 1) / GW));
     for (int it = 0; it < p.iters; it++) {
         const bool last = it == p.iters - 1;
         const int64_t vstride = it == 0 ? (int64_t)p.d : (int64_t)p.b1 * p.d;

@@ -18,6 +18,11 @@
 //                       strides over b2 (P^T folded into the load); online
 //                       softmax over the b1 blocks with logits s q.Ktil + H,
 //                       O accumulated in TMEM, rows written back strided.
+// The entropy enters the L-step's logit MMA: the R-step stores, per key row of
+// Ktil, a 16-column bfloat16 panel [H'_hi, H'_lo, 0, ...] with H' = H / (s ln 2)
+// (split in two bfloat16 parts that sum to H' within 2^-16 relative), and the
+// L-step adds one K-step of an all-ones query panel times that panel, so S
+// arrives in TMEM as (s q.Ktil + H) / (s ln 2) with no per-element entropy work.
 // Warp roles (384 threads): warp 0 TMA producer (in the L-step: queries, Ktil
 // and entropies; warp 2 produces Z), warp 1 MMA issuer and TMEM owner, warps
 // 4-7 and 8-11 the two softmax (L-step) or the softmax and epilogue (R-step)
@@ -60,7 +65,9 @@ __global__ void __launch_bounds__(128) tc_qbar_kernel(const __nv_bfloat16 *__res
     const int row_elems = p.b2 * kD;
     const int nchunk = (row_elems / 8 + 127) / 128;
     const int chunk = blockIdx.x % nchunk;
-    const int bhg = blockIdx.x / nchunk;
+    // every tile of the heads that the unit range touches (the R-step reads all
+    // of a head's aggregated rows, padding included)
+    const int bhg = blockIdx.x / nchunk + p.head_begin() * p.tiles;
     const int g = bhg % p.tiles, bh = bhg / p.tiles;
     const int col = (chunk * 128 + threadIdx.x) * 8;
     const int u0 = tile_begin(g, p.b1, p.tiles), u1 = tile_begin(g + 1, p.b1, p.tiles);
@@ -123,25 +130,31 @@ __global__ void __launch_bounds__(128) tc_qbar_kernel(const __nv_bfloat16 *__res
 // 16 warps.  Warps 0-3 and 4-7: the softmax warpgroups of query tiles 0 and 1
 // (one query row per thread); warps 8-11: the epilogue warpgroup (O / l to
 // bfloat16 rows of Y, off the softmax warps' chain); warp 12: the TMA producer
-// of the queries, Ktil and the entropies; warp 13: the MMA issuer; warp 14:
-// the producer of Z; warp 15 idles.  setmaxnreg moves registers from the
+// of Ktil and its entropy panel; warp 13: the MMA issuer; warp 14: the
+// producer of Z; warp 15: the producer of the query tiles.  setmaxnreg moves registers from the
 // producer and epilogue warpgroups to the softmax warpgroups.
 // Tensor memory: S_0 | S_1 | O_0 | O_1 (128 columns each); P_t overwrites the
 // first 64 columns of S_t as packed bfloat16 pairs.
 // =====================================================================
 namespace ls {
 constexpr int kThreads = 512;
-constexpr int kSoftmaxRegs = 184, kEpilogueRegs = 88, kProducerRegs = 56;
+constexpr int kSoftmaxRegs = 176, kEpilogueRegs = 96, kProducerRegs = 64;
 static_assert(2 * kSoftmaxRegs + kEpilogueRegs + kProducerRegs == 4 * (65536 / kThreads),
               "the warpgroups' registers must add up to the launch's 128 per thread");
-// one pair of every kPolyEvery takes its exponentials on the FMA pipe (0: none)
-constexpr int kPolyEvery = 4;
+// one pair of every kPolyEvery takes its exponentials on the FMA pipe (0: none).
+// Measured at 720p: the softmax is bound by issue slots, not by the MUFU, so the
+// polynomial's extra instructions cost more than the exponentials it moves
+// (1.30 ms per step with a quarter on the polynomial, 1.25 ms with none).
+constexpr int kPolyEvery = 0;
 constexpr uint32_t kQ = 0;                          // query tiles 0, 1
 constexpr uint32_t kK = 2 * kTile;                  // Ktil stages 0, 1
 constexpr uint32_t kZ = kK + 2 * kTile;             // Z stages 0, 1
-constexpr uint32_t kH = kZ + 2 * kTile;             // entropies: 4 buffers of 128 floats
-constexpr uint32_t kL = kH + 2048;                  // row sums [problem parity][tile][128]
-constexpr uint32_t kBar = kL + 2048;
+constexpr uint32_t kHx = kZ + 2 * kTile;            // entropy panels (128 x 32 B) of the Ktil stages
+constexpr uint32_t kPanelHx = 128 * 32;
+constexpr uint32_t kQx = kHx + 2 * kPanelHx;        // the all-ones query panel
+constexpr uint32_t kL = kQx + kPanelHx;             // row sums [problem parity][tile][128]
+constexpr uint32_t kStg = kL + 2048;                // epilogue: 4 warps x 32 rows x 128 B
+constexpr uint32_t kBar = kStg + 4 * 4096;
 constexpr uint32_t kSmem = kBar + 512;              // the base is 1024-aligned (checked)
 static_assert(kSmem <= (uint32_t)kMaxSmem, "L-step shared memory");
 }  // namespace ls
@@ -150,10 +163,9 @@ struct LsArgs {
     Problem p;
     int nchunks;    // key chunks of 128 blocks
     int npairs;     // pairs of 128-query tiles per (g, v)
-    int nprob;      // BH * t * b2 * npairs
-    int hstride;    // row length of the entropy array
+    int nprob;      // problems of the unit range: units * b2 * npairs
+    int prob0;      // first problem: unit_begin * b2 * npairs
     float c_log2;   // (1/sqrt(d)) * log2(e)
-    const float *hent;
     __nv_bfloat16 *out;
     int *status;
     long long limit;
@@ -161,12 +173,13 @@ struct LsArgs {
 };
 
 struct LsProblem {
-    int bh, g, v, u_start, u1, key_row0, h_row0;
+    int bh, g, v, u_start, u1, key_row0;
 };
 
 __device__ __forceinline__ LsProblem ls_problem(const LsArgs &a, int unit) {
     const Problem &p = a.p;
     LsProblem q;
+    unit += a.prob0;
     const int pair = unit % a.npairs;
     unit /= a.npairs;
     q.v = unit % p.b2;
@@ -176,13 +189,13 @@ __device__ __forceinline__ LsProblem ls_problem(const LsArgs &a, int unit) {
     q.u1 = tile_begin(q.g + 1, p.b1, p.tiles);
     q.u_start = tile_begin(q.g, p.b1, p.tiles) + 256 * pair;
     q.key_row0 = ((q.bh * p.tiles + q.g) * p.b2 + q.v) * p.b1;
-    q.h_row0 = ((q.bh * p.tiles + q.g) * p.b2 + q.v) * a.hstride;
     return q;
 }
 
 __global__ void __launch_bounds__(ls::kThreads, 1)
 tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmZ, LsArgs a) {
+                const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmHx,
+                LsArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // the SW128 operand tiles need a 1024-byte aligned base; the layout leaves no
     // room to align by hand, so a misaligned base is reported, not worked around
@@ -194,11 +207,10 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + ls::kBar);
     uint64_t *q_full = bars + 0;     // [2 tiles]
     uint64_t *q_empty = bars + 2;    // [2 tiles]: the tile's last S MMA of a problem done
-    uint64_t *k_full = bars + 4;     // [2 stages]
+    uint64_t *k_full = bars + 4;     // [2 stages]: Ktil and its entropy panel
     uint64_t *k_empty = bars + 6;    // [2 stages]: both S MMAs of the chunk done
     uint64_t *z_full = bars + 8;     // [2 stages]
     uint64_t *z_empty = bars + 10;   // [2 stages]: both PV MMAs of the chunk done
-    uint64_t *h_full = bars + 12;    // [4 buffers]: bulk copy of the chunk's entropies
     uint64_t *s_full = bars + 16;    // [2 tiles]
     uint64_t *p_full = bars + 18;    // [2 tiles], one arrival per softmax warp
     uint64_t *o_full = bars + 20;    // [2 tiles]: the last PV MMA of a problem done
@@ -230,12 +242,17 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             mbar_init(o_free + t, 4);   // one arrival per epilogue warp
             mbar_init(l_full + t, 4);   // one arrival per softmax warp
         }
-        for (int s = 0; s < 4; s++) mbar_init(h_full + s, 1);
         mbar_init(mma_done, 1);
         mbar_init(stall_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
+    // the all-ones query panel (every bfloat16 = 1.0, so its swizzle is moot):
+    // the entropy K-step adds 1 * H'_hi + 1 * H'_lo (the panel's other columns are 0)
+    for (int i = threadIdx.x; i < (int)(ls::kPanelHx / 16); i += blockDim.x)
+        reinterpret_cast<uint4 *>(sm + ls::kQx)[i] =
+            make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    fence_proxy_async_smem();   // generic writes -> the tensor cores' async proxy
     if (warp == 13) tmem_alloc(tmem_slot, 512);
     tc_fence_before();
     __syncthreads();
@@ -246,18 +263,44 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     if (warp >= 12) {
         regs_dec<ls::kProducerRegs>();
         if (warp == 12) {
-            // ---------------- producer: queries per problem; per chunk Ktil and H as
-            // soon as the S MMAs of two chunks back are done.  H has four buffers:
-            // S_1 of chunk jc - 2 (whose completion frees the Ktil stage of chunk jc)
-            // is issued only after both softmax warpgroups finished chunk jc - 3,
-            // so buffer jc & 3 (last read for chunk jc - 4) is free.
-            int issued[2] = {0, 0}, qloads = 0, issued_h = 0;
+            // ---------------- producer of Ktil and its entropy panel: per chunk as
+            // soon as the S MMAs of two chunks back are done (never behind a query
+            // load, which has its own warp)
+            int issued[2] = {0, 0};
             bool ok = true;
             for (int pi = 0; ok && pi < nmine; pi++) {
                 const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
-                // each query tile reloads as soon as its own last S MMA of the
-                // previous problem is done
-                for (int t = 0; ok && t < 2; t++) {
+                for (int j = 0; j < nch; j++) {
+                    const int jc = pi * nch + j, sk = jc & 1;
+                    if (jc >= 2 && !wait_warp(k_empty + sk, ((jc >> 1) - 1) & 1, w)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        // keys past b1 in the ragged last chunk belong to the next
+                        // row (or are zero-filled past the array): masked later
+                        mbar_expect_tx(k_full + sk, kTile + ls::kPanelHx);
+                        for (int pn = 0; pn < 2; pn++)
+                            tma_load_2d(sm + ls::kK + sk * kTile + pn * kPanel, &tmK, pn * 64,
+                                        pr.key_row0 + j * 128, k_full + sk);
+                        tma_load_2d(sm + ls::kHx + sk * ls::kPanelHx, &tmHx, 0,
+                                    pr.key_row0 + j * 128, k_full + sk);
+                    }
+                    issued[sk]++;
+                }
+            }
+            if (lane == 0)   // every issued copy lands before the CTA may exit
+                for (int s = 0; s < 2; s++)
+                    if (issued[s] > 0) wait_phase_cleanup(k_full + s, (issued[s] - 1) & 1, kCleanupPolls);
+        } else if (warp == 15) {
+            // ---------------- query producer: each query tile reloads as soon as its
+            // own last S MMA of the previous problem is done; the next problem's
+            // rows (a strided gather) are prefetched into L2 a whole problem ahead
+            int qloads = 0;
+            bool ok = true;
+            for (int pi = 0; ok && pi < nmine; pi++) {
+                const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
+                for (int t = 0; t < 2; t++) {
                     if (pi > 0 && !wait_warp(q_empty + t, (pi - 1) & 1, w)) {
                         ok = false;
                         break;
@@ -271,37 +314,16 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 }
                 if (!ok) break;
                 qloads++;
-                for (int j = 0; j < nch; j++) {
-                    const int jc = pi * nch + j, sk = jc & 1;
-                    if (jc >= 2 && !wait_warp(k_empty + sk, ((jc >> 1) - 1) & 1, w)) {
-                        ok = false;
-                        break;
-                    }
-                    if (lane == 0) {
-                        mbar_expect_tx(k_full + sk, kTile);
+                if (lane == 0 && pi + 1 < nmine) {
+                    const LsProblem nx = ls_problem(a, blockIdx.x + (pi + 1) * gridDim.x);
+                    for (int t = 0; t < 2; t++)
                         for (int pn = 0; pn < 2; pn++)
-                            tma_load_2d(sm + ls::kK + sk * kTile + pn * kPanel, &tmK, pn * 64,
-                                        pr.key_row0 + j * 128, k_full + sk);
-                        // the chunk's entropies (log2 units; keys past b1 are masked later)
-                        mbar_expect_tx(h_full + (jc & 3), 512);
-                        bulk_load(sm + ls::kH + (jc & 3) * 512, a.hent + pr.h_row0 + j * 128, 512,
-                                  h_full + (jc & 3));
-                    }
-                    issued[sk]++;
-                    issued_h++;
+                            tma_prefetch_3d(&tmQ, pn * 64, nx.v, nx.bh * p.b1 + nx.u_start + t * 128);
                 }
             }
-            if (lane == 0) {   // every issued copy lands before the CTA may exit
+            if (lane == 0)
                 for (int t = 0; t < 2; t++)
                     if (qloads > 0) wait_phase_cleanup(q_full + t, (qloads - 1) & 1, kCleanupPolls);
-                for (int s = 0; s < 2; s++)
-                    if (issued[s] > 0) wait_phase_cleanup(k_full + s, (issued[s] - 1) & 1, kCleanupPolls);
-                for (int hb = 0; hb < 4; hb++) {   // the last copy into each entropy buffer
-                    if (issued_h <= hb) continue;
-                    const int last = hb + ((issued_h - 1 - hb) / 4) * 4;
-                    wait_phase_cleanup(h_full + hb, (last >> 2) & 1, kCleanupPolls);
-                }
-            }
         } else if (warp == 14) {
             // ---------------- Z producer: its own warp, so that a Ktil load never
             // queues behind the wait for a Z stage (released one PV later than Ktil)
@@ -341,7 +363,9 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             const uint64_t dQ = smem_desc_sw128(smem_u32(sm + ls::kQ), 16, 1024);
             const uint64_t dK = smem_desc_sw128(smem_u32(sm + ls::kK), 16, 1024);
             const uint64_t dZ = smem_desc_sw128(smem_u32(sm + ls::kZ), kPanel, 1024);
-            constexpr uint32_t kTileDesc = kTile >> 4;
+            const uint64_t dQx = smem_desc_sw32(smem_u32(sm + ls::kQx));
+            const uint64_t dHx = smem_desc_sw32(smem_u32(sm + ls::kHx));
+            constexpr uint32_t kTileDesc = kTile >> 4, kHxDesc = ls::kPanelHx >> 4;
             const int total = nmine * nch;
             // fault injection: a wait that can only give up (bounded, then abort)
             bool ok = !a.stall || spin_warp(stall_bar, 0, w);
@@ -351,6 +375,7 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 if (t == 0 && !spin_warp(k_full + sk, (jc >> 1) & 1, w)) return false;
                 tc_fence_after();
                 mma8_ss_k128(tmem + t * 128, dQ + t * kTileDesc, dK + sk * kTileDesc, idS, 0u);
+                mma1_ss_acc(tmem + t * 128, dQx, dHx + sk * kHxDesc, idS);   // + H'
                 mma_commit_warp(s_full + t);
                 if (t == 1) mma_commit_warp(k_empty + sk);
                 if (jc % nch == nch - 1) mma_commit_warp(q_empty + t);   // tile t no longer read
@@ -396,28 +421,48 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 }
                 tc_fence_after();
                 const float inv_l = 1.f / lsum[((pi & 1) * 2 + t) * 128 + wq * 32 + lane];
-                const int u = pr.u_start + t * 128 + wq * 32 + lane;
-                uint4 *dst = reinterpret_cast<uint4 *>(
-                    a.out + ((int64_t)pr.bh * p.N + (int64_t)u * p.b2 + pr.v) * kD);
+                // O_t leaves tensor memory 32 columns at a time, straight into
+                // bfloat16 pairs; once all of it is in registers the next
+                // problem's first PV may overwrite it, and only then do the
+                // global stores run
+                uint32_t pk[64];
 #pragma unroll
-                for (int c = 0; c < 4; c++) {   // 32 columns at a time
+                for (int c = 0; c < 4; c++) {
                     float o[32];
                     tmem_ld32f(tmem + lane_off + 256 + t * 128 + c * 32, o);
                     tmem_wait_ld();
-                    if (c == 3) {   // all of O_t is in registers: the next PV may start
-                        tc_fence_before();
-                        mbar_arrive_warp(o_free + t);
-                    }
-                    uint32_t pk[16];
 #pragma unroll
                     for (int k = 0; k < 16; k++)
-                        pk[k] = pack_bf16(o[2 * k] * inv_l, o[2 * k + 1] * inv_l);
-                    if (u < pr.u1) {
+                        pk[c * 16 + k] = pack_bf16(o[2 * k] * inv_l, o[2 * k + 1] * inv_l);
+                }
+                tc_fence_before();
+                mbar_arrive_warp(o_free + t);
+                // the warp's 32 rows leave through shared memory, half a row (128 B)
+                // at a time: each lane writes its own row, then every store
+                // instruction covers four whole row halves (eight 16-byte chunks
+                // each), instead of 32 scattered 16-byte pieces
+                uint8_t *stg = sm + ls::kStg + wq * 4096;
+                const int u0w = pr.u_start + t * 128 + wq * 32;
 #pragma unroll
-                        for (int ch = 0; ch < 4; ch++)
-                            dst[c * 4 + ch] = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2],
-                                                         pk[4 * ch + 3]);
+                for (int hf = 0; hf < 2; hf++) {
+#pragma unroll
+                    for (int c = 0; c < 8; c++)   // chunk c at slot (c + row) mod 8: no bank pile-up
+                        *reinterpret_cast<uint4 *>(stg + lane * 128 + ((c + lane) & 7) * 16) =
+                            make_uint4(pk[hf * 32 + 4 * c], pk[hf * 32 + 4 * c + 1],
+                                       pk[hf * 32 + 4 * c + 2], pk[hf * 32 + 4 * c + 3]);
+                    __syncwarp();
+#pragma unroll
+                    for (int rr = 0; rr < 8; rr++) {
+                        const int row = rr * 4 + (lane >> 3), c = lane & 7;
+                        const uint4 val =
+                            *reinterpret_cast<const uint4 *>(stg + row * 128 + ((c + row) & 7) * 16);
+                        const int u = u0w + row;
+                        if (u < pr.u1)
+                            *reinterpret_cast<uint4 *>(
+                                a.out + ((int64_t)pr.bh * p.N + (int64_t)u * p.b2 + pr.v) * kD +
+                                hf * 64 + c * 8) = val;
                     }
+                    __syncwarp();
                 }
             }
         }
@@ -435,64 +480,49 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             float m_run = -INFINITY, l_run = 0.f;
             for (int j = 0; j < nch; j++) {
                 const int jc = pi * nch + j;
-                if (!wait_warp(s_full + t, jc & 1, w) ||
-                    !wait_warp(h_full + (jc & 3), (jc >> 2) & 1, w)) {
+                if (!wait_warp(s_full + t, jc & 1, w)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                // S = (s q.Ktil + H) / (s ln 2): scaled by c_log2 it is the logit in
+                // log2 units, so the maximum is taken on S itself
                 float x[128];
 #pragma unroll
                 for (int c = 0; c < 4; c++) tmem_ld32f(tS + c * 32, &x[c * 32]);
                 tmem_wait_ld();
-                // logits in log2 units: x * s * log2(e) + H / ln 2 (the entropy
-                // arrives in log2 units)
-                const uint64_t *hs = reinterpret_cast<const uint64_t *>(sm + ls::kH + (jc & 3) * 512);
-                uint64_t xp[64];
                 float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
                 const int nvalid = p.b1 - j * 128;   // keys of this chunk inside the row
-                const bool full = nvalid >= 128;
-                if (full) {
+                if (nvalid < 128) {
+                    // the ragged last chunk: keys past b1 belong to the next row
+                    // (or are zero fill), so mask them by selection
 #pragma unroll
-                    for (int i = 0; i < 64; i++) {
-                        xp[i] = f2_fma(f2_pack(x[2 * i], x[2 * i + 1]), c2, hs[i]);
-                        float lo, hi;
-                        f2_unpack(xp[i], lo, hi);
-                        mx4[i & 3] = fmax3(mx4[i & 3], lo, hi);
-                    }
-                } else {
-                    // the ragged last chunk: S and the entropy copy run past the row
-                    // (into the next row or the workspace slack), so mask by selection
-#pragma unroll
-                    for (int i = 0; i < 64; i++) {
-                        float lo, hi;
-                        f2_unpack(f2_fma(f2_pack(x[2 * i], x[2 * i + 1]), c2, hs[i]), lo, hi);
-                        lo = 2 * i < nvalid ? lo : -INFINITY;
-                        hi = 2 * i + 1 < nvalid ? hi : -INFINITY;
-                        xp[i] = f2_pack(lo, hi);
-                        mx4[i & 3] = fmax3(mx4[i & 3], lo, hi);
-                    }
+                    for (int i = 0; i < 128; i++) x[i] = i < nvalid ? x[i] : -INFINITY;
                 }
+#pragma unroll
+                for (int i = 0; i < 64; i++) mx4[i & 3] = fmax3(mx4[i & 3], x[2 * i], x[2 * i + 1]);
                 const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-                // the running maximum moves only when it grows by more than 2^8: the
-                // probabilities stay below 256 and O is rescaled rarely
+                // the running maximum moves only when it grows by more than 2^8 in
+                // log2 units: the probabilities stay below 256 and O is rescaled rarely
                 float alpha = 1.f;
                 bool rescale = false;
-                if (mx > m_run + 8.f) {
-                    alpha = fast_exp2(m_run - mx);
+                if ((mx - m_run) * a.c_log2 > 8.f) {
+                    alpha = fast_exp2((m_run - mx) * a.c_log2);
                     m_run = mx;
                     rescale = true;
                 }
-                const uint64_t nm2 = f2_pack(-m_run, -m_run);
+                const uint64_t nmc2 = f2_pack(-m_run * a.c_log2, -m_run * a.c_log2);
                 uint64_t sum2[4] = {0, 0, 0, 0};
 #pragma unroll
                 for (int h = 0; h < 2; h++) {
                     uint32_t pk[32];
 #pragma unroll
                     for (int i = 0; i < 32; i++) {
-                        const uint64_t d2 = f2_add(xp[h * 32 + i], nm2);
+                        const int e = h * 32 + i;
+                        const uint64_t d2 = f2_fma(f2_pack(x[2 * e], x[2 * e + 1]), c2, nmc2);
                         uint64_t e2;
-                        if (ls::kPolyEvery > 0 && (i % ls::kPolyEvery) == ls::kPolyEvery - 1 && full) {
+                        constexpr int kEvery = ls::kPolyEvery > 0 ? ls::kPolyEvery : 1;
+                        if (ls::kPolyEvery > 0 && (i % kEvery) == kEvery - 1 && nvalid >= 128) {
                             e2 = exp2_poly_x2(d2);
                         } else {
                             float lo, hi;
@@ -550,9 +580,8 @@ struct RsArgs {
     int nmt;             // 128-row tiles of qbar (t*b2 padded)
     int mpad;            // nmt * 128
     int bpc;             // blocks per CTA (flattened over heads and blocks)
-    int hstride;         // row length of the entropy array (b1 rounded up to 4)
     float c_log2;
-    float *hent;
+
     int *status;
     long long limit;
     int stall;           // test hook: the MMA warp first waits on a barrier nothing completes
@@ -565,7 +594,9 @@ struct RsLayout {
     static constexpr uint32_t kPanelKV = B2P * 128;
     __host__ __device__ static uint32_t kv(int nmt) { return (uint32_t)nmt * kTile; }
     __host__ __device__ static uint32_t stg(int nmt) { return kv(nmt) + 2 * kStage; }
-    __host__ __device__ static uint32_t bar(int nmt) { return stg(nmt) + 4 * 8192; }
+    // entropy-panel staging of the softmax warps: 4 warps x 32 rows x 32 B
+    __host__ __device__ static uint32_t hstg(int nmt) { return stg(nmt) + 4 * 8192; }
+    __host__ __device__ static uint32_t bar(int nmt) { return hstg(nmt) + 4 * 1024; }
     __host__ __device__ static uint32_t smem(int nmt) { return bar(nmt) + 256 + 1024; }
 };
 
@@ -573,7 +604,8 @@ template <int B2P>
 __global__ void __launch_bounds__(384, 1)
 tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmZs,
-                const __grid_constant__ CUtensorMap tmKs, RsArgs a) {
+                const __grid_constant__ CUtensorMap tmKs, const __grid_constant__ CUtensorMap tmHs,
+                RsArgs a) {
     using L = RsLayout<B2P>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
@@ -595,8 +627,9 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
 
     const Problem &p = a.p;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int total = p.BH * p.b1;
-    const int first = blockIdx.x * a.bpc;
+    // (head, block) items of the heads that the unit range touches
+    const int total = p.head_end() * p.b1;
+    const int first = p.head_begin() * p.b1 + blockIdx.x * a.bpc;
     const int nblk = min(a.bpc, total - first);
     const int nitems = nblk * nmt;
     const int tb2 = p.tiles * p.b2;
@@ -735,45 +768,83 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
             if (!wait_warp(s_full + (i & 1), (i >> 1) & 1, w)) break;
             tc_fence_after();
             const uint32_t tS = tmem + lane_off + (i & 1) * 128;
+            // the row's B2P logits: all TMEM loads in flight together, one wait
             float x[B2P];
-            float mx = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < B2P / 16; c++) {
-                uint32_t raw[16];
-                tmem_ld16(tS + c * 16, raw);
-                tmem_wait_ld();
+            for (int c = 0; c < B2P / 16; c++) tmem_ld16f(tS + c * 16, &x[c * 16]);
+            tmem_wait_ld();
+            if (p.b2 < B2P) {   // padded key columns (uniform branch)
+                // a large finite logit, not -inf: its probability is exactly 0 and
+                // 0 * x stays finite in the entropy sum (no per-column condition)
 #pragma unroll
-                for (int k = 0; k < 16; k++) {
-                    const int col = c * 16 + k;
-                    x[col] = col < p.b2 ? __uint_as_float(raw[k]) * a.c_log2 : -INFINITY;
-                    mx = fmaxf(mx, x[col]);
+                for (int col = 0; col < B2P; col++) x[col] = col < p.b2 ? x[col] : -1e30f;
+            }
+            // maximum with four independent chains
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int k = 0; k < B2P / 2; k++) mx4[k & 3] = fmax3(mx4[k & 3], x[2 * k], x[2 * k + 1]);
+            const float mxr = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+            // base-2 exponentials of c * (x - max), packed in pairs; the row sum and
+            // sum p * x (for the entropy) accumulate in four packed chains each
+            const uint64_t c2 = f2_pack(a.c_log2, a.c_log2);
+            const uint64_t nm2 = f2_pack(-mxr * a.c_log2, -mxr * a.c_log2);
+            uint64_t l2[4] = {0, 0, 0, 0}, e2[4] = {0, 0, 0, 0};
+            uint64_t pp[B2P / 2];
+#pragma unroll
+            for (int k = 0; k < B2P / 2; k++) {
+                const uint64_t xs = f2_mul(f2_pack(x[2 * k], x[2 * k + 1]), c2);   // log2 units
+                float d0, d1;
+                f2_unpack(f2_add(xs, nm2), d0, d1);
+                pp[k] = f2_pack(fast_exp2(d0), fast_exp2(d1));
+                l2[k & 3] = f2_add(l2[k & 3], pp[k]);
+                e2[k & 3] = f2_fma(pp[k], xs, e2[k & 3]);
+            }
+            float la, lb, ea, eb;
+            f2_unpack(f2_add(f2_add(l2[0], l2[1]), f2_add(l2[2], l2[3])), la, lb);
+            f2_unpack(f2_add(f2_add(e2[0], e2[1]), f2_add(e2[2], e2[3])), ea, eb);
+            const float l = la + lb, inv = 1.f / l;
+            const int row = mt * 128 + r;
+            // entropy of the row in log2 units, log2(sum 2^x) - E_R[x] = H / ln 2,
+            // stored divided by c_log2 = s log2(e) (the L-step's logits are
+            // S * c_log2) as a bfloat16 pair hi + lo in the row's entropy panel
+            {
+                const float hp = (mxr * a.c_log2 + log2f(l) - (ea + eb) * inv) / a.c_log2;
+                const __nv_bfloat16 hi = __float2bfloat16_rn(hp);
+                const __nv_bfloat16 lo = __float2bfloat16_rn(hp - __bfloat162float(hi));
+                const uint32_t pair = (uint32_t)__bfloat16_as_ushort(hi) |
+                                      ((uint32_t)__bfloat16_as_ushort(lo) << 16);
+                // the warp's 32 panel rows (32 B each) leave in one TMA store, which
+                // clips the rows past t*b2; the previous item's store must have
+                // finished reading the staging first
+                uint8_t *hs = sm + L::hstg(nmt) + wq * 1024;
+                if (lane == 0) tma_store_wait_read_all();
+                __syncwarp();
+                *reinterpret_cast<uint4 *>(hs + lane * 32) = make_uint4(pair, 0u, 0u, 0u);
+                *reinterpret_cast<uint4 *>(hs + lane * 32 + 16) = make_uint4(0u, 0u, 0u, 0u);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_4d(&tmHs, hs, 0, up, mt * 128 + wq * 32, bh);
+                    tma_store_commit();
                 }
             }
-            float l = 0.f, e = 0.f;
-#pragma unroll
-            for (int col = 0; col < B2P; col++) {
-                const float pr = fast_exp2(x[col] - mx);
-                l += pr;
-                e += col < p.b2 ? pr * x[col] : 0.f;
-                x[col] = pr;
-            }
-            const float inv = 1.f / l;
-            const int row = mt * 128 + r;
-            // entropy of the row in log2 units (the L-step works in base 2):
-            // log2(sum 2^x) - E_R[x] = H / ln 2
-            if (row < tb2) a.hent[((int64_t)bh * tb2 + row) * a.hstride + up] = mx + log2f(l) - e * inv;
+            const uint64_t inv2 = f2_pack(inv, inv);
 #pragma unroll
             for (int c = 0; c < B2P / 16; c++) {
                 uint32_t pk[8];
 #pragma unroll
-                for (int k = 0; k < 8; k++)
-                    pk[k] = pack_bf16(x[c * 16 + 2 * k] * inv, x[c * 16 + 2 * k + 1] * inv);
+                for (int k = 0; k < 8; k++) {
+                    float p0, p1;
+                    f2_unpack(f2_mul(pp[c * 8 + k], inv2), p0, p1);
+                    pk[k] = pack_bf16(p0, p1);
+                }
                 tmem_st8(tS + c * 8, pk);
             }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive_warp(p_full + (i & 1));
         }
+        if (lane == 0) tma_store_wait_all();   // the entropy stores complete before exit
     } else if (warp >= 8) {
         // ---------------- epilogue: Z and Ktil rows -> bf16 -> staging -> TMA store
         const int wq = warp & 3;
@@ -855,20 +926,18 @@ EncodeTiledFn encode_fn() {
 
 // bf16 tensor map, 128-byte swizzle; dims innermost first, strides in bytes for dims 1..rank-1
 bool make_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims,
-              const uint64_t *strides, const uint32_t *box) {
+              const uint64_t *strides, const uint32_t *box,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base),
-              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int b2_padded(int b2) { return (b2 + 15) / 16 * 16; }
-// entropy rows start on 16-byte boundaries (bulk copies); the L-step's copy of
-// the last chunk of a row runs up to 512 bytes past it, hence the tail slack
-int h_stride(const Problem &p) { return (p.b1 + 3) / 4 * 4; }
+
 int qbar_tiles(const Problem &p) { return (p.tiles * p.b2 + 127) / 128; }
 size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -885,7 +954,7 @@ uint32_t rstep_smem(int b2p, int nmt) {
 
 struct TcWorkspace {
     __nv_bfloat16 *qbar, *ktil, *z;
-    float *hent;
+    uint4 *hx;   // [BH][t][b2][b1] rows of 32 bytes
 };
 
 TcWorkspace carve(const Problem &p, void *base) {
@@ -899,7 +968,7 @@ TcWorkspace carve(const Problem &p, void *base) {
     c += al256(kz);
     ws.z = (__nv_bfloat16 *)c;
     c += al256(kz);
-    ws.hent = (float *)c;
+    ws.hx = (uint4 *)c;
     return ws;
 }
 
@@ -913,7 +982,8 @@ cudaError_t launch_rstep(const CUtensorMap *maps, const RsArgs &a, int grid, cud
     const uint32_t smem = RsLayout<B2P>::smem(a.nmt);
     cudaError_t e = set_smem(tc_rstep_kernel<B2P>, smem);
     if (e != cudaSuccess) return e;
-    tc_rstep_kernel<B2P><<<grid, 384, smem, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], a);
+    tc_rstep_kernel<B2P><<<grid, 384, smem, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
+                                                   maps[5], a);
     return cudaGetLastError();
 }
 
@@ -932,7 +1002,7 @@ bool sm100_supports(const Problem &p, monarch_dtype dtype) {
     // TMA coordinates are 32-bit: every row index must fit
     if ((int64_t)p.BH * p.tiles * p.N + 256 >= (1LL << 31)) return false;
     if ((int64_t)p.BH * qbar_tiles(p) * 128 >= (1LL << 31)) return false;
-    if ((int64_t)p.BH * p.tiles * p.b2 * h_stride(p) + 128 >= (1LL << 31)) return false;
+
     if (encode_fn() == nullptr) return false;
     return true;
 }
@@ -941,9 +1011,8 @@ size_t sm100_workspace_bytes(const Problem &p, bool &overflow) {
     overflow = false;
     const size_t mpad = (size_t)qbar_tiles(p) * 128;
     const size_t kz = (size_t)p.BH * p.tiles * p.N * kD * 2;
-    const size_t hrows = (size_t)p.BH * p.tiles * p.b2;
-    return al256((size_t)p.BH * mpad * kD * 2) + 2 * al256(kz) +
-           al256(hrows * h_stride(p) * 4 + 512);
+    const size_t hx = (size_t)p.BH * p.tiles * p.N * 32;
+    return al256((size_t)p.BH * mpad * kD * 2) + 2 * al256(kz) + al256(hx);
 }
 
 cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const void *v,
@@ -957,14 +1026,14 @@ cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const 
     {
         const int nchunk = (p.b2 * kD / 8 + 127) / 128;
         ProfileScope scope(K_TC_QBAR, stream);
-        tc_qbar_kernel<<<p.BH * p.tiles * nchunk, 128, 0, stream>>>(
+        tc_qbar_kernel<<<(p.head_end() - p.head_begin()) * p.tiles * nchunk, 128, 0, stream>>>(
             (const __nv_bfloat16 *)q, ws.qbar, p, mpad);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     // S2
     {
-        CUtensorMap maps[5];
+        CUtensorMap maps[6];
         const uint64_t dq[2] = {(uint64_t)kD, (uint64_t)p.BH * mpad};
         const uint64_t dkv[2] = {(uint64_t)kD, (uint64_t)p.BH * p.N};
         const uint64_t s2[1] = {kD * 2};
@@ -979,11 +1048,17 @@ cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const 
             !make_map(&maps[2], v, 2, dkv, s2, bkv) || !make_map(&maps[3], ws.z, 4, dst, sst, bst) ||
             !make_map(&maps[4], ws.ktil, 4, dst, sst, bst))
             return cudaErrorInvalidValue;
-        const int total = p.BH * p.b1;
+        // entropy panels, [bh][t*b2 rows][b1][16], stored 32 rows x 32 B per warp
+        const uint64_t dhx[4] = {16, (uint64_t)p.b1, (uint64_t)p.tiles * p.b2, (uint64_t)p.BH};
+        const uint64_t shx[3] = {32, (uint64_t)p.b1 * 32, (uint64_t)p.tiles * p.b2 * p.b1 * 32};
+        const uint32_t bhx[4] = {16, 1, 32, 1};
+        if (!make_map(&maps[5], ws.hx, 4, dhx, shx, bhx, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+        const int total = (p.head_end() - p.head_begin()) * p.b1;
         const int sms = sm_count();
         const int bpc = (total + sms - 1) / sms;
         const int grid = (total + bpc - 1) / bpc;
-        RsArgs a{p, nmt, mpad, bpc, h_stride(p), c_log2, ws.hent, status, wait_limit, stall};
+        RsArgs a{p, nmt, mpad, bpc, c_log2, status, wait_limit, stall};
         ProfileScope scope(K_TC_RSTEP, stream);
         cudaError_t e = cudaErrorInvalidValue;
         switch (b2p) {
@@ -1000,27 +1075,31 @@ cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const 
     }
     // S3
     {
-        CUtensorMap maps[3];
+        CUtensorMap maps[4];
         const uint64_t dq[3] = {(uint64_t)kD, (uint64_t)p.b2, (uint64_t)p.BH * p.b1};
         const uint64_t sq[2] = {kD * 2, (uint64_t)p.b2 * kD * 2};
         const uint32_t bq[3] = {64, 1, 128};
         const uint64_t dk[2] = {(uint64_t)kD, (uint64_t)p.BH * p.tiles * p.N};
         const uint64_t sk[1] = {kD * 2};
         const uint32_t bk[2] = {64, 128};
+        const uint64_t dh[2] = {16, (uint64_t)p.BH * p.tiles * p.N};
+        const uint64_t sh[1] = {32};
+        const uint32_t bh[2] = {16, 128};
         if (!make_map(&maps[0], q, 3, dq, sq, bq) || !make_map(&maps[1], ws.ktil, 2, dk, sk, bk) ||
-            !make_map(&maps[2], ws.z, 2, dk, sk, bk))
+            !make_map(&maps[2], ws.z, 2, dk, sk, bk) ||
+            !make_map(&maps[3], ws.hx, 2, dh, sh, bh, CU_TENSOR_MAP_SWIZZLE_32B))
             return cudaErrorInvalidValue;
         const int nq_max = tile_max_rows(p.b1, p.tiles);
         const int npairs = ((nq_max + 127) / 128 + 1) / 2;
-        const int nprob = p.BH * p.tiles * p.b2 * npairs;
-        LsArgs a{p, (p.b1 + 127) / 128, npairs, nprob, h_stride(p), c_log2, ws.hent,
-                 (__nv_bfloat16 *)out,
-                 status, wait_limit, stall};
+        const int nprob = (p.unit_end - p.unit_begin) * p.b2 * npairs;
+        LsArgs a{p, (p.b1 + 127) / 128, npairs, nprob, p.unit_begin * p.b2 * npairs, c_log2,
+                 (__nv_bfloat16 *)out, status, wait_limit, stall};
         cudaError_t e = set_smem(tc_lstep_kernel, ls::kSmem);
         if (e != cudaSuccess) return e;
         const int grid = nprob < sm_count() ? nprob : sm_count();
         ProfileScope scope(K_TC_LSTEP, stream);
-        tc_lstep_kernel<<<grid, ls::kThreads, ls::kSmem, stream>>>(maps[0], maps[1], maps[2], a);
+        tc_lstep_kernel<<<grid, ls::kThreads, ls::kSmem, stream>>>(maps[0], maps[1], maps[2],
+                                                                   maps[3], a);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

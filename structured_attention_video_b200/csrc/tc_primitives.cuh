@@ -346,6 +346,17 @@ __device__ __forceinline__ void mma8_ts_mn128(uint32_t d_tmem, uint32_t a_tmem, 
         : "memory");
 }
 
+// One K-step (K = 16) of D += A B^T, both operands one 32-byte-swizzled K atom.
+__device__ __forceinline__ void mma1_ss_acc(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                            uint32_t idesc) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, 1;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc)
+        : "memory");
+}
+
 // Warpgroup register reallocation (all four warps of a warpgroup execute the
 // same call): dec returns registers to the CTA's pool, inc waits until the pool
 // can give the warp N registers per thread.  The pool is what the block was
@@ -407,6 +418,15 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
           "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
 }
+__device__ __forceinline__ void tmem_ld16f(uint32_t taddr, float *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=f"(r[0]), "=f"(r[1]), "=f"(r[2]), "=f"(r[3]), "=f"(r[4]), "=f"(r[5]), "=f"(r[6]),
+          "=f"(r[7]), "=f"(r[8]), "=f"(r[9]), "=f"(r[10]), "=f"(r[11]), "=f"(r[12]),
+          "=f"(r[13]), "=f"(r[14]), "=f"(r[15])
+        : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -450,6 +470,19 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo,
     d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
     d |= (uint64_t)1 << 46;
     d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// The same for the 32-byte swizzle (layout type 6): K-major rows of 16
+// bfloat16 (32 bytes), 8-row atoms of 256 bytes (SBO); the tile base must be
+// 256-byte aligned.
+__device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;                       // LBO: unused for one K atom
+    d |= (uint64_t)((256u >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)6 << 61;
     return d;
 }
 

@@ -241,6 +241,44 @@ def test_entry_points_agree(tiny64):
     assert torch.equal(oh, ref.cpu())
 
 
+@pytest.mark.parametrize("name,dtype,kw,cuts", [
+    ("480p_chunk", "bf16", dict(H=4, tiles=3), (0, 5, 7, 12)),     # tensor-core path
+    ("tiny", "f32", dict(tiles=5, iters=2), (0, 3, 4, 10)),         # generic path, iters > 1
+])
+def test_unit_ranges_partition_the_output(name, dtype, kw, cuts):
+    """Calls over a partition of the (head, tile) units give the full call's output
+    bit for bit, and a call writes no row outside its units."""
+    wl = synth.WORKLOADS[name].replace(dtype=dtype, **kw)
+    q64, k64, v64 = (synth.round_to_dtype(x, dtype) for x in synth.make_inputs(wl))
+    q, k, v = (to_torch(x, dtype) for x in (q64, k64, v64))
+    dt = _lib.F32 if dtype == "f32" else _lib.BF16
+    shape = (wl.B, wl.H, wl.f, wl.h, wl.w, wl.d, wl.b1, wl.b2, wl.tiles, wl.iters)
+    need = _lib.monarch_attn_workspace_bytes(*shape, dt)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    full = run(wl, q, k, v)
+    assert cuts[-1] == wl.B * wl.H * wl.tiles
+    parts = torch.full_like(q, float("nan"))
+    for b, e in zip(cuts, cuts[1:]):
+        one = torch.full_like(q, float("nan"))
+        for out in (parts, one):
+            assert _lib.monarch_attn_fwd_units_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                  out.data_ptr(), *shape, dt, b, e,
+                                                  ws.data_ptr(), need, None) == 0
+        torch.cuda.synchronize()
+        mine = torch.zeros(q.shape[:3], dtype=torch.bool)
+        for unit in range(b, e):
+            bh, g = divmod(unit, wl.tiles)
+            rows = oracle.tile_rows(wl.b1, wl.tiles, g)[:, None] * wl.b2 + np.arange(wl.b2)
+            mine[bh // wl.H, bh % wl.H, torch.as_tensor(rows.ravel())] = True
+        written = ~torch.isnan(one.float()).any(dim=-1).cpu()
+        assert torch.equal(written, mine)
+    assert _lib.monarch_last_device_status(None) == 0
+    assert torch.equal(parts, full)
+    assert _lib.monarch_attn_fwd_units_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                          parts.data_ptr(), *shape, dt, 0, cuts[-1] + 1,
+                                          ws.data_ptr(), need, None) == 2
+
+
 def test_device_entry_points_reject_bad_buffers(tiny64):
     q = to_torch(tiny64[0], "f32")
     shape = (1, 2, 3, 8, 8, 32, 24, 8, 1, 1)
