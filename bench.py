@@ -235,7 +235,9 @@ def kernel_roofline(name: str, ms_per_launch: float, wl: synth.Workload, peaks, 
         flops = 6.0 * t * N * wl.b2 * d * BH
     elif name.endswith("lstep_kernel"):
         flops = 4.0 * N * wl.b1 * d * BH
-    elif name == "qbar_weighted_kernel":
+    elif name == "tc_lstat_kernel":       # logits only (no products with Z)
+        flops = 2.0 * N * wl.b1 * d * BH
+    elif name in ("qbar_weighted_kernel", "tc_qagg_kernel"):
         flops = 4.0 * N * wl.b1 * d * BH
     else:
         flops = None

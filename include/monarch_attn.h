@@ -173,6 +173,36 @@ MONARCH_API monarch_status monarch_attn_fwd_units_ws(const void *q, const void *
                                                      size_t ws_bytes, monarch_stream_t stream);
 
 /*
+ * Queries of a chunk of frames against keys and values that also hold earlier
+ * frames (a key/value cache), as in chunk-by-chunk autoregressive video
+ * generation (the Self-Forcing setting of the MonarchRT pages: summary page,
+ * "Setup"; explainer page, the autoregressive models it evaluates).
+ *   q, out   [B][H][fq*h*w][d]: the chunk's queries and output.
+ *   k, v     [B][H][fk*h*w][d]: keys and values of fk >= 1 frames (the cached
+ *            frames followed by the chunk's own, or any other order).
+ *   b1*b2 = fq*h*w, b1k*b2 = fk*h*w: b2 tokens per block row on both sides
+ *            (aligned: b2 = w, b1 = fq*h, b1k = fk*h); the tiles split the b1
+ *            query block rows.
+ * The Monarch factors become L_v of b1 x b1k and R_{u',g} of b2 x b2 for the b1k
+ * key blocks; every step is that of monarch_attn_fwd with the key blocks
+ * running over [b1k].  fq = fk with the same tensors is monarch_attn_fwd.
+ * Workspace: monarch_attn_kv_workspace_bytes (0 if the arguments fail
+ * validation).  Errors and ownership as monarch_attn_fwd_ws.
+ * monarch_attn_kv_path reports the kernel family as monarch_attn_path does.
+ */
+MONARCH_API size_t monarch_attn_kv_workspace_bytes(int B, int H, int fq, int fk, int h, int w,
+                                                   int d, int b1, int b1k, int b2, int tiles,
+                                                   int iters, monarch_dtype dtype);
+MONARCH_API int monarch_attn_kv_path(int B, int H, int fq, int fk, int h, int w, int d, int b1,
+                                     int b1k, int b2, int tiles, int iters, monarch_dtype dtype);
+MONARCH_API monarch_status monarch_attn_fwd_kv_ws(const void *q, const void *k, const void *v,
+                                                  void *out, int B, int H, int fq, int fk, int h,
+                                                  int w, int d, int b1, int b1k, int b2,
+                                                  int tiles, int iters, monarch_dtype dtype,
+                                                  void *workspace, size_t ws_bytes,
+                                                  monarch_stream_t stream);
+
+/*
  * Forward pass on HOST buffers: q, k, v, out are host pointers (pinned memory
  * gives full PCIe bandwidth; pageable memory works but is slower).  Device
  * copies of the inputs and output and the workspace are taken with

@@ -81,47 +81,51 @@ int oracle_index_maps(int f, int h, int w, int b1, int b2, int tiles,
     return ORACLE_OK;
 }
 
-static size_t workspace_doubles(int d, int b1, int b2, int tiles)
+static size_t workspace_doubles(int d, int b1, int b1k, int b2, int tiles)
 {
     int nq_max = (b1 + tiles - 1) / tiles + 1;
-    int mx = b1 > b2 ? b1 : b2;
-    return (size_t)nq_max * b1 + (size_t)b1 * b2 + 2 * (size_t)b1 * d + b1 + d + mx;
+    int mx = b1k > b2 ? b1k : b2;
+    return (size_t)nq_max * b1k + (size_t)b1k * b2 + 2 * (size_t)b1k * d + b1k + d + mx;
 }
 
 /*
  * One (tile g, column c) problem of one head: runs `half_steps` alternating
  * half-steps (R, L, R, L, ...) and writes y for the rows (u, c), u in T_g.
- * q, k, v, y: one head, [N][d] row-major.
- * L_out (optional) [b2][b1][b1]: L_c[u][u'] for u in T_g.
- * R_out (optional) [b1][tiles][b2][b2]: R_{u',g}[c][:].
+ * q, y: one head, [b1*b2][d] row-major (the queries; b1 block rows split
+ * into the tiles); k, v: one head, [b1k*b2][d] (the keys and values in b1k
+ * blocks of b2 tokens).  b1k = b1 is self-attention over one clip; b1k > b1
+ * is the chunked setting in which the queries of the current chunk of frames
+ * attend to a cache of earlier frames as well as to their own.
+ * L_out (optional) [b2][b1][b1k]: L_c[u][u'] for u in T_g.
+ * R_out (optional) [b1k][tiles][b2][b2]: R_{u',g}[c][:].
  */
 static void solve_problem(const double *q, const double *k, const double *v, double *y,
-                          int d, int b1, int b2, int tiles, int g, int c, int half_steps,
-                          double *L_out, double *R_out, double *ws)
+                          int d, int b1, int b1k, int b2, int tiles, int g, int c,
+                          int half_steps, double *L_out, double *R_out, double *ws)
 {
     const double s = 1.0 / sqrt((double)d);
     const int u0 = tile_first_row(g, b1, tiles), u1 = tile_first_row(g + 1, b1, tiles);
     const int nq = u1 - u0;
-    double *L = ws;                          /* [nq][b1]  L_c[u][u'], u in T_g */
-    double *R = L + (size_t)nq * b1;         /* [b1][b2]  R_{u',g}[c][:]       */
-    double *Kt = R + (size_t)b1 * b2;        /* [b1][d]   Ktil[g][c][u']       */
-    double *Z = Kt + (size_t)b1 * d;         /* [b1][d]   Z[g][c][u']          */
-    double *H = Z + (size_t)b1 * d;          /* [b1]      entropy of R row     */
-    double *qbar = H + b1;                   /* [d]                            */
-    double *logit = qbar + d;                /* [max(b1, b2)]                  */
+    double *L = ws;                          /* [nq][b1k]  L_c[u][u'], u in T_g */
+    double *R = L + (size_t)nq * b1k;        /* [b1k][b2]  R_{u',g}[c][:]       */
+    double *Kt = R + (size_t)b1k * b2;       /* [b1k][d]   Ktil[g][c][u']       */
+    double *Z = Kt + (size_t)b1k * d;        /* [b1k][d]   Z[g][c][u']          */
+    double *H = Z + (size_t)b1k * d;         /* [b1k]      entropy of R row     */
+    double *qbar = H + b1k;                  /* [d]                             */
+    double *logit = qbar + d;                /* [max(b1k, b2)]                  */
 
-    for (size_t i = 0; i < (size_t)nq * b1; i++)
-        L[i] = 1.0 / b1;
+    for (size_t i = 0; i < (size_t)nq * b1k; i++)
+        L[i] = 1.0 / b1k;
 
     for (int step = 0; step < half_steps; step++) {
         if ((step & 1) == 0) {
             /* R-step: every block u' of tile g, row c of R_{u',g} */
-            for (int up = 0; up < b1; up++) {
+            for (int up = 0; up < b1k; up++) {
                 double wsum = 0.0;
                 for (int j = 0; j < d; j++)
                     qbar[j] = 0.0;
                 for (int u = u0; u < u1; u++) {
-                    double wgt = L[(size_t)(u - u0) * b1 + up];
+                    double wgt = L[(size_t)(u - u0) * b1k + up];
                     const double *qr = q + ((int64_t)u * b2 + c) * d;
                     wsum += wgt;
                     for (int j = 0; j < d; j++)
@@ -169,7 +173,7 @@ static void solve_problem(const double *q, const double *k, const double *v, dou
             for (int u = u0; u < u1; u++) {
                 const double *qr = q + ((int64_t)u * b2 + c) * d;
                 double mx = -INFINITY;
-                for (int up = 0; up < b1; up++) {
+                for (int up = 0; up < b1k; up++) {
                     double acc = 0.0;
                     for (int j = 0; j < d; j++)
                         acc += qr[j] * Kt[(size_t)up * d + j];
@@ -178,11 +182,11 @@ static void solve_problem(const double *q, const double *k, const double *v, dou
                         mx = logit[up];
                 }
                 double sum = 0.0;
-                for (int up = 0; up < b1; up++)
+                for (int up = 0; up < b1k; up++)
                     sum += exp(logit[up] - mx);
                 double lse = mx + log(sum);
-                for (int up = 0; up < b1; up++)
-                    L[(size_t)(u - u0) * b1 + up] = exp(logit[up] - lse);
+                for (int up = 0; up < b1k; up++)
+                    L[(size_t)(u - u0) * b1k + up] = exp(logit[up] - lse);
             }
         }
     }
@@ -192,18 +196,18 @@ static void solve_problem(const double *q, const double *k, const double *v, dou
         double *yr = y + ((int64_t)u * b2 + c) * d;
         for (int j = 0; j < d; j++) {
             double acc = 0.0;
-            for (int up = 0; up < b1; up++)
-                acc += L[(size_t)(u - u0) * b1 + up] * Z[(size_t)up * d + j];
+            for (int up = 0; up < b1k; up++)
+                acc += L[(size_t)(u - u0) * b1k + up] * Z[(size_t)up * d + j];
             yr[j] = acc;
         }
     }
 
     if (L_out)
         for (int u = u0; u < u1; u++)
-            for (int up = 0; up < b1; up++)
-                L_out[((int64_t)c * b1 + u) * b1 + up] = L[(size_t)(u - u0) * b1 + up];
+            for (int up = 0; up < b1k; up++)
+                L_out[((int64_t)c * b1 + u) * b1k + up] = L[(size_t)(u - u0) * b1k + up];
     if (R_out)
-        for (int up = 0; up < b1; up++)
+        for (int up = 0; up < b1k; up++)
             for (int vp = 0; vp < b2; vp++)
                 R_out[(((int64_t)up * tiles + g) * b2 + c) * b2 + vp] = R[(size_t)up * b2 + vp];
 }
@@ -229,7 +233,7 @@ int oracle_monarch_attn(const double *q, const double *k, const double *v, doubl
     if (BH < 1 || check_shape(N, d, b1, b2, tiles, half_steps))
         return ORACLE_EINVAL;
     const int64_t nprob = (int64_t)BH * tiles * b2;
-    const size_t wsz = workspace_doubles(d, b1, b2, tiles);
+    const size_t wsz = workspace_doubles(d, b1, b1, b2, tiles);
     int err = ORACLE_OK;
 #ifdef _OPENMP
     if (nthreads <= 0)
@@ -254,7 +258,7 @@ int oracle_monarch_attn(const double *q, const double *k, const double *v, doubl
             int g = (int)((p / b2) % tiles);
             int c = (int)(p % b2);
             size_t off = (size_t)bh * N * d;
-            solve_problem(q + off, k + off, v + off, y + off, d, b1, b2, tiles, g, c,
+            solve_problem(q + off, k + off, v + off, y + off, d, b1, b1, b2, tiles, g, c,
                           half_steps,
                           L_out ? L_out + (size_t)bh * b2 * b1 * b1 : NULL,
                           R_out ? R_out + (size_t)bh * b1 * tiles * b2 * b2 : NULL, ws);
@@ -279,7 +283,7 @@ int oracle_monarch_problems(const double *q, const double *k, const double *v, d
         if (probs[3 * i] < 0 || probs[3 * i] >= BH || probs[3 * i + 1] < 0 ||
             probs[3 * i + 1] >= tiles || probs[3 * i + 2] < 0 || probs[3 * i + 2] >= b2)
             return ORACLE_EINVAL;
-    const size_t wsz = workspace_doubles(d, b1, b2, tiles);
+    const size_t wsz = workspace_doubles(d, b1, b1, b2, tiles);
     int err = ORACLE_OK;
 #ifdef _OPENMP
     if (nthreads <= 0)
@@ -302,8 +306,58 @@ int oracle_monarch_problems(const double *q, const double *k, const double *v, d
                 continue;
             int bh = probs[3 * i], g = probs[3 * i + 1], c = probs[3 * i + 2];
             size_t off = (size_t)bh * N * d;
-            solve_problem(q + off, k + off, v + off, y + off, d, b1, b2, tiles, g, c,
+            solve_problem(q + off, k + off, v + off, y + off, d, b1, b1, b2, tiles, g, c,
                           half_steps, NULL, NULL, ws);
+        }
+        free(ws);
+    }
+    return err;
+}
+
+/*
+ * Queries of one chunk of frames against keys and values that also hold
+ * earlier frames (a cache): q, y [BH][b1*b2][d], k, v [BH][b1k*b2][d], with
+ * the b2 tokens of a block row shared by both (the video width for the
+ * aligned blocks) and b1k >= 1 key blocks.  Every step is the one above with
+ * the key blocks u' running over [b1k]; the tiles split the b1 query block
+ * rows.  L_out [BH][b2][b1][b1k] and R_out [BH][b1k][tiles][b2][b2] optional.
+ */
+int oracle_monarch_attn_kv(const double *q, const double *k, const double *v, double *y,
+                           int BH, int d, int b1, int b1k, int b2, int tiles, int half_steps,
+                           double *L_out, double *R_out, int nthreads)
+{
+    if (BH < 1 || b1k < 1 || check_shape(b1 * b2, d, b1, b2, tiles, half_steps))
+        return ORACLE_EINVAL;
+    const int64_t nprob = (int64_t)BH * tiles * b2;
+    const size_t wsz = workspace_doubles(d, b1, b1k, b2, tiles);
+    const size_t nq = (size_t)b1 * b2 * d, nk = (size_t)b1k * b2 * d;
+    int err = ORACLE_OK;
+#ifdef _OPENMP
+    if (nthreads <= 0)
+        nthreads = omp_get_max_threads();
+#pragma omp parallel num_threads(nthreads)
+#endif
+    {
+        double *ws = (double *)malloc(wsz * sizeof(double));
+        if (!ws) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            err = ORACLE_ENOMEM;
+        }
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+        for (int64_t p = 0; p < nprob; p++) {
+            if (!ws)
+                continue;
+            int bh = (int)(p / ((int64_t)tiles * b2));
+            int g = (int)((p / b2) % tiles);
+            int c = (int)(p % b2);
+            solve_problem(q + bh * nq, k + bh * nk, v + bh * nk, y + bh * nq, d, b1, b1k, b2,
+                          tiles, g, c, half_steps,
+                          L_out ? L_out + (size_t)bh * b2 * b1 * b1k : NULL,
+                          R_out ? R_out + (size_t)bh * b1k * tiles * b2 * b2 : NULL, ws);
         }
         free(ws);
     }

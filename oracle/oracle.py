@@ -44,6 +44,8 @@ def _load(path: str | None = None):
         lib.oracle_monarch_attn.restype = i
         lib.oracle_monarch_problems.argtypes = [dp, dp, dp, dp, i, i, i, i, i, i, i, i, ip, i]
         lib.oracle_monarch_problems.restype = i
+        lib.oracle_monarch_attn_kv.argtypes = [dp, dp, dp, dp, i, i, i, i, i, i, i, dp, dp, i]
+        lib.oracle_monarch_attn_kv.restype = i
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = i
         _libs[key] = lib
@@ -97,6 +99,31 @@ def monarch_attn(q, k, v, b1, b2, tiles=1, iters=1, half_steps=None, factors=Fal
                                      b2, tiles, hs, _dptr(L), _dptr(R), nthreads)
     if rc != 0:
         raise ValueError("oracle_monarch_attn failed with code %d" % rc)
+    y = y.reshape(shape)
+    if factors:
+        return y, L.reshape(shape[:-2] + L.shape[1:]), R.reshape(shape[:-2] + R.shape[1:])
+    return y
+
+
+def monarch_attn_kv(q, k, v, b1, b1k, b2, tiles=1, iters=1, half_steps=None, factors=False,
+                    nthreads=0, lib=None):
+    """Queries [..., b1*b2, d] against keys and values [..., b1k*b2, d] (a chunk of
+    frames attending to a cache that also holds earlier frames).  Returns y (and L
+    [..., b2, b1, b1k], R [..., b1k, tiles, b2, b2] if factors)."""
+    qh, shape = _heads(q)
+    kh, _ = _heads(k)
+    vh, _ = _heads(v)
+    BH, Nq, d = qh.shape
+    if Nq != b1 * b2 or kh.shape != (BH, b1k * b2, d) or vh.shape != kh.shape:
+        raise ValueError("monarch_attn_kv: shapes do not match the blocks")
+    hs = 2 * iters if half_steps is None else half_steps
+    y = np.zeros_like(qh)
+    L = np.zeros((BH, b2, b1, b1k)) if factors else None
+    R = np.zeros((BH, b1k, tiles, b2, b2)) if factors else None
+    rc = _load(lib).oracle_monarch_attn_kv(_dptr(qh), _dptr(kh), _dptr(vh), _dptr(y), BH, d, b1,
+                                           b1k, b2, tiles, hs, _dptr(L), _dptr(R), nthreads)
+    if rc != 0:
+        raise ValueError("oracle_monarch_attn_kv failed with code %d" % rc)
     y = y.reshape(shape)
     if factors:
         return y, L.reshape(shape[:-2] + L.shape[1:]), R.reshape(shape[:-2] + R.shape[1:])

@@ -34,6 +34,9 @@ SIGNATURES = {
     "monarch_attn_workspace_bytes": (_SHAPE + [_i], _sz),
     "monarch_attn_fwd_ws": ([_vp, _vp, _vp, _vp] + _SHAPE + [_i, _vp, _sz, _vp], _i),
     "monarch_attn_fwd_host": ([_vp, _vp, _vp, _vp] + _SHAPE + [_i, _vp], _i),
+    "monarch_attn_kv_workspace_bytes": ([_i] * 12 + [_i], _sz),
+    "monarch_attn_kv_path": ([_i] * 12 + [_i], _i),
+    "monarch_attn_fwd_kv_ws": ([_vp, _vp, _vp, _vp] + [_i] * 12 + [_i, _vp, _sz, _vp], _i),
     "monarch_attn_fwd_units_ws": ([_vp, _vp, _vp, _vp] + _SHAPE + [_i, _i, _i, _vp, _sz, _vp], _i),
     "monarch_attn_fwd_noalloc": ([_vp, _vp, _vp, _vp] + _SHAPE + [_i, _vp], _i),
     "monarch_index_maps": ([_i] * 6 + [_ip, _ip, _ip, _ip], _i),
@@ -80,6 +83,21 @@ def monarch_attn_fwd_ws(q, k, v, out, B, H, f, h, w, d, b1, b2, tiles, iters, dt
                         ws_bytes, stream):
     return _lib.monarch_attn_fwd_ws(q, k, v, out, B, H, f, h, w, d, b1, b2, tiles, iters, dtype,
                                     workspace, ws_bytes, stream)
+
+
+def monarch_attn_kv_workspace_bytes(B, H, fq, fk, h, w, d, b1, b1k, b2, tiles, iters, dtype):
+    return _lib.monarch_attn_kv_workspace_bytes(B, H, fq, fk, h, w, d, b1, b1k, b2, tiles, iters,
+                                                dtype)
+
+
+def monarch_attn_kv_path(B, H, fq, fk, h, w, d, b1, b1k, b2, tiles, iters, dtype):
+    return _lib.monarch_attn_kv_path(B, H, fq, fk, h, w, d, b1, b1k, b2, tiles, iters, dtype)
+
+
+def monarch_attn_fwd_kv_ws(q, k, v, out, B, H, fq, fk, h, w, d, b1, b1k, b2, tiles, iters, dtype,
+                           workspace, ws_bytes, stream):
+    return _lib.monarch_attn_fwd_kv_ws(q, k, v, out, B, H, fq, fk, h, w, d, b1, b1k, b2, tiles,
+                                       iters, dtype, workspace, ws_bytes, stream)
 
 
 def monarch_attn_fwd_units_ws(q, k, v, out, B, H, f, h, w, d, b1, b2, tiles, iters, dtype,

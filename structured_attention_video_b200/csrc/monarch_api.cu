@@ -114,8 +114,31 @@ monarch_status validate_shape(int B, int H, int f, int h, int w, int d, int b1, 
     p->scale = (float)(1.0 / sqrt((double)d));
     p->unit_begin = 0;
     p->unit_end = B * H * tiles;
+    p->Nk = p->N;
+    p->b1k = b1;
     return MONARCH_OK;
 }
+
+namespace {
+
+// The chunk-and-cache form: queries over fq frames, keys and values over fk,
+// b1*b2 = fq*h*w and b1k*b2 = fk*h*w.
+monarch_status validate_kv(int B, int H, int fq, int fk, int h, int w, int d, int b1, int b1k,
+                           int b2, int tiles, int iters, monarch_dtype dtype, Problem *p) {
+    monarch_status st = validate_shape(B, H, fq, h, w, d, b1, b2, tiles, iters, dtype, p);
+    if (st != MONARCH_OK) return st;
+    if (fk < 1 || b1k < 1) return MONARCH_ERR_INVALID_ARG;
+    const int64_t Nk = (int64_t)fk * h * w;
+    if (Nk > (1LL << 30) || (int64_t)b1k * b2 != Nk) return MONARCH_ERR_SHAPE;
+    const int64_t BHt = (int64_t)B * H * tiles;
+    if (BHt * b1k * ((b2 + 7) / 8) >= (1LL << 31) || BHt * b2 * ((b1k + 7) / 8) >= (1LL << 31))
+        return MONARCH_ERR_SHAPE;
+    p->Nk = (int)Nk;
+    p->b1k = b1k;
+    return MONARCH_OK;
+}
+
+}  // namespace
 
 namespace {
 
@@ -251,6 +274,43 @@ monarch_status monarch_attn_fwd_units_ws(const void *q, const void *k, const voi
     if (unit_begin == unit_end) return MONARCH_OK;   // nothing to compute
     p.unit_begin = unit_begin;
     p.unit_end = unit_end;
+    return run_forward(p, dtype, q, k, v, out, workspace, (cudaStream_t)stream);
+}
+
+size_t monarch_attn_kv_workspace_bytes(int B, int H, int fq, int fk, int h, int w, int d,
+                                       int b1, int b1k, int b2, int tiles, int iters,
+                                       monarch_dtype dtype) {
+    Problem p;
+    if (validate_kv(B, H, fq, fk, h, w, d, b1, b1k, b2, tiles, iters, dtype, &p) != MONARCH_OK)
+        return 0;
+    bool overflow = false;
+    const size_t n = workspace_bytes_for(p, dtype, choose_path(p, dtype), overflow);
+    return overflow ? 0 : n;
+}
+
+int monarch_attn_kv_path(int B, int H, int fq, int fk, int h, int w, int d, int b1, int b1k,
+                         int b2, int tiles, int iters, monarch_dtype dtype) {
+    Problem p;
+    if (validate_kv(B, H, fq, fk, h, w, d, b1, b1k, b2, tiles, iters, dtype, &p) != MONARCH_OK)
+        return -1;
+    return choose_path(p, dtype);
+}
+
+monarch_status monarch_attn_fwd_kv_ws(const void *q, const void *k, const void *v, void *out,
+                                      int B, int H, int fq, int fk, int h, int w, int d, int b1,
+                                      int b1k, int b2, int tiles, int iters, monarch_dtype dtype,
+                                      void *workspace, size_t ws_bytes, monarch_stream_t stream) {
+    if (!q || !k || !v || !out || !workspace) return MONARCH_ERR_INVALID_ARG;
+    Problem p;
+    monarch_status st = validate_kv(B, H, fq, fk, h, w, d, b1, b1k, b2, tiles, iters, dtype, &p);
+    if (st != MONARCH_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        ((uintptr_t)workspace & 255u))
+        return MONARCH_ERR_ALIGN;
+    bool overflow = false;
+    const size_t need = workspace_bytes_for(p, dtype, choose_path(p, dtype), overflow);
+    if (overflow) return MONARCH_ERR_SHAPE;
+    if (ws_bytes < need) return MONARCH_ERR_NO_MEMORY;
     return run_forward(p, dtype, q, k, v, out, workspace, (cudaStream_t)stream);
 }
 
@@ -403,7 +463,8 @@ const char *monarch_profile_kernel_name(int k) {
     static const char *names[K_COUNT] = {"qbar_mean_kernel",     "rstep_kernel",
                                          "lstep_kernel",         "qbar_weighted_kernel",
                                          "tc_qbar_kernel",       "tc_rstep_kernel",
-                                         "tc_lstep_kernel"};
+                                         "tc_lstep_kernel",      "tc_lstat_kernel",
+                                         "tc_qagg_kernel"};
     return (k >= 0 && k < K_COUNT) ? names[k] : nullptr;
 }
 

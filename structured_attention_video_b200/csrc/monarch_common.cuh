@@ -43,6 +43,10 @@ struct Problem {
     // [unit_begin, unit_end); every unit is independent from the aggregated
     // query to its output rows (all of them by default)
     int unit_begin, unit_end;
+    // keys and values: Nk = b1k * b2 tokens in b1k blocks (Nk = N, b1k = b1 for
+    // self-attention over one clip; more when the queries of a chunk of frames
+    // also attend to a cache of earlier frames)
+    int Nk, b1k;
     __host__ __device__ int head_begin() const { return unit_begin / tiles; }
     __host__ __device__ int head_end() const { return (unit_end + tiles - 1) / tiles; }
 };
@@ -65,7 +69,9 @@ enum KernelId {
     K_TC_QBAR = 4,        // S1, tensor-core path
     K_TC_RSTEP = 5,       // S2, tensor-core path
     K_TC_LSTEP = 6,       // S3, tensor-core path
-    K_COUNT = 7
+    K_TC_LSTAT = 7,       // S3 row statistics of the iterations before the last (tensor-core)
+    K_TC_QAGG = 8,        // S4 re-aggregated queries (tensor-core)
+    K_COUNT = 9
 };
 
 // Brackets one kernel launch with CUDA events while profiling is enabled.
@@ -139,10 +145,10 @@ monarch_status validate_shape(int B, int H, int f, int h, int w, int d, int b1, 
 
 // Generic (SIMT) path: float32 intermediates.
 struct GenericWorkspace {
-    float *qbar;   // iters == 1: [BH][t][b2][d];  iters > 1: [BH][t][b2][b1][d]
-    float *ktil;   // [BH][t][b2][b1][d]   Ktil[g][v][u'] = sum_v' R_{u',g}[v,v'] k_(u',v')
-    float *z;      // [BH][t][b2][b1][d]   Z[g][v][u']    = sum_v' R_{u',g}[v,v'] v_(u',v')
-    float *hent;   // [BH][t][b2][b1]      entropy of R_{u',g}[v,:]
+    float *qbar;   // iters == 1: [BH][t][b2][d];  iters > 1: [BH][t][b2][b1k][d]
+    float *ktil;   // [BH][t][b2][b1k][d]  Ktil[g][v][u'] = sum_v' R_{u',g}[v,v'] k_(u',v')
+    float *z;      // [BH][t][b2][b1k][d]  Z[g][v][u']    = sum_v' R_{u',g}[v,v'] v_(u',v')
+    float *hent;   // [BH][t][b2][b1k]     entropy of R_{u',g}[v,:]
     float *lse;    // [BH][N]              row log-sum-exp of the L-step (iters > 1)
 };
 

@@ -71,11 +71,11 @@ rstep_kernel(const T *__restrict__ k, const T *__restrict__ v, const float *__re
     float *sv = sk + KC * DS;     // [KC][DS]
 
     const int nvg = (p.b2 + GW - 1) / GW;
-    int64_t bid = blockIdx.x + (int64_t)p.unit_begin * p.b1 * nvg;   // from the first unit
+    int64_t bid = blockIdx.x + (int64_t)p.unit_begin * p.b1k * nvg;   // from the first unit
     const int vg = (int)(bid % nvg);
     bid /= nvg;
-    const int up = (int)(bid % p.b1);
-    bid /= p.b1;
+    const int up = (int)(bid % p.b1k);   // key block
+    bid /= p.b1k;
     const int g = (int)(bid % p.tiles);
     const int bh = (int)(bid / p.tiles);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -87,7 +87,7 @@ rstep_kernel(const T *__restrict__ k, const T *__restrict__ v, const float *__re
         const float *qr = qbar + (bhg * p.b2 + vrow) * qbar_v_stride + (int64_t)up * qbar_up_stride;
         for (int j = lane; j < D; j += 32) sq[warp * D + j] = qr[j];
     }
-    const int64_t base = ((int64_t)bh * p.N + (int64_t)up * p.b2) * D;
+    const int64_t base = ((int64_t)bh * p.Nk + (int64_t)up * p.b2) * D;
     float m = -INFINITY, l = 0.f, e = 0.f;
     float acck[NJ], accv[NJ];
 #pragma unroll
@@ -133,7 +133,7 @@ rstep_kernel(const T *__restrict__ k, const T *__restrict__ v, const float *__re
     }
     if (active) {
         const float inv = 1.f / l;
-        const int64_t row = (bhg * p.b2 + vrow) * p.b1 + up;
+        const int64_t row = (bhg * p.b2 + vrow) * p.b1k + up;
 #pragma unroll
         for (int i = 0; i < NJ; i++) {
             ktil[row * D + lane + 32 * i] = acck[i] * inv;
@@ -175,14 +175,14 @@ lstep_kernel(const T *__restrict__ q, const float *__restrict__ ktil, const floa
 
     if (active)
         for (int j = lane; j < D; j += 32) sq[warp * D + j] = to_f32(q[tok * D + j]);
-    const int64_t kbase = (bhg * p.b2 + vcol) * p.b1;   // row of block u' = 0
+    const int64_t kbase = (bhg * p.b2 + vcol) * p.b1k;   // row of block u' = 0
     float m = -INFINITY, l = 0.f;
     float acc[NJ];
 #pragma unroll
     for (int i = 0; i < NJ; i++) acc[i] = 0.f;
 
-    for (int c0 = 0; c0 < p.b1; c0 += KC) {
-        const int nk = min(KC, p.b1 - c0);
+    for (int c0 = 0; c0 < p.b1k; c0 += KC) {
+        const int nk = min(KC, p.b1k - c0);
         __syncthreads();
         for (int idx = threadIdx.x; idx < nk * D; idx += blockDim.x) {
             const int r = idx / D, j = idx % D;
@@ -236,7 +236,7 @@ qbar_weighted_kernel(const T *__restrict__ q, const float *__restrict__ ktil,
     float *sq = skt + GW * D;     // [KC][DS]  query rows of the chunk
     float *sl = sq + KC * DS;     // [KC]
 
-    const int nupg = (p.b1 + GW - 1) / GW;
+    const int nupg = (p.b1k + GW - 1) / GW;
     int64_t bid = blockIdx.x + (int64_t)p.unit_begin * p.b2 * nupg;   // from the first unit
     const int upg = (int)(bid % nupg);
     bid /= nupg;
@@ -246,10 +246,10 @@ qbar_weighted_kernel(const T *__restrict__ q, const float *__restrict__ ktil,
     const int bh = (int)(bid / p.tiles);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int up = upg * GW + warp;
-    const bool active = up < p.b1;
+    const bool active = up < p.b1k;
     const int u0 = tile_begin(g, p.b1, p.tiles), u1 = tile_begin(g + 1, p.b1, p.tiles);
     const int64_t bhg = (int64_t)bh * p.tiles + g;
-    const int64_t row = (bhg * p.b2 + vcol) * p.b1 + up;
+    const int64_t row = (bhg * p.b2 + vcol) * p.b1k + up;
 
     if (active)
         for (int j = lane; j < D; j += 32) skt[warp * D + j] = ktil[row * D + j];
@@ -327,12 +327,12 @@ cudaError_t run_generic(const Problem &p, const T *q, const T *k, const T *v, T 
         ProfileScope scope(K_QBAR_MEAN, stream);
         qbar_mean_kernel<T><<<mean_blocks, 256, 0, stream>>>(q, ws.qbar, p);
     }
-    const unsigned r_blocks = (unsigned)(units * p.b1 * ((p.b2 + GW - 1) / GW));
+    const unsigned r_blocks = (unsigned)(units * p.b1k * ((p.b2 + GW - 1) / GW));
     const unsigned l_blocks = (unsigned)(units * p.b2 * ((tile_max_rows(p.b1, p.tiles) + GW - 1) / GW));
-    const unsigned w_blocks = (unsigned)(units * p.b2 * ((p.b1 + GW - 1) / GW));
+    const unsigned w_blocks = (unsigned)(units * p.b2 * ((p.b1k + GW - 1) / GW));
     for (int it = 0; it < p.iters; it++) {
         const bool last = it == p.iters - 1;
-        const int64_t vstride = it == 0 ? (int64_t)p.d : (int64_t)p.b1 * p.d;
+        const int64_t vstride = it == 0 ? (int64_t)p.d : (int64_t)p.b1k * p.d;
         const int64_t upstride = it == 0 ? 0 : (int64_t)p.d;
         {
             ProfileScope scope(K_RSTEP, stream);
@@ -369,17 +369,17 @@ cudaError_t dispatch_d(const Problem &p, const void *q, const void *k, const voi
 }  // namespace
 
 size_t generic_workspace_bytes(const Problem &p, bool &overflow) {
-    const long double big = (long double)p.BH * p.tiles * p.N * p.d * 4.0L * 4.0L;
+    const long double big = (long double)p.BH * p.tiles * p.Nk * p.d * 4.0L * 4.0L;
     overflow = big > (long double)(1ULL << 62);
     if (overflow) return 0;
-    const size_t td = (size_t)p.BH * p.tiles * p.N * p.d;   // one [BH][t][b2][b1][d] array
+    const size_t td = (size_t)p.BH * p.tiles * p.Nk * p.d;   // one [BH][t][b2][b1k][d] array
     const size_t qb = p.iters > 1 ? td : (size_t)p.BH * p.tiles * p.b2 * p.d;
-    return align256(qb * 4) + 2 * align256(td * 4) + align256((size_t)p.BH * p.tiles * p.N * 4) +
+    return align256(qb * 4) + 2 * align256(td * 4) + align256((size_t)p.BH * p.tiles * p.Nk * 4) +
            (p.iters > 1 ? align256((size_t)p.BH * p.N * 4) : 0);
 }
 
 GenericWorkspace generic_workspace_carve(const Problem &p, void *base) {
-    const size_t td = (size_t)p.BH * p.tiles * p.N * p.d;
+    const size_t td = (size_t)p.BH * p.tiles * p.Nk * p.d;
     const size_t qb = p.iters > 1 ? td : (size_t)p.BH * p.tiles * p.b2 * p.d;
     char *c = (char *)base;
     GenericWorkspace ws;
@@ -390,7 +390,7 @@ GenericWorkspace generic_workspace_carve(const Problem &p, void *base) {
     ws.z = (float *)c;
     c += align256(td * 4);
     ws.hent = (float *)c;
-    c += align256((size_t)p.BH * p.tiles * p.N * 4);
+    c += align256((size_t)p.BH * p.tiles * p.Nk * 4);
     ws.lse = p.iters > 1 ? (float *)c : nullptr;
     return ws;
 }

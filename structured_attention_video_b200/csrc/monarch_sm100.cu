@@ -159,21 +159,43 @@ constexpr uint32_t kSmem = kBar + 512;              // the base is 1024-aligned 
 static_assert(kSmem <= (uint32_t)kMaxSmem, "L-step shared memory");
 }  // namespace ls
 
+// What one launch of the L-step kernel computes (mode):
+//   kLsOut   the L-step with the output.  M side: the query rows (u, v), u in
+//            T_g (a strided gather); N side: the Ktil rows [g][v][u'] with their
+//            entropy panels; values: Z.  Writes the rows of Y.
+//   kLsStat  (iterations before the last) the same logits without the products
+//            with Z: writes each query row's log-sum-exp lam (raw logit units,
+//            i.e. of S = q.Ktil + H') as a panel row [-lam_hi, -lam_lo, 0...].
+//   kLsAgg   (query re-aggregation for the next R-step) the roles transposed:
+//            M side: the Ktil rows u' of (g, v); N side and values: the query rows
+//            (u, v), u in T_g, with the panels of -lam.  The row softmax over u of
+//            q.Ktil[u'] - lam(u) (the entropy of block u' is constant along the row
+//            and cancels) is L_v[u, u'] / sum_u L_v[u, u'], so the output row is the
+//            aggregated query qbar[g][v][u'], written to the per-block buffer
+//            [bh][u'][g*b2 + v][d] that the next R-step reads.
+enum LsMode { kLsOut = 0, kLsStat = 1, kLsAgg = 2 };
+
 struct LsArgs {
     Problem p;
-    int nchunks;    // key chunks of 128 blocks
-    int npairs;     // pairs of 128-query tiles per (g, v)
+    int mode;
+    int npairs;     // pairs of 128-row M tiles per (g, v)
     int nprob;      // problems of the unit range: units * b2 * npairs
     int prob0;      // first problem: unit_begin * b2 * npairs
+    int mpad;       // kLsAgg: rows per block of the per-block aggregated queries
     float c_log2;   // (1/sqrt(d)) * log2(e)
-    __nv_bfloat16 *out;
+    __nv_bfloat16 *out;   // kLsOut: Y; kLsAgg: aggregated queries [BH][b1][mpad][d]
+    uint4 *lam;           // kLsStat: lam panels [BH][N] rows of 32 bytes
     int *status;
     long long limit;
     int stall;      // test hook: the MMA warp first waits on a barrier nothing completes
 };
 
+// One problem: (bh, g, v) and a pair of 128-row M tiles.  M rows m = m_first +
+// t*128 + r are valid below m_end; the 3-D tensor maps take coordinates (x, y, z).
 struct LsProblem {
-    int bh, g, v, u_start, u1, key_row0;
+    int bh, g, v;
+    int m_y, m_z, m_first, m_end;   // M side: tile t starts at z = m_z + t*128
+    int n_y, n_z, nkeys, nch;       // N side: chunk j starts at z = n_z + j*128
 };
 
 __device__ __forceinline__ LsProblem ls_problem(const LsArgs &a, int unit) {
@@ -186,15 +208,41 @@ __device__ __forceinline__ LsProblem ls_problem(const LsArgs &a, int unit) {
     unit /= p.b2;
     q.g = unit % p.tiles;
     q.bh = unit / p.tiles;
-    q.u1 = tile_begin(q.g + 1, p.b1, p.tiles);
-    q.u_start = tile_begin(q.g, p.b1, p.tiles) + 256 * pair;
-    q.key_row0 = ((q.bh * p.tiles + q.g) * p.b2 + q.v) * p.b1;
+    const int u_lo = tile_begin(q.g, p.b1, p.tiles), u_hi = tile_begin(q.g + 1, p.b1, p.tiles);
+    const int slab = ((q.bh * p.tiles + q.g) * p.b2 + q.v) * p.b1k;   // Ktil row of block 0
+    if (a.mode != kLsAgg) {
+        q.m_y = q.v;
+        q.m_first = u_lo + 256 * pair;
+        q.m_z = q.bh * p.b1 + q.m_first;
+        q.m_end = u_hi;
+        q.n_y = 0;
+        q.n_z = slab;
+        q.nkeys = p.b1k;
+    } else {
+        q.m_y = 0;
+        q.m_first = 256 * pair;
+        q.m_z = slab + q.m_first;
+        q.m_end = p.b1k;
+        q.n_y = q.v;
+        q.n_z = q.bh * p.b1 + u_lo;
+        q.nkeys = u_hi - u_lo;
+    }
+    q.nch = (q.nkeys + 127) / 128;
     return q;
 }
 
+// One TMA tile load of the L-step: a 3-D gather (x, y, z) or a 2-D row box (x, z).
+__device__ __forceinline__ void ls_load(void *dst, const CUtensorMap *map, bool gather, int x,
+                                        int y, int z, uint64_t *bar) {
+    if (gather)
+        tma_load_3d(dst, map, x, y, z, bar);
+    else
+        tma_load_2d(dst, map, x, z, bar);
+}
+
 __global__ void __launch_bounds__(ls::kThreads, 1)
-tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmHx,
+tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__ CUtensorMap tmN,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmX,
                 LsArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // the SW128 operand tiles need a 1024-byte aligned base; the layout leaves no
@@ -205,11 +253,11 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     uint8_t *sm = smem_raw;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + ls::kBar);
-    uint64_t *q_full = bars + 0;     // [2 tiles]
+    uint64_t *q_full = bars + 0;     // [2 tiles]: M tile loaded
     uint64_t *q_empty = bars + 2;    // [2 tiles]: the tile's last S MMA of a problem done
-    uint64_t *k_full = bars + 4;     // [2 stages]: Ktil and its entropy panel
+    uint64_t *k_full = bars + 4;     // [2 stages]: N chunk and its panel
     uint64_t *k_empty = bars + 6;    // [2 stages]: both S MMAs of the chunk done
-    uint64_t *z_full = bars + 8;     // [2 stages]
+    uint64_t *z_full = bars + 8;     // [2 stages]: value chunk
     uint64_t *z_empty = bars + 10;   // [2 stages]: both PV MMAs of the chunk done
     uint64_t *s_full = bars + 16;    // [2 tiles]
     uint64_t *p_full = bars + 18;    // [2 tiles], one arrival per softmax warp
@@ -226,7 +274,10 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nmine = a.nprob > (int)blockIdx.x
                           ? (a.nprob - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-    const int nch = a.nchunks;
+    const bool values = a.mode != kLsStat;   // products with the values (Z or the queries)
+    // the strided query gather (3-D map) is the M side, or in kLsAgg the N side;
+    // the other side reads contiguous rows (2-D map)
+    const bool n_gather = a.mode == kLsAgg;
 
     if (threadIdx.x == 0) {
         for (int t = 0; t < 2; t++) {
@@ -247,8 +298,9 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         *abort_flag = 0;
         fence_mbar_init();
     }
-    // the all-ones query panel (every bfloat16 = 1.0, so its swizzle is moot):
-    // the entropy K-step adds 1 * H'_hi + 1 * H'_lo (the panel's other columns are 0)
+    // the M side's extra K-step panel, all ones (so its swizzle is moot): times the
+    // N side's panel [x_hi, x_lo, 0, ..., 0] it adds x = x_hi + x_lo to every logit
+    // of the N row (the entropy H' of a key block, or -lam of a query row)
     for (int i = threadIdx.x; i < (int)(ls::kPanelHx / 16); i += blockDim.x)
         reinterpret_cast<uint4 *>(sm + ls::kQx)[i] =
             make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
@@ -263,39 +315,40 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     if (warp >= 12) {
         regs_dec<ls::kProducerRegs>();
         if (warp == 12) {
-            // ---------------- producer of Ktil and its entropy panel: per chunk as
-            // soon as the S MMAs of two chunks back are done (never behind a query
+            // ---------------- producer of the N chunks and their panels: per chunk as
+            // soon as the S MMAs of two chunks back are done (never behind an M-tile
             // load, which has its own warp)
-            int issued[2] = {0, 0};
+            int issued[2] = {0, 0}, jc0 = 0;
             bool ok = true;
             for (int pi = 0; ok && pi < nmine; pi++) {
                 const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
-                for (int j = 0; j < nch; j++) {
-                    const int jc = pi * nch + j, sk = jc & 1;
+                for (int j = 0; j < pr.nch; j++) {
+                    const int jc = jc0 + j, sk = jc & 1;
                     if (jc >= 2 && !wait_warp(k_empty + sk, ((jc >> 1) - 1) & 1, w)) {
                         ok = false;
                         break;
                     }
                     if (lane == 0) {
-                        // keys past b1 in the ragged last chunk belong to the next
-                        // row (or are zero-filled past the array): masked later
+                        // rows past nkeys in the ragged last chunk belong to the next
+                        // row block (or are zero-filled past the array): masked later
                         mbar_expect_tx(k_full + sk, kTile + ls::kPanelHx);
                         for (int pn = 0; pn < 2; pn++)
-                            tma_load_2d(sm + ls::kK + sk * kTile + pn * kPanel, &tmK, pn * 64,
-                                        pr.key_row0 + j * 128, k_full + sk);
-                        tma_load_2d(sm + ls::kHx + sk * ls::kPanelHx, &tmHx, 0,
-                                    pr.key_row0 + j * 128, k_full + sk);
+                            ls_load(sm + ls::kK + sk * kTile + pn * kPanel, &tmN, n_gather,
+                                    pn * 64, pr.n_y, pr.n_z + j * 128, k_full + sk);
+                        ls_load(sm + ls::kHx + sk * ls::kPanelHx, &tmX, n_gather, 0, pr.n_y,
+                                pr.n_z + j * 128, k_full + sk);
                     }
                     issued[sk]++;
                 }
+                jc0 += pr.nch;
             }
             if (lane == 0)   // every issued copy lands before the CTA may exit
                 for (int s = 0; s < 2; s++)
                     if (issued[s] > 0) wait_phase_cleanup(k_full + s, (issued[s] - 1) & 1, kCleanupPolls);
         } else if (warp == 15) {
-            // ---------------- query producer: each query tile reloads as soon as its
-            // own last S MMA of the previous problem is done; the next problem's
-            // rows (a strided gather) are prefetched into L2 a whole problem ahead
+            // ---------------- M-tile producer: each tile reloads as soon as its own
+            // last S MMA of the previous problem is done; the next problem's rows
+            // are prefetched into L2 a whole problem ahead
             int qloads = 0;
             bool ok = true;
             for (int pi = 0; ok && pi < nmine; pi++) {
@@ -308,8 +361,8 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     if (lane == 0) {
                         mbar_expect_tx(q_full + t, kTile);
                         for (int pn = 0; pn < 2; pn++)
-                            tma_load_3d(sm + ls::kQ + t * kTile + pn * kPanel, &tmQ, pn * 64, pr.v,
-                                        pr.bh * p.b1 + pr.u_start + t * 128, q_full + t);
+                            ls_load(sm + ls::kQ + t * kTile + pn * kPanel, &tmM, !n_gather,
+                                    pn * 64, pr.m_y, pr.m_z + t * 128, q_full + t);
                     }
                 }
                 if (!ok) break;
@@ -317,22 +370,26 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 if (lane == 0 && pi + 1 < nmine) {
                     const LsProblem nx = ls_problem(a, blockIdx.x + (pi + 1) * gridDim.x);
                     for (int t = 0; t < 2; t++)
-                        for (int pn = 0; pn < 2; pn++)
-                            tma_prefetch_3d(&tmQ, pn * 64, nx.v, nx.bh * p.b1 + nx.u_start + t * 128);
+                        for (int pn = 0; pn < 2; pn++) {
+                            if (!n_gather)
+                                tma_prefetch_3d(&tmM, pn * 64, nx.m_y, nx.m_z + t * 128);
+                            else
+                                tma_prefetch_2d(&tmM, pn * 64, nx.m_z + t * 128);
+                        }
                 }
             }
             if (lane == 0)
                 for (int t = 0; t < 2; t++)
                     if (qloads > 0) wait_phase_cleanup(q_full + t, (qloads - 1) & 1, kCleanupPolls);
-        } else if (warp == 14) {
-            // ---------------- Z producer: its own warp, so that a Ktil load never
-            // queues behind the wait for a Z stage (released one PV later than Ktil)
-            int issued_z[2] = {0, 0};
+        } else if (warp == 14 && values) {
+            // ---------------- value producer: its own warp, so that an N-chunk load
+            // never queues behind the wait for a value stage (released one PV later)
+            int issued_z[2] = {0, 0}, jc0 = 0;
             bool ok = true;
             for (int pi = 0; ok && pi < nmine; pi++) {
                 const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
-                for (int j = 0; j < nch; j++) {
-                    const int jc = pi * nch + j, st = jc & 1;
+                for (int j = 0; j < pr.nch; j++) {
+                    const int jc = jc0 + j, st = jc & 1;
                     if (jc >= 2 && !wait_warp(z_empty + st, ((jc >> 1) - 1) & 1, w)) {
                         ok = false;
                         break;
@@ -340,11 +397,12 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     if (lane == 0) {
                         mbar_expect_tx(z_full + st, kTile);
                         for (int pn = 0; pn < 2; pn++)
-                            tma_load_2d(sm + ls::kZ + st * kTile + pn * kPanel, &tmZ, pn * 64,
-                                        pr.key_row0 + j * 128, z_full + st);
+                            ls_load(sm + ls::kZ + st * kTile + pn * kPanel, &tmV, n_gather,
+                                    pn * 64, pr.n_y, pr.n_z + j * 128, z_full + st);
                     }
                     issued_z[st]++;
                 }
+                jc0 += pr.nch;
             }
             if (lane == 0)
                 for (int s = 0; s < 2; s++)
@@ -357,7 +415,9 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             // the next chunk overwrites the columns that PV_t reads as P: tcgen05
             // MMAs issued by one thread execute in issue order, so it follows PV_t
             // without a wait, and its commit (s_full) also covers PV_t, which orders
-            // the softmax's rescale of O_t after PV_t.
+            // the softmax's rescale of O_t after PV_t.  Without values (kLsStat)
+            // there is no PV: S_t of the next chunk waits for the softmax to have
+            // read S_t (p_full).
             constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t idO = idesc_bf16(128, 128, 0, 1);
             const uint64_t dQ = smem_desc_sw128(smem_u32(sm + ls::kQ), 16, 1024);
@@ -366,29 +426,29 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             const uint64_t dQx = smem_desc_sw32(smem_u32(sm + ls::kQx));
             const uint64_t dHx = smem_desc_sw32(smem_u32(sm + ls::kHx));
             constexpr uint32_t kTileDesc = kTile >> 4, kHxDesc = ls::kPanelHx >> 4;
-            const int total = nmine * nch;
             // fault injection: a wait that can only give up (bounded, then abort)
             bool ok = !a.stall || spin_warp(stall_bar, 0, w);
-            auto issue_s = [&](int t, int jc) -> bool {
+            // S_t of global chunk jc, chunk j of problem pi (nch chunks)
+            auto issue_s = [&](int t, int jc, int j, int pi, int nch) -> bool {
                 const int sk = jc & 1;
-                if (jc % nch == 0 && !spin_warp(q_full + t, (jc / nch) & 1, w)) return false;
+                if (j == 0 && !spin_warp(q_full + t, pi & 1, w)) return false;
                 if (t == 0 && !spin_warp(k_full + sk, (jc >> 1) & 1, w)) return false;
                 tc_fence_after();
                 mma8_ss_k128(tmem + t * 128, dQ + t * kTileDesc, dK + sk * kTileDesc, idS, 0u);
-                mma1_ss_acc(tmem + t * 128, dQx, dHx + sk * kHxDesc, idS);   // + H'
+                mma1_ss_acc(tmem + t * 128, dQx, dHx + sk * kHxDesc, idS);   // + panel value
                 mma_commit_warp(s_full + t);
                 if (t == 1) mma_commit_warp(k_empty + sk);
-                if (jc % nch == nch - 1) mma_commit_warp(q_empty + t);   // tile t no longer read
+                if (j == nch - 1) mma_commit_warp(q_empty + t);   // tile t no longer read
                 return true;
             };
-            auto issue_pv = [&](int t, int jc) -> bool {
-                const int st = jc & 1, j = jc % nch;
-                if (t == 0 && !spin_warp(z_full + st, (jc >> 1) & 1, w)) return false;
+            auto issue_pv = [&](int t, int jc, int j, int pi, int nch) -> bool {
+                const int st = jc & 1;
+                if (values && t == 0 && !spin_warp(z_full + st, (jc >> 1) & 1, w)) return false;
                 if (!spin_warp(p_full + t, jc & 1, w)) return false;
+                if (!values) return true;
                 // the first PV of a problem overwrites O_t: the epilogue of the
                 // previous problem must have read it
-                if (j == 0 && jc >= nch && !spin_warp(o_free + t, ((jc / nch) - 1) & 1, w))
-                    return false;
+                if (j == 0 && pi > 0 && !spin_warp(o_free + t, (pi - 1) & 1, w)) return false;
                 tc_fence_after();
                 mma8_ts_mn128(tmem + 256 + t * 128, tmem + t * 128, dZ + st * kTileDesc, idO,
                               j > 0 ? 1u : 0u);
@@ -396,22 +456,34 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 if (j == nch - 1) mma_commit_warp(o_full + t);
                 return true;
             };
-            if (ok && total > 0) ok = issue_s(0, 0) && issue_s(1, 0);
-            for (int jc = 0; ok && jc < total; jc++) {
-                const bool more = jc + 1 < total;
-                ok = issue_pv(0, jc) && (!more || issue_s(0, jc + 1)) && issue_pv(1, jc) &&
-                     (!more || issue_s(1, jc + 1));
+            int jc0 = 0;
+            LsProblem pr = nmine > 0 ? ls_problem(a, blockIdx.x) : LsProblem{};
+            if (ok && nmine > 0) ok = issue_s(0, 0, 0, 0, pr.nch) && issue_s(1, 0, 0, 0, pr.nch);
+            for (int pi = 0; ok && pi < nmine; pi++) {
+                const bool has_next = pi + 1 < nmine;
+                const LsProblem nx = has_next ? ls_problem(a, blockIdx.x + (pi + 1) * gridDim.x) : pr;
+                for (int j = 0; ok && j < pr.nch; j++) {
+                    const int jc = jc0 + j;
+                    const bool last = j == pr.nch - 1, more = !last || has_next;
+                    // the chunk after jc: j + 1 of this problem, or 0 of the next
+                    const int jn = last ? 0 : j + 1, pn = last ? pi + 1 : pi;
+                    const int nn = last ? nx.nch : pr.nch;
+                    ok = issue_pv(0, jc, j, pi, pr.nch) && (!more || issue_s(0, jc + 1, jn, pn, nn)) &&
+                         issue_pv(1, jc, j, pi, pr.nch) && (!more || issue_s(1, jc + 1, jn, pn, nn));
+                }
+                jc0 += pr.nch;
+                pr = nx;
             }
             mma_commit_warp(mma_done);
             wait_phase_cleanup(mma_done, 0, kCleanupPolls);
         }
     } else if (warp >= 8) {
         // ---------------- epilogue warpgroup: per problem and tile, O_t / l to
-        // bfloat16; each thread writes its own output row as sixteen 16-byte stores
+        // bfloat16 rows of the output (Y, or the aggregated queries)
         regs_dec<ls::kEpilogueRegs>();
         const int wq = warp & 3;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-        bool ok = true;
+        bool ok = values;
         for (int pi = 0; ok && pi < nmine; pi++) {
             const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
             for (int t = 0; t < 2; t++) {
@@ -442,7 +514,7 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 // instruction covers four whole row halves (eight 16-byte chunks
                 // each), instead of 32 scattered 16-byte pieces
                 uint8_t *stg = sm + ls::kStg + wq * 4096;
-                const int u0w = pr.u_start + t * 128 + wq * 32;
+                const int m0w = pr.m_first + t * 128 + wq * 32;
 #pragma unroll
                 for (int hf = 0; hf < 2; hf++) {
 #pragma unroll
@@ -456,11 +528,16 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                         const int row = rr * 4 + (lane >> 3), c = lane & 7;
                         const uint4 val =
                             *reinterpret_cast<const uint4 *>(stg + row * 128 + ((c + row) & 7) * 16);
-                        const int u = u0w + row;
-                        if (u < pr.u1)
-                            *reinterpret_cast<uint4 *>(
-                                a.out + ((int64_t)pr.bh * p.N + (int64_t)u * p.b2 + pr.v) * kD +
-                                hf * 64 + c * 8) = val;
+                        const int m = m0w + row;
+                        if (m < pr.m_end) {
+                            // kLsOut: Y row (u, v); kLsAgg: aggregated query of block
+                            // u' = m for row g*b2 + v
+                            const int64_t orow =
+                                a.mode == kLsOut
+                                    ? (int64_t)pr.bh * p.N + (int64_t)m * p.b2 + pr.v
+                                    : ((int64_t)pr.bh * p.b1k + m) * a.mpad + pr.g * p.b2 + pr.v;
+                            *reinterpret_cast<uint4 *>(a.out + orow * kD + hf * 64 + c * 8) = val;
+                        }
                     }
                     __syncwarp();
                 }
@@ -476,26 +553,28 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const uint32_t tO = tmem + lane_off + 256 + t * 128;
         const uint64_t c2 = f2_pack(a.c_log2, a.c_log2);
         bool ok = true;
+        int jc0 = 0;
         for (int pi = 0; ok && pi < nmine; pi++) {
+            const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
             float m_run = -INFINITY, l_run = 0.f;
-            for (int j = 0; j < nch; j++) {
-                const int jc = pi * nch + j;
+            for (int j = 0; j < pr.nch; j++) {
+                const int jc = jc0 + j;
                 if (!wait_warp(s_full + t, jc & 1, w)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                // S = (s q.Ktil + H) / (s ln 2): scaled by c_log2 it is the logit in
-                // log2 units, so the maximum is taken on S itself
+                // S = q.Ktil + H' (kLsAgg: Ktil.q - lam): scaled by c_log2 it is the
+                // logit in log2 units, so the maximum is taken on S itself
                 float x[128];
 #pragma unroll
                 for (int c = 0; c < 4; c++) tmem_ld32f(tS + c * 32, &x[c * 32]);
                 tmem_wait_ld();
                 float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-                const int nvalid = p.b1 - j * 128;   // keys of this chunk inside the row
+                const int nvalid = pr.nkeys - j * 128;   // N rows of this chunk inside the row
                 if (nvalid < 128) {
-                    // the ragged last chunk: keys past b1 belong to the next row
-                    // (or are zero fill), so mask them by selection
+                    // the ragged last chunk: rows past nkeys belong to the next row
+                    // block (or are zero fill), so mask them by selection
 #pragma unroll
                     for (int i = 0; i < 128; i++) x[i] = i < nvalid ? x[i] : -INFINITY;
                 }
@@ -534,12 +613,12 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                         f2_unpack(e2, p0, p1);
                         pk[i] = pack_bf16(p0, p1);
                     }
-                    tmem_st32(tS + h * 32, pk);
+                    if (values) tmem_st32(tS + h * 32, pk);
                 }
                 float s0, s1;
                 f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), s0, s1);
                 l_run = l_run * alpha + (s0 + s1);
-                if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+                if (values && j > 0 && __any_sync(0xffffffffu, rescale)) {
                     // O_t is complete up to the previous chunk (the commit of this
                     // chunk's S covers the previous PV); scale it in four slices
 #pragma unroll
@@ -552,16 +631,37 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                         tmem_st32f(tO + c * 32, o);
                     }
                 }
-                tmem_wait_st();
+                if (values) tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive_warp(p_full + t);
             }
             if (!ok) break;
-            // the row sums for the epilogue; slot pi & 1 is rewritten two problems
-            // later, when the epilogue has released O_t (o_free) of this problem,
-            // which the first PV of the problem after next waits for
-            lsum[((pi & 1) * 2 + t) * 128 + wq * 32 + lane] = l_run;
-            mbar_arrive_warp(l_full + t);
+            jc0 += pr.nch;
+            if (values) {
+                // the row sums for the epilogue.  Before publishing those of problem
+                // pi the epilogue must have taken those of pi - 1 (its o_free
+                // arrival follows its l_full wait): otherwise l_full could run two
+                // phases ahead of the epilogue's parity wait when problems are short.
+                // o_free cannot itself run ahead here, since the epilogue releases
+                // problem pi only after these row sums.
+                if (pi > 0 && !wait_warp(o_free + t, (pi - 1) & 1, w)) break;
+                lsum[((pi & 1) * 2 + t) * 128 + wq * 32 + lane] = l_run;
+                mbar_arrive_warp(l_full + t);
+            } else {
+                // the row's log-sum-exp in raw logit units, stored negated as a
+                // bfloat16 pair (hi + lo within 2^-16 relative) in its panel row
+                const int m = pr.m_first + t * 128 + wq * 32 + lane;
+                if (m < pr.m_end) {
+                    const float lam = m_run + fast_log2(l_run) / a.c_log2;
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(-lam);
+                    const __nv_bfloat16 lo = __float2bfloat16_rn(-lam - __bfloat162float(hi));
+                    const uint32_t pair = (uint32_t)__bfloat16_as_ushort(hi) |
+                                          ((uint32_t)__bfloat16_as_ushort(lo) << 16);
+                    uint4 *dst = a.lam + ((int64_t)pr.bh * p.N + (int64_t)m * p.b2 + pr.v) * 2;
+                    dst[0] = make_uint4(pair, 0u, 0u, 0u);
+                    dst[1] = make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
         }
     }
     tc_fence_before();
@@ -581,11 +681,16 @@ struct RsArgs {
     int mpad;            // nmt * 128
     int bpc;             // blocks per CTA (flattened over heads and blocks)
     float c_log2;
-
+    float inv_c_log2;
+    // 0: one set of aggregated queries per head (the first iteration, uniform L),
+    // loaded once per head; 1: per block u' (later iterations), tile mt of block
+    // u' at rows (bh*b1 + u')*mpad + mt*128, loaded per item into slot mt
+    int qblk;
     int *status;
     long long limit;
     int stall;           // test hook: the MMA warp first waits on a barrier nothing completes
 };
+constexpr int kMaxQbarTiles = 4;   // slots of the per-block aggregated-query ring
 
 template <int B2P>
 struct RsLayout {
@@ -624,15 +729,16 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 17);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 18);
     uint64_t *stall_bar = bars + 19;   // never completed (fault-injection hook)
+    uint64_t *qs_full = bars + 20;     // [kMaxQbarTiles] per-block mode: slot mt loaded
+    uint64_t *qs_empty = bars + 24;    // [kMaxQbarTiles] per-block mode: slot mt's S MMA done
 
     const Problem &p = a.p;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // (head, block) items of the heads that the unit range touches
-    const int total = p.head_end() * p.b1;
-    const int first = p.head_begin() * p.b1 + blockIdx.x * a.bpc;
+    const int total = p.head_end() * p.b1k;
+    const int first = p.head_begin() * p.b1k + blockIdx.x * a.bpc;
     const int nblk = min(a.bpc, total - first);
     const int nitems = nblk * nmt;
-    const int tb2 = p.tiles * p.b2;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -648,6 +754,10 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
         }
         mbar_init(mma_done, 1);
         mbar_init(stall_bar, 1);
+        for (int s = 0; s < kMaxQbarTiles; s++) {
+            mbar_init(qs_full + s, 1);
+            mbar_init(qs_empty + s, 1);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -659,13 +769,28 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
     const WaitCtx w{a.limit, a.status, abort_flag};
 
     if (warp == 0) {
-        // ---------------- producer: qbar tiles per head, K and V per block
+        // ---------------- producer: qbar tiles per head (or per block), K and V per block
         if (lane == 0) {
-            int heads = 0, cur = -1, issued[2] = {0, 0};
+            int heads = 0, cur = -1, issued[2] = {0, 0}, qissued[kMaxQbarTiles] = {0, 0, 0, 0};
             bool ok = true;
             for (int ib = 0; ib < nblk && ok; ib++) {
-                const int fb = first + ib, bh = fb / p.b1, up = fb % p.b1;
-                if (bh != cur) {
+                const int fb = first + ib, bh = fb / p.b1k, up = fb % p.b1k;
+                if (a.qblk) {
+                    // slot mt takes tile mt of this block once the S MMA of the
+                    // previous block's tile mt is done
+                    for (int mt = 0; mt < nmt && ok; mt++) {
+                        if (ib >= 1 && !wait_phase(qs_empty + mt, (ib - 1) & 1, w)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_expect_tx(qs_full + mt, kTile);
+                        for (int pn = 0; pn < 2; pn++)
+                            tma_load_2d(sm + mt * kTile + pn * kPanel, &tmQb, pn * 64,
+                                        fb * a.mpad + mt * 128, qs_full + mt);
+                        qissued[mt]++;
+                    }
+                    if (!ok) break;
+                } else if (bh != cur) {
                     if (heads > 0 && !wait_phase(q_empty, (heads - 1) & 1, w)) break;
                     mbar_expect_tx(q_full, nmt * kTile);
                     for (int mt = 0; mt < nmt; mt++)
@@ -679,7 +804,7 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 if (ib >= 2 && !wait_phase(kv_empty + st, ((ib >> 1) - 1) & 1, w)) break;
                 uint8_t *stage = sm + L::kv(nmt) + st * L::kStage;
                 mbar_expect_tx(kv_full + st, L::kStage);
-                const int row = bh * p.N + up * p.b2;
+                const int row = bh * p.Nk + up * p.b2;
                 for (int pn = 0; pn < 2; pn++) {
                     tma_load_2d(stage + pn * L::kPanelKV, &tmK, pn * 64, row, kv_full + st);
                     tma_load_2d(stage + L::kVOff + pn * L::kPanelKV, &tmV, pn * 64, row,
@@ -691,6 +816,9 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
             for (int s = 0; s < 2; s++)
                 if (issued[s] > 0)
                     wait_phase_cleanup(kv_full + s, (issued[s] - 1) & 1, kCleanupPolls);
+            for (int mt = 0; mt < kMaxQbarTiles; mt++)   // the last load into each slot
+                if (qissued[mt] > 0)
+                    wait_phase_cleanup(qs_full + mt, (qissued[mt] - 1) & 1, kCleanupPolls);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer: the whole warp runs the loop, one elected
@@ -707,14 +835,14 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
             // S = qbar_mt K_u'^T for item i into S buffer i & 1
             auto gemm1 = [&](int i) -> bool {
                 const int ib = i / nmt, mt = i % nmt;
-                const int fb = first + ib, bh = fb / p.b1;
-                if (mt == 0) {
-                    if (ib == 0 || (fb - 1) / p.b1 != bh) {
-                        if (!wait_warp(q_full, heads & 1, w)) return false;
-                        heads++;
-                    }
-                    if (!wait_warp(kv_full + (ib & 1), (ib >> 1) & 1, w)) return false;
+                const int fb = first + ib, bh = fb / p.b1k;
+                if (a.qblk) {
+                    if (!wait_warp(qs_full + mt, ib & 1, w)) return false;
+                } else if (mt == 0 && (ib == 0 || (fb - 1) / p.b1k != bh)) {
+                    if (!wait_warp(q_full, heads & 1, w)) return false;
+                    heads++;
                 }
+                if (mt == 0 && !wait_warp(kv_full + (ib & 1), (ib >> 1) & 1, w)) return false;
                 if (i >= 2 && !wait_warp(s_free + (i & 1), ((i >> 1) - 1) & 1, w)) return false;
                 tc_fence_after();
                 const uint64_t a0 = desc_plus(dQ, mt * kTile);
@@ -725,8 +853,12 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                            desc_plus(a0, (kk >> 2) * kPanel + (kk & 3) * 32),
                            desc_plus(b0, (kk >> 2) * L::kPanelKV + (kk & 3) * 32), id1, kk > 0);
                 mma_commit_warp(s_full + (i & 1));
-                const bool head_ends = (ib == nblk - 1) || ((fb + 1) / p.b1 != bh);
-                if (mt == nmt - 1 && head_ends) mma_commit_warp(q_empty);
+                if (a.qblk) {
+                    mma_commit_warp(qs_empty + mt);   // slot mt may take the next block's tile
+                } else {
+                    const bool head_ends = (ib == nblk - 1) || ((fb + 1) / p.b1k != bh);
+                    if (mt == nmt - 1 && head_ends) mma_commit_warp(q_empty);
+                }
                 return true;
             };
             if (ok && nitems > 0) ok = gemm1(0);
@@ -760,11 +892,10 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
     } else if (warp >= 4 && warp < 8) {
         // ---------------- softmax: R rows, entropy, normalised P back to TMEM (bf16)
         const int wq = warp & 3;
-        const int r = wq * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
         for (int i = 0; i < nitems; i++) {
             const int ib = i / nmt, mt = i % nmt;
-            const int fb = first + ib, bh = fb / p.b1, up = fb % p.b1;
+            const int fb = first + ib, bh = fb / p.b1k, up = fb % p.b1k;
             if (!wait_warp(s_full + (i & 1), (i >> 1) & 1, w)) break;
             tc_fence_after();
             const uint32_t tS = tmem + lane_off + (i & 1) * 128;
@@ -803,12 +934,13 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
             f2_unpack(f2_add(f2_add(l2[0], l2[1]), f2_add(l2[2], l2[3])), la, lb);
             f2_unpack(f2_add(f2_add(e2[0], e2[1]), f2_add(e2[2], e2[3])), ea, eb);
             const float l = la + lb, inv = 1.f / l;
-            const int row = mt * 128 + r;
             // entropy of the row in log2 units, log2(sum 2^x) - E_R[x] = H / ln 2,
             // stored divided by c_log2 = s log2(e) (the L-step's logits are
             // S * c_log2) as a bfloat16 pair hi + lo in the row's entropy panel
             {
-                const float hp = (mxr * a.c_log2 + log2f(l) - (ea + eb) * inv) / a.c_log2;
+                // (l >= 1: the row maximum contributes 2^0, so the approximate
+                // log2 is accurate to a few ulp of its result)
+                const float hp = (mxr * a.c_log2 + fast_log2(l) - (ea + eb) * inv) * a.inv_c_log2;
                 const __nv_bfloat16 hi = __float2bfloat16_rn(hp);
                 const __nv_bfloat16 lo = __float2bfloat16_rn(hp - __bfloat162float(hi));
                 const uint32_t pair = (uint32_t)__bfloat16_as_ushort(hi) |
@@ -853,7 +985,7 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
         bool ok = true;
         for (int i = 0; ok && i < nitems; i++) {
             const int ib = i / nmt, mt = i % nmt;
-            const int fb = first + ib, bh = fb / p.b1, up = fb % p.b1;
+            const int fb = first + ib, bh = fb / p.b1k, up = fb % p.b1k;
             for (int part = 0; part < 2; part++) {
                 if (!wait_warp(o_full + part, i & 1, w)) {
                     ok = false;
@@ -954,12 +1086,14 @@ uint32_t rstep_smem(int b2p, int nmt) {
 
 struct TcWorkspace {
     __nv_bfloat16 *qbar, *ktil, *z;
-    uint4 *hx;   // [BH][t][b2][b1] rows of 32 bytes
+    uint4 *hx;            // [BH][t][b2][b1] rows of 32 bytes
+    __nv_bfloat16 *qblk;  // iters > 1: aggregated queries per block [BH][b1][mpad][d]
+    uint4 *lam;           // iters > 1: log-sum-exp panels [BH][N] rows of 32 bytes
 };
 
 TcWorkspace carve(const Problem &p, void *base) {
     const size_t mpad = (size_t)qbar_tiles(p) * 128;
-    const size_t kz = (size_t)p.BH * p.tiles * p.N * kD * 2;
+    const size_t kz = (size_t)p.BH * p.tiles * p.Nk * kD * 2;
     char *c = (char *)base;
     TcWorkspace ws;
     ws.qbar = (__nv_bfloat16 *)c;
@@ -969,6 +1103,14 @@ TcWorkspace carve(const Problem &p, void *base) {
     ws.z = (__nv_bfloat16 *)c;
     c += al256(kz);
     ws.hx = (uint4 *)c;
+    c += al256((size_t)p.BH * p.tiles * p.Nk * 32);
+    ws.qblk = nullptr;
+    ws.lam = nullptr;
+    if (p.iters > 1) {
+        ws.qblk = (__nv_bfloat16 *)c;
+        c += al256((size_t)p.BH * p.b1k * mpad * kD * 2);
+        ws.lam = (uint4 *)c;
+    }
     return ws;
 }
 
@@ -997,10 +1139,15 @@ int sm_count() {
 }  // namespace
 
 bool sm100_supports(const Problem &p, monarch_dtype dtype) {
-    if (dtype != MONARCH_BF16 || p.d != kD || p.iters != 1 || p.b2 > 128) return false;
+    if (dtype != MONARCH_BF16 || p.d != kD || p.b2 > 128) return false;
+    // later iterations keep one slot per aggregated-query tile
+    if (p.iters > 1 && qbar_tiles(p) > kMaxQbarTiles) return false;
+    if (p.iters > 1 && (int64_t)p.BH * p.b1k * qbar_tiles(p) * 128 + 256 >= (1LL << 31)) return false;
     if (rstep_smem(b2_padded(p.b2), qbar_tiles(p)) > (uint32_t)kMaxSmem) return false;
     // TMA coordinates are 32-bit: every row index must fit
-    if ((int64_t)p.BH * p.tiles * p.N + 256 >= (1LL << 31)) return false;
+    if ((int64_t)p.BH * p.tiles * p.Nk + 256 >= (1LL << 31)) return false;
+    if ((int64_t)p.BH * p.Nk + 256 >= (1LL << 31) || (int64_t)p.BH * p.N + 256 >= (1LL << 31))
+        return false;
     if ((int64_t)p.BH * qbar_tiles(p) * 128 >= (1LL << 31)) return false;
 
     if (encode_fn() == nullptr) return false;
@@ -1010,19 +1157,119 @@ bool sm100_supports(const Problem &p, monarch_dtype dtype) {
 size_t sm100_workspace_bytes(const Problem &p, bool &overflow) {
     overflow = false;
     const size_t mpad = (size_t)qbar_tiles(p) * 128;
-    const size_t kz = (size_t)p.BH * p.tiles * p.N * kD * 2;
-    const size_t hx = (size_t)p.BH * p.tiles * p.N * 32;
-    return al256((size_t)p.BH * mpad * kD * 2) + 2 * al256(kz) + al256(hx);
+    const size_t kz = (size_t)p.BH * p.tiles * p.Nk * kD * 2;
+    const size_t hx = (size_t)p.BH * p.tiles * p.Nk * 32;
+    size_t bytes = al256((size_t)p.BH * mpad * kD * 2) + 2 * al256(kz) + al256(hx);
+    if (p.iters > 1)
+        bytes += al256((size_t)p.BH * p.b1k * mpad * kD * 2) + al256((size_t)p.BH * p.N * 32);
+    return bytes;
 }
+
+namespace {
+
+// bfloat16 tensor maps of the L-step (128-row boxes): rows of a [rows][d] array
+// (2-D), the strided query gather (3-D: y = column v, z = bh*b1 + u), and the
+// same two forms for 32-byte panel rows.
+bool map_rows(CUtensorMap *m, const void *base, uint64_t rows, uint32_t width,
+              CUtensorMapSwizzle sw) {
+    const uint64_t dims[2] = {width, rows};
+    const uint64_t str[1] = {(uint64_t)width * 2};
+    const uint32_t box[2] = {width == 16 ? 16u : 64u, 128};
+    return make_map(m, base, 2, dims, str, box, sw);
+}
+bool map_gather(CUtensorMap *m, const void *base, const Problem &p, uint32_t width,
+                CUtensorMapSwizzle sw) {
+    const uint64_t dims[3] = {width, (uint64_t)p.b2, (uint64_t)p.BH * p.b1};
+    const uint64_t str[2] = {(uint64_t)width * 2, (uint64_t)p.b2 * width * 2};
+    const uint32_t box[3] = {width == 16 ? 16u : 64u, 1, 128};
+    return make_map(m, base, 3, dims, str, box, sw);
+}
+
+cudaError_t run_rstep(const Problem &p, const TcWorkspace &ws, const void *k, const void *v,
+                      int qblk, float c_log2, int *status, long long wait_limit, int stall,
+                      cudaStream_t stream) {
+    const int nmt = qbar_tiles(p), mpad = nmt * 128, b2p = b2_padded(p.b2);
+    CUtensorMap maps[6];
+    const uint64_t dq[2] = {(uint64_t)kD, qblk ? (uint64_t)p.BH * p.b1k * mpad : (uint64_t)p.BH * mpad};
+    const uint64_t dkv[2] = {(uint64_t)kD, (uint64_t)p.BH * p.Nk};
+    const uint64_t s2[1] = {kD * 2};
+    const uint32_t bq[2] = {64, 128};
+    const uint32_t bkv[2] = {64, (uint32_t)b2p};
+    const uint64_t dst[4] = {(uint64_t)kD, (uint64_t)p.b1k, (uint64_t)p.tiles * p.b2,
+                             (uint64_t)p.BH};
+    const uint64_t sst[3] = {kD * 2, (uint64_t)p.b1k * kD * 2,
+                             (uint64_t)p.tiles * p.b2 * p.b1k * kD * 2};
+    const uint32_t bst[4] = {64, 1, 32, 1};
+    // entropy panels, [bh][t*b2 rows][b1][16], stored 32 rows x 32 B per warp
+    const uint64_t dhx[4] = {16, (uint64_t)p.b1k, (uint64_t)p.tiles * p.b2, (uint64_t)p.BH};
+    const uint64_t shx[3] = {32, (uint64_t)p.b1k * 32, (uint64_t)p.tiles * p.b2 * p.b1k * 32};
+    const uint32_t bhx[4] = {16, 1, 32, 1};
+    if (!make_map(&maps[0], qblk ? ws.qblk : ws.qbar, 2, dq, s2, bq) ||
+        !make_map(&maps[1], k, 2, dkv, s2, bkv) || !make_map(&maps[2], v, 2, dkv, s2, bkv) ||
+        !make_map(&maps[3], ws.z, 4, dst, sst, bst) || !make_map(&maps[4], ws.ktil, 4, dst, sst, bst) ||
+        !make_map(&maps[5], ws.hx, 4, dhx, shx, bhx, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    const int total = (p.head_end() - p.head_begin()) * p.b1k;
+    const int sms = sm_count();
+    const int bpc = (total + sms - 1) / sms;
+    const int grid = (total + bpc - 1) / bpc;
+    RsArgs a{p, nmt, mpad, bpc, c_log2, 1.f / c_log2, qblk, status, wait_limit, stall};
+    ProfileScope scope(K_TC_RSTEP, stream);
+    switch (b2p) {
+        case 16: return launch_rstep<16>(maps, a, grid, stream);
+        case 32: return launch_rstep<32>(maps, a, grid, stream);
+        case 48: return launch_rstep<48>(maps, a, grid, stream);
+        case 64: return launch_rstep<64>(maps, a, grid, stream);
+        case 80: return launch_rstep<80>(maps, a, grid, stream);
+        case 96: return launch_rstep<96>(maps, a, grid, stream);
+        case 112: return launch_rstep<112>(maps, a, grid, stream);
+        case 128: return launch_rstep<128>(maps, a, grid, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t run_lstep(const Problem &p, const TcWorkspace &ws, const void *q, void *out, int mode,
+                      float c_log2, int *status, long long wait_limit, int stall,
+                      cudaStream_t stream) {
+    const int mpad = qbar_tiles(p) * 128;
+    CUtensorMap qg, kt, zt, xp;
+    const uint64_t rows = (uint64_t)p.BH * p.tiles * p.Nk;
+    if (!map_gather(&qg, q, p, kD, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map_rows(&kt, ws.ktil, rows, kD, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map_rows(&zt, ws.z, rows, kD, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    const bool agg = mode == kLsAgg;
+    if (agg ? !map_gather(&xp, ws.lam, p, 16, CU_TENSOR_MAP_SWIZZLE_32B)
+            : !map_rows(&xp, ws.hx, rows, 16, CU_TENSOR_MAP_SWIZZLE_32B))
+        return cudaErrorInvalidValue;
+    // M-side rows per (g, v): the tile's queries, or (kLsAgg) the b1 Ktil rows
+    const int mrows = agg ? p.b1k : tile_max_rows(p.b1, p.tiles);
+    const int npairs = ((mrows + 127) / 128 + 1) / 2;
+    const int nprob = (p.unit_end - p.unit_begin) * p.b2 * npairs;
+    LsArgs a{p, mode, npairs, nprob, p.unit_begin * p.b2 * npairs, mpad, c_log2,
+             agg ? ws.qblk : (__nv_bfloat16 *)out, ws.lam, status, wait_limit, stall};
+    cudaError_t e = set_smem(tc_lstep_kernel, ls::kSmem);
+    if (e != cudaSuccess) return e;
+    const int grid = nprob < sm_count() ? nprob : sm_count();
+    ProfileScope scope(mode == kLsOut ? K_TC_LSTEP : mode == kLsStat ? K_TC_LSTAT : K_TC_QAGG,
+                       stream);
+    if (agg)
+        tc_lstep_kernel<<<grid, ls::kThreads, ls::kSmem, stream>>>(kt, qg, qg, xp, a);
+    else
+        tc_lstep_kernel<<<grid, ls::kThreads, ls::kSmem, stream>>>(qg, kt, zt, xp, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
 
 cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const void *v,
                           void *out, void *workspace, int *status, long long wait_limit,
                           int stall, cudaStream_t stream) {
     const TcWorkspace ws = carve(p, workspace);
-    const int nmt = qbar_tiles(p), mpad = nmt * 128, b2p = b2_padded(p.b2);
+    const int mpad = qbar_tiles(p) * 128;
     const float c_log2 = p.scale * kLog2e;
 
-    // S1
+    // S1: the first R-step's aggregated queries (uniform L: plain means)
     {
         const int nchunk = (p.b2 * kD / 8 + 127) / 128;
         ProfileScope scope(K_TC_QBAR, stream);
@@ -1031,79 +1278,19 @@ cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const 
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    // S2
-    {
-        CUtensorMap maps[6];
-        const uint64_t dq[2] = {(uint64_t)kD, (uint64_t)p.BH * mpad};
-        const uint64_t dkv[2] = {(uint64_t)kD, (uint64_t)p.BH * p.N};
-        const uint64_t s2[1] = {kD * 2};
-        const uint32_t bq[2] = {64, 128};
-        const uint32_t bkv[2] = {64, (uint32_t)b2p};
-        const uint64_t dst[4] = {(uint64_t)kD, (uint64_t)p.b1, (uint64_t)p.tiles * p.b2,
-                                 (uint64_t)p.BH};
-        const uint64_t sst[3] = {kD * 2, (uint64_t)p.b1 * kD * 2,
-                                 (uint64_t)p.tiles * p.b2 * p.b1 * kD * 2};
-        const uint32_t bst[4] = {64, 1, 32, 1};
-        if (!make_map(&maps[0], ws.qbar, 2, dq, s2, bq) || !make_map(&maps[1], k, 2, dkv, s2, bkv) ||
-            !make_map(&maps[2], v, 2, dkv, s2, bkv) || !make_map(&maps[3], ws.z, 4, dst, sst, bst) ||
-            !make_map(&maps[4], ws.ktil, 4, dst, sst, bst))
-            return cudaErrorInvalidValue;
-        // entropy panels, [bh][t*b2 rows][b1][16], stored 32 rows x 32 B per warp
-        const uint64_t dhx[4] = {16, (uint64_t)p.b1, (uint64_t)p.tiles * p.b2, (uint64_t)p.BH};
-        const uint64_t shx[3] = {32, (uint64_t)p.b1 * 32, (uint64_t)p.tiles * p.b2 * p.b1 * 32};
-        const uint32_t bhx[4] = {16, 1, 32, 1};
-        if (!make_map(&maps[5], ws.hx, 4, dhx, shx, bhx, CU_TENSOR_MAP_SWIZZLE_NONE))
-            return cudaErrorInvalidValue;
-        const int total = (p.head_end() - p.head_begin()) * p.b1;
-        const int sms = sm_count();
-        const int bpc = (total + sms - 1) / sms;
-        const int grid = (total + bpc - 1) / bpc;
-        RsArgs a{p, nmt, mpad, bpc, c_log2, status, wait_limit, stall};
-        ProfileScope scope(K_TC_RSTEP, stream);
-        cudaError_t e = cudaErrorInvalidValue;
-        switch (b2p) {
-            case 16: e = launch_rstep<16>(maps, a, grid, stream); break;
-            case 32: e = launch_rstep<32>(maps, a, grid, stream); break;
-            case 48: e = launch_rstep<48>(maps, a, grid, stream); break;
-            case 64: e = launch_rstep<64>(maps, a, grid, stream); break;
-            case 80: e = launch_rstep<80>(maps, a, grid, stream); break;
-            case 96: e = launch_rstep<96>(maps, a, grid, stream); break;
-            case 112: e = launch_rstep<112>(maps, a, grid, stream); break;
-            case 128: e = launch_rstep<128>(maps, a, grid, stream); break;
-        }
-        if (e != cudaSuccess) return e;
+    // S2, then for every further iteration: the L-step's row statistics, the
+    // re-aggregated queries (S4) and the R-step on them; then S3 with the output
+    cudaError_t e = run_rstep(p, ws, k, v, 0, c_log2, status, wait_limit, stall, stream);
+    for (int it = 1; e == cudaSuccess && it < p.iters; it++) {
+        e = run_lstep(p, ws, q, out, kLsStat, c_log2, status, wait_limit, stall, stream);
+        if (e == cudaSuccess)
+            e = run_lstep(p, ws, q, out, kLsAgg, c_log2, status, wait_limit, stall, stream);
+        if (e == cudaSuccess)
+            e = run_rstep(p, ws, k, v, 1, c_log2, status, wait_limit, stall, stream);
     }
-    // S3
-    {
-        CUtensorMap maps[4];
-        const uint64_t dq[3] = {(uint64_t)kD, (uint64_t)p.b2, (uint64_t)p.BH * p.b1};
-        const uint64_t sq[2] = {kD * 2, (uint64_t)p.b2 * kD * 2};
-        const uint32_t bq[3] = {64, 1, 128};
-        const uint64_t dk[2] = {(uint64_t)kD, (uint64_t)p.BH * p.tiles * p.N};
-        const uint64_t sk[1] = {kD * 2};
-        const uint32_t bk[2] = {64, 128};
-        const uint64_t dh[2] = {16, (uint64_t)p.BH * p.tiles * p.N};
-        const uint64_t sh[1] = {32};
-        const uint32_t bh[2] = {16, 128};
-        if (!make_map(&maps[0], q, 3, dq, sq, bq) || !make_map(&maps[1], ws.ktil, 2, dk, sk, bk) ||
-            !make_map(&maps[2], ws.z, 2, dk, sk, bk) ||
-            !make_map(&maps[3], ws.hx, 2, dh, sh, bh, CU_TENSOR_MAP_SWIZZLE_32B))
-            return cudaErrorInvalidValue;
-        const int nq_max = tile_max_rows(p.b1, p.tiles);
-        const int npairs = ((nq_max + 127) / 128 + 1) / 2;
-        const int nprob = (p.unit_end - p.unit_begin) * p.b2 * npairs;
-        LsArgs a{p, (p.b1 + 127) / 128, npairs, nprob, p.unit_begin * p.b2 * npairs, c_log2,
-                 (__nv_bfloat16 *)out, status, wait_limit, stall};
-        cudaError_t e = set_smem(tc_lstep_kernel, ls::kSmem);
-        if (e != cudaSuccess) return e;
-        const int grid = nprob < sm_count() ? nprob : sm_count();
-        ProfileScope scope(K_TC_LSTEP, stream);
-        tc_lstep_kernel<<<grid, ls::kThreads, ls::kSmem, stream>>>(maps[0], maps[1], maps[2],
-                                                                   maps[3], a);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
+    if (e == cudaSuccess)
+        e = run_lstep(p, ws, q, out, kLsOut, c_log2, status, wait_limit, stall, stream);
+    return e;
 }
 
 }  // namespace monarch

@@ -22,8 +22,8 @@ MUTANTS = {
                              "const double *kr = k + ((int64_t)vp * b1 + up) * d;"),
     "values_from_keys": ("z += r * v[((int64_t)up * b2 + vp) * d + j];",
                          "z += r * k[((int64_t)up * b2 + vp) * d + j];"),
-    "output_from_ktilde": ("acc += L[(size_t)(u - u0) * b1 + up] * Z[(size_t)up * d + j];",
-                           "acc += L[(size_t)(u - u0) * b1 + up] * Kt[(size_t)up * d + j];"),
+    "output_from_ktilde": ("acc += L[(size_t)(u - u0) * b1k + up] * Z[(size_t)up * d + j];",
+                           "acc += L[(size_t)(u - u0) * b1k + up] * Kt[(size_t)up * d + j];"),
     "query_column_swapped": ("const double *qr = q + ((int64_t)u * b2 + c) * d;\n"
                              "                double mx",
                              "const double *qr = q + ((int64_t)c * b1 + u) * d;\n"

@@ -271,3 +271,70 @@ def test_golden_regression_rows():
         assert abs(got - float(val)) <= 1e-12 * max(1.0, abs(float(val)))
         n += 1
     assert n > 0
+
+
+# --------------------------------------------------------------------------
+# queries of a chunk of frames against a key/value cache (N_q != N_k)
+# --------------------------------------------------------------------------
+@pytest.fixture(scope="module")
+def chunk_and_cache():
+    """Queries of the last frame of a 3-frame clip against keys and values of all three
+    frames (the cache holds the two earlier ones): f_q = 1, f_k = 3, h = w = 8."""
+    q, k, v = synth.make_inputs(TINY)          # [1, 2, 192, 32]: frames of 64 tokens
+    return q[0][:, 128:], k[0], v[0]           # queries [2, 64, 32], keys/values [2, 192, 32]
+
+
+def brute_force_m_kv(L, R, b1, b1k, b2, tiles):
+    """M[(u,v),(u',v')] = L_v[u,u'] R_{u',g(u)}[v,v'] as a (b1*b2) x (b1k*b2) matrix."""
+    lo = [(g * b1) // tiles for g in range(tiles + 1)]
+    M = np.zeros((b1 * b2, b1k * b2))
+    for g in range(tiles):
+        for u in range(lo[g], lo[g + 1]):
+            for v in range(b2):
+                for up in range(b1k):
+                    M[u * b2 + v, up * b2:(up + 1) * b2] = L[v, u, up] * R[up, g, v, :]
+    return M
+
+
+def test_kv_with_the_clip_itself_is_the_self_attention_oracle(tiny):
+    q, k, v = tiny
+    for b1, b2, t, it in [(24, 8, 3, 2), (8, 24, 2, 1)]:
+        a = oracle.monarch_attn(q, k, v, b1, b2, t, it)
+        b = oracle.monarch_attn_kv(q, k, v, b1, b1, b2, t, it)
+        assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("iters", [1, 3])
+def test_kv_single_token_blocks_are_exact_rectangular_attention(chunk_and_cache, iters):
+    """b2 = 1: every R block is 1 x 1 and the L-step is softmax over all N_k keys."""
+    q, k, v = chunk_and_cache
+    y = oracle.monarch_attn_kv(q, k, v, 64, 192, 1, 1, iters)
+    assert rel(y, dense_attention(q, k, v)) < 1e-12
+
+
+@pytest.mark.parametrize("b1,b1k,b2", [(8, 24, 8), (1, 3, 64), (4, 12, 16)])
+def test_kv_one_query_row_per_tile_is_exact_rectangular_attention(chunk_and_cache, b1, b1k, b2):
+    """t = b1: each tile holds one query row, so R is that row's exact softmax within
+    each key block and L weighs the blocks by their log-sum-exp."""
+    q, k, v = chunk_and_cache
+    y = oracle.monarch_attn_kv(q, k, v, b1, b1k, b2, b1, 1)
+    assert rel(y, dense_attention(q, k, v)) < 1e-12
+
+
+def test_kv_zero_queries_give_the_mean_of_all_values(chunk_and_cache):
+    _, k, v = chunk_and_cache
+    q = np.zeros((2, 64, 32))
+    y = oracle.monarch_attn_kv(q, k, v, 8, 24, 8, 3, 2)
+    assert np.abs(y - v.mean(-2, keepdims=True)).max() < 1e-12
+
+
+@pytest.mark.parametrize("tiles,iters", [(1, 1), (3, 2)])
+def test_kv_brute_force_m_is_row_stochastic_and_reproduces_y(chunk_and_cache, tiles, iters):
+    q, k, v = chunk_and_cache
+    b1, b1k, b2 = 8, 24, 8
+    y, L, R = oracle.monarch_attn_kv(q, k, v, b1, b1k, b2, tiles, iters, factors=True)
+    for h in range(q.shape[0]):
+        M = brute_force_m_kv(L[h], R[h], b1, b1k, b2, tiles)
+        assert (M >= 0).all()
+        assert np.abs(M.sum(1) - 1).max() < 1e-12
+        assert rel(M @ v[h], y[h]) < 1e-12

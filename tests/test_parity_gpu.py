@@ -116,6 +116,31 @@ def test_tensor_core_edge_shapes(f, h, w, b1, b2, tiles):
     assert rel_fro(got, ref) <= TOL["bf16"]
 
 
+TC_ITER_EDGES = [
+    # f, h, w, b1, b2, tiles, iters
+    (2, 3, 100, 6, 100, 2, 2),      # b2 padded to 112, two aggregated-query tiles per block
+    (5, 60, 48, 300, 48, 5, 3),     # 60 queries per tile, three alternating rounds
+    (10, 100, 16, 1000, 16, 1, 2),  # 1000 queries per tile: 8 query chunks in the aggregation
+    (1, 64, 1, 64, 1, 2, 2),        # b2 = 1
+    (3, 4, 16, 12, 16, 12, 2),      # one query row per tile (t = b1)
+    (2, 100, 7, 200, 7, 3, 4),      # ragged chunks of 128 on both sides
+]
+
+
+@pytest.mark.parametrize("f,h,w,b1,b2,tiles,iters", TC_ITER_EDGES)
+def test_tensor_core_iterations_whole_output(f, h, w, b1, b2, tiles, iters):
+    """iters > 1 on the tensor cores: the L-step's row statistics, the re-aggregated
+    queries (S4) and the R-step on per-block queries, against the oracle."""
+    wl = TINY.replace(H=2, d=128, f=f, h=h, w=w, b1=b1, b2=b2, tiles=tiles, iters=iters)
+    q64, k64, v64 = (synth.round_to_dtype(x, "bf16") for x in synth.make_inputs(wl))
+    q, k, v = (to_torch(x, "bf16") for x in (q64, k64, v64))
+    assert kernel_path(q, f=f, h=h, w=w, b1=b1, b2=b2, tiles=tiles, iters=iters) == 1
+    ref = oracle.monarch_attn(q64, k64, v64, b1, b2, tiles, iters)
+    got = from_torch(run(wl, q, k, v), "bf16")
+    assert np.isfinite(got).all()
+    assert rel_fro(got, ref) <= TOL["bf16"]
+
+
 def test_chunk_480p_whole_output():
     wl = synth.WORKLOADS["480p_chunk"]
     q, k, v = device_inputs(wl)
@@ -195,9 +220,11 @@ def inputs_14b():
 def test_full_14b_iteration_sweep(inputs_14b, iters):
     wl = synth.WORKLOADS["14b"].replace(iters=iters)
     q, k, v = inputs_14b
+    assert kernel_path(q, f=wl.f, h=wl.h, w=wl.w, b1=wl.b1, b2=wl.b2, tiles=wl.tiles,
+                       iters=iters) == 1
     out = run(wl, q, k, v)
     convex_hull_check(out, v)
-    probs = sample_problems(wl, 8, seed=iters)
+    probs = sample_problems(wl, 64, seed=iters)
     assert sampled_error(wl, out, probs) <= TOL[wl.dtype]
 
 
@@ -331,3 +358,46 @@ def test_tensor_core_path_survives_a_tiny_wait_limit():
     q64, k64, v64 = (from_torch(x, wl.dtype) for x in (q, k, v))
     ref = oracle.monarch_attn(q64, k64, v64, wl.b1, wl.b2, wl.tiles, wl.iters)
     assert rel_fro(from_torch(out, wl.dtype), ref) <= TOL[wl.dtype]
+
+
+# --------------------------------------------------------------------------
+# a chunk of frames against a key/value cache (N_q != N_k)
+# --------------------------------------------------------------------------
+KV_CASES = [
+    # name, dtype, d, fq, fk, h, w, b2, tiles, iters, path
+    ("tiny", "f32", 32, 1, 3, 8, 8, 8, 3, 2, 0),
+    ("tiny", "bf16", 32, 2, 3, 8, 8, 8, 1, 1, 0),
+    ("480p_chunk", "bf16", 128, 1, 3, 8, 32, 32, 2, 1, 1),
+    ("480p_chunk", "bf16", 128, 2, 6, 30, 52, 52, 2, 2, 1),
+    ("480p_chunk", "bf16", 128, 3, 2, 10, 16, 16, 4, 1, 1),      # fewer key frames than query frames
+    ("480p_chunk", "bf16", 128, 1, 4, 64, 1, 1, 2, 1, 1),        # b2 = 1
+]
+
+
+@pytest.mark.parametrize("name,dtype,d,fq,fk,h,w,b2,tiles,iters,path", KV_CASES)
+def test_chunk_against_kv_cache_whole_output(name, dtype, d, fq, fk, h, w, b2, tiles, iters, path):
+    """Queries of the newest fq frames of a clip against keys and values of all fk frames."""
+    wl = synth.WORKLOADS[name].replace(H=2, d=d, f=max(fq, fk), h=h, w=w, b1=max(fq, fk) * h * w // b2,
+                                       b2=b2, tiles=1, iters=1, dtype=dtype)
+    q64, k64, v64 = (synth.round_to_dtype(x, dtype) for x in synth.make_inputs(wl))
+    nq, nk = fq * h * w, fk * h * w
+    q64 = np.ascontiguousarray(q64[..., wl.N - nq:, :])   # the chunk: the newest frames
+    k64 = np.ascontiguousarray(k64[..., wl.N - nk:, :])
+    v64 = np.ascontiguousarray(v64[..., wl.N - nk:, :])
+    b1, b1k = nq // b2, nk // b2
+    ref = oracle.monarch_attn_kv(q64, k64, v64, b1, b1k, b2, tiles, iters)
+    q, k, v = (to_torch(x, dtype) for x in (q64, k64, v64))
+    dt = _lib.F32 if dtype == "f32" else _lib.BF16
+    shape = (wl.B, wl.H, fq, fk, h, w, d, b1, b1k, b2, tiles, iters)
+    assert _lib.monarch_attn_kv_path(*shape, dt) == path
+    need = _lib.monarch_attn_kv_workspace_bytes(*shape, dt)
+    assert need > 0
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    out = torch.full_like(q, float("nan"))
+    assert _lib.monarch_attn_fwd_kv_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                       *shape, dt, ws.data_ptr(), need, None) == 0
+    torch.cuda.synchronize()
+    assert _lib.monarch_last_device_status(None) == 0
+    got = from_torch(out, dtype)
+    assert np.isfinite(got).all()
+    assert rel_fro(got, ref) <= TOL[dtype]
