@@ -67,3 +67,46 @@ def monarch_attention(q, k, v, *, f, h, w, b1, b2, tiles=1, iters=1, out=None, w
                                         workspace.numel() * workspace.element_size(), stream),
                "monarch_attn_fwd_ws")
     return out
+
+
+def monarch_attention_kv(q, k, v, *, fq, fk, h, w, b1, b1k, b2, tiles=1, iters=1, out=None):
+    """Queries of a chunk of fq frames [B, H, fq*h*w, d] against keys and values of
+    fk frames [B, H, fk*h*w, d] (a cache of earlier frames and the chunk's own)."""
+    if q.dim() != 4 or k.dim() != 4 or k.shape != v.shape:
+        raise ValueError("expected [B, H, N, d] tensors, k and v alike")
+    B, H, nq, d = q.shape
+    if nq != fq * h * w or k.shape != (B, H, fk * h * w, d):
+        raise ValueError("query or key/value lengths do not match the frame counts")
+    if out is None:
+        out = torch.empty_like(q)
+    for t in (q, k, v, out):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != q.dtype:
+            raise ValueError("contiguous CUDA tensors of one dtype expected")
+    dt = _DTYPES[q.dtype]
+    args = (B, H, fq, fk, h, w, d, b1, b1k, b2, tiles, iters)
+    need = _lib.monarch_attn_kv_workspace_bytes(*args, dt)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    _lib.check(_lib.monarch_attn_fwd_kv_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                           out.data_ptr(), *args, dt, ws.data_ptr(), need,
+                                           stream), "monarch_attn_fwd_kv_ws")
+    return out
+
+
+def monarch_attention_units(q, k, v, out, *, f, h, w, b1, b2, tiles=1, iters=1, unit_begin=0,
+                            unit_end=None):
+    """Computes only the (head, tile) units [unit_begin, unit_end) of the forward pass
+    (unit = (b*H + h)*tiles + g) into their rows of `out`; other rows are untouched."""
+    _check_tensors(q, k, v, out)
+    args = _shape_args(q, f, h, w, b1, b2, tiles, iters)
+    if unit_end is None:
+        unit_end = q.shape[0] * q.shape[1] * tiles
+    dt = _DTYPES[q.dtype]
+    need = _lib.monarch_attn_workspace_bytes(*args, dt)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    _lib.check(_lib.monarch_attn_fwd_units_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                              out.data_ptr(), *args, dt, unit_begin, unit_end,
+                                              ws.data_ptr(), need, stream),
+               "monarch_attn_fwd_units_ws")
+    return out

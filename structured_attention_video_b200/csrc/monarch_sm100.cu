@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(128) tc_qbar_kernel(const __nv_bfloat16 *__res
 // =====================================================================
 namespace ls {
 constexpr int kThreads = 512;
-constexpr int kSoftmaxRegs = 176, kEpilogueRegs = 96, kProducerRegs = 64;
+constexpr int kSoftmaxRegs = 160, kEpilogueRegs = 128, kProducerRegs = 64;
 static_assert(2 * kSoftmaxRegs + kEpilogueRegs + kProducerRegs == 4 * (65536 / kThreads),
               "the warpgroups' registers must add up to the launch's 128 per thread");
 // one pair of every kPolyEvery takes its exponentials on the FMA pipe (0: none).
@@ -198,6 +198,7 @@ struct LsProblem {
     int n_y, n_z, nkeys, nch;       // N side: chunk j starts at z = n_z + j*128
 };
 
+template <int MODE>
 __device__ __forceinline__ LsProblem ls_problem(const LsArgs &a, int unit) {
     const Problem &p = a.p;
     LsProblem q;
@@ -210,7 +211,7 @@ __device__ __forceinline__ LsProblem ls_problem(const LsArgs &a, int unit) {
     q.bh = unit / p.tiles;
     const int u_lo = tile_begin(q.g, p.b1, p.tiles), u_hi = tile_begin(q.g + 1, p.b1, p.tiles);
     const int slab = ((q.bh * p.tiles + q.g) * p.b2 + q.v) * p.b1k;   // Ktil row of block 0
-    if (a.mode != kLsAgg) {
+    if (MODE != kLsAgg) {
         q.m_y = q.v;
         q.m_first = u_lo + 256 * pair;
         q.m_z = q.bh * p.b1 + q.m_first;
@@ -240,6 +241,7 @@ __device__ __forceinline__ void ls_load(void *dst, const CUtensorMap *map, bool 
         tma_load_2d(dst, map, x, z, bar);
 }
 
+template <int MODE>
 __global__ void __launch_bounds__(ls::kThreads, 1)
 tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__ CUtensorMap tmN,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmX,
@@ -274,10 +276,10 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nmine = a.nprob > (int)blockIdx.x
                           ? (a.nprob - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-    const bool values = a.mode != kLsStat;   // products with the values (Z or the queries)
+    constexpr bool values = MODE != kLsStat;   // products with the values (Z or the queries)
     // the strided query gather (3-D map) is the M side, or in kLsAgg the N side;
     // the other side reads contiguous rows (2-D map)
-    const bool n_gather = a.mode == kLsAgg;
+    constexpr bool n_gather = MODE == kLsAgg;
 
     if (threadIdx.x == 0) {
         for (int t = 0; t < 2; t++) {
@@ -321,7 +323,7 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
             int issued[2] = {0, 0}, jc0 = 0;
             bool ok = true;
             for (int pi = 0; ok && pi < nmine; pi++) {
-                const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
+                const LsProblem pr = ls_problem<MODE>(a, blockIdx.x + pi * gridDim.x);
                 for (int j = 0; j < pr.nch; j++) {
                     const int jc = jc0 + j, sk = jc & 1;
                     if (jc >= 2 && !wait_warp(k_empty + sk, ((jc >> 1) - 1) & 1, w)) {
@@ -352,7 +354,7 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
             int qloads = 0;
             bool ok = true;
             for (int pi = 0; ok && pi < nmine; pi++) {
-                const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
+                const LsProblem pr = ls_problem<MODE>(a, blockIdx.x + pi * gridDim.x);
                 for (int t = 0; t < 2; t++) {
                     if (pi > 0 && !wait_warp(q_empty + t, (pi - 1) & 1, w)) {
                         ok = false;
@@ -368,7 +370,7 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                 if (!ok) break;
                 qloads++;
                 if (lane == 0 && pi + 1 < nmine) {
-                    const LsProblem nx = ls_problem(a, blockIdx.x + (pi + 1) * gridDim.x);
+                    const LsProblem nx = ls_problem<MODE>(a, blockIdx.x + (pi + 1) * gridDim.x);
                     for (int t = 0; t < 2; t++)
                         for (int pn = 0; pn < 2; pn++) {
                             if (!n_gather)
@@ -387,7 +389,7 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
             int issued_z[2] = {0, 0}, jc0 = 0;
             bool ok = true;
             for (int pi = 0; ok && pi < nmine; pi++) {
-                const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
+                const LsProblem pr = ls_problem<MODE>(a, blockIdx.x + pi * gridDim.x);
                 for (int j = 0; j < pr.nch; j++) {
                     const int jc = jc0 + j, st = jc & 1;
                     if (jc >= 2 && !wait_warp(z_empty + st, ((jc >> 1) - 1) & 1, w)) {
@@ -457,11 +459,11 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                 return true;
             };
             int jc0 = 0;
-            LsProblem pr = nmine > 0 ? ls_problem(a, blockIdx.x) : LsProblem{};
+            LsProblem pr = nmine > 0 ? ls_problem<MODE>(a, blockIdx.x) : LsProblem{};
             if (ok && nmine > 0) ok = issue_s(0, 0, 0, 0, pr.nch) && issue_s(1, 0, 0, 0, pr.nch);
             for (int pi = 0; ok && pi < nmine; pi++) {
                 const bool has_next = pi + 1 < nmine;
-                const LsProblem nx = has_next ? ls_problem(a, blockIdx.x + (pi + 1) * gridDim.x) : pr;
+                const LsProblem nx = has_next ? ls_problem<MODE>(a, blockIdx.x + (pi + 1) * gridDim.x) : pr;
                 for (int j = 0; ok && j < pr.nch; j++) {
                     const int jc = jc0 + j;
                     const bool last = j == pr.nch - 1, more = !last || has_next;
@@ -485,7 +487,7 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
         bool ok = values;
         for (int pi = 0; ok && pi < nmine; pi++) {
-            const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
+            const LsProblem pr = ls_problem<MODE>(a, blockIdx.x + pi * gridDim.x);
             for (int t = 0; t < 2; t++) {
                 if (!wait_warp(o_full + t, pi & 1, w) || !wait_warp(l_full + t, pi & 1, w)) {
                     ok = false;
@@ -533,7 +535,7 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                             // kLsOut: Y row (u, v); kLsAgg: aggregated query of block
                             // u' = m for row g*b2 + v
                             const int64_t orow =
-                                a.mode == kLsOut
+                                MODE == kLsOut
                                     ? (int64_t)pr.bh * p.N + (int64_t)m * p.b2 + pr.v
                                     : ((int64_t)pr.bh * p.b1k + m) * a.mpad + pr.g * p.b2 + pr.v;
                             *reinterpret_cast<uint4 *>(a.out + orow * kD + hf * 64 + c * 8) = val;
@@ -555,7 +557,7 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
         bool ok = true;
         int jc0 = 0;
         for (int pi = 0; ok && pi < nmine; pi++) {
-            const LsProblem pr = ls_problem(a, blockIdx.x + pi * gridDim.x);
+            const LsProblem pr = ls_problem<MODE>(a, blockIdx.x + pi * gridDim.x);
             float m_run = -INFINITY, l_run = 0.f;
             for (int j = 0; j < pr.nch; j++) {
                 const int jc = jc0 + j;
@@ -686,6 +688,8 @@ struct RsArgs {
     // loaded once per head; 1: per block u' (later iterations), tile mt of block
     // u' at rows (bh*b1 + u')*mpad + mt*128, loaded per item into slot mt
     int qblk;
+    int hdirect;         // 1: entropy panel rows by plain stores (no staging room)
+    uint4 *hx;           // entropy panels [BH][t*b2][b1k] rows of 32 bytes (hdirect)
     int *status;
     long long limit;
     int stall;           // test hook: the MMA warp first waits on a barrier nothing completes
@@ -699,10 +703,16 @@ struct RsLayout {
     static constexpr uint32_t kPanelKV = B2P * 128;
     __host__ __device__ static uint32_t kv(int nmt) { return (uint32_t)nmt * kTile; }
     __host__ __device__ static uint32_t stg(int nmt) { return kv(nmt) + 2 * kStage; }
-    // entropy-panel staging of the softmax warps: 4 warps x 32 rows x 32 B
+    // entropy-panel staging of the softmax warps: 4 warps x 32 rows x 32 B, when
+    // it fits (hdirect = 0); otherwise each softmax thread stores its panel row
+    // with plain stores (hdirect = 1, no staging)
     __host__ __device__ static uint32_t hstg(int nmt) { return stg(nmt) + 4 * 8192; }
-    __host__ __device__ static uint32_t bar(int nmt) { return hstg(nmt) + 4 * 1024; }
-    __host__ __device__ static uint32_t smem(int nmt) { return bar(nmt) + 256 + 1024; }
+    __host__ __device__ static uint32_t bar(int nmt, int hdirect) {
+        return hstg(nmt) + (hdirect ? 0 : 4 * 1024);
+    }
+    __host__ __device__ static uint32_t smem(int nmt, int hdirect) {
+        return bar(nmt, hdirect) + 256 + 1024;
+    }
 };
 
 template <int B2P>
@@ -715,7 +725,7 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     const int nmt = a.nmt;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::bar(nmt));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::bar(nmt, a.hdirect));
     uint64_t *q_full = bars + 0;
     uint64_t *q_empty = bars + 1;
     uint64_t *kv_full = bars + 2;    // [2]
@@ -945,19 +955,28 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 const __nv_bfloat16 lo = __float2bfloat16_rn(hp - __bfloat162float(hi));
                 const uint32_t pair = (uint32_t)__bfloat16_as_ushort(hi) |
                                       ((uint32_t)__bfloat16_as_ushort(lo) << 16);
-                // the warp's 32 panel rows (32 B each) leave in one TMA store, which
-                // clips the rows past t*b2; the previous item's store must have
-                // finished reading the staging first
-                uint8_t *hs = sm + L::hstg(nmt) + wq * 1024;
-                if (lane == 0) tma_store_wait_read_all();
-                __syncwarp();
-                *reinterpret_cast<uint4 *>(hs + lane * 32) = make_uint4(pair, 0u, 0u, 0u);
-                *reinterpret_cast<uint4 *>(hs + lane * 32 + 16) = make_uint4(0u, 0u, 0u, 0u);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_4d(&tmHs, hs, 0, up, mt * 128 + wq * 32, bh);
-                    tma_store_commit();
+                if (a.hdirect) {
+                    const int row = mt * 128 + wq * 32 + lane;
+                    if (row < p.tiles * p.b2) {
+                        uint4 *dst = a.hx + (((int64_t)bh * p.tiles * p.b2 + row) * p.b1k + up) * 2;
+                        dst[0] = make_uint4(pair, 0u, 0u, 0u);
+                        dst[1] = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                } else {
+                    // the warp's 32 panel rows (32 B each) leave in one TMA store,
+                    // which clips the rows past t*b2; the previous item's store must
+                    // have finished reading the staging first
+                    uint8_t *hs = sm + L::hstg(nmt) + wq * 1024;
+                    if (lane == 0) tma_store_wait_read_all();
+                    __syncwarp();
+                    *reinterpret_cast<uint4 *>(hs + lane * 32) = make_uint4(pair, 0u, 0u, 0u);
+                    *reinterpret_cast<uint4 *>(hs + lane * 32 + 16) = make_uint4(0u, 0u, 0u, 0u);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_4d(&tmHs, hs, 0, up, mt * 128 + wq * 32, bh);
+                        tma_store_commit();
+                    }
                 }
             }
             const uint64_t inv2 = f2_pack(inv, inv);
@@ -1073,10 +1092,10 @@ int b2_padded(int b2) { return (b2 + 15) / 16 * 16; }
 int qbar_tiles(const Problem &p) { return (p.tiles * p.b2 + 127) / 128; }
 size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-uint32_t rstep_smem(int b2p, int nmt) {
+uint32_t rstep_smem(int b2p, int nmt, int hdirect) {
     switch (b2p) {
 #define MONARCH_RS_CASE(V) \
-    case V: return RsLayout<V>::smem(nmt);
+    case V: return RsLayout<V>::smem(nmt, hdirect);
         MONARCH_RS_CASE(16) MONARCH_RS_CASE(32) MONARCH_RS_CASE(48) MONARCH_RS_CASE(64)
         MONARCH_RS_CASE(80) MONARCH_RS_CASE(96) MONARCH_RS_CASE(112) MONARCH_RS_CASE(128)
 #undef MONARCH_RS_CASE
@@ -1121,7 +1140,7 @@ cudaError_t set_smem(K kernel, uint32_t bytes) {
 
 template <int B2P>
 cudaError_t launch_rstep(const CUtensorMap *maps, const RsArgs &a, int grid, cudaStream_t s) {
-    const uint32_t smem = RsLayout<B2P>::smem(a.nmt);
+    const uint32_t smem = RsLayout<B2P>::smem(a.nmt, a.hdirect);
     cudaError_t e = set_smem(tc_rstep_kernel<B2P>, smem);
     if (e != cudaSuccess) return e;
     tc_rstep_kernel<B2P><<<grid, 384, smem, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
@@ -1143,7 +1162,7 @@ bool sm100_supports(const Problem &p, monarch_dtype dtype) {
     // later iterations keep one slot per aggregated-query tile
     if (p.iters > 1 && qbar_tiles(p) > kMaxQbarTiles) return false;
     if (p.iters > 1 && (int64_t)p.BH * p.b1k * qbar_tiles(p) * 128 + 256 >= (1LL << 31)) return false;
-    if (rstep_smem(b2_padded(p.b2), qbar_tiles(p)) > (uint32_t)kMaxSmem) return false;
+    if (rstep_smem(b2_padded(p.b2), qbar_tiles(p), 1) > (uint32_t)kMaxSmem) return false;
     // TMA coordinates are 32-bit: every row index must fit
     if ((int64_t)p.BH * p.tiles * p.Nk + 256 >= (1LL << 31)) return false;
     if ((int64_t)p.BH * p.Nk + 256 >= (1LL << 31) || (int64_t)p.BH * p.N + 256 >= (1LL << 31))
@@ -1213,7 +1232,9 @@ cudaError_t run_rstep(const Problem &p, const TcWorkspace &ws, const void *k, co
     const int sms = sm_count();
     const int bpc = (total + sms - 1) / sms;
     const int grid = (total + bpc - 1) / bpc;
-    RsArgs a{p, nmt, mpad, bpc, c_log2, 1.f / c_log2, qblk, status, wait_limit, stall};
+    const int hdirect = rstep_smem(b2p, nmt, 0) > (uint32_t)kMaxSmem ? 1 : 0;
+    RsArgs a{p, nmt, mpad, bpc, c_log2, 1.f / c_log2, qblk, hdirect, ws.hx, status, wait_limit,
+             stall};
     ProfileScope scope(K_TC_RSTEP, stream);
     switch (b2p) {
         case 16: return launch_rstep<16>(maps, a, grid, stream);
@@ -1248,15 +1269,27 @@ cudaError_t run_lstep(const Problem &p, const TcWorkspace &ws, const void *q, vo
     const int nprob = (p.unit_end - p.unit_begin) * p.b2 * npairs;
     LsArgs a{p, mode, npairs, nprob, p.unit_begin * p.b2 * npairs, mpad, c_log2,
              agg ? ws.qblk : (__nv_bfloat16 *)out, ws.lam, status, wait_limit, stall};
-    cudaError_t e = set_smem(tc_lstep_kernel, ls::kSmem);
-    if (e != cudaSuccess) return e;
     const int grid = nprob < sm_count() ? nprob : sm_count();
     ProfileScope scope(mode == kLsOut ? K_TC_LSTEP : mode == kLsStat ? K_TC_LSTAT : K_TC_QAGG,
                        stream);
-    if (agg)
-        tc_lstep_kernel<<<grid, ls::kThreads, ls::kSmem, stream>>>(kt, qg, qg, xp, a);
-    else
-        tc_lstep_kernel<<<grid, ls::kThreads, ls::kSmem, stream>>>(qg, kt, zt, xp, a);
+    cudaError_t e;
+    switch (mode) {
+        case kLsOut:
+            e = set_smem(tc_lstep_kernel<kLsOut>, ls::kSmem);
+            if (e != cudaSuccess) return e;
+            tc_lstep_kernel<kLsOut><<<grid, ls::kThreads, ls::kSmem, stream>>>(qg, kt, zt, xp, a);
+            break;
+        case kLsStat:
+            e = set_smem(tc_lstep_kernel<kLsStat>, ls::kSmem);
+            if (e != cudaSuccess) return e;
+            tc_lstep_kernel<kLsStat><<<grid, ls::kThreads, ls::kSmem, stream>>>(qg, kt, zt, xp, a);
+            break;
+        default:
+            e = set_smem(tc_lstep_kernel<kLsAgg>, ls::kSmem);
+            if (e != cudaSuccess) return e;
+            tc_lstep_kernel<kLsAgg><<<grid, ls::kThreads, ls::kSmem, stream>>>(kt, qg, qg, xp, a);
+            break;
+    }
     return cudaGetLastError();
 }
 

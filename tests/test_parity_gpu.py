@@ -182,6 +182,7 @@ def inputs_480p():
 def test_full_480p_tile_sweep(inputs_480p, tiles):
     wl = synth.WORKLOADS["480p_full"].replace(tiles=tiles)
     q, k, v = inputs_480p
+    assert kernel_path(q, f=wl.f, h=wl.h, w=wl.w, b1=wl.b1, b2=wl.b2, tiles=tiles) == 1
     out = run(wl, q, k, v)
     convex_hull_check(out, v)
     probs = sample_problems(wl, 12, seed=tiles)
