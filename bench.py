@@ -682,6 +682,9 @@ def main():
                     help="timed steps of the 480p full clip reported beside the line (0: skip)")
     ap.add_argument("--heads", type=int, default=0,
                     help="override H (smaller cases for ncu captures; not a bench line)")
+    ap.add_argument("--iters", type=int, default=0,
+                    help="override the alternating rounds (captures of the iteration kernels; "
+                         "not a bench line)")
     ap.add_argument("--shard", action="store_true",
                     help="N > 1: split ONE clip's (head, tile) units across the ranks "
                          "(strong scaling) instead of one clip per rank")
@@ -707,6 +710,8 @@ def main():
     wl = synth.WORKLOADS[args.workload]
     if args.heads > 0:
         wl = wl.replace(H=args.heads)
+    if args.iters > 0:
+        wl = wl.replace(iters=args.iters)
 
     if args.impl == "reference":
         run_reference(args, wl, world, rank)

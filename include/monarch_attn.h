@@ -87,6 +87,10 @@ typedef enum {
  *   tiles     tiles per block, 1 <= tiles <= b1.   iters  alternating rounds, >= 1.
  * The workspace (monarch_attn_workspace_bytes) is taken with stream-ordered
  * cudaMallocAsync on `stream` and released with cudaFreeAsync on it.
+ * Source: MonarchRT explainer page, "Monarch矩阵" (M = P L P^T R), "创新一"
+ * (blocks aligned to the latent grid) and "创新二" (tiles); the entropy term
+ * and the alternating rounds: VMonarch abstract (MonarchAttention's
+ * variational form).
  */
 MONARCH_API monarch_status monarch_attn_fwd(const void *q, const void *k, const void *v, void *out,
                                 int B, int H, int f, int h, int w, int d, int b1, int b2,
@@ -119,6 +123,8 @@ MONARCH_API monarch_status monarch_attn_fwd(const void *q, const void *k, const 
  * the contents of the last call; nothing in it needs to start at zero.  Calls
  * that overlap on the GPU (different streams without ordering, or several host
  * threads) race on the array and give wrong results: serialise them.
+ * Source: the operation of monarch_attn_fwd; the allocation-free form has no
+ * counterpart in the pages.
  */
 #define MONARCH_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 
@@ -133,7 +139,8 @@ MONARCH_API monarch_status monarch_attn_fwd_noalloc(const void *q, const void *k
  * the arguments fail validation.  Pure host function; enqueues nothing.
  * The workspace holds the aggregated queries, Ktil = R K and Z = R V for
  * every (head, tile, column, block), the entropies H and, for iters > 1,
- * the row log-sum-exp of the L-step.
+ * the per-block aggregated queries and the row log-sum-exp of the L-step.
+ * Source: no counterpart in the pages (a property of this implementation).
  */
 MONARCH_API size_t monarch_attn_workspace_bytes(int B, int H, int f, int h, int w, int d, int b1, int b2,
                                     int tiles, int iters, monarch_dtype dtype);
@@ -144,6 +151,7 @@ MONARCH_API size_t monarch_attn_workspace_bytes(int B, int H, int f, int h, int 
  * as monarch_attn_fwd.  Returns MONARCH_ERR_NO_MEMORY if ws_bytes is too small.
  * The workspace contents need no initialisation and are garbage afterwards.
  * Two calls that share a workspace must not overlap on the GPU.
+ * Source: as monarch_attn_fwd.
  */
 MONARCH_API monarch_status monarch_attn_fwd_ws(const void *q, const void *k, const void *v, void *out,
                                    int B, int H, int f, int h, int w, int d, int b1, int b2,
@@ -164,6 +172,7 @@ MONARCH_API monarch_status monarch_attn_fwd_ws(const void *q, const void *k, con
  * workspace size does not depend on the range; the tensor-core path computes
  * the R-step of every tile of the heads that the range touches).
  * Returns MONARCH_ERR_SHAPE for a range outside [0, B*H*tiles].
+ * Source: explainer page, "创新二：平铺Monarch参数化" (independent tiles).
  */
 MONARCH_API monarch_status monarch_attn_fwd_units_ws(const void *q, const void *k, const void *v,
                                                      void *out, int B, int H, int f, int h, int w,
@@ -189,6 +198,9 @@ MONARCH_API monarch_status monarch_attn_fwd_units_ws(const void *q, const void *
  * Workspace: monarch_attn_kv_workspace_bytes (0 if the arguments fail
  * validation).  Errors and ownership as monarch_attn_fwd_ws.
  * monarch_attn_kv_path reports the kernel family as monarch_attn_path does.
+ * Source: summary page, "Setup" (chunked autoregressive generation with a
+ * cache of earlier frames); the factor shapes b1 x b1k are this library's
+ * reading of the method for unequal query and key lengths.
  */
 MONARCH_API size_t monarch_attn_kv_workspace_bytes(int B, int H, int fq, int fk, int h, int w,
                                                    int d, int b1, int b1k, int b2, int tiles,
@@ -209,6 +221,7 @@ MONARCH_API monarch_status monarch_attn_fwd_kv_ws(const void *q, const void *k, 
  * cudaMallocAsync on `stream`; the call enqueues host-to-device copies, the
  * forward pass and the device-to-host copy of `out`, then releases the device
  * memory, all on `stream`.  `out` is valid once the stream has synchronised.
+ * Source: as monarch_attn_fwd (host buffers: no counterpart in the pages).
  */
 MONARCH_API monarch_status monarch_attn_fwd_host(const void *q, const void *k, const void *v, void *out,
                                      int B, int H, int f, int h, int w, int d, int b1, int b2,
@@ -221,6 +234,9 @@ MONARCH_API monarch_status monarch_attn_fwd_host(const void *q, const void *k, c
  *   u_of_n[n] = n / b2, v_of_n[n] = n % b2, perm[n] = v*b1 + u   (each N entries),
  *   tile_begin[g] = floor(g*b1/tiles) for g = 0..tiles        (tiles + 1 entries).
  * Any output pointer may be NULL to skip it.
+ * Source: explainer page, "Monarch矩阵" (the permutation between the two
+ * block-diagonal factors), "创新一" (N = f*h*w in blocks of (f*h, w)) and
+ * "创新二" (tiles of the block rows).
  */
 MONARCH_API monarch_status monarch_index_maps(int f, int h, int w, int b1, int b2, int tiles,
                                   int32_t *u_of_n, int32_t *v_of_n, int32_t *perm,
@@ -229,6 +245,7 @@ MONARCH_API monarch_status monarch_index_maps(int f, int h, int w, int b1, int b
 /*
  * The same maps computed by a kernel on the device into device buffers
  * (sizes as above; NULL skips a map), enqueued on `stream`.
+ * Source: as monarch_index_maps.
  */
 MONARCH_API monarch_status monarch_index_maps_device(int f, int h, int w, int b1, int b2, int tiles,
                                          int32_t *u_of_n, int32_t *v_of_n, int32_t *perm,
@@ -240,6 +257,7 @@ MONARCH_API monarch_status monarch_index_maps_device(int f, int h, int w, int b1
  * gives up it records MONARCH_ERR_TIMEOUT there and the kernel returns early
  * (its output is then incomplete).  Returns MONARCH_OK if no wait gave up,
  * MONARCH_ERR_CUDA if the synchronisation failed.
+ * Source: no counterpart in the pages (failure detection of this library).
  */
 MONARCH_API monarch_status monarch_last_device_status(monarch_stream_t stream);
 
@@ -247,6 +265,7 @@ MONARCH_API monarch_status monarch_last_device_status(monarch_stream_t stream);
  * Test hook: the iteration limit of the device-side bounded waits (spins on an
  * mbarrier).  0 restores the default.  Takes effect for launches enqueued after
  * the call, on every device.  Returns the previous limit.
+ * Source: no counterpart in the pages (a test facility of this library).
  */
 MONARCH_API long long monarch_set_wait_limit(long long spins);
 
@@ -267,6 +286,7 @@ MONARCH_API int monarch_debug_inject_stall(int on);
  * Benchmark hook: per-kernel timing.  While enabled (on != 0), every kernel
  * launch of the forward pass is bracketed by CUDA events recorded on its launch
  * stream; the launches themselves are unchanged.  Disabling keeps the counters.
+ * Source: no counterpart in the pages (a measurement facility).
  */
 MONARCH_API monarch_status monarch_profile_enable(int on);
 
@@ -276,20 +296,25 @@ MONARCH_API monarch_status monarch_profile_enable(int on);
  * (ms[k]) and launch count (launches[k]) since the previous call, then resets
  * the counters.  Either array may be NULL.  Returns the number of kernel
  * families (the valid k), or -1 if waiting on an event failed.
+ * Source: no counterpart in the pages (a measurement facility).
  */
 MONARCH_API int monarch_profile_collect(double *ms, long long *launches, int max_kernels);
 
-/* Name of kernel family k (static string), or NULL if k is out of range. */
+/* Name of kernel family k (static string), or NULL if k is out of range.
+ * Source: no counterpart in the pages. */
 MONARCH_API const char *monarch_profile_kernel_name(int k);
 
-/* Static, NUL-terminated description of a status code. */
+/* Static, NUL-terminated description of a status code.
+ * Source: no counterpart in the pages. */
 MONARCH_API const char *monarch_status_string(monarch_status status);
 
 /*
  * Which kernel family a call with these arguments dispatches to:
  * 0 = generic SIMT kernels (any supported shape, float32 or bfloat16),
- * 1 = sm_100a tensor-core kernels (bfloat16, d = 128, b2 <= 128, iters = 1),
+ * 1 = sm_100a tensor-core kernels (bfloat16, d = 128, b2 <= 128, the R-step's
+ *     shared-memory plan fits; any iteration count),
  * -1 = the arguments fail validation.  Pure host function.
+ * Source: no counterpart in the pages (dispatch of this library).
  */
 MONARCH_API int monarch_attn_path(int B, int H, int f, int h, int w, int d, int b1, int b2, int tiles,
                       int iters, monarch_dtype dtype);

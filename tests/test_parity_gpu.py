@@ -2,10 +2,10 @@
 
 Tolerances: relative Frobenius error <= 1e-5 for float32 inputs and <= 1e-2 for
 bfloat16 inputs (float32 accumulation); index maps bit-exact.  Small shapes
-compare the whole output; the full-size shapes of the benchmark compare sampled
-(head, tile, column) problems, which the oracle computes one by one, plus
-properties that hold at any size (every output row is a convex combination of
-value rows)."""
+compare the whole output, and so does the 720p clip of the benchmark (every
+head, tile and column, the oracle solving them one by one); the other full-size
+shapes compare sampled (head, tile, column) problems plus properties that hold
+at any size (every output row is a convex combination of value rows)."""
 import numpy as np
 import pytest
 
@@ -15,7 +15,8 @@ from oracle import oracle  # noqa: E402
 from structured_attention_video_b200 import _lib, synth  # noqa: E402
 from structured_attention_video_b200.attention import kernel_path, monarch_attention  # noqa: E402
 
-from helpers import TOL, device_inputs, from_torch, rel_fro, sample_problems, sampled_error, to_torch  # noqa: E402
+from helpers import (TOL, device_inputs, from_torch, oracle_on_samples, rel_fro,  # noqa: E402
+                     sample_problems, sampled_error, to_torch)
 
 pytestmark = pytest.mark.gpu
 
@@ -202,6 +203,29 @@ def test_full_720p_headline(inputs_720p):
     convex_hull_check(out, v)
     probs = sample_problems(wl, 24, seed=720)
     assert sampled_error(wl, out, probs) <= TOL[wl.dtype]
+
+
+def test_full_720p_whole_output(inputs_720p):
+    """Every output element of the 720p clip against the oracle: all heads x tiles x
+    columns, head by head (the oracle regenerates each head from the seeded
+    generator); the error bound holds for the whole output and for every head."""
+    wl = synth.WORKLOADS["720p"]
+    q, k, v = inputs_720p
+    out = run(wl, q, k, v)
+    probs = [(bh, g, c) for bh in range(wl.B * wl.H) for g in range(wl.tiles)
+             for c in range(wl.b2)]
+    ref = oracle_on_samples(wl, probs)
+    num = den = 0.0
+    for bh in range(wl.B * wl.H):
+        b, h = divmod(bh, wl.H)
+        got = from_torch(out[b, h], wl.dtype)
+        assert not np.isnan(ref[bh]).any()
+        e2 = float(np.sum((got - ref[bh]) ** 2))
+        r2 = float(np.sum(ref[bh] ** 2))
+        assert np.sqrt(e2 / r2) <= TOL[wl.dtype], bh
+        num += e2
+        den += r2
+    assert np.sqrt(num / den) <= TOL[wl.dtype]
 
 
 def test_full_720p_deterministic(inputs_720p):
