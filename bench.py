@@ -301,11 +301,14 @@ def kernel_traffic(name: str):
         rec = json.load(fh).get(name)
     if not rec:
         return None
-    src = os.path.join(ROOT, "structured_attention_video_b200", "csrc", rec["source"])
-    if not os.path.exists(src):
-        return None
-    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    return rec["dram_bytes_per_launch"] if digest == rec["source_sha256"] else None
+    # the kernel's sources (its .cu and the headers it inlines), hashed in order
+    h = hashlib.sha256()
+    for name_ in rec["sources"]:
+        src = os.path.join(ROOT, "structured_attention_video_b200", "csrc", name_)
+        if not os.path.exists(src):
+            return None
+        h.update(open(src, "rb").read())
+    return rec["dram_bytes_per_launch"] if h.hexdigest() == rec["sources_sha256"] else None
 
 
 # ---------------------------------------------------------------------------

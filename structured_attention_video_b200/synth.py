@@ -73,17 +73,18 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
     def monarch_flops(self) -> float:
-        """Algorithmic FLOPs of the forward pass (multiply-add = 2).
+        """Algorithmic FLOPs of the forward pass (multiply-add = 2): the work the
+        method needs, not what a given kernel schedule issues.
 
-        Per (b, h) and iteration: the R-step does 6*t*N*b2*d (logits plus the
-        two products with [V | K]); the L-step does 4*N*b1*d (logits plus the
-        product with Z); every iteration after the first re-aggregates the
-        queries with L (2*N*b1*d).
+        Per (b, h): every iteration's R-step takes the logits of the aggregated
+        queries against each key block and Ktil = R K (2 + 2 = 4*t*N*b2*d); the
+        last one also forms Z = R V (2*t*N*b2*d more).  Every iteration's L-step
+        takes the logits q.Ktil (2*N*b1*d) and then either re-aggregates the
+        queries with L (iterations before the last) or forms Y = L Z (the last),
+        2*N*b1*d either way.  Total (4T + 2)*t*N*b2*d + 4T*N*b1*d.
         """
         T, t, N = self.iters, self.tiles, self.N
-        per_head = (6 * t * N * self.b2 * self.d * T
-                    + 4 * N * self.b1 * self.d * T
-                    + 2 * N * self.b1 * self.d * (T - 1))
+        per_head = (4 * T + 2) * t * N * self.b2 * self.d + 4 * T * N * self.b1 * self.d
         return float(self.B * self.H * per_head)
 
     def dense_flops(self) -> float:

@@ -88,13 +88,14 @@ def test_generic_kernels_report_against_the_alu_peak():
     assert r["peak"] == pytest.approx(148 * 128 * 2 * 1965.0e6 / 1e12)
 
 
-def _fake_tree(tmp_path, source_text, recorded_text):
+def _fake_tree(tmp_path, source_text, recorded_text, header_text="h", recorded_header="h"):
     csrc = tmp_path / "structured_attention_video_b200" / "csrc"
     csrc.mkdir(parents=True)
     (csrc / "k.cu").write_text(source_text)
+    (csrc / "k.cuh").write_text(header_text)
     (tmp_path / "profiles").mkdir()
-    rec = {"tc_lstep_kernel": {"source": "k.cu",
-                               "source_sha256": hashlib.sha256(recorded_text.encode()).hexdigest(),
+    digest = hashlib.sha256((recorded_text + recorded_header).encode()).hexdigest()
+    rec = {"tc_lstep_kernel": {"sources": ["k.cu", "k.cuh"], "sources_sha256": digest,
                                "dram_bytes_per_launch": 123.0}}
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
 
@@ -112,12 +113,19 @@ def test_traffic_is_null_once_the_kernel_changed(tmp_path, monkeypatch):
     assert bench.kernel_traffic("tc_lstep_kernel") is None
 
 
+def test_traffic_is_null_once_an_inlined_header_changed(tmp_path, monkeypatch):
+    _fake_tree(tmp_path, "kernel v1", "kernel v1", header_text="h2", recorded_header="h1")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.kernel_traffic("tc_lstep_kernel") is None
+
+
 def test_committed_traffic_record_names_existing_sources():
     with open(os.path.join(ROOT, "profiles", "traffic.json")) as fh:
         rec = json.load(fh)
     for name, entry in rec.items():
-        assert os.path.exists(os.path.join(ROOT, "structured_attention_video_b200", "csrc",
-                                           entry["source"])), name
+        for src in entry["sources"]:
+            assert os.path.exists(os.path.join(ROOT, "structured_attention_video_b200", "csrc",
+                                               src)), name
         assert entry["dram_bytes_per_launch"] > 0
 
 
