@@ -59,29 +59,39 @@ __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, const 
 // =====================================================================
 // S1: aggregated queries
 // =====================================================================
-__global__ void __launch_bounds__(128) tc_qbar_kernel(const __nv_bfloat16 *__restrict__ q,
-                                                      __nv_bfloat16 *__restrict__ qbar, Problem p,
-                                                      int mpad) {
+// Block: 512 threads = 4 row groups x 128 column threads.  Column thread c owns
+// 8 consecutive elements of the flattened (v, d) row; row group r sums a quarter
+// of the tile's rows, so four times as many 16-byte loads are in flight as with
+// one thread per column (the kernel is bound by memory latency, not bandwidth,
+// with B*H*t*ceil(b2*d/1024) blocks).  The four partial sums meet in shared
+// memory in a fixed order.
+constexpr int kQbarGroups = 4;
+__global__ void __launch_bounds__(128 * kQbarGroups) tc_qbar_kernel(
+    const __nv_bfloat16 *__restrict__ q, __nv_bfloat16 *__restrict__ qbar, Problem p, int mpad) {
+    __shared__ float part[kQbarGroups - 1][8][128];
     const int row_elems = p.b2 * kD;
     const int nchunk = (row_elems / 8 + 127) / 128;
     const int chunk = blockIdx.x % nchunk;
+    const int grp = threadIdx.x >> 7, tid = threadIdx.x & 127;
     // every tile of the heads that the unit range touches (the R-step reads all
     // of a head's aggregated rows, padding included)
     const int bhg = blockIdx.x / nchunk + p.head_begin() * p.tiles;
     const int g = bhg % p.tiles, bh = bhg / p.tiles;
-    const int col = (chunk * 128 + threadIdx.x) * 8;
+    const int col = (chunk * 128 + tid) * 8;
     const int u0 = tile_begin(g, p.b1, p.tiles), u1 = tile_begin(g + 1, p.b1, p.tiles);
-    if (col < row_elems) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(q + (int64_t)bh * p.N * kD +
-                                                           (int64_t)u0 * row_elems + col);
-        const int64_t stride = row_elems / 8;
-        float acc[8];
+    // rows [r0, r1) of this group: a contiguous quarter of the tile
+    const int n = u1 - u0;
+    const int r0 = u0 + (grp * n) / kQbarGroups, r1 = u0 + ((grp + 1) * n) / kQbarGroups;
+    const bool active = col < row_elems;
+    float acc[8];
 #pragma unroll
-        for (int i = 0; i < 8; i++) acc[i] = 0.f;
-        int u = u0;
-        // eight independent 16-byte loads in flight per thread: the grid has only
-        // B*H*t*ceil(b2*d/1024) blocks, too few warps to cover the memory latency
-        for (; u + 8 <= u1; u += 8) {
+    for (int i = 0; i < 8; i++) acc[i] = 0.f;
+    if (active) {
+        const int64_t stride = row_elems / 8;
+        const uint4 *src = reinterpret_cast<const uint4 *>(q + (int64_t)bh * p.N * kD +
+                                                           (int64_t)r0 * row_elems + col);
+        int u = r0;
+        for (; u + 8 <= r1; u += 8) {   // eight independent 16-byte loads in flight
             uint4 x[8];
 #pragma unroll
             for (int k = 0; k < 8; k++) x[k] = __ldg(src + k * stride);
@@ -97,7 +107,7 @@ __global__ void __launch_bounds__(128) tc_qbar_kernel(const __nv_bfloat16 *__res
                 }
             }
         }
-        for (; u < u1; u++) {
+        for (; u < r1; u++) {
             uint4 x = __ldg(src);
             src += stride;
             const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&x);
@@ -108,14 +118,25 @@ __global__ void __launch_bounds__(128) tc_qbar_kernel(const __nv_bfloat16 *__res
                 acc[2 * i + 1] += f.y;
             }
         }
-        const float inv = 1.f / (float)(u1 - u0);
+    }
+    if (grp > 0) {
+#pragma unroll
+        for (int i = 0; i < 8; i++) part[grp - 1][i][tid] = acc[i];
+    }
+    __syncthreads();
+    if (grp == 0 && active) {
+#pragma unroll
+        for (int r = 0; r < kQbarGroups - 1; r++)
+#pragma unroll
+            for (int i = 0; i < 8; i++) acc[i] += part[r][i][tid];
+        const float inv = 1.f / (float)n;
         uint4 o;
         uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
 #pragma unroll
         for (int i = 0; i < 4; i++) ow[i] = pack_bf16(acc[2 * i] * inv, acc[2 * i + 1] * inv);
         *reinterpret_cast<uint4 *>(qbar + ((int64_t)bh * mpad + (int64_t)g * p.b2) * kD + col) = o;
     }
-    if (g == 0) {   // zero the padding rows [t*b2, mpad) of this head
+    if (g == 0 && grp == 0) {   // zero the padding rows [t*b2, mpad) of this head
         const int64_t pad = (int64_t)(mpad - p.tiles * p.b2) * kD;
         __nv_bfloat16 *base = qbar + ((int64_t)bh * mpad + (int64_t)p.tiles * p.b2) * kD;
         for (int64_t e = col; e < pad; e += (int64_t)nchunk * 128 * 8)
@@ -131,14 +152,18 @@ __global__ void __launch_bounds__(128) tc_qbar_kernel(const __nv_bfloat16 *__res
 // (one query row per thread); warps 8-11: the epilogue warpgroup (O / l to
 // bfloat16 rows of Y, off the softmax warps' chain); warp 12: the TMA producer
 // of Ktil and its entropy panel; warp 13: the MMA issuer; warp 14: the
-// producer of Z; warp 15: the producer of the query tiles.  setmaxnreg moves registers from the
-// producer and epilogue warpgroups to the softmax warpgroups.
-// Tensor memory: S_0 | S_1 | O_0 | O_1 (128 columns each); P_t overwrites the
-// first 64 columns of S_t as packed bfloat16 pairs.
+// producer of Z; warp 15: the producer of the query tiles.  setmaxnreg gives the
+// softmax warpgroups 136 registers, the epilogue 128 and the producer warpgroup
+// 112 (the MMA issuer keeps two cursors over the problems).  The keys are
+// consumed in halves of 64: one 128-key chunk of Ktil and Z in shared memory
+// serves two halves.
+// Tensor memory: S_t,0 | S_t,1 (64 columns each, the two S buffers of tile t)
+// at t*128, then O_0 | O_1 (128 columns each); P of a half overwrites the first
+// 32 columns of its S buffer as packed bfloat16 pairs.
 // =====================================================================
 namespace ls {
 constexpr int kThreads = 512;
-constexpr int kSoftmaxRegs = 160, kEpilogueRegs = 128, kProducerRegs = 64;
+constexpr int kSoftmaxRegs = 136, kEpilogueRegs = 128, kProducerRegs = 112;
 static_assert(2 * kSoftmaxRegs + kEpilogueRegs + kProducerRegs == 4 * (65536 / kThreads),
               "the warpgroups' registers must add up to the launch's 128 per thread");
 // one pair of every kPolyEvery takes its exponentials on the FMA pipe (0: none).
@@ -196,6 +221,7 @@ struct LsProblem {
     int bh, g, v;
     int m_y, m_z, m_first, m_end;   // M side: tile t starts at z = m_z + t*128
     int n_y, n_z, nkeys, nch;       // N side: chunk j starts at z = n_z + j*128
+    int nh;                         // 64-key halves of the N side (the softmax's unit)
 };
 
 template <int MODE>
@@ -229,6 +255,7 @@ __device__ __forceinline__ LsProblem ls_problem(const LsArgs &a, int unit) {
         q.nkeys = u_hi - u_lo;
     }
     q.nch = (q.nkeys + 127) / 128;
+    q.nh = (q.nkeys + 63) / 64;
     return q;
 }
 
@@ -261,8 +288,8 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
     uint64_t *k_empty = bars + 6;    // [2 stages]: both S MMAs of the chunk done
     uint64_t *z_full = bars + 8;     // [2 stages]: value chunk
     uint64_t *z_empty = bars + 10;   // [2 stages]: both PV MMAs of the chunk done
-    uint64_t *s_full = bars + 16;    // [2 tiles]
-    uint64_t *p_full = bars + 18;    // [2 tiles], one arrival per softmax warp
+    uint64_t *s_full = bars + 12;    // [2 tiles][2 S buffers]: S of a 64-key half
+    uint64_t *p_full = bars + 16;    // [2 tiles][2 S buffers], one arrival per softmax warp
     uint64_t *o_full = bars + 20;    // [2 tiles]: the last PV MMA of a problem done
     uint64_t *o_free = bars + 22;    // [2 tiles], one arrival per epilogue warp: O_t read
     uint64_t *l_full = bars + 24;    // [2 tiles], one arrival per softmax warp: row sums written
@@ -270,6 +297,7 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
     uint64_t *stall_bar = bars + 27;   // never completed (fault-injection hook)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 28);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 29);
+    uint64_t *pv_done = bars + 30;   // [2 tiles]: one phase per PV MMA of the tile
     float *lsum = reinterpret_cast<float *>(sm + ls::kL);   // [2][2][128]
 
     const Problem &p = a.p;
@@ -286,16 +314,19 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
             mbar_init(q_full + t, 1);
             mbar_init(q_empty + t, 1);
             mbar_init(k_full + t, 1);
-            mbar_init(k_empty + t, 1);
+            mbar_init(k_empty + t, 2);   // one commit per tile's MMA issuer
             mbar_init(z_full + t, 1);
-            mbar_init(z_empty + t, 1);
-            mbar_init(s_full + t, 1);
-            mbar_init(p_full + t, 4);   // one arrival per softmax warp
+            mbar_init(z_empty + t, 2);   // one commit per tile's MMA issuer
+            for (int b = 0; b < 2; b++) {
+                mbar_init(s_full + 2 * t + b, 1);
+                mbar_init(p_full + 2 * t + b, 4);   // one arrival per softmax warp
+            }
+            mbar_init(pv_done + t, 1);
             mbar_init(o_full + t, 1);
             mbar_init(o_free + t, 4);   // one arrival per epilogue warp
             mbar_init(l_full + t, 4);   // one arrival per softmax warp
         }
-        mbar_init(mma_done, 1);
+        mbar_init(mma_done, 2);   // one commit per MMA issuer
         mbar_init(stall_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -347,11 +378,15 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
             if (lane == 0)   // every issued copy lands before the CTA may exit
                 for (int s = 0; s < 2; s++)
                     if (issued[s] > 0) wait_phase_cleanup(k_full + s, (issued[s] - 1) & 1, kCleanupPolls);
-        } else if (warp == 15) {
-            // ---------------- M-tile producer: each tile reloads as soon as its own
-            // last S MMA of the previous problem is done; the next problem's rows
-            // are prefetched into L2 a whole problem ahead
-            int qloads = 0;
+        } else if (warp == 14) {
+            // ---------------- producer of the M tiles and the values.  Per problem:
+            // first the two M tiles (each as soon as its own last S MMA of the
+            // previous problem is done), with the next problem's rows prefetched
+            // into L2, then the problem's value chunks (each as soon as the PV MMAs
+            // of two chunks back are done).  Every wait points at an MMA that the
+            // issuers reach without these loads: a tile's last S of the previous
+            // problem follows that problem's value chunks in the issue order.
+            int qloads = 0, issued_z[2] = {0, 0}, jc0 = 0;
             bool ok = true;
             for (int pi = 0; ok && pi < nmine; pi++) {
                 const LsProblem pr = ls_problem<MODE>(a, blockIdx.x + pi * gridDim.x);
@@ -379,18 +414,7 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                                 tma_prefetch_2d(&tmM, pn * 64, nx.m_z + t * 128);
                         }
                 }
-            }
-            if (lane == 0)
-                for (int t = 0; t < 2; t++)
-                    if (qloads > 0) wait_phase_cleanup(q_full + t, (qloads - 1) & 1, kCleanupPolls);
-        } else if (warp == 14 && values) {
-            // ---------------- value producer: its own warp, so that an N-chunk load
-            // never queues behind the wait for a value stage (released one PV later)
-            int issued_z[2] = {0, 0}, jc0 = 0;
-            bool ok = true;
-            for (int pi = 0; ok && pi < nmine; pi++) {
-                const LsProblem pr = ls_problem<MODE>(a, blockIdx.x + pi * gridDim.x);
-                for (int j = 0; j < pr.nch; j++) {
+                for (int j = 0; values && j < pr.nch; j++) {
                     const int jc = jc0 + j, st = jc & 1;
                     if (jc >= 2 && !wait_warp(z_empty + st, ((jc >> 1) - 1) & 1, w)) {
                         ok = false;
@@ -406,75 +430,99 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                 }
                 jc0 += pr.nch;
             }
-            if (lane == 0)
-                for (int s = 0; s < 2; s++)
-                    if (issued_z[s] > 0)
-                        wait_phase_cleanup(z_full + s, (issued_z[s] - 1) & 1, kCleanupPolls);
-        } else if (warp == 13) {
-            // ---------------- MMA issuer.  Order: S_0 and S_1 of the first chunk, then
-            // per chunk PV_0, S_0 of the next chunk, PV_1, S_1 of the next chunk, so
-            // that a tile's chain never waits on the other tile's softmax.  S_t of
-            // the next chunk overwrites the columns that PV_t reads as P: tcgen05
-            // MMAs issued by one thread execute in issue order, so it follows PV_t
-            // without a wait, and its commit (s_full) also covers PV_t, which orders
-            // the softmax's rescale of O_t after PV_t.  Without values (kLsStat)
-            // there is no PV: S_t of the next chunk waits for the softmax to have
-            // read S_t (p_full).
-            constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
+            if (lane == 0) {   // every issued copy lands before the CTA may exit
+                for (int t = 0; t < 2; t++)
+                    if (qloads > 0) wait_phase_cleanup(q_full + t, (qloads - 1) & 1, kCleanupPolls);
+                for (int st = 0; st < 2; st++)
+                    if (issued_z[st] > 0)
+                        wait_phase_cleanup(z_full + st, (issued_z[st] - 1) & 1, kCleanupPolls);
+            }
+        } else if (warp == 13 || warp == 15) {
+            // ---------------- MMA issuers: warp 13 for tile 0, warp 15 for tile 1, so
+            // that one tile's MMAs never queue behind a wait for the other tile's
+            // softmax.  The unit is a 64-key half of a 128-key chunk; tile t has two
+            // S buffers of 64 columns (tensor-memory columns t*128 + b*64), and half
+            // hc (counted over the CTA's problems) uses buffer hc & 1.  Order: S of
+            // the first two halves, then per half hc: PV(hc), S(hc + 2).  So the S
+            // of the next half is already in its buffer while the softmax works on
+            // this one.  S(hc + 2) overwrites the columns that PV(hc) reads as P:
+            // tcgen05 MMAs issued by one thread execute in issue order, so it
+            // follows PV(hc) without a wait.  Without values (kLsStat) there is no
+            // PV: S(hc + 2) waits for the softmax to have read S(hc) (p_full).  The
+            // stages of Ktil and Z are released by one commit from each issuer.
+            const int t = warp == 13 ? 0 : 1;
+            constexpr uint32_t idS = idesc_bf16(128, 64, 0, 0);
             constexpr uint32_t idO = idesc_bf16(128, 128, 0, 1);
-            const uint64_t dQ = smem_desc_sw128(smem_u32(sm + ls::kQ), 16, 1024);
+            const uint64_t dQ = smem_desc_sw128(smem_u32(sm + ls::kQ + t * kTile), 16, 1024);
             const uint64_t dK = smem_desc_sw128(smem_u32(sm + ls::kK), 16, 1024);
             const uint64_t dZ = smem_desc_sw128(smem_u32(sm + ls::kZ), kPanel, 1024);
             const uint64_t dQx = smem_desc_sw32(smem_u32(sm + ls::kQx));
             const uint64_t dHx = smem_desc_sw32(smem_u32(sm + ls::kHx));
             constexpr uint32_t kTileDesc = kTile >> 4, kHxDesc = ls::kPanelHx >> 4;
+            // rows 64..127 of a 128-row stage: 64 rows x 128 B (SW128), 64 rows x
+            // 32 B (SW32), in descriptor units of 16 bytes
+            constexpr uint32_t kHalfDesc = 64 * 128 >> 4, kHalfHxDesc = 64 * 32 >> 4;
+            const uint32_t tS = tmem + t * 128, tO = tmem + 256 + t * 128;
             // fault injection: a wait that can only give up (bounded, then abort)
             bool ok = !a.stall || spin_warp(stall_bar, 0, w);
-            // S_t of global chunk jc, chunk j of problem pi (nch chunks)
-            auto issue_s = [&](int t, int jc, int j, int pi, int nch) -> bool {
-                const int sk = jc & 1;
-                if (j == 0 && !spin_warp(q_full + t, pi & 1, w)) return false;
-                if (t == 0 && !spin_warp(k_full + sk, (jc >> 1) & 1, w)) return false;
+            // a position in the CTA's sequence of halves: half i of problem pi,
+            // global half hc, chunk jc0 + i / 2
+            struct Cursor {
+                int pi, i, hc, jc0;
+                LsProblem pr;
+            };
+            auto advance = [&](Cursor &c) {
+                c.hc++;
+                if (++c.i == c.pr.nh) {
+                    c.i = 0;
+                    c.jc0 += c.pr.nch;
+                    if (++c.pi < nmine) c.pr = ls_problem<MODE>(a, blockIdx.x + c.pi * gridDim.x);
+                }
+            };
+            auto issue_s = [&](const Cursor &c) -> bool {
+                const int jc = c.jc0 + (c.i >> 1), sk = jc & 1, kh = c.i & 1, b = c.hc & 1;
+                if (c.i == 0 && !spin_warp(q_full + t, c.pi & 1, w)) return false;
+                if (kh == 0 && !spin_warp(k_full + sk, (jc >> 1) & 1, w)) return false;
                 tc_fence_after();
-                mma8_ss_k128(tmem + t * 128, dQ + t * kTileDesc, dK + sk * kTileDesc, idS, 0u);
-                mma1_ss_acc(tmem + t * 128, dQx, dHx + sk * kHxDesc, idS);   // + panel value
-                mma_commit_warp(s_full + t);
-                if (t == 1) mma_commit_warp(k_empty + sk);
-                if (j == nch - 1) mma_commit_warp(q_empty + t);   // tile t no longer read
+                const uint32_t d = tS + b * 64;
+                mma8_ss_k128(d, dQ, dK + sk * kTileDesc + kh * kHalfDesc, idS, 0u);
+                mma1_ss_acc(d, dQx, dHx + sk * kHxDesc + kh * kHalfHxDesc, idS);   // + panel value
+                mma_commit_warp(s_full + 2 * t + b);
+                const bool last = c.i == c.pr.nh - 1;
+                if (kh == 1 || last) mma_commit_warp(k_empty + sk);   // this tile read the stage
+                if (last) mma_commit_warp(q_empty + t);   // tile t no longer read
                 return true;
             };
-            auto issue_pv = [&](int t, int jc, int j, int pi, int nch) -> bool {
-                const int st = jc & 1;
-                if (values && t == 0 && !spin_warp(z_full + st, (jc >> 1) & 1, w)) return false;
-                if (!spin_warp(p_full + t, jc & 1, w)) return false;
+            auto issue_pv = [&](const Cursor &c) -> bool {
+                const int jc = c.jc0 + (c.i >> 1), st = jc & 1, kh = c.i & 1, b = c.hc & 1;
+                if (values && kh == 0 && !spin_warp(z_full + st, (jc >> 1) & 1, w)) return false;
+                if (!spin_warp(p_full + 2 * t + b, (c.hc >> 1) & 1, w)) return false;
                 if (!values) return true;
                 // the first PV of a problem overwrites O_t: the epilogue of the
                 // previous problem must have read it
-                if (j == 0 && pi > 0 && !spin_warp(o_free + t, (pi - 1) & 1, w)) return false;
+                if (c.i == 0 && c.pi > 0 && !spin_warp(o_free + t, (c.pi - 1) & 1, w)) return false;
                 tc_fence_after();
-                mma8_ts_mn128(tmem + 256 + t * 128, tmem + t * 128, dZ + st * kTileDesc, idO,
-                              j > 0 ? 1u : 0u);
-                if (t == 1) mma_commit_warp(z_empty + st);
-                if (j == nch - 1) mma_commit_warp(o_full + t);
+                mma4_ts_mn64(tO, tS + b * 64, dZ + st * kTileDesc + kh * kHalfDesc, idO,
+                             c.i > 0 ? 1u : 0u);
+                mma_commit_warp(pv_done + t);
+                const bool last = c.i == c.pr.nh - 1;
+                if (kh == 1 || last) mma_commit_warp(z_empty + st);   // this tile read the stage
+                if (last) mma_commit_warp(o_full + t);
                 return true;
             };
-            int jc0 = 0;
-            LsProblem pr = nmine > 0 ? ls_problem<MODE>(a, blockIdx.x) : LsProblem{};
-            if (ok && nmine > 0) ok = issue_s(0, 0, 0, 0, pr.nch) && issue_s(1, 0, 0, 0, pr.nch);
-            for (int pi = 0; ok && pi < nmine; pi++) {
-                const bool has_next = pi + 1 < nmine;
-                const LsProblem nx = has_next ? ls_problem<MODE>(a, blockIdx.x + (pi + 1) * gridDim.x) : pr;
-                for (int j = 0; ok && j < pr.nch; j++) {
-                    const int jc = jc0 + j;
-                    const bool last = j == pr.nch - 1, more = !last || has_next;
-                    // the chunk after jc: j + 1 of this problem, or 0 of the next
-                    const int jn = last ? 0 : j + 1, pn = last ? pi + 1 : pi;
-                    const int nn = last ? nx.nch : pr.nch;
-                    ok = issue_pv(0, jc, j, pi, pr.nch) && (!more || issue_s(0, jc + 1, jn, pn, nn)) &&
-                         issue_pv(1, jc, j, pi, pr.nch) && (!more || issue_s(1, jc + 1, jn, pn, nn));
+            if (nmine > 0) {
+                Cursor cs{0, 0, 0, 0, ls_problem<MODE>(a, blockIdx.x)};   // next S to issue
+                Cursor cp = cs;                                          // next PV to issue
+                for (int k = 0; ok && k < 2 && cs.pi < nmine; k++) {
+                    ok = issue_s(cs);
+                    advance(cs);
                 }
-                jc0 += pr.nch;
-                pr = nx;
+                while (ok && cp.pi < nmine) {
+                    const bool more = cs.pi < nmine;
+                    ok = issue_pv(cp) && (!more || issue_s(cs));
+                    if (more) advance(cs);
+                    advance(cp);
+                }
             }
             mma_commit_warp(mma_done);
             wait_phase_cleanup(mma_done, 0, kCleanupPolls);
@@ -551,37 +599,38 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
         const int t = warp >> 2;
         const int wq = warp & 3;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-        const uint32_t tS = tmem + lane_off + t * 128;
+        const uint32_t tS0 = tmem + lane_off + t * 128;   // S buffer b at + b * 64
         const uint32_t tO = tmem + lane_off + 256 + t * 128;
         const uint64_t c2 = f2_pack(a.c_log2, a.c_log2);
         bool ok = true;
-        int jc0 = 0;
+        int hc = 0;   // 64-key halves done by this tile over the CTA's problems
         for (int pi = 0; ok && pi < nmine; pi++) {
             const LsProblem pr = ls_problem<MODE>(a, blockIdx.x + pi * gridDim.x);
             float m_run = -INFINITY, l_run = 0.f;
-            for (int j = 0; j < pr.nch; j++) {
-                const int jc = jc0 + j;
-                if (!wait_warp(s_full + t, jc & 1, w)) {
+            for (int i = 0; i < pr.nh; i++, hc++) {
+                const int b = hc & 1;
+                if (!wait_warp(s_full + 2 * t + b, (hc >> 1) & 1, w)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint32_t tS = tS0 + b * 64;
                 // S = q.Ktil + H' (kLsAgg: Ktil.q - lam): scaled by c_log2 it is the
                 // logit in log2 units, so the maximum is taken on S itself
-                float x[128];
-#pragma unroll
-                for (int c = 0; c < 4; c++) tmem_ld32f(tS + c * 32, &x[c * 32]);
+                float x[64];
+                tmem_ld32f(tS, &x[0]);
+                tmem_ld32f(tS + 32, &x[32]);
                 tmem_wait_ld();
-                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-                const int nvalid = pr.nkeys - j * 128;   // N rows of this chunk inside the row
-                if (nvalid < 128) {
-                    // the ragged last chunk: rows past nkeys belong to the next row
+                const int nvalid = pr.nkeys - i * 64;   // N rows of this half inside the row
+                if (nvalid < 64) {
+                    // the ragged last half: rows past nkeys belong to the next row
                     // block (or are zero fill), so mask them by selection
 #pragma unroll
-                    for (int i = 0; i < 128; i++) x[i] = i < nvalid ? x[i] : -INFINITY;
+                    for (int k = 0; k < 64; k++) x[k] = k < nvalid ? x[k] : -INFINITY;
                 }
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int i = 0; i < 64; i++) mx4[i & 3] = fmax3(mx4[i & 3], x[2 * i], x[2 * i + 1]);
+                for (int k = 0; k < 32; k++) mx4[k & 3] = fmax3(mx4[k & 3], x[2 * k], x[2 * k + 1]);
                 const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
                 // the running maximum moves only when it grows by more than 2^8 in
                 // log2 units: the probabilities stay below 256 and O is rescaled rarely
@@ -594,51 +643,53 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                 }
                 const uint64_t nmc2 = f2_pack(-m_run * a.c_log2, -m_run * a.c_log2);
                 uint64_t sum2[4] = {0, 0, 0, 0};
+                uint32_t pk[32];
 #pragma unroll
-                for (int h = 0; h < 2; h++) {
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int i = 0; i < 32; i++) {
-                        const int e = h * 32 + i;
-                        const uint64_t d2 = f2_fma(f2_pack(x[2 * e], x[2 * e + 1]), c2, nmc2);
-                        uint64_t e2;
-                        constexpr int kEvery = ls::kPolyEvery > 0 ? ls::kPolyEvery : 1;
-                        if (ls::kPolyEvery > 0 && (i % kEvery) == kEvery - 1 && nvalid >= 128) {
-                            e2 = exp2_poly_x2(d2);
-                        } else {
-                            float lo, hi;
-                            f2_unpack(d2, lo, hi);
-                            e2 = f2_pack(fast_exp2(lo), fast_exp2(hi));
-                        }
-                        sum2[i & 3] = f2_add(sum2[i & 3], e2);
-                        float p0, p1;
-                        f2_unpack(e2, p0, p1);
-                        pk[i] = pack_bf16(p0, p1);
+                for (int k = 0; k < 32; k++) {
+                    const uint64_t d2 = f2_fma(f2_pack(x[2 * k], x[2 * k + 1]), c2, nmc2);
+                    uint64_t e2;
+                    constexpr int kEvery = ls::kPolyEvery > 0 ? ls::kPolyEvery : 1;
+                    if (ls::kPolyEvery > 0 && (k % kEvery) == kEvery - 1 && nvalid >= 64) {
+                        e2 = exp2_poly_x2(d2);
+                    } else {
+                        float lo, hi;
+                        f2_unpack(d2, lo, hi);
+                        e2 = f2_pack(fast_exp2(lo), fast_exp2(hi));
                     }
-                    if (values) tmem_st32(tS + h * 32, pk);
+                    sum2[k & 3] = f2_add(sum2[k & 3], e2);
+                    float p0, p1;
+                    f2_unpack(e2, p0, p1);
+                    pk[k] = pack_bf16(p0, p1);
                 }
+                // P (packed bfloat16 pairs) over the first 32 columns of the buffer
+                if (values) tmem_st32(tS, pk);
                 float s0, s1;
                 f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), s0, s1);
                 l_run = l_run * alpha + (s0 + s1);
-                if (values && j > 0 && __any_sync(0xffffffffu, rescale)) {
-                    // O_t is complete up to the previous chunk (the commit of this
-                    // chunk's S covers the previous PV); scale it in four slices
+                if (values && i > 0 && __any_sync(0xffffffffu, rescale)) {
+                    // O_t holds the products up to the previous half once PV_t of
+                    // that half is done (it may still be running: S of this half
+                    // was issued two halves back); then scale it in four slices
+                    if (!wait_warp(pv_done + t, (hc - 1) & 1, w)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
 #pragma unroll
                     for (int c = 0; c < 4; c++) {
                         float o[32];
                         tmem_ld32f(tO + c * 32, o);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; i++) o[i] *= alpha;
+                        for (int k = 0; k < 32; k++) o[k] *= alpha;
                         tmem_st32f(tO + c * 32, o);
                     }
                 }
                 if (values) tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive_warp(p_full + t);
+                mbar_arrive_warp(p_full + 2 * t + b);
             }
             if (!ok) break;
-            jc0 += pr.nch;
             if (values) {
                 // the row sums for the epilogue.  Before publishing those of problem
                 // pi the epilogue must have taken those of pi - 1 (its o_free
@@ -1024,22 +1075,27 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 }
                 tc_fence_before();
                 mbar_arrive_warp(o_empty + part);
-                // the previous store of this warp must have finished reading staging
-                if (lane == 0) tma_store_wait_read_all();
-                __syncwarp();
+                // each 64-column panel leaves in its own store group from staging
+                // slot pn; the group that last read slot pn is two groups back, so
+                // one younger group may still be reading while this panel is written
 #pragma unroll
-                for (int c = 0; c < 16; c++) {   // 16-byte chunk c of the 256-byte row
-                    const int pn = c >> 3, pos = (c & 7) ^ (lane & 7);
-                    *reinterpret_cast<uint4 *>(stg + pn * 4096 + lane * 128 + pos * 16) =
-                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    const CUtensorMap *map = part == 0 ? &tmZs : &tmKs;
-                    for (int pn = 0; pn < 2; pn++)
-                        tma_store_4d(map, stg + pn * 4096, pn * 64, up, mt * 128 + wq * 32, bh);
-                    tma_store_commit();
+                for (int pn = 0; pn < 2; pn++) {
+                    if (lane == 0) tma_store_wait_read_le1();
+                    __syncwarp();
+#pragma unroll
+                    for (int c = 0; c < 8; c++) {   // 16-byte chunk c of the panel's 128-byte row
+                        const int pos = c ^ (lane & 7);
+                        *reinterpret_cast<uint4 *>(stg + pn * 4096 + lane * 128 + pos * 16) =
+                            make_uint4(pk[pn * 32 + 4 * c], pk[pn * 32 + 4 * c + 1],
+                                       pk[pn * 32 + 4 * c + 2], pk[pn * 32 + 4 * c + 3]);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_4d(part == 0 ? &tmZs : &tmKs, stg + pn * 4096, pn * 64, up,
+                                     mt * 128 + wq * 32, bh);
+                        tma_store_commit();
+                    }
                 }
             }
         }
@@ -1306,7 +1362,8 @@ cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const 
     {
         const int nchunk = (p.b2 * kD / 8 + 127) / 128;
         ProfileScope scope(K_TC_QBAR, stream);
-        tc_qbar_kernel<<<(p.head_end() - p.head_begin()) * p.tiles * nchunk, 128, 0, stream>>>(
+        tc_qbar_kernel<<<(p.head_end() - p.head_begin()) * p.tiles * nchunk, 128 * kQbarGroups, 0,
+                         stream>>>(
             (const __nv_bfloat16 *)q, ws.qbar, p, mpad);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;

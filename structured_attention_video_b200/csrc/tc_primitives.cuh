@@ -143,6 +143,11 @@ __device__ __forceinline__ void tma_store_commit() {
 __device__ __forceinline__ void tma_store_wait_read_all() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
+// Waits until at most one of this thread's bulk store groups still reads its
+// shared-memory source (the older ones are done reading).
+__device__ __forceinline__ void tma_store_wait_read_le1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
 __device__ __forceinline__ void tma_store_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
@@ -347,6 +352,27 @@ __device__ __forceinline__ void mma8_ts_mn128(uint32_t d_tmem, uint32_t a_tmem, 
 }
 
 // One K-step (K = 16) of D += A B^T, both operands one 32-byte-swizzled K atom.
+// D (+)= A * B over K = 64: A (M = 128 x 64, bfloat16) in tensor memory, B an
+// MN-major SW128 shared-memory operand; four K-steps of 16 (A advances 8
+// columns, B 16 rows = 2 KB per step).
+__device__ __forceinline__ void mma4_ts_mn64(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                             uint32_t idesc, uint32_t acc0) {
+    asm volatile(
+        "{\n\t.reg .pred e, p0;\n\t"
+        ".reg .b32 a1, a2, a3;\n\t"
+        ".reg .b64 b1, b2, b3;\n\t"
+        "add.u32 a1, %1, 8;\n\tadd.u32 a2, %1, 16;\n\tadd.u32 a3, %1, 24;\n\t"
+        "add.s64 b1, %2, 128;\n\tadd.s64 b2, %2, 256;\n\tadd.s64 b3, %2, 384;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.and.b32 p0, %4, 0, e;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, 1;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc0)
+        : "memory");
+}
+
 __device__ __forceinline__ void mma1_ss_acc(uint32_t d_tmem, uint64_t a, uint64_t b,
                                             uint32_t idesc) {
     asm volatile(

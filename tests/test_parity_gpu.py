@@ -102,6 +102,8 @@ TC_EDGES = [
     (2, 100, 7, 200, 7, 3),      # b2 padded to 16; ragged last key chunk (200 = 128 + 72)
     (5, 60, 48, 300, 48, 5),     # 60 rows per tile: the second query tile of a pair is empty
     (10, 100, 16, 1000, 16, 1),  # 1000 query rows per tile: four pairs of query tiles
+    (1, 65, 4, 65, 4, 2),        # 65 keys: a second 64-key half with one valid key
+    (1, 129, 8, 129, 8, 3),      # 129 keys: the last 128-key chunk has a single half
 ]
 
 
