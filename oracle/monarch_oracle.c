@@ -365,6 +365,204 @@ int oracle_monarch_attn_kv(const double *q, const double *k, const double *v, do
 }
 
 /* Number of threads the OpenMP runtime would use (1 without OpenMP). */
+/*
+ * Backward pass of one iteration (iters = 1) by the chain rule, step by step.
+ * There is no backward in the pages; this is the derivative of the forward
+ * map above (its plain definition, written out), which the finetuning of the
+ * summary page ("Approach") and the explainer page ("创新三") trains through.
+ * Given dy = dPhi/dy for some scalar Phi, it returns dPhi/dq, dPhi/dk and
+ * dPhi/dv.  Per (tile g, column c) problem, with the forward quantities of
+ * solve_problem (qbar, R, H, Ktil, Z, L):
+ *   L-step and output (y_u = sum_u' L[u,u'] Z[u'], b = s q_u.Ktil + H):
+ *     dL[u,u'] = dy_u.Z[u'],  db[u,u'] = L[u,u'] (dL[u,u'] - sum_u'' L dL),
+ *     dq_u += s sum_u' db Ktil[u'],   dKtil[u'] += s sum_u db q_u,
+ *     dZ[u'] += sum_u L[u,u'] dy_u,   dH[u'] += sum_u db[u,u'].
+ *   R-step (a = s qbar.k_(u',v'), R = softmax(a), H = lse(a) - sum R a,
+ *   Ktil = sum R k, Z = sum R v):
+ *     dR[v'] = dKtil[u'].k_(u',v') + dZ[u'].v_(u',v'),
+ *     da[v'] = R (dR - sum R dR) - dH[u'] R (a - sum R a)   (dH/da = -R (a - E_R a)),
+ *     dqbar += s sum_v' da k_(u',v'),
+ *     dk_(u',v') += s da qbar + R dKtil[u'],   dv_(u',v') += R dZ[u'].
+ *   Aggregation (qbar = mean over u in T_g of q_(u,c)):  dq_(u,c) += dqbar / |T_g|.
+ * q, k, v, dy, dq, dk, dv: [BH][N][d]; dq, dk, dv are overwritten.
+ */
+int oracle_monarch_attn_bwd(const double *q, const double *k, const double *v,
+                            const double *dy, double *dq, double *dk, double *dv, int BH,
+                            int N, int d, int b1, int b2, int tiles, int nthreads)
+{
+    if (BH < 1 || check_shape(N, d, b1, b2, tiles, 2))
+        return ORACLE_EINVAL;
+    const double s = 1.0 / sqrt((double)d);
+    const size_t per_head = (size_t)N * d;
+    memset(dq, 0, (size_t)BH * per_head * sizeof(double));
+    memset(dk, 0, (size_t)BH * per_head * sizeof(double));
+    memset(dv, 0, (size_t)BH * per_head * sizeof(double));
+    const int nq_max = (b1 + tiles - 1) / tiles + 1;
+    /* per thread: A, R [b1][b2]; Kt, Z, dKt, dZ [b1][d]; H, dH [b1];
+     * L, dB [nq_max][b1]; qbar, dqbar [d]; row [max(b1, b2)] */
+    const size_t wsz = 2 * (size_t)b1 * b2 + 4 * (size_t)b1 * d + 2 * (size_t)b1 +
+                       2 * (size_t)nq_max * b1 + 2 * (size_t)d + (size_t)(b1 > b2 ? b1 : b2);
+    int err = ORACLE_OK;
+#ifdef _OPENMP
+    if (nthreads <= 0)
+        nthreads = omp_get_max_threads();
+#pragma omp parallel num_threads(nthreads)
+#endif
+    {
+        double *ws = (double *)malloc(wsz * sizeof(double));
+        if (!ws) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            err = ORACLE_ENOMEM;
+        }
+        /* heads in parallel: the problems of one head all add into its dk, dv */
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+        for (int bh = 0; bh < BH; bh++) {
+            if (!ws)
+                continue;
+            const double *qh = q + (size_t)bh * per_head, *kh = k + (size_t)bh * per_head;
+            const double *vh = v + (size_t)bh * per_head, *dyh = dy + (size_t)bh * per_head;
+            double *dqh = dq + (size_t)bh * per_head, *dkh = dk + (size_t)bh * per_head;
+            double *dvh = dv + (size_t)bh * per_head;
+            double *A = ws, *R = A + (size_t)b1 * b2, *Kt = R + (size_t)b1 * b2;
+            double *Z = Kt + (size_t)b1 * d, *dKt = Z + (size_t)b1 * d, *dZ = dKt + (size_t)b1 * d;
+            double *H = dZ + (size_t)b1 * d, *dH = H + b1, *L = dH + b1;
+            double *dB = L + (size_t)nq_max * b1, *qbar = dB + (size_t)nq_max * b1;
+            double *dqbar = qbar + d, *row = dqbar + d;
+            for (int g = 0; g < tiles; g++) {
+                const int u0 = tile_first_row(g, b1, tiles), u1 = tile_first_row(g + 1, b1, tiles);
+                const int nq = u1 - u0;
+                for (int c = 0; c < b2; c++) {
+                    /* ---- forward, as in solve_problem (one R-step from uniform L) */
+                    for (int j = 0; j < d; j++) {
+                        double acc = 0.0;
+                        for (int u = u0; u < u1; u++)
+                            acc += qh[((int64_t)u * b2 + c) * d + j];
+                        qbar[j] = acc / nq;
+                    }
+                    for (int up = 0; up < b1; up++) {
+                        double mx = -INFINITY;
+                        for (int vp = 0; vp < b2; vp++) {
+                            double acc = 0.0;
+                            for (int j = 0; j < d; j++)
+                                acc += qbar[j] * kh[((int64_t)up * b2 + vp) * d + j];
+                            A[(size_t)up * b2 + vp] = s * acc;
+                            if (s * acc > mx)
+                                mx = s * acc;
+                        }
+                        double sum = 0.0;
+                        for (int vp = 0; vp < b2; vp++)
+                            sum += exp(A[(size_t)up * b2 + vp] - mx);
+                        const double lse = mx + log(sum);
+                        double ent = lse;
+                        for (int vp = 0; vp < b2; vp++) {
+                            R[(size_t)up * b2 + vp] = exp(A[(size_t)up * b2 + vp] - lse);
+                            ent -= R[(size_t)up * b2 + vp] * A[(size_t)up * b2 + vp];
+                        }
+                        H[up] = ent;
+                        for (int j = 0; j < d; j++) {
+                            double kt = 0.0, z = 0.0;
+                            for (int vp = 0; vp < b2; vp++) {
+                                kt += R[(size_t)up * b2 + vp] * kh[((int64_t)up * b2 + vp) * d + j];
+                                z += R[(size_t)up * b2 + vp] * vh[((int64_t)up * b2 + vp) * d + j];
+                            }
+                            Kt[(size_t)up * d + j] = kt;
+                            Z[(size_t)up * d + j] = z;
+                        }
+                    }
+                    for (int u = u0; u < u1; u++) {
+                        const double *qr = qh + ((int64_t)u * b2 + c) * d;
+                        double mx = -INFINITY;
+                        for (int up = 0; up < b1; up++) {
+                            double acc = 0.0;
+                            for (int j = 0; j < d; j++)
+                                acc += qr[j] * Kt[(size_t)up * d + j];
+                            row[up] = s * acc + H[up];
+                            if (row[up] > mx)
+                                mx = row[up];
+                        }
+                        double sum = 0.0;
+                        for (int up = 0; up < b1; up++)
+                            sum += exp(row[up] - mx);
+                        const double lse = mx + log(sum);
+                        for (int up = 0; up < b1; up++)
+                            L[(size_t)(u - u0) * b1 + up] = exp(row[up] - lse);
+                    }
+                    /* ---- L-step and output backward */
+                    memset(dKt, 0, (size_t)b1 * d * sizeof(double));
+                    memset(dZ, 0, (size_t)b1 * d * sizeof(double));
+                    memset(dH, 0, (size_t)b1 * sizeof(double));
+                    for (int u = u0; u < u1; u++) {
+                        const double *qr = qh + ((int64_t)u * b2 + c) * d;
+                        const double *dyr = dyh + ((int64_t)u * b2 + c) * d;
+                        double *Lr = L + (size_t)(u - u0) * b1, *dBr = dB + (size_t)(u - u0) * b1;
+                        double ldl = 0.0;
+                        for (int up = 0; up < b1; up++) {
+                            double acc = 0.0;
+                            for (int j = 0; j < d; j++)
+                                acc += dyr[j] * Z[(size_t)up * d + j];
+                            row[up] = acc;   /* dL[u,u'] */
+                            ldl += Lr[up] * acc;
+                        }
+                        for (int up = 0; up < b1; up++)
+                            dBr[up] = Lr[up] * (row[up] - ldl);
+                        double *dqr = dqh + ((int64_t)u * b2 + c) * d;
+                        for (int j = 0; j < d; j++) {
+                            double acc = 0.0;
+                            for (int up = 0; up < b1; up++)
+                                acc += dBr[up] * Kt[(size_t)up * d + j];
+                            dqr[j] += s * acc;
+                        }
+                        for (int up = 0; up < b1; up++) {
+                            for (int j = 0; j < d; j++) {
+                                dKt[(size_t)up * d + j] += s * dBr[up] * qr[j];
+                                dZ[(size_t)up * d + j] += Lr[up] * dyr[j];
+                            }
+                            dH[up] += dBr[up];
+                        }
+                    }
+                    /* ---- R-step backward */
+                    for (int j = 0; j < d; j++)
+                        dqbar[j] = 0.0;
+                    for (int up = 0; up < b1; up++) {
+                        const double *Rr = R + (size_t)up * b2, *Ar = A + (size_t)up * b2;
+                        double rdr = 0.0, ea = 0.0;
+                        for (int vp = 0; vp < b2; vp++) {
+                            const double *kr = kh + ((int64_t)up * b2 + vp) * d;
+                            const double *vr = vh + ((int64_t)up * b2 + vp) * d;
+                            double acc = 0.0;
+                            for (int j = 0; j < d; j++)
+                                acc += dKt[(size_t)up * d + j] * kr[j] + dZ[(size_t)up * d + j] * vr[j];
+                            row[vp] = acc;   /* dR[v'] */
+                            rdr += Rr[vp] * acc;
+                            ea += Rr[vp] * Ar[vp];
+                        }
+                        for (int vp = 0; vp < b2; vp++) {
+                            const double da = Rr[vp] * (row[vp] - rdr) - dH[up] * Rr[vp] * (Ar[vp] - ea);
+                            const double *kr = kh + ((int64_t)up * b2 + vp) * d;
+                            double *dkr = dkh + ((int64_t)up * b2 + vp) * d;
+                            double *dvr = dvh + ((int64_t)up * b2 + vp) * d;
+                            for (int j = 0; j < d; j++) {
+                                dqbar[j] += s * da * kr[j];
+                                dkr[j] += s * da * qbar[j] + Rr[vp] * dKt[(size_t)up * d + j];
+                                dvr[j] += Rr[vp] * dZ[(size_t)up * d + j];
+                            }
+                        }
+                    }
+                    for (int u = u0; u < u1; u++)
+                        for (int j = 0; j < d; j++)
+                            dqh[((int64_t)u * b2 + c) * d + j] += dqbar[j] / nq;
+                }
+            }
+        }
+        free(ws);
+    }
+    return err;
+}
+
 int oracle_max_threads(void)
 {
 #ifdef _OPENMP

@@ -46,6 +46,8 @@ def _load(path: str | None = None):
         lib.oracle_monarch_problems.restype = i
         lib.oracle_monarch_attn_kv.argtypes = [dp, dp, dp, dp, i, i, i, i, i, i, i, dp, dp, i]
         lib.oracle_monarch_attn_kv.restype = i
+        lib.oracle_monarch_attn_bwd.argtypes = [dp] * 7 + [i] * 7
+        lib.oracle_monarch_attn_bwd.restype = i
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = i
         _libs[key] = lib
@@ -128,6 +130,24 @@ def monarch_attn_kv(q, k, v, b1, b1k, b2, tiles=1, iters=1, half_steps=None, fac
     if factors:
         return y, L.reshape(shape[:-2] + L.shape[1:]), R.reshape(shape[:-2] + R.shape[1:])
     return y
+
+
+def monarch_attn_bwd(q, k, v, dy, b1, b2, tiles=1, nthreads=0, lib=None):
+    """Gradients (dq, dk, dv) of sum(dy * y) for one iteration of the forward pass
+    (the chain rule through the output, the L-step, the R-step and the query
+    aggregation); float64 arrays [..., N, d]."""
+    qh, shape = _heads(q)
+    kh, _ = _heads(k)
+    vh, _ = _heads(v)
+    dyh, _ = _heads(dy)
+    BH, N, d = qh.shape
+    dq, dk, dv = (np.zeros_like(qh) for _ in range(3))
+    rc = _load(lib).oracle_monarch_attn_bwd(_dptr(qh), _dptr(kh), _dptr(vh), _dptr(dyh),
+                                            _dptr(dq), _dptr(dk), _dptr(dv), BH, N, d, b1, b2,
+                                            tiles, nthreads)
+    if rc != 0:
+        raise ValueError("oracle_monarch_attn_bwd failed with code %d" % rc)
+    return dq.reshape(shape), dk.reshape(shape), dv.reshape(shape)
 
 
 def monarch_problems(q, k, v, b1, b2, tiles, iters, probs, nthreads=0, y=None):
