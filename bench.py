@@ -456,6 +456,72 @@ def time_forward(wl: synth.Workload, q, k, v, out, steps: int, warmup: int, flus
     return times, _lib.monarch_attn_path(*sargs, _lib.BF16)
 
 
+def run_backward(args, wl: synth.Workload) -> None:
+    """One JSON line: device ms of the backward pass of one iteration
+    (monarch_attn_bwd_ws on resident bfloat16 inputs and upstream gradient), its
+    algorithmic FLOPs against the float32 SIMT roofline of its kernels, and the
+    per-family split.  Parity is checked by the GPU tests, not here."""
+    import torch
+    from structured_attention_video_b200 import _lib
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    peaks, peak_kind = load_peaks()
+    shape = (wl.B, wl.H, wl.N, wl.d)
+    hq, hk, hv = (torch.empty(shape, dtype=torch.int16) for _ in range(3))
+    synth.fill_device_bits(wl, hq.numpy().view(np.uint16), hk.numpy().view(np.uint16),
+                           hv.numpy().view(np.uint16), 0)
+    q, k, v = (x.to(dev).view(torch.bfloat16) for x in (hq, hk, hv))
+    dy = torch.randn(shape, generator=torch.Generator().manual_seed(3)).to(dev, torch.bfloat16)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    sargs = (wl.B, wl.H, wl.f, wl.h, wl.w, wl.d, wl.b1, wl.b2, wl.tiles, 1)
+    nb = _lib.monarch_attn_bwd_workspace_bytes(*sargs, _lib.BF16)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+
+    def step():
+        _lib.check(_lib.monarch_attn_bwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                            dy.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                            dv.data_ptr(), *sargs, _lib.BF16, ws.data_ptr(), nb,
+                                            sh), "monarch_attn_bwd_ws")
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    _lib.monarch_profile_enable(1)
+    _lib.monarch_profile_collect()
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    _lib.monarch_profile_enable(0)
+    prof = _lib.monarch_profile_collect()
+    _lib.check(_lib.monarch_last_device_status(sh), "device status (backward)")
+    kernels = {name: ms_tot / max(1, args.steps) for name, (ms_tot, cnt) in prof.items() if cnt > 0}
+    ms = float(np.median(times))
+    flops = wl.backward_flops()
+    achieved = flops / (ms * 1e-3) / 1e12
+    peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    print(json.dumps({
+        "metric": "Monarch-attn backward ms (one iteration)", "value": ms, "unit": "ms",
+        "higher_is_better": False, "steps": args.steps, "warmup": args.warmup,
+        "ms_stats": step_stats(times), "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(wl, 1),
+        "backward_gflop": flops / 1e9,
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak,
+                     "peak_source": "derived: 148 SMs x 128 FP32 FMA lanes x 2 x %s sm_max_mhz"
+                                    % peak_kind},
+        "kernels_ms_per_step": kernels, "workspace_bytes": nb,
+        "gpu": torch.cuda.get_device_name(0)}), flush=True)
+
+
 SWEEPS = (("480p_full", "tiles", (1, 2, 4, 8), None),
           ("14b", "iters", (1, 2, 5, 10), (0, 13, 27, 40, 53, 79)))
 
@@ -694,6 +760,9 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="error-vs-cost sweeps (tiles on 480p, iterations on Wan-14B) instead "
                          "of the bench line; one GPU")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass of one iteration on --workload instead of "
+                         "the forward bench line; one GPU")
     ap.add_argument("--sweep-steps", type=int, default=20)
     ap.add_argument("--sweep-rows", type=int, default=1024)
     args = ap.parse_args()
@@ -723,6 +792,11 @@ def main():
         if world != 1:
             ap.error("--sweep runs on one GPU")
         run_sweeps(args)
+        return
+    if args.backward:
+        if world != 1:
+            ap.error("--backward runs on one GPU")
+        run_backward(args, wl)
         return
 
     import torch

@@ -215,6 +215,41 @@ MONARCH_API monarch_status monarch_attn_fwd_kv_ws(const void *q, const void *k, 
                                                   monarch_stream_t stream);
 
 /*
+ * Backward pass of one iteration (iters must be 1; else MONARCH_ERR_UNSUPPORTED).
+ * Given dy = dPhi/dY for a scalar loss Phi of the output of monarch_attn_fwd with
+ * the same arguments, writes dq = dPhi/dQ, dk = dPhi/dK, dv = dPhi/dV: the chain
+ * rule through the output, the L-step (L = softmax(s q.Ktil + H)), the R-step
+ * (R = softmax(s qbar.k), its entropy H, Ktil = R K, Z = R V) and the query
+ * aggregation (qbar = mean of the tile's queries).
+ *   q, k, v, dy   device pointers, [B][H][N][d] in `dtype`, read only.
+ *   dq, dk, dv    device pointers, [B][H][N][d] in `dtype`, fully overwritten.
+ * Other arguments as monarch_attn_fwd.  The generic float32 kernels run for every
+ * supported shape and dtype (recomputing the forward's R-step); each gradient
+ * element is written by one warp, so results are deterministic.  The workspace
+ * (monarch_attn_bwd_workspace_bytes, 0 if the arguments fail validation or
+ * iters != 1) holds the forward intermediates and the backward's, all float32.
+ * monarch_attn_bwd takes it with cudaMallocAsync on `stream`; monarch_attn_bwd_ws
+ * uses the caller's (256-byte aligned; MONARCH_ERR_NO_MEMORY if too small).
+ * Source: the pages print no backward; they finetune through the attention
+ * (summary page, "Approach"; explainer page, "创新三：微调与高效内核").  This is
+ * the derivative of the forward map above.
+ */
+MONARCH_API size_t monarch_attn_bwd_workspace_bytes(int B, int H, int f, int h, int w, int d,
+                                                    int b1, int b2, int tiles, int iters,
+                                                    monarch_dtype dtype);
+MONARCH_API monarch_status monarch_attn_bwd_ws(const void *q, const void *k, const void *v,
+                                               const void *dy, void *dq, void *dk, void *dv,
+                                               int B, int H, int f, int h, int w, int d, int b1,
+                                               int b2, int tiles, int iters, monarch_dtype dtype,
+                                               void *workspace, size_t ws_bytes,
+                                               monarch_stream_t stream);
+MONARCH_API monarch_status monarch_attn_bwd(const void *q, const void *k, const void *v,
+                                            const void *dy, void *dq, void *dk, void *dv, int B,
+                                            int H, int f, int h, int w, int d, int b1, int b2,
+                                            int tiles, int iters, monarch_dtype dtype,
+                                            monarch_stream_t stream);
+
+/*
  * Forward pass on HOST buffers: q, k, v, out are host pointers (pinned memory
  * gives full PCIe bandwidth; pageable memory works but is slower).  Device
  * copies of the inputs and output and the workspace are taken with

@@ -39,6 +39,9 @@ SIGNATURES = {
     "monarch_attn_fwd_kv_ws": ([_vp, _vp, _vp, _vp] + [_i] * 12 + [_i, _vp, _sz, _vp], _i),
     "monarch_attn_fwd_units_ws": ([_vp, _vp, _vp, _vp] + _SHAPE + [_i, _i, _i, _vp, _sz, _vp], _i),
     "monarch_attn_fwd_noalloc": ([_vp, _vp, _vp, _vp] + _SHAPE + [_i, _vp], _i),
+    "monarch_attn_bwd_workspace_bytes": (_SHAPE + [_i], _sz),
+    "monarch_attn_bwd_ws": ([_vp] * 7 + _SHAPE + [_i, _vp, _sz, _vp], _i),
+    "monarch_attn_bwd": ([_vp] * 7 + _SHAPE + [_i, _vp], _i),
     "monarch_index_maps": ([_i] * 6 + [_ip, _ip, _ip, _ip], _i),
     "monarch_index_maps_device": ([_i] * 6 + [_vp, _vp, _vp, _vp, _vp], _i),
     "monarch_last_device_status": ([_vp], _i),
@@ -116,6 +119,22 @@ def monarch_attn_fwd_noalloc(q, k, v, out, B, H, f, h, w, d, b1, b2, tiles, iter
                              stream):
     return _lib.monarch_attn_fwd_noalloc(q, k, v, out, B, H, f, h, w, d, b1, b2, tiles, iters,
                                          dtype, stream)
+
+
+def monarch_attn_bwd_workspace_bytes(B, H, f, h, w, d, b1, b2, tiles, iters, dtype):
+    return _lib.monarch_attn_bwd_workspace_bytes(B, H, f, h, w, d, b1, b2, tiles, iters, dtype)
+
+
+def monarch_attn_bwd_ws(q, k, v, dy, dq, dk, dv, B, H, f, h, w, d, b1, b2, tiles, iters, dtype,
+                        workspace, ws_bytes, stream):
+    return _lib.monarch_attn_bwd_ws(q, k, v, dy, dq, dk, dv, B, H, f, h, w, d, b1, b2, tiles,
+                                    iters, dtype, workspace, ws_bytes, stream)
+
+
+def monarch_attn_bwd(q, k, v, dy, dq, dk, dv, B, H, f, h, w, d, b1, b2, tiles, iters, dtype,
+                     stream):
+    return _lib.monarch_attn_bwd(q, k, v, dy, dq, dk, dv, B, H, f, h, w, d, b1, b2, tiles, iters,
+                                 dtype, stream)
 
 
 def monarch_index_maps(f, h, w, b1, b2, tiles, u_of_n, v_of_n, perm, tile_begin):

@@ -110,3 +110,28 @@ def monarch_attention_units(q, k, v, out, *, f, h, w, b1, b2, tiles=1, iters=1, 
                                               ws.data_ptr(), need, stream),
                "monarch_attn_fwd_units_ws")
     return out
+
+
+def monarch_attention_backward(q, k, v, dy, *, f, h, w, b1, b2, tiles=1, iters=1, workspace=None):
+    """Gradients (dq, dk, dv) of a loss whose gradient with respect to
+    monarch_attention(q, k, v, ...) is dy (one iteration)."""
+    _check_tensors(q, k, v, dy)
+    args = _shape_args(q, f, h, w, b1, b2, tiles, iters)
+    dt = _DTYPES[q.dtype]
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    need = _lib.monarch_attn_bwd_workspace_bytes(*args, dt)
+    if need == 0:
+        # validation failed or iters != 1: let the library report why
+        _lib.check(_lib.monarch_attn_bwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                            dy.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                            dv.data_ptr(), *args, dt, 0, 0, 0),
+                   "monarch_attn_bwd_ws")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    _lib.check(_lib.monarch_attn_bwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(), dy.data_ptr(),
+                                        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), *args, dt,
+                                        workspace.data_ptr(),
+                                        workspace.numel() * workspace.element_size(), stream),
+               "monarch_attn_bwd_ws")
+    return dq, dk, dv

@@ -337,6 +337,66 @@ monarch_status monarch_attn_fwd(const void *q, const void *k, const void *v, voi
     return st;
 }
 
+// Backward pass of one iteration (generic SIMT kernels): see the header.
+size_t monarch_attn_bwd_workspace_bytes(int B, int H, int f, int h, int w, int d, int b1, int b2,
+                                        int tiles, int iters, monarch_dtype dtype) {
+    Problem p;
+    if (validate_shape(B, H, f, h, w, d, b1, b2, tiles, iters, dtype, &p) != MONARCH_OK ||
+        iters != 1)
+        return 0;
+    bool overflow = false;
+    const size_t n = backward_workspace_bytes(p, overflow);
+    return overflow ? 0 : n;
+}
+
+monarch_status monarch_attn_bwd_ws(const void *q, const void *k, const void *v, const void *dy,
+                                   void *dq, void *dk, void *dv, int B, int H, int f, int h,
+                                   int w, int d, int b1, int b2, int tiles, int iters,
+                                   monarch_dtype dtype, void *workspace, size_t ws_bytes,
+                                   monarch_stream_t stream) {
+    if (!q || !k || !v || !dy || !dq || !dk || !dv || !workspace) return MONARCH_ERR_INVALID_ARG;
+    Problem p;
+    monarch_status st = validate_shape(B, H, f, h, w, d, b1, b2, tiles, iters, dtype, &p);
+    if (st != MONARCH_OK) return st;
+    if (iters != 1) return MONARCH_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dy) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv) || ((uintptr_t)workspace & 255u))
+        return MONARCH_ERR_ALIGN;
+    bool overflow = false;
+    const size_t need = backward_workspace_bytes(p, overflow);
+    if (overflow) return MONARCH_ERR_SHAPE;
+    if (ws_bytes < need) return MONARCH_ERR_NO_MEMORY;
+    return generic_backward(p, dtype, q, k, v, dy, dq, dk, dv, workspace,
+                            (cudaStream_t)stream) == cudaSuccess
+               ? MONARCH_OK
+               : MONARCH_ERR_CUDA;
+}
+
+monarch_status monarch_attn_bwd(const void *q, const void *k, const void *v, const void *dy,
+                                void *dq, void *dk, void *dv, int B, int H, int f, int h, int w,
+                                int d, int b1, int b2, int tiles, int iters, monarch_dtype dtype,
+                                monarch_stream_t stream) {
+    const size_t need = monarch_attn_bwd_workspace_bytes(B, H, f, h, w, d, b1, b2, tiles, iters,
+                                                         dtype);
+    if (need == 0) {
+        Problem p;
+        monarch_status st = validate_shape(B, H, f, h, w, d, b1, b2, tiles, iters, dtype, &p);
+        return st != MONARCH_OK ? st : (iters != 1 ? MONARCH_ERR_UNSUPPORTED : MONARCH_ERR_SHAPE);
+    }
+    if (!q || !k || !v || !dy || !dq || !dk || !dv) return MONARCH_ERR_INVALID_ARG;
+    configure_pool_once();
+    void *ws = nullptr;
+    if (cudaMallocAsync(&ws, need, (cudaStream_t)stream) != cudaSuccess) {
+        cudaGetLastError();
+        return MONARCH_ERR_NO_MEMORY;
+    }
+    monarch_status st = monarch_attn_bwd_ws(q, k, v, dy, dq, dk, dv, B, H, f, h, w, d, b1, b2,
+                                            tiles, iters, dtype, ws, need, stream);
+    if (cudaFreeAsync(ws, (cudaStream_t)stream) != cudaSuccess && st == MONARCH_OK)
+        st = MONARCH_ERR_CUDA;
+    return st;
+}
+
 monarch_status monarch_attn_fwd_host(const void *q, const void *k, const void *v, void *out,
                                      int B, int H, int f, int h, int w, int d, int b1, int b2,
                                      int tiles, int iters, monarch_dtype dtype,
@@ -464,7 +524,8 @@ const char *monarch_profile_kernel_name(int k) {
                                          "lstep_kernel",         "qbar_weighted_kernel",
                                          "tc_qbar_kernel",       "tc_rstep_kernel",
                                          "tc_lstep_kernel",      "tc_lstat_kernel",
-                                         "tc_qagg_kernel"};
+                                         "tc_qagg_kernel", "bwd_lstep_kernels",
+                                         "bwd_rstep_kernels"};
     return (k >= 0 && k < K_COUNT) ? names[k] : nullptr;
 }
 

@@ -71,7 +71,9 @@ enum KernelId {
     K_TC_LSTEP = 6,       // S3, tensor-core path
     K_TC_LSTAT = 7,       // S3 row statistics of the iterations before the last (tensor-core)
     K_TC_QAGG = 8,        // S4 re-aggregated queries (tensor-core)
-    K_COUNT = 9
+    K_BWD_L = 9,          // backward of the L-step and the output (generic)
+    K_BWD_R = 10,         // backward of the R-step and the aggregation (generic)
+    K_COUNT = 11
 };
 
 // Brackets one kernel launch with CUDA events while profiling is enabled.
@@ -154,6 +156,25 @@ struct GenericWorkspace {
 
 size_t generic_workspace_bytes(const Problem &p, bool &overflow);
 GenericWorkspace generic_workspace_carve(const Problem &p, void *base);
+// S1 and the first R-step only (qbar, Ktil, Z, H into the workspace), for the
+// backward pass of one iteration.
+cudaError_t generic_rstep_only(const Problem &p, monarch_dtype dtype, const void *q,
+                               const void *k, const void *v, const GenericWorkspace &ws,
+                               cudaStream_t stream);
+
+// Backward pass of one iteration (float32 intermediates after the forward's).
+struct BwdWorkspace {
+    float *lse, *delta;   // [BH][N]  per query row: L-step log-sum-exp, dy.y
+    float *dql;           // [BH][N][d]  the L-step's part of dq
+    float *dkt, *dz;      // [BH][t][b2][b1k][d]  dKtil, dZ
+    float *dh;            // [BH][t][b2][b1k]     dH
+    float *lsea, *ea, *rho;   // [BH][t][b2][b1k]  per R row: lse(a), E_R[a], sum R dR
+    float *dqbar;         // [BH][t][b2][d]
+};
+size_t backward_workspace_bytes(const Problem &p, bool &overflow);
+cudaError_t generic_backward(const Problem &p, monarch_dtype dtype, const void *q, const void *k,
+                             const void *v, const void *dy, void *dq, void *dk, void *dv,
+                             void *workspace, cudaStream_t stream);
 cudaError_t generic_forward(const Problem &p, monarch_dtype dtype, const void *q, const void *k,
                             const void *v, void *out, const GenericWorkspace &ws,
                             cudaStream_t stream);

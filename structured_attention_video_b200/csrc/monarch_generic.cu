@@ -353,6 +353,24 @@ cudaError_t run_generic(const Problem &p, const T *q, const T *k, const T *v, T 
     return cudaGetLastError();
 }
 
+template <typename T, int D>
+cudaError_t run_rstep_only(const Problem &p, const T *q, const T *k, const T *v,
+                           const GenericWorkspace &ws, cudaStream_t stream) {
+    const size_t smem_r = (GW * D + 2 * KC * (D + 1)) * sizeof(float);
+    const int64_t units = p.unit_end - p.unit_begin;
+    const int64_t nmean = units * p.b2 * p.d;
+    const int mean_blocks = (int)((nmean + 255) / 256 < 148 * 64 ? (nmean + 255) / 256 : 148 * 64);
+    {
+        ProfileScope scope(K_QBAR_MEAN, stream);
+        qbar_mean_kernel<T><<<mean_blocks, 256, 0, stream>>>(q, ws.qbar, p);
+    }
+    const unsigned r_blocks = (unsigned)(units * p.b1k * ((p.b2 + GW - 1) / GW));
+    ProfileScope scope(K_RSTEP, stream);
+    rstep_kernel<T, D><<<r_blocks, GW * 32, smem_r, stream>>>(k, v, ws.qbar, (int64_t)p.d, 0,
+                                                            ws.ktil, ws.z, ws.hent, p);
+    return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t dispatch_d(const Problem &p, const void *q, const void *k, const void *v, void *out,
                        const GenericWorkspace &ws, cudaStream_t stream) {
@@ -400,6 +418,24 @@ cudaError_t generic_forward(const Problem &p, monarch_dtype dtype, const void *q
                             cudaStream_t stream) {
     if (dtype == MONARCH_F32) return dispatch_d<float>(p, q, k, v, out, ws, stream);
     return dispatch_d<__nv_bfloat16>(p, q, k, v, out, ws, stream);
+}
+
+cudaError_t generic_rstep_only(const Problem &p, monarch_dtype dtype, const void *q,
+                               const void *k, const void *v, const GenericWorkspace &ws,
+                               cudaStream_t stream) {
+    switch (p.d) {
+#define MONARCH_RO_CASE(D)                                                                    \
+    case D:                                                                                   \
+        return dtype == MONARCH_F32                                                           \
+                   ? run_rstep_only<float, D>(p, (const float *)q, (const float *)k,          \
+                                              (const float *)v, ws, stream)                   \
+                   : run_rstep_only<__nv_bfloat16, D>(p, (const __nv_bfloat16 *)q,            \
+                                                      (const __nv_bfloat16 *)k,               \
+                                                      (const __nv_bfloat16 *)v, ws, stream);
+        MONARCH_RO_CASE(32) MONARCH_RO_CASE(64) MONARCH_RO_CASE(128)
+#undef MONARCH_RO_CASE
+    }
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t index_maps_device(int N, int b1, int b2, int tiles, int32_t *u_of_n, int32_t *v_of_n,

@@ -1064,14 +1064,18 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 tc_fence_after();
                 uint32_t pk[64];
 #pragma unroll
-                for (int c = 0; c < 4; c++) {
-                    uint32_t o[32];
-                    tmem_ld32(tmem + lane_off + 256 + part * 128 + c * 32, o);
+                for (int c = 0; c < 4; c += 2) {   // two 32-column loads per wait
+                    uint32_t o0[32], o1[32];
+                    tmem_ld32(tmem + lane_off + 256 + part * 128 + c * 32, o0);
+                    tmem_ld32(tmem + lane_off + 256 + part * 128 + c * 32 + 32, o1);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int k = 0; k < 16; k++)
+                    for (int k = 0; k < 16; k++) {
                         pk[c * 16 + k] =
-                            pack_bf16(__uint_as_float(o[2 * k]), __uint_as_float(o[2 * k + 1]));
+                            pack_bf16(__uint_as_float(o0[2 * k]), __uint_as_float(o0[2 * k + 1]));
+                        pk[c * 16 + 16 + k] =
+                            pack_bf16(__uint_as_float(o1[2 * k]), __uint_as_float(o1[2 * k + 1]));
+                    }
                 }
                 tc_fence_before();
                 mbar_arrive_warp(o_empty + part);

@@ -87,6 +87,18 @@ class Workload:
         per_head = (4 * T + 2) * t * N * self.b2 * self.d + 4 * T * N * self.b1 * self.d
         return float(self.B * self.H * per_head)
 
+    def backward_flops(self) -> float:
+        """Algorithmic FLOPs of the backward pass of one iteration (multiply-add =
+        2), without recomputing the forward's R-step.
+
+        Per (b, h): the L-step side takes the logits again, dL = dY Z^T, dq = dB
+        Ktil, dKtil = dB^T Q and dZ = L^T dY (5 x 2*N*b1*d); the R-step side
+        takes its logits again, dR = dKtil k + dZ v (two products), dqbar = dA k,
+        dk = dA qbar + R^T dKtil (two) and dv = R^T dZ (7 x 2*t*N*b2*d).
+        """
+        return float(self.B * self.H * (10 * self.N * self.b1 + 14 * self.tiles * self.N * self.b2)
+                     * self.d)
+
     def dense_flops(self) -> float:
         """FLOPs of exact softmax attention on the same shape (4*N^2*d per head)."""
         return float(4 * self.B * self.H * self.N * self.N * self.d)

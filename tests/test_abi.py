@@ -109,3 +109,23 @@ def test_workspace_covers_intermediates():
     wl = synth.WORKLOADS["720p"]
     need = _lib.monarch_attn_workspace_bytes(*SHAPE_720P, _lib.BF16)
     assert need >= 2 * wl.B * wl.H * wl.tiles * wl.N * wl.d * 2
+
+
+def test_backward_workspace_and_validation():
+    """The backward's workspace: 0 for iters != 1 or a failing shape; otherwise at
+    least the forward's intermediates plus the backward's float32 arrays; the
+    calls reject bad arguments before touching the device."""
+    shape = (1, 2, 3, 8, 8, 32, 24, 8, 5)   # B, H, f, h, w, d, b1, b2, tiles
+    fw = _lib.monarch_attn_workspace_bytes(*shape, 1, _lib.F32)
+    bw = _lib.monarch_attn_bwd_workspace_bytes(*shape, 1, _lib.F32)
+    B, H, N, d, t = 1, 2, 192, 32, 5
+    floats = (2 * B * H * N + B * H * N * d + 2 * B * H * t * N * d + 4 * B * H * t * N)
+    assert bw >= fw + 4 * floats
+    assert _lib.monarch_attn_bwd_workspace_bytes(*shape, 2, _lib.F32) == 0
+    assert _lib.monarch_attn_bwd_workspace_bytes(1, 2, 3, 8, 8, 32, 25, 8, 5, 1, _lib.F32) == 0
+    # iters = 2: refused before anything is enqueued
+    assert _lib.monarch_attn_bwd(16, 16, 16, 16, 16, 16, 16, *shape, 2, _lib.F32,
+                                 None) == 4   # MONARCH_ERR_UNSUPPORTED
+    # a null gradient pointer
+    assert _lib.monarch_attn_bwd_ws(16, 16, 16, 16, None, 16, 16, *shape, 1, _lib.F32, 256,
+                                    bw, None) == 1   # MONARCH_ERR_INVALID_ARG
