@@ -182,6 +182,27 @@ MONARCH_API monarch_status monarch_attn_fwd_units_ws(const void *q, const void *
                                                      size_t ws_bytes, monarch_stream_t stream);
 
 /*
+ * Forward pass on tensors in another layout.  layout = MONARCH_LAYOUT_BHND is
+ * [B][H][N][d] (monarch_attn_fwd_ws); MONARCH_LAYOUT_BNHD is [B][N][H][d], the
+ * heads of each token contiguous, as in the attention layers of video diffusion
+ * transformers.  q, k, v and out all use `layout`; the workspace
+ * (monarch_attn_workspace_bytes, the same for both layouts) and every other
+ * argument are those of monarch_attn_fwd_ws.  Both kernel families read the
+ * strided rows directly (no transposed copies).  Returns MONARCH_ERR_INVALID_ARG
+ * for another layout value.
+ * Source: the survey's strided-input variant of the explainer page's video token
+ * layout ("创新一：块对齐策略": N = f*h*w tokens per head).
+ */
+typedef enum { MONARCH_LAYOUT_BHND = 0, MONARCH_LAYOUT_BNHD = 1 } monarch_layout;
+
+MONARCH_API monarch_status monarch_attn_fwd_layout_ws(const void *q, const void *k, const void *v,
+                                                      void *out, int B, int H, int f, int h,
+                                                      int w, int d, int b1, int b2, int tiles,
+                                                      int iters, monarch_dtype dtype,
+                                                      monarch_layout layout, void *workspace,
+                                                      size_t ws_bytes, monarch_stream_t stream);
+
+/*
  * Queries of a chunk of frames against keys and values that also hold earlier
  * frames (a key/value cache), as in chunk-by-chunk autoregressive video
  * generation (the Self-Forcing setting of the MonarchRT pages: summary page,

@@ -39,6 +39,7 @@ SIGNATURES = {
     "monarch_attn_fwd_kv_ws": ([_vp, _vp, _vp, _vp] + [_i] * 12 + [_i, _vp, _sz, _vp], _i),
     "monarch_attn_fwd_units_ws": ([_vp, _vp, _vp, _vp] + _SHAPE + [_i, _i, _i, _vp, _sz, _vp], _i),
     "monarch_attn_fwd_noalloc": ([_vp, _vp, _vp, _vp] + _SHAPE + [_i, _vp], _i),
+    "monarch_attn_fwd_layout_ws": ([_vp, _vp, _vp, _vp] + _SHAPE + [_i, _i, _vp, _sz, _vp], _i),
     "monarch_attn_bwd_workspace_bytes": (_SHAPE + [_i], _sz),
     "monarch_attn_bwd_ws": ([_vp] * 7 + _SHAPE + [_i, _vp, _sz, _vp], _i),
     "monarch_attn_bwd": ([_vp] * 7 + _SHAPE + [_i, _vp], _i),
@@ -119,6 +120,15 @@ def monarch_attn_fwd_noalloc(q, k, v, out, B, H, f, h, w, d, b1, b2, tiles, iter
                              stream):
     return _lib.monarch_attn_fwd_noalloc(q, k, v, out, B, H, f, h, w, d, b1, b2, tiles, iters,
                                          dtype, stream)
+
+
+BHND, BNHD = 0, 1   # monarch_layout
+
+
+def monarch_attn_fwd_layout_ws(q, k, v, out, B, H, f, h, w, d, b1, b2, tiles, iters, dtype,
+                               layout, workspace, ws_bytes, stream):
+    return _lib.monarch_attn_fwd_layout_ws(q, k, v, out, B, H, f, h, w, d, b1, b2, tiles, iters,
+                                           dtype, layout, workspace, ws_bytes, stream)
 
 
 def monarch_attn_bwd_workspace_bytes(B, H, f, h, w, d, b1, b2, tiles, iters, dtype):

@@ -135,3 +135,34 @@ def monarch_attention_backward(q, k, v, dy, *, f, h, w, b1, b2, tiles=1, iters=1
                                         workspace.numel() * workspace.element_size(), stream),
                "monarch_attn_bwd_ws")
     return dq, dk, dv
+
+
+def monarch_attention_bnhd(q, k, v, *, f, h, w, b1, b2, tiles=1, iters=1, out=None,
+                           workspace=None):
+    """monarch_attention on [B, N, H, d] tensors (the heads of each token
+    contiguous); the kernels read the strided rows directly."""
+    if out is None:
+        out = torch.empty_like(q)
+    _check_tensors(q, k, v, out)
+    if q.dim() != 4:
+        raise ValueError("expected [B, N, H, d] tensors")
+    B, N, H, d = q.shape
+    if N != f * h * w:
+        raise ValueError("N = %d but f*h*w = %d" % (N, f * h * w))
+    args = (B, H, f, h, w, d, b1, b2, tiles, iters)
+    dt = _DTYPES[q.dtype]
+    need = _lib.monarch_attn_workspace_bytes(*args, dt)
+    if need == 0:
+        _lib.check(_lib.monarch_attn_fwd_layout_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                   out.data_ptr(), *args, dt, _lib.BNHD, 0, 0, 0),
+                   "monarch_attn_fwd_layout_ws")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    _lib.check(_lib.monarch_attn_fwd_layout_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                               out.data_ptr(), *args, dt, _lib.BNHD,
+                                               workspace.data_ptr(),
+                                               workspace.numel() * workspace.element_size(),
+                                               stream),
+               "monarch_attn_fwd_layout_ws")
+    return out

@@ -116,6 +116,7 @@ monarch_status validate_shape(int B, int H, int f, int h, int w, int d, int b1, 
     p->unit_end = B * H * tiles;
     p->Nk = p->N;
     p->b1k = b1;
+    p->layout = kLayoutBHND;
     return MONARCH_OK;
 }
 
@@ -244,6 +245,28 @@ monarch_status monarch_attn_fwd_ws(const void *q, const void *k, const void *v, 
     Problem p;
     monarch_status st = validate_shape(B, H, f, h, w, d, b1, b2, tiles, iters, dtype, &p);
     if (st != MONARCH_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        ((uintptr_t)workspace & 255u))
+        return MONARCH_ERR_ALIGN;
+    bool overflow = false;
+    const size_t need = workspace_bytes_for(p, dtype, choose_path(p, dtype), overflow);
+    if (overflow) return MONARCH_ERR_SHAPE;
+    if (ws_bytes < need) return MONARCH_ERR_NO_MEMORY;
+    return run_forward(p, dtype, q, k, v, out, workspace, (cudaStream_t)stream);
+}
+
+monarch_status monarch_attn_fwd_layout_ws(const void *q, const void *k, const void *v, void *out,
+                                          int B, int H, int f, int h, int w, int d, int b1,
+                                          int b2, int tiles, int iters, monarch_dtype dtype,
+                                          monarch_layout layout, void *workspace,
+                                          size_t ws_bytes, monarch_stream_t stream) {
+    if (!q || !k || !v || !out || !workspace) return MONARCH_ERR_INVALID_ARG;
+    if (layout != MONARCH_LAYOUT_BHND && layout != MONARCH_LAYOUT_BNHD)
+        return MONARCH_ERR_INVALID_ARG;
+    Problem p;
+    monarch_status st = validate_shape(B, H, f, h, w, d, b1, b2, tiles, iters, dtype, &p);
+    if (st != MONARCH_OK) return st;
+    p.layout = layout == MONARCH_LAYOUT_BNHD ? kLayoutBNHD : kLayoutBHND;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
         ((uintptr_t)workspace & 255u))
         return MONARCH_ERR_ALIGN;

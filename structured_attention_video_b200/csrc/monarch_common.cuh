@@ -47,9 +47,26 @@ struct Problem {
     // self-attention over one clip; more when the queries of a chunk of frames
     // also attend to a cache of earlier frames)
     int Nk, b1k;
+    // layout of q, k, v and the output: kLayoutBHND or kLayoutBNHD (below)
+    int layout;
     __host__ __device__ int head_begin() const { return unit_begin / tiles; }
     __host__ __device__ int head_end() const { return (unit_end + tiles - 1) / tiles; }
 };
+
+// Layouts of the inputs and the output: [B][H][N][d] (the tokens of a head are
+// contiguous rows) or [B][N][H][d] (the heads of a token are contiguous).
+// Element j of token n of head bh = b*H + h sits at
+//   head_base(p, bh, n_tokens) + n * tok_stride(p) + j.
+// Every intermediate in the workspace keeps its own [B*H]-major layout.
+constexpr int kLayoutBHND = 0, kLayoutBNHD = 1;
+__host__ __device__ __forceinline__ int64_t tok_stride(const Problem &p) {
+    return p.layout == kLayoutBNHD ? (int64_t)p.H * p.d : (int64_t)p.d;
+}
+__host__ __device__ __forceinline__ int64_t head_base(const Problem &p, int bh, int ntok) {
+    return p.layout == kLayoutBNHD
+               ? ((int64_t)(bh / p.H) * ntok * p.H + bh % p.H) * p.d
+               : (int64_t)bh * ntok * p.d;
+}
 
 // Kernels that can give up a bounded wait receive a pointer to the device
 // status word of the library (one int per device, read and cleared by

@@ -50,9 +50,10 @@ __global__ void qbar_mean_kernel(const T *__restrict__ q, float *__restrict__ qb
         const int64_t bhg = idx / row_elems, col = idx % row_elems;
         const int g = (int)(bhg % p.tiles), bh = (int)(bhg / p.tiles);
         const int u0 = tile_begin(g, p.b1, p.tiles), u1 = tile_begin(g + 1, p.b1, p.tiles);
-        const T *src = q + (int64_t)bh * p.N * p.d + col;
+        const int64_t ts = tok_stride(p);
+        const T *src = q + head_base(p, bh, p.N) + (col / p.d) * ts + col % p.d;
         float acc = 0.f;
-        for (int u = u0; u < u1; u++) acc += to_f32(src[(int64_t)u * row_elems]);
+        for (int u = u0; u < u1; u++) acc += to_f32(src[(int64_t)u * p.b2 * ts]);
         qbar[idx] = acc / (float)(u1 - u0);
     }
 }
@@ -87,7 +88,8 @@ rstep_kernel(const T *__restrict__ k, const T *__restrict__ v, const float *__re
         const float *qr = qbar + (bhg * p.b2 + vrow) * qbar_v_stride + (int64_t)up * qbar_up_stride;
         for (int j = lane; j < D; j += 32) sq[warp * D + j] = qr[j];
     }
-    const int64_t base = ((int64_t)bh * p.Nk + (int64_t)up * p.b2) * D;
+    const int64_t ts = tok_stride(p);
+    const int64_t base = head_base(p, bh, p.Nk) + (int64_t)up * p.b2 * ts;
     float m = -INFINITY, l = 0.f, e = 0.f;
     float acck[NJ], accv[NJ];
 #pragma unroll
@@ -98,8 +100,8 @@ rstep_kernel(const T *__restrict__ k, const T *__restrict__ v, const float *__re
         __syncthreads();
         for (int idx = threadIdx.x; idx < nk * D; idx += blockDim.x) {
             const int r = idx / D, j = idx % D;
-            sk[r * DS + j] = to_f32(k[base + (int64_t)(c0 + r) * D + j]);
-            sv[r * DS + j] = to_f32(v[base + (int64_t)(c0 + r) * D + j]);
+            sk[r * DS + j] = to_f32(k[base + (int64_t)(c0 + r) * ts + j]);
+            sv[r * DS + j] = to_f32(v[base + (int64_t)(c0 + r) * ts + j]);
         }
         __syncthreads();
         if (!active) continue;
@@ -171,10 +173,11 @@ lstep_kernel(const T *__restrict__ q, const float *__restrict__ ktil, const floa
     const int u = u0 + ug * GW + warp;
     const bool active = u < u1;
     const int64_t bhg = (int64_t)bh * p.tiles + g;
-    const int64_t tok = (int64_t)bh * p.N + (int64_t)u * p.b2 + vcol;
+    const int64_t tok = (int64_t)bh * p.N + (int64_t)u * p.b2 + vcol;   // workspace index
+    const int64_t qoff = head_base(p, bh, p.N) + ((int64_t)u * p.b2 + vcol) * tok_stride(p);
 
     if (active)
-        for (int j = lane; j < D; j += 32) sq[warp * D + j] = to_f32(q[tok * D + j]);
+        for (int j = lane; j < D; j += 32) sq[warp * D + j] = to_f32(q[qoff + j]);
     const int64_t kbase = (bhg * p.b2 + vcol) * p.b1k;   // row of block u' = 0
     float m = -INFINITY, l = 0.f;
     float acc[NJ];
@@ -216,7 +219,7 @@ lstep_kernel(const T *__restrict__ q, const float *__restrict__ ktil, const floa
         if (out) {
             const float inv = 1.f / l;
 #pragma unroll
-            for (int i = 0; i < NJ; i++) out[tok * D + lane + 32 * i] = from_f32<T>(acc[i] * inv);
+            for (int i = 0; i < NJ; i++) out[qoff + lane + 32 * i] = from_f32<T>(acc[i] * inv);
         }
         if (lse_out && lane == 0) lse_out[tok] = m + logf(l);
     }
@@ -263,8 +266,8 @@ qbar_weighted_kernel(const T *__restrict__ q, const float *__restrict__ ktil,
         __syncthreads();
         for (int idx = threadIdx.x; idx < nk * D; idx += blockDim.x) {
             const int r = idx / D, j = idx % D;
-            const int64_t tok = (int64_t)bh * p.N + (int64_t)(c0 + r) * p.b2 + vcol;
-            sq[r * DS + j] = to_f32(q[tok * D + j]);
+            const int64_t tok = (int64_t)(c0 + r) * p.b2 + vcol;
+            sq[r * DS + j] = to_f32(q[head_base(p, bh, p.N) + tok * tok_stride(p) + j]);
         }
         if (threadIdx.x < nk)
             sl[threadIdx.x] = lse[(int64_t)bh * p.N + (int64_t)(c0 + threadIdx.x) * p.b2 + vcol];

@@ -87,9 +87,11 @@ __global__ void __launch_bounds__(128 * kQbarGroups) tc_qbar_kernel(
 #pragma unroll
     for (int i = 0; i < 8; i++) acc[i] = 0.f;
     if (active) {
-        const int64_t stride = row_elems / 8;
-        const uint4 *src = reinterpret_cast<const uint4 *>(q + (int64_t)bh * p.N * kD +
-                                                           (int64_t)r0 * row_elems + col);
+        // element (u, v, j) of the head: token u*b2 + v; col = v*d + j
+        const int64_t ts = tok_stride(p);
+        const int64_t stride = p.b2 * ts / 8;   // one block row u, in 16-byte units
+        const uint4 *src = reinterpret_cast<const uint4 *>(
+            q + head_base(p, bh, p.N) + (int64_t)r0 * p.b2 * ts + (col / kD) * ts + col % kD);
         int u = r0;
         for (; u + 8 <= r1; u += 8) {   // eight independent 16-byte loads in flight
             uint4 x[8];
@@ -222,6 +224,9 @@ struct LsProblem {
     int m_y, m_z, m_first, m_end;   // M side: tile t starts at z = m_z + t*128
     int n_y, n_z, nkeys, nch;       // N side: chunk j starts at z = n_z + j*128
     int nh;                         // 64-key halves of the N side (the softmax's unit)
+    // the side that reads the query rows (M, or N in kLsAgg) through the 5-D query
+    // map (x, v, u, head, batch): column qv, first row qu, head qh, batch qb
+    int qv, qu, qh, qb;
 };
 
 template <int MODE>
@@ -256,7 +261,22 @@ __device__ __forceinline__ LsProblem ls_problem(const LsArgs &a, int unit) {
     }
     q.nch = (q.nkeys + 127) / 128;
     q.nh = (q.nkeys + 63) / 64;
+    q.qv = q.v;
+    q.qu = MODE != kLsAgg ? q.m_first : u_lo;
+    q.qh = q.bh % p.H;
+    q.qb = q.bh / p.H;
     return q;
+}
+
+// One 128-row tile of query rows (u, v), u = u0 .. u0 + 127 at column v, through the
+// 5-D query map: (x, v, u, head, batch), or (x, head, v, u, batch) for [B][N][H][d]
+// (the map's dimensions run in order of increasing stride); rows past b1 read zeros.
+__device__ __forceinline__ void ls_load_q(void *dst, const CUtensorMap *map, int x,
+                                          const LsProblem &pr, int u0, bool bnhd, uint64_t *bar) {
+    if (bnhd)
+        tma_load_5d(dst, map, x, pr.qh, pr.qv, u0, pr.qb, bar);
+    else
+        tma_load_5d(dst, map, x, pr.qv, u0, pr.qh, pr.qb, bar);
 }
 
 // One TMA tile load of the L-step: a 3-D gather (x, y, z) or a 2-D row box (x, z).
@@ -365,9 +385,14 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                         // rows past nkeys in the ragged last chunk belong to the next
                         // row block (or are zero-filled past the array): masked later
                         mbar_expect_tx(k_full + sk, kTile + ls::kPanelHx);
-                        for (int pn = 0; pn < 2; pn++)
-                            ls_load(sm + ls::kK + sk * kTile + pn * kPanel, &tmN, n_gather,
-                                    pn * 64, pr.n_y, pr.n_z + j * 128, k_full + sk);
+                        for (int pn = 0; pn < 2; pn++) {
+                            if (n_gather)
+                                ls_load_q(sm + ls::kK + sk * kTile + pn * kPanel, &tmN, pn * 64,
+                                          pr, pr.qu + j * 128, p.layout == kLayoutBNHD, k_full + sk);
+                            else
+                                ls_load(sm + ls::kK + sk * kTile + pn * kPanel, &tmN, false,
+                                        pn * 64, pr.n_y, pr.n_z + j * 128, k_full + sk);
+                        }
                         ls_load(sm + ls::kHx + sk * ls::kPanelHx, &tmX, n_gather, 0, pr.n_y,
                                 pr.n_z + j * 128, k_full + sk);
                     }
@@ -397,9 +422,14 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                     }
                     if (lane == 0) {
                         mbar_expect_tx(q_full + t, kTile);
-                        for (int pn = 0; pn < 2; pn++)
-                            ls_load(sm + ls::kQ + t * kTile + pn * kPanel, &tmM, !n_gather,
-                                    pn * 64, pr.m_y, pr.m_z + t * 128, q_full + t);
+                        for (int pn = 0; pn < 2; pn++) {
+                            if (!n_gather)
+                                ls_load_q(sm + ls::kQ + t * kTile + pn * kPanel, &tmM, pn * 64,
+                                          pr, pr.qu + t * 128, p.layout == kLayoutBNHD, q_full + t);
+                            else
+                                ls_load(sm + ls::kQ + t * kTile + pn * kPanel, &tmM, false,
+                                        pn * 64, pr.m_y, pr.m_z + t * 128, q_full + t);
+                        }
                     }
                 }
                 if (!ok) break;
@@ -408,8 +438,12 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                     const LsProblem nx = ls_problem<MODE>(a, blockIdx.x + (pi + 1) * gridDim.x);
                     for (int t = 0; t < 2; t++)
                         for (int pn = 0; pn < 2; pn++) {
-                            if (!n_gather)
-                                tma_prefetch_3d(&tmM, pn * 64, nx.m_y, nx.m_z + t * 128);
+                            if (!n_gather && p.layout == kLayoutBNHD)
+                                tma_prefetch_5d(&tmM, pn * 64, nx.qh, nx.qv, nx.qu + t * 128,
+                                                nx.qb);
+                            else if (!n_gather)
+                                tma_prefetch_5d(&tmM, pn * 64, nx.qv, nx.qu + t * 128, nx.qh,
+                                                nx.qb);
                             else
                                 tma_prefetch_2d(&tmM, pn * 64, nx.m_z + t * 128);
                         }
@@ -422,9 +456,14 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                     }
                     if (lane == 0) {
                         mbar_expect_tx(z_full + st, kTile);
-                        for (int pn = 0; pn < 2; pn++)
-                            ls_load(sm + ls::kZ + st * kTile + pn * kPanel, &tmV, n_gather,
-                                    pn * 64, pr.n_y, pr.n_z + j * 128, z_full + st);
+                        for (int pn = 0; pn < 2; pn++) {
+                            if (n_gather)
+                                ls_load_q(sm + ls::kZ + st * kTile + pn * kPanel, &tmV, pn * 64,
+                                          pr, pr.qu + j * 128, p.layout == kLayoutBNHD, z_full + st);
+                            else
+                                ls_load(sm + ls::kZ + st * kTile + pn * kPanel, &tmV, false,
+                                        pn * 64, pr.n_y, pr.n_z + j * 128, z_full + st);
+                        }
                     }
                     issued_z[st]++;
                 }
@@ -582,11 +621,13 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                         if (m < pr.m_end) {
                             // kLsOut: Y row (u, v); kLsAgg: aggregated query of block
                             // u' = m for row g*b2 + v
-                            const int64_t orow =
+                            const int64_t off =
                                 MODE == kLsOut
-                                    ? (int64_t)pr.bh * p.N + (int64_t)m * p.b2 + pr.v
-                                    : ((int64_t)pr.bh * p.b1k + m) * a.mpad + pr.g * p.b2 + pr.v;
-                            *reinterpret_cast<uint4 *>(a.out + orow * kD + hf * 64 + c * 8) = val;
+                                    ? head_base(p, pr.bh, p.N) +
+                                          ((int64_t)m * p.b2 + pr.v) * tok_stride(p)
+                                    : (((int64_t)pr.bh * p.b1k + m) * a.mpad + pr.g * p.b2 + pr.v) *
+                                          kD;
+                            *reinterpret_cast<uint4 *>(a.out + off + hf * 64 + c * 8) = val;
                         }
                     }
                     __syncwarp();
@@ -865,10 +906,14 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 if (ib >= 2 && !wait_phase(kv_empty + st, ((ib >> 1) - 1) & 1, w)) break;
                 uint8_t *stage = sm + L::kv(nmt) + st * L::kStage;
                 mbar_expect_tx(kv_full + st, L::kStage);
-                const int row = bh * p.Nk + up * p.b2;
+                // the block's b2 tokens of head bh: (x, token, head, batch), or
+                // (x, head, token, batch) for [B][N][H][d] (increasing strides)
+                const bool bnhd = p.layout == kLayoutBNHD;
+                const int tok0 = up * p.b2, hh = bh % p.H, bb = bh / p.H;
+                const int c1 = bnhd ? hh : tok0, c2 = bnhd ? tok0 : hh;
                 for (int pn = 0; pn < 2; pn++) {
-                    tma_load_2d(stage + pn * L::kPanelKV, &tmK, pn * 64, row, kv_full + st);
-                    tma_load_2d(stage + L::kVOff + pn * L::kPanelKV, &tmV, pn * 64, row,
+                    tma_load_4d(stage + pn * L::kPanelKV, &tmK, pn * 64, c1, c2, bb, kv_full + st);
+                    tma_load_4d(stage + L::kVOff + pn * L::kPanelKV, &tmV, pn * 64, c1, c2, bb,
                                 kv_full + st);
                 }
                 issued[st]++;
@@ -1264,16 +1309,50 @@ bool map_gather(CUtensorMap *m, const void *base, const Problem &p, uint32_t wid
     return make_map(m, base, 3, dims, str, box, sw);
 }
 
+// Keys or values in the call's layout as a 4-D map (x, token, head, batch), box
+// (64, rows): a block's rows of one head; rows past Nk read zeros.
+bool map_keys(CUtensorMap *m, const void *base, const Problem &p, uint32_t rows) {
+    const uint64_t batch = (uint64_t)p.Nk * p.H * kD * 2;
+    if (p.layout == kLayoutBNHD) {   // (x, head, token, batch)
+        const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)p.H, (uint64_t)p.Nk, (uint64_t)p.B};
+        const uint64_t str[3] = {(uint64_t)kD * 2, (uint64_t)p.H * kD * 2, batch};
+        const uint32_t box[4] = {64, 1, rows, 1};
+        return make_map(m, base, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+    const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)p.Nk, (uint64_t)p.H, (uint64_t)p.B};
+    const uint64_t str[3] = {(uint64_t)kD * 2, (uint64_t)p.Nk * kD * 2, batch};
+    const uint32_t box[4] = {64, rows, 1, 1};
+    return make_map(m, base, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+// Queries in the call's layout as a 5-D map (x, v, u, head, batch), box (64, 1,
+// 128): 128 block rows u at one column v (the inverse shuffle); rows past b1
+// read zeros.
+bool map_queries(CUtensorMap *m, const void *base, const Problem &p) {
+    const uint64_t batch = (uint64_t)p.N * p.H * kD * 2;
+    if (p.layout == kLayoutBNHD) {   // (x, head, v, u, batch)
+        const uint64_t tok = (uint64_t)p.H * kD * 2;
+        const uint64_t dims[5] = {(uint64_t)kD, (uint64_t)p.H, (uint64_t)p.b2, (uint64_t)p.b1,
+                                  (uint64_t)p.B};
+        const uint64_t str[4] = {(uint64_t)kD * 2, tok, (uint64_t)p.b2 * tok, batch};
+        const uint32_t box[5] = {64, 1, 1, 128, 1};
+        return make_map(m, base, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+    const uint64_t dims[5] = {(uint64_t)kD, (uint64_t)p.b2, (uint64_t)p.b1, (uint64_t)p.H,
+                              (uint64_t)p.B};
+    const uint64_t str[4] = {(uint64_t)kD * 2, (uint64_t)p.b2 * kD * 2, (uint64_t)p.N * kD * 2,
+                             batch};
+    const uint32_t box[5] = {64, 1, 128, 1, 1};
+    return make_map(m, base, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 cudaError_t run_rstep(const Problem &p, const TcWorkspace &ws, const void *k, const void *v,
                       int qblk, float c_log2, int *status, long long wait_limit, int stall,
                       cudaStream_t stream) {
     const int nmt = qbar_tiles(p), mpad = nmt * 128, b2p = b2_padded(p.b2);
     CUtensorMap maps[6];
     const uint64_t dq[2] = {(uint64_t)kD, qblk ? (uint64_t)p.BH * p.b1k * mpad : (uint64_t)p.BH * mpad};
-    const uint64_t dkv[2] = {(uint64_t)kD, (uint64_t)p.BH * p.Nk};
     const uint64_t s2[1] = {kD * 2};
     const uint32_t bq[2] = {64, 128};
-    const uint32_t bkv[2] = {64, (uint32_t)b2p};
     const uint64_t dst[4] = {(uint64_t)kD, (uint64_t)p.b1k, (uint64_t)p.tiles * p.b2,
                              (uint64_t)p.BH};
     const uint64_t sst[3] = {kD * 2, (uint64_t)p.b1k * kD * 2,
@@ -1284,7 +1363,7 @@ cudaError_t run_rstep(const Problem &p, const TcWorkspace &ws, const void *k, co
     const uint64_t shx[3] = {32, (uint64_t)p.b1k * 32, (uint64_t)p.tiles * p.b2 * p.b1k * 32};
     const uint32_t bhx[4] = {16, 1, 32, 1};
     if (!make_map(&maps[0], qblk ? ws.qblk : ws.qbar, 2, dq, s2, bq) ||
-        !make_map(&maps[1], k, 2, dkv, s2, bkv) || !make_map(&maps[2], v, 2, dkv, s2, bkv) ||
+        !map_keys(&maps[1], k, p, (uint32_t)b2p) || !map_keys(&maps[2], v, p, (uint32_t)b2p) ||
         !make_map(&maps[3], ws.z, 4, dst, sst, bst) || !make_map(&maps[4], ws.ktil, 4, dst, sst, bst) ||
         !make_map(&maps[5], ws.hx, 4, dhx, shx, bhx, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
@@ -1315,7 +1394,7 @@ cudaError_t run_lstep(const Problem &p, const TcWorkspace &ws, const void *q, vo
     const int mpad = qbar_tiles(p) * 128;
     CUtensorMap qg, kt, zt, xp;
     const uint64_t rows = (uint64_t)p.BH * p.tiles * p.Nk;
-    if (!map_gather(&qg, q, p, kD, CU_TENSOR_MAP_SWIZZLE_128B) ||
+    if (!map_queries(&qg, q, p) ||
         !map_rows(&kt, ws.ktil, rows, kD, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map_rows(&zt, ws.z, rows, kD, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;

@@ -428,3 +428,35 @@ def test_chunk_against_kv_cache_whole_output(name, dtype, d, fq, fk, h, w, b2, t
     got = from_torch(out, dtype)
     assert np.isfinite(got).all()
     assert rel_fro(got, ref) <= TOL[dtype]
+
+
+# --------------------------------------------------------------------------
+# [B, N, H, d] inputs: the kernels read the strided rows directly; the result is
+# the [B, H, N, d] computation's, bit for bit (only the addresses differ)
+# --------------------------------------------------------------------------
+LAYOUT_CASES = [
+    # f, h, w, b1, b2, tiles, iters, d, dtype, kernel path
+    (2, 3, 100, 6, 100, 2, 1, 128, "bf16", 1),
+    (5, 60, 48, 300, 48, 5, 2, 128, "bf16", 1),    # iters > 1: queries on both MMA sides
+    (2, 100, 7, 200, 7, 3, 1, 128, "bf16", 1),
+    (3, 8, 8, 24, 8, 5, 2, 64, "f32", 0),
+    (3, 8, 8, 24, 8, 3, 1, 32, "bf16", 0),
+]
+
+
+@pytest.mark.parametrize("f,h,w,b1,b2,tiles,iters,d,dtype,path", LAYOUT_CASES)
+def test_bnhd_layout_matches_bhnd_bit_for_bit(f, h, w, b1, b2, tiles, iters, d, dtype, path):
+    from structured_attention_video_b200.attention import monarch_attention_bnhd
+    wl = TINY.replace(B=2, H=3, d=d, f=f, h=h, w=w, b1=b1, b2=b2, tiles=tiles, iters=iters)
+    q64, k64, v64 = (synth.round_to_dtype(x, dtype) for x in synth.make_inputs(wl))
+    q, k, v = (to_torch(x, dtype) for x in (q64, k64, v64))
+    assert kernel_path(q, f=f, h=h, w=w, b1=b1, b2=b2, tiles=tiles, iters=iters) == path
+    ref = run(wl, q, k, v)
+    qt, kt, vt = (x.transpose(1, 2).contiguous() for x in (q, k, v))
+    out = monarch_attention_bnhd(qt, kt, vt, f=f, h=h, w=w, b1=b1, b2=b2, tiles=tiles,
+                                 iters=iters)
+    torch.cuda.synchronize()
+    assert _lib.monarch_last_device_status(None) == 0
+    assert torch.equal(out.transpose(1, 2), ref)
+    want = oracle.monarch_attn(q64, k64, v64, b1, b2, tiles, iters)
+    assert rel_fro(from_torch(ref, dtype), want) <= TOL[dtype]
