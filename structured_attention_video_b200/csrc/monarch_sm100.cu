@@ -66,7 +66,7 @@ __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, const 
 // with B*H*t*ceil(b2*d/1024) blocks).  The four partial sums meet in shared
 // memory in a fixed order.
 constexpr int kQbarGroups = 4;
-__global__ void __launch_bounds__(128 * kQbarGroups) tc_qbar_kernel(
+__global__ void __launch_bounds__(128 * kQbarGroups, 2) tc_qbar_kernel(
     const __nv_bfloat16 *__restrict__ q, __nv_bfloat16 *__restrict__ qbar, Problem p, int mpad) {
     __shared__ float part[kQbarGroups - 1][8][128];
     const int row_elems = p.b2 * kD;
@@ -224,9 +224,6 @@ struct LsProblem {
     int m_y, m_z, m_first, m_end;   // M side: tile t starts at z = m_z + t*128
     int n_y, n_z, nkeys, nch;       // N side: chunk j starts at z = n_z + j*128
     int nh;                         // 64-key halves of the N side (the softmax's unit)
-    // the side that reads the query rows (M, or N in kLsAgg) through the 5-D query
-    // map (x, v, u, head, batch): column qv, first row qu, head qh, batch qb
-    int qv, qu, qh, qb;
 };
 
 template <int MODE>
@@ -261,22 +258,20 @@ __device__ __forceinline__ LsProblem ls_problem(const LsArgs &a, int unit) {
     }
     q.nch = (q.nkeys + 127) / 128;
     q.nh = (q.nkeys + 63) / 64;
-    q.qv = q.v;
-    q.qu = MODE != kLsAgg ? q.m_first : u_lo;
-    q.qh = q.bh % p.H;
-    q.qb = q.bh / p.H;
     return q;
 }
 
-// One 128-row tile of query rows (u, v), u = u0 .. u0 + 127 at column v, through the
-// 5-D query map: (x, v, u, head, batch), or (x, head, v, u, batch) for [B][N][H][d]
-// (the map's dimensions run in order of increasing stride); rows past b1 read zeros.
-__device__ __forceinline__ void ls_load_q(void *dst, const CUtensorMap *map, int x,
-                                          const LsProblem &pr, int u0, bool bnhd, uint64_t *bar) {
-    if (bnhd)
-        tma_load_5d(dst, map, x, pr.qh, pr.qv, u0, pr.qb, bar);
+// One 128-row tile of query rows (u, v), u = u0 .. u0 + 127 at column v of head bh,
+// through the 5-D query map: (x, v, u, head, batch), or (x, head, v, u, batch) for
+// [B][N][H][d] (the map's dimensions run in order of increasing stride); rows past
+// b1 read zeros.
+__device__ __forceinline__ void ls_load_q(void *dst, const CUtensorMap *map, int x, int v, int u0,
+                                          int bh, const Problem &p, uint64_t *bar) {
+    const int hh = bh % p.H, bb = bh / p.H;
+    if (p.layout == kLayoutBNHD)
+        tma_load_5d(dst, map, x, hh, v, u0, bb, bar);
     else
-        tma_load_5d(dst, map, x, pr.qv, u0, pr.qh, pr.qb, bar);
+        tma_load_5d(dst, map, x, v, u0, hh, bb, bar);
 }
 
 // One TMA tile load of the L-step: a 3-D gather (x, y, z) or a 2-D row box (x, z).
@@ -388,7 +383,8 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                         for (int pn = 0; pn < 2; pn++) {
                             if (n_gather)
                                 ls_load_q(sm + ls::kK + sk * kTile + pn * kPanel, &tmN, pn * 64,
-                                          pr, pr.qu + j * 128, p.layout == kLayoutBNHD, k_full + sk);
+                                          pr.v, pr.n_z - pr.bh * p.b1 + j * 128, pr.bh, p,
+                                          k_full + sk);
                             else
                                 ls_load(sm + ls::kK + sk * kTile + pn * kPanel, &tmN, false,
                                         pn * 64, pr.n_y, pr.n_z + j * 128, k_full + sk);
@@ -425,7 +421,7 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                         for (int pn = 0; pn < 2; pn++) {
                             if (!n_gather)
                                 ls_load_q(sm + ls::kQ + t * kTile + pn * kPanel, &tmM, pn * 64,
-                                          pr, pr.qu + t * 128, p.layout == kLayoutBNHD, q_full + t);
+                                          pr.v, pr.m_first + t * 128, pr.bh, p, q_full + t);
                             else
                                 ls_load(sm + ls::kQ + t * kTile + pn * kPanel, &tmM, false,
                                         pn * 64, pr.m_y, pr.m_z + t * 128, q_full + t);
@@ -439,11 +435,11 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                     for (int t = 0; t < 2; t++)
                         for (int pn = 0; pn < 2; pn++) {
                             if (!n_gather && p.layout == kLayoutBNHD)
-                                tma_prefetch_5d(&tmM, pn * 64, nx.qh, nx.qv, nx.qu + t * 128,
-                                                nx.qb);
+                                tma_prefetch_5d(&tmM, pn * 64, nx.bh % p.H, nx.v,
+                                                nx.m_first + t * 128, nx.bh / p.H);
                             else if (!n_gather)
-                                tma_prefetch_5d(&tmM, pn * 64, nx.qv, nx.qu + t * 128, nx.qh,
-                                                nx.qb);
+                                tma_prefetch_5d(&tmM, pn * 64, nx.v, nx.m_first + t * 128,
+                                                nx.bh % p.H, nx.bh / p.H);
                             else
                                 tma_prefetch_2d(&tmM, pn * 64, nx.m_z + t * 128);
                         }
@@ -459,7 +455,8 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                         for (int pn = 0; pn < 2; pn++) {
                             if (n_gather)
                                 ls_load_q(sm + ls::kZ + st * kTile + pn * kPanel, &tmV, pn * 64,
-                                          pr, pr.qu + j * 128, p.layout == kLayoutBNHD, z_full + st);
+                                          pr.v, pr.n_z - pr.bh * p.b1 + j * 128, pr.bh, p,
+                                          z_full + st);
                             else
                                 ls_load(sm + ls::kZ + st * kTile + pn * kPanel, &tmV, false,
                                         pn * 64, pr.n_y, pr.n_z + j * 128, z_full + st);
@@ -604,6 +601,13 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                 // each), instead of 32 scattered 16-byte pieces
                 uint8_t *stg = sm + ls::kStg + wq * 4096;
                 const int m0w = pr.m_first + t * 128 + wq * 32;
+                // kLsOut: Y row (u, v) = token m*b2 + v of head bh in the call's layout,
+                // at obase + (m - m0w) * ostride
+                const int64_t ostride = MODE == kLsOut ? (int64_t)p.b2 * tok_stride(p) : 0;
+                __nv_bfloat16 *const obase =
+                    MODE == kLsOut ? a.out + head_base(p, pr.bh, p.N) +
+                                         ((int64_t)m0w * p.b2 + pr.v) * tok_stride(p)
+                                   : a.out;
 #pragma unroll
                 for (int hf = 0; hf < 2; hf++) {
 #pragma unroll
@@ -619,15 +623,13 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                             *reinterpret_cast<const uint4 *>(stg + row * 128 + ((c + row) & 7) * 16);
                         const int m = m0w + row;
                         if (m < pr.m_end) {
-                            // kLsOut: Y row (u, v); kLsAgg: aggregated query of block
-                            // u' = m for row g*b2 + v
-                            const int64_t off =
+                            // kLsAgg: the aggregated query of block u' = m for row g*b2 + v
+                            __nv_bfloat16 *dst =
                                 MODE == kLsOut
-                                    ? head_base(p, pr.bh, p.N) +
-                                          ((int64_t)m * p.b2 + pr.v) * tok_stride(p)
-                                    : (((int64_t)pr.bh * p.b1k + m) * a.mpad + pr.g * p.b2 + pr.v) *
-                                          kD;
-                            *reinterpret_cast<uint4 *>(a.out + off + hf * 64 + c * 8) = val;
+                                    ? obase + row * ostride
+                                    : a.out + (((int64_t)pr.bh * p.b1k + m) * a.mpad +
+                                               pr.g * p.b2 + pr.v) * kD;
+                            *reinterpret_cast<uint4 *>(dst + hf * 64 + c * 8) = val;
                         }
                     }
                     __syncwarp();
