@@ -364,6 +364,222 @@ int oracle_monarch_attn_kv(const double *q, const double *k, const double *v, do
     return err;
 }
 
+/*
+ * The other reading of the tiles ("创新二：平铺Monarch参数化": each block is split
+ * into tiles that are factorised independently): the tiles split the KEY
+ * columns v' of every block instead of the query rows u.
+ *   Key tile g' holds the columns T'_g' = [floor(g'*b2/t), floor((g'+1)*b2/t)),
+ *   t in [1, b2].  A super-key is a (block u', key tile g') pair; there are
+ *   b1k*t of them.
+ *   M[(u,v),(u',v')] = L_v[u, (u',g'(v'))] * R_{u',g'(v')}[v,v'], where L_v[u,:]
+ *   is a distribution over the super-keys and R_{u',g'}[v,:] one over the
+ *   columns of tile g'.
+ * The same variational objective gives the same two half-steps:
+ *   init      L_v[u,:] = 1/(b1k*t)
+ *   R-step    per (u', g', v): qbar = sum_u L_v[u,(u',g')] q_(u,v) / sum_u L,
+ *             over ALL query rows u in [b1];  R = softmax over v' in T'_g' of
+ *             s*qbar.k_(u',v');  H = its entropy;  Ktil, Z = sum_v' R k, R v
+ *   L-step    per (u, v): L_v[u,:] = softmax over (u',g') of
+ *             s*q_(u,v).Ktil[v,(u',g')] + H[v,(u',g')]
+ *   output    y_(u,v) = sum_(u',g') L_v[u,(u',g')] Z[v,(u',g')]
+ * t = 1 is plain Monarch (the same map as one query tile); t = b2 makes every
+ * tile a single key column, R = 1, H = 0, and the L-step a softmax over all
+ * N keys: exact attention.  Every step for column v reads all query rows
+ * (u, v), all keys and all values and writes only the rows (u, v), so the
+ * oracle loops over independent (head, v) problems.
+ * Super-key j = g'*b1k + u'.  L_out (optional) [b2][b1][t*b1k];
+ * R_out (optional) [b1k][t][b2][b2] with zeros outside the tile's columns.
+ */
+static int key_tile_first_col(int g, int b2, int tiles)
+{
+    return (int)(((int64_t)g * b2) / tiles);
+}
+
+static size_t keytiles_workspace_doubles(int d, int b1, int b1k, int b2, int tiles)
+{
+    size_t nsk = (size_t)tiles * b1k;
+    size_t mx = nsk > (size_t)b2 ? nsk : (size_t)b2;
+    return (size_t)b1 * nsk + nsk * b2 + 2 * nsk * d + nsk + d + mx;
+}
+
+static void solve_problem_keytiles(const double *q, const double *k, const double *v,
+                                   double *y, int d, int b1, int b1k, int b2, int tiles,
+                                   int c, int half_steps, double *L_out, double *R_out,
+                                   double *ws)
+{
+    const double s = 1.0 / sqrt((double)d);
+    const int nsk = tiles * b1k;
+    double *L = ws;                          /* [b1][nsk]   L_c[u][j]            */
+    double *R = L + (size_t)b1 * nsk;        /* [nsk][b2]   R_{u',g'}[c][:]      */
+    double *Kt = R + (size_t)nsk * b2;       /* [nsk][d]    Ktil[c][j]           */
+    double *Z = Kt + (size_t)nsk * d;        /* [nsk][d]    Z[c][j]              */
+    double *H = Z + (size_t)nsk * d;         /* [nsk]       entropy of R row     */
+    double *qbar = H + nsk;                  /* [d]                              */
+    double *logit = qbar + d;                /* [max(nsk, b2)]                   */
+
+    for (size_t i = 0; i < (size_t)b1 * nsk; i++)
+        L[i] = 1.0 / nsk;
+
+    for (int step = 0; step < half_steps; step++) {
+        if ((step & 1) == 0) {
+            /* R-step: every super-key j = (u', g'), row c of R_{u',g'} */
+            for (int g = 0; g < tiles; g++) {
+                const int c0 = key_tile_first_col(g, b2, tiles);
+                const int c1 = key_tile_first_col(g + 1, b2, tiles);
+                for (int up = 0; up < b1k; up++) {
+                    const int j = g * b1k + up;
+                    double wsum = 0.0;
+                    for (int jj = 0; jj < d; jj++)
+                        qbar[jj] = 0.0;
+                    for (int u = 0; u < b1; u++) {
+                        double wgt = L[(size_t)u * nsk + j];
+                        const double *qr = q + ((int64_t)u * b2 + c) * d;
+                        wsum += wgt;
+                        for (int jj = 0; jj < d; jj++)
+                            qbar[jj] += wgt * qr[jj];
+                    }
+                    for (int jj = 0; jj < d; jj++)
+                        qbar[jj] = wsum > 0.0 ? qbar[jj] / wsum : 0.0;
+
+                    double mx = -INFINITY;
+                    for (int vp = c0; vp < c1; vp++) {
+                        const double *kr = k + ((int64_t)up * b2 + vp) * d;
+                        double acc = 0.0;
+                        for (int jj = 0; jj < d; jj++)
+                            acc += qbar[jj] * kr[jj];
+                        logit[vp] = s * acc;
+                        if (logit[vp] > mx)
+                            mx = logit[vp];
+                    }
+                    double sum = 0.0;
+                    for (int vp = c0; vp < c1; vp++)
+                        sum += exp(logit[vp] - mx);
+                    double lse = mx + log(sum);
+                    double ent = lse;
+                    for (int vp = 0; vp < b2; vp++)
+                        R[(size_t)j * b2 + vp] = 0.0;
+                    for (int vp = c0; vp < c1; vp++) {
+                        double r = exp(logit[vp] - lse);
+                        R[(size_t)j * b2 + vp] = r;
+                        ent -= r * logit[vp];
+                    }
+                    H[j] = ent;
+                    for (int jj = 0; jj < d; jj++) {
+                        double kt = 0.0, z = 0.0;
+                        for (int vp = c0; vp < c1; vp++) {
+                            double r = R[(size_t)j * b2 + vp];
+                            kt += r * k[((int64_t)up * b2 + vp) * d + jj];
+                            z += r * v[((int64_t)up * b2 + vp) * d + jj];
+                        }
+                        Kt[(size_t)j * d + jj] = kt;
+                        Z[(size_t)j * d + jj] = z;
+                    }
+                }
+            }
+        } else {
+            /* L-step: every query row u at column c, over all super-keys */
+            for (int u = 0; u < b1; u++) {
+                const double *qr = q + ((int64_t)u * b2 + c) * d;
+                double mx = -INFINITY;
+                for (int j = 0; j < nsk; j++) {
+                    double acc = 0.0;
+                    for (int jj = 0; jj < d; jj++)
+                        acc += qr[jj] * Kt[(size_t)j * d + jj];
+                    logit[j] = s * acc + H[j];
+                    if (logit[j] > mx)
+                        mx = logit[j];
+                }
+                double sum = 0.0;
+                for (int j = 0; j < nsk; j++)
+                    sum += exp(logit[j] - mx);
+                double lse = mx + log(sum);
+                for (int j = 0; j < nsk; j++)
+                    L[(size_t)u * nsk + j] = exp(logit[j] - lse);
+            }
+        }
+    }
+
+    /* output: y_(u,c) = sum_j L_c[u,j] Z[j] */
+    for (int u = 0; u < b1; u++) {
+        double *yr = y + ((int64_t)u * b2 + c) * d;
+        for (int jj = 0; jj < d; jj++) {
+            double acc = 0.0;
+            for (int j = 0; j < nsk; j++)
+                acc += L[(size_t)u * nsk + j] * Z[(size_t)j * d + jj];
+            yr[jj] = acc;
+        }
+    }
+
+    if (L_out)
+        for (int u = 0; u < b1; u++)
+            for (int j = 0; j < nsk; j++)
+                L_out[((int64_t)c * b1 + u) * nsk + j] = L[(size_t)u * nsk + j];
+    if (R_out)
+        for (int g = 0; g < tiles; g++)
+            for (int up = 0; up < b1k; up++)
+                for (int vp = 0; vp < b2; vp++)
+                    R_out[(((int64_t)up * tiles + g) * b2 + c) * b2 + vp] =
+                        R[(size_t)(g * b1k + up) * b2 + vp];
+}
+
+/*
+ * Key-column tiles over BH heads of self-attention: q, k, v, y [BH][N][d],
+ * t in [1, b2].  With nprob >= 0 only the listed (bh, c) problems
+ * (probs[2*i], probs[2*i+1]) run, writing the rows (u, c) of head bh of y and
+ * leaving the others untouched; with nprob < 0 every problem runs and the
+ * optional L_out [BH][b2][b1][t*b1] and R_out [BH][b1][t][b2][b2] are filled.
+ */
+int oracle_monarch_attn_keytiles(const double *q, const double *k, const double *v,
+                                 double *y, int BH, int N, int d, int b1, int b2, int tiles,
+                                 int half_steps, double *L_out, double *R_out, int nprob,
+                                 const int32_t *probs, int nthreads)
+{
+    if (BH < 1 || N < 1 || d < 1 || b1 < 1 || b2 < 1 || (int64_t)b1 * b2 != N ||
+        tiles < 1 || tiles > b2 || half_steps < 1)
+        return ORACLE_EINVAL;
+    for (int i = 0; i < nprob; i++)
+        if (probs[2 * i] < 0 || probs[2 * i] >= BH || probs[2 * i + 1] < 0 ||
+            probs[2 * i + 1] >= b2)
+            return ORACLE_EINVAL;
+    const int64_t ntask = nprob >= 0 ? nprob : (int64_t)BH * b2;
+    const size_t wsz = keytiles_workspace_doubles(d, b1, b1, b2, tiles);
+    const size_t nsk = (size_t)tiles * b1;
+    int err = ORACLE_OK;
+#ifdef _OPENMP
+    if (nthreads <= 0)
+        nthreads = omp_get_max_threads();
+#pragma omp parallel num_threads(nthreads)
+#endif
+    {
+        double *ws = (double *)malloc(wsz * sizeof(double));
+        if (!ws) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            err = ORACLE_ENOMEM;
+        }
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+        for (int64_t p = 0; p < ntask; p++) {
+            if (!ws)
+                continue;
+            int bh = nprob >= 0 ? probs[2 * p] : (int)(p / b2);
+            int c = nprob >= 0 ? probs[2 * p + 1] : (int)(p % b2);
+            size_t off = (size_t)bh * N * d;
+            int full = nprob < 0;
+            solve_problem_keytiles(q + off, k + off, v + off, y + off, d, b1, b1, b2, tiles, c,
+                                   half_steps,
+                                   (full && L_out) ? L_out + (size_t)bh * b2 * b1 * nsk : NULL,
+                                   (full && R_out) ? R_out + (size_t)bh * b1 * tiles * b2 * b2
+                                                   : NULL,
+                                   ws);
+        }
+        free(ws);
+    }
+    return err;
+}
+
 /* Number of threads the OpenMP runtime would use (1 without OpenMP). */
 /*
  * Backward pass of one iteration (iters = 1) by the chain rule, step by step.

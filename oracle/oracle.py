@@ -46,6 +46,9 @@ def _load(path: str | None = None):
         lib.oracle_monarch_problems.restype = i
         lib.oracle_monarch_attn_kv.argtypes = [dp, dp, dp, dp, i, i, i, i, i, i, i, dp, dp, i]
         lib.oracle_monarch_attn_kv.restype = i
+        lib.oracle_monarch_attn_keytiles.argtypes = [dp, dp, dp, dp, i, i, i, i, i, i, i, dp,
+                                                     dp, i, ip, i]
+        lib.oracle_monarch_attn_keytiles.restype = i
         lib.oracle_monarch_attn_bwd.argtypes = [dp] * 7 + [i] * 7
         lib.oracle_monarch_attn_bwd.restype = i
         lib.oracle_max_threads.argtypes = []
@@ -130,6 +133,44 @@ def monarch_attn_kv(q, k, v, b1, b1k, b2, tiles=1, iters=1, half_steps=None, fac
     if factors:
         return y, L.reshape(shape[:-2] + L.shape[1:]), R.reshape(shape[:-2] + R.shape[1:])
     return y
+
+
+def monarch_attn_keytiles(q, k, v, b1, b2, tiles=1, iters=1, half_steps=None, factors=False,
+                          probs=None, nthreads=0, lib=None, y=None):
+    """The tiles split the key columns v' of every block (the other reading of the
+    tiled parameterisation); float64 arrays [..., N, d], tiles in [1, b2].  Returns y
+    (and L [..., b2, b1, tiles*b1] with super-key j = g'*b1 + u', R [..., b1, tiles,
+    b2, b2] if factors).  With probs, a list of (bh, c) pairs, only the rows (u, c) of
+    those problems are written (the rest of y is NaN, or taken from `y`)."""
+    qh, shape = _heads(q)
+    kh, _ = _heads(k)
+    vh, _ = _heads(v)
+    BH, N, d = qh.shape
+    hs = 2 * iters if half_steps is None else half_steps
+    if probs is None:
+        pr, npr = None, -1
+        out = np.zeros_like(qh)
+    else:
+        pr = np.ascontiguousarray(np.asarray(probs, dtype=np.int32).reshape(-1, 2))
+        npr = pr.shape[0]
+        out = np.full_like(qh, np.nan) if y is None else y.reshape(qh.shape)
+    full = factors and probs is None
+    L = np.zeros((BH, b2, b1, tiles * b1)) if full else None
+    R = np.zeros((BH, b1, tiles, b2, b2)) if full else None
+    rc = _load(lib).oracle_monarch_attn_keytiles(
+        _dptr(qh), _dptr(kh), _dptr(vh), _dptr(out), BH, N, d, b1, b2, tiles, hs, _dptr(L),
+        _dptr(R), npr, _iptr(pr) if pr is not None else None, nthreads)
+    if rc != 0:
+        raise ValueError("oracle_monarch_attn_keytiles failed with code %d" % rc)
+    out = out.reshape(shape)
+    if full:
+        return out, L.reshape(shape[:-2] + L.shape[1:]), R.reshape(shape[:-2] + R.shape[1:])
+    return out
+
+
+def key_tile_cols(b2, tiles, g):
+    """Key columns of key tile g: [floor(g*b2/t), floor((g+1)*b2/t))."""
+    return np.arange((g * b2) // tiles, ((g + 1) * b2) // tiles)
 
 
 def monarch_attn_bwd(q, k, v, dy, b1, b2, tiles=1, nthreads=0, lib=None):
