@@ -522,6 +522,118 @@ def run_backward(args, wl: synth.Workload) -> None:
         "gpu": torch.cuda.get_device_name(0)}), flush=True)
 
 
+def keytile_cpu_baseline(wl: synth.Workload, got_bits: np.ndarray, samples: int) -> dict:
+    """The float64 oracle of key-column tiles on `samples` seeded (head, column)
+    problems, all query rows of each, on the host's cores: its time scaled to a
+    whole step (B*H*b2 problems), and the rel-Frobenius error of the device output
+    (`got_bits`, bfloat16 storage [B][H][N][d]) on those rows."""
+    from oracle import oracle
+    rng = np.random.default_rng(5)
+    probs = sorted({(int(rng.integers(wl.B * wl.H)), int(rng.integers(wl.b2)))
+                    for _ in range(samples)})
+    pos = synth.positional_code(wl.f, wl.h, wl.w, wl.d)
+    num = den = 0.0
+    secs = 0.0
+    for bh in sorted({pr[0] for pr in probs}):
+        b, h = divmod(bh, wl.H)
+        x = synth.make_head(wl, b, h, 0, pos)
+        cols = [c for (hh, c) in probs if hh == bh]
+        t0 = time.perf_counter()
+        y = oracle.monarch_attn_keytiles(x["q"][None], x["k"][None], x["v"][None], wl.b1, wl.b2,
+                                         wl.tiles, wl.iters, probs=[(0, c) for c in cols])[0]
+        secs += time.perf_counter() - t0
+        for c in cols:
+            rows = np.arange(wl.b1) * wl.b2 + c
+            o = synth.from_device_bits(got_bits[b, h, rows], "bf16")
+            num += float(((o - y[rows]) ** 2).sum())
+            den += float((y[rows] ** 2).sum())
+    total = wl.B * wl.H * wl.b2
+    return {"value": secs * 1e3 * total / len(probs), "unit": "ms", "cores": oracle.max_threads(),
+            "kind": "oracle", "seconds": secs,
+            "sample": "%d (head, column) problems of the workload (%.2f%% of one step's output "
+                      "rows), float64 C oracle with OpenMP, scaled to a whole step"
+                      % (len(probs), 100.0 * len(probs) / total),
+            "rel_err": {"value": float(np.sqrt(num / den)), "rows": len(probs) * wl.b1,
+                        "vs": "float64 oracle, same seeded inputs", "tolerance": 0.01}}
+
+
+def run_keytiles(args, wl: synth.Workload) -> None:
+    """One JSON line: device ms of the forward pass with key-column tiles (the
+    key columns of every block split into wl.tiles tiles; each query row's L over
+    the b1*t super-keys) on resident bfloat16 inputs, its algorithmic FLOPs against
+    the path roofline, the per-kernel split, and the rel-Frobenius error of sampled
+    (head, column) problems against the float64 oracle."""
+    import torch
+    from structured_attention_video_b200 import _lib
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    peaks, peak_kind = load_peaks()
+    shape = (wl.B, wl.H, wl.N, wl.d)
+    hq, hk, hv = (torch.empty(shape, dtype=torch.int16) for _ in range(3))
+    synth.fill_device_bits(wl, hq.numpy().view(np.uint16), hk.numpy().view(np.uint16),
+                           hv.numpy().view(np.uint16), 0)
+    q, k, v = (x.to(dev).view(torch.bfloat16) for x in (hq, hk, hv))
+    out = torch.empty_like(q)
+    sargs = (wl.B, wl.H, wl.f, wl.h, wl.w, wl.d, wl.b1, wl.b2, wl.tiles, wl.iters)
+    axis = _lib.TILE_KEY_COLUMNS
+    nb = _lib.monarch_attn_tiled_workspace_bytes(*sargs, _lib.BF16, axis)
+    path = _lib.monarch_attn_tiled_path(*sargs, _lib.BF16, axis)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+
+    def step():
+        _lib.check(_lib.monarch_attn_fwd_tiled_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                  out.data_ptr(), *sargs, _lib.BF16, axis,
+                                                  _lib.BHND, ws.data_ptr(), nb, sh),
+                   "monarch_attn_fwd_tiled_ws")
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    _lib.monarch_profile_enable(1)
+    _lib.monarch_profile_collect()
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    _lib.monarch_profile_enable(0)
+    prof = _lib.monarch_profile_collect()
+    _lib.check(_lib.monarch_last_device_status(sh), "device status (key tiles)")
+    kernels = {name: ms_tot / max(1, args.steps) for name, (ms_tot, cnt) in prof.items() if cnt > 0}
+    ms = float(np.median(times))
+    flops = wl.monarch_flops_keytiles()
+    io = wl.io_bytes()
+    roof_ms = max(flops / (peaks["bf16_tflops"] * 1e12), io / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    # the CPU-baseline leg: the oracle on sampled (head, column) problems (every
+    # query row of each), timed and scaled to a whole step; the same rows give the
+    # rel-Frobenius error of the device output
+    base = None
+    if not args.no_cpu_baseline and args.keytile_samples > 0:
+        got = out.view(torch.int16).cpu().numpy().view(np.uint16)
+        base = keytile_cpu_baseline(wl, got, args.keytile_samples)
+    cfg = workload_config(wl, 1)
+    cfg["tile_axis"] = "key columns"
+    print(json.dumps({
+        "metric": "Monarch-attn forward ms, key-column tiles", "value": ms, "unit": "ms",
+        "higher_is_better": False, "steps": args.steps, "warmup": args.warmup,
+        "ms_stats": step_stats(times), "dtype": "bf16", "data": "synthetic", "config": cfg,
+        "monarch_gflop": flops / 1e9, "monarch_tflops": flops / (ms * 1e-3) / 1e12,
+        "path_roofline": {"roofline_ms": roof_ms, "frac": roof_ms / ms,
+                          "peak_source": "%s bf16_tflops (burst) and hbm_gbs" % peak_kind},
+        "kernels_ms_per_step": kernels,
+        "kernel_path": "sm100 tensor-core" if path == 1 else "generic SIMT",
+        "rel_err": None if base is None else base.pop("rel_err"), "cpu_baseline": base,
+        "workspace_bytes": nb,
+        "gpu": torch.cuda.get_device_name(0)}), flush=True)
+
+
 SWEEPS = (("480p_full", "tiles", (1, 2, 4, 8), None),
           ("14b", "iters", (1, 2, 5, 10), (0, 13, 27, 40, 53, 79)))
 
@@ -763,6 +875,11 @@ def main():
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass of one iteration on --workload instead of "
                          "the forward bench line; one GPU")
+    ap.add_argument("--key-tiles", action="store_true",
+                    help="time the forward pass with key-column tiles (the other reading of "
+                         "the tiles) on --workload instead of the bench line; one GPU")
+    ap.add_argument("--keytile-samples", type=int, default=8,
+                    help="(head, column) problems checked against the oracle by --key-tiles")
     ap.add_argument("--sweep-steps", type=int, default=20)
     ap.add_argument("--sweep-rows", type=int, default=1024)
     args = ap.parse_args()
@@ -797,6 +914,11 @@ def main():
         if world != 1:
             ap.error("--backward runs on one GPU")
         run_backward(args, wl)
+        return
+    if args.key_tiles:
+        if world != 1:
+            ap.error("--key-tiles runs on one GPU")
+        run_keytiles(args, wl)
         return
 
     import torch

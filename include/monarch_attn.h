@@ -203,6 +203,46 @@ MONARCH_API monarch_status monarch_attn_fwd_layout_ws(const void *q, const void 
                                                       size_t ws_bytes, monarch_stream_t stream);
 
 /*
+ * Forward pass with the tiles on either axis.  The tiled parameterisation splits
+ * every block into t tiles that are factorised independently; which axis is
+ * split is a reading:
+ *   MONARCH_TILE_QUERY_ROWS   (every other entry point) the query rows u of each
+ *       block: tile g = rows [floor(g*b1/t), floor((g+1)*b1/t)) owns its own
+ *       R_{u',g}; 1 <= tiles <= b1; tiles = b1 is exact attention.
+ *   MONARCH_TILE_KEY_COLUMNS  the key columns v' of each block: key tile g' =
+ *       columns [floor(g'*b2/t), floor((g'+1)*b2/t)); R_{u',g'}[v,:] is a softmax
+ *       over the tile's columns of s*qbar.k with qbar aggregated over all b1
+ *       query rows of column v, and each query row's L is a softmax over the
+ *       b1*t (block u', key tile g') super-keys of s*q.Ktil + H;
+ *       1 <= tiles <= b2; tiles = b2 is exact attention.
+ * tiles = 1 is plain Monarch on both axes.  `layout` as monarch_attn_fwd_layout_ws;
+ * the workspace is monarch_attn_tiled_workspace_bytes (0 if the arguments fail
+ * validation; MONARCH_ERR_NO_MEMORY if ws_bytes is smaller), 256-byte aligned;
+ * monarch_attn_tiled_path reports the kernel family as monarch_attn_path does
+ * (key-column tiles take the tensor-core kernels for one iteration, the generic
+ * kernels for more).  Other arguments, errors and
+ * ownership as monarch_attn_fwd_ws; MONARCH_ERR_INVALID_ARG for another axis value.
+ * Source: explainer page, "创新二：平铺Monarch参数化" (each block split into tiles
+ * factorised independently; the axis is not stated there).
+ */
+typedef enum { MONARCH_TILE_QUERY_ROWS = 0, MONARCH_TILE_KEY_COLUMNS = 1 } monarch_tile_axis;
+
+MONARCH_API size_t monarch_attn_tiled_workspace_bytes(int B, int H, int f, int h, int w, int d,
+                                                      int b1, int b2, int tiles, int iters,
+                                                      monarch_dtype dtype,
+                                                      monarch_tile_axis axis);
+MONARCH_API int monarch_attn_tiled_path(int B, int H, int f, int h, int w, int d, int b1, int b2,
+                                        int tiles, int iters, monarch_dtype dtype,
+                                        monarch_tile_axis axis);
+MONARCH_API monarch_status monarch_attn_fwd_tiled_ws(const void *q, const void *k, const void *v,
+                                                     void *out, int B, int H, int f, int h,
+                                                     int w, int d, int b1, int b2, int tiles,
+                                                     int iters, monarch_dtype dtype,
+                                                     monarch_tile_axis axis,
+                                                     monarch_layout layout, void *workspace,
+                                                     size_t ws_bytes, monarch_stream_t stream);
+
+/*
  * Queries of a chunk of frames against keys and values that also hold earlier
  * frames (a key/value cache), as in chunk-by-chunk autoregressive video
  * generation (the Self-Forcing setting of the MonarchRT pages: summary page,

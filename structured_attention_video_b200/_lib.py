@@ -40,6 +40,10 @@ SIGNATURES = {
     "monarch_attn_fwd_units_ws": ([_vp, _vp, _vp, _vp] + _SHAPE + [_i, _i, _i, _vp, _sz, _vp], _i),
     "monarch_attn_fwd_noalloc": ([_vp, _vp, _vp, _vp] + _SHAPE + [_i, _vp], _i),
     "monarch_attn_fwd_layout_ws": ([_vp, _vp, _vp, _vp] + _SHAPE + [_i, _i, _vp, _sz, _vp], _i),
+    "monarch_attn_tiled_workspace_bytes": (_SHAPE + [_i, _i], _sz),
+    "monarch_attn_tiled_path": (_SHAPE + [_i, _i], _i),
+    "monarch_attn_fwd_tiled_ws": ([_vp, _vp, _vp, _vp] + _SHAPE + [_i, _i, _i, _vp, _sz, _vp],
+                                  _i),
     "monarch_attn_bwd_workspace_bytes": (_SHAPE + [_i], _sz),
     "monarch_attn_bwd_ws": ([_vp] * 7 + _SHAPE + [_i, _vp, _sz, _vp], _i),
     "monarch_attn_bwd": ([_vp] * 7 + _SHAPE + [_i, _vp], _i),
@@ -129,6 +133,24 @@ def monarch_attn_fwd_layout_ws(q, k, v, out, B, H, f, h, w, d, b1, b2, tiles, it
                                layout, workspace, ws_bytes, stream):
     return _lib.monarch_attn_fwd_layout_ws(q, k, v, out, B, H, f, h, w, d, b1, b2, tiles, iters,
                                            dtype, layout, workspace, ws_bytes, stream)
+
+
+TILE_QUERY_ROWS, TILE_KEY_COLUMNS = 0, 1   # monarch_tile_axis
+
+
+def monarch_attn_tiled_workspace_bytes(B, H, f, h, w, d, b1, b2, tiles, iters, dtype, axis):
+    return _lib.monarch_attn_tiled_workspace_bytes(B, H, f, h, w, d, b1, b2, tiles, iters, dtype,
+                                                   axis)
+
+
+def monarch_attn_tiled_path(B, H, f, h, w, d, b1, b2, tiles, iters, dtype, axis):
+    return _lib.monarch_attn_tiled_path(B, H, f, h, w, d, b1, b2, tiles, iters, dtype, axis)
+
+
+def monarch_attn_fwd_tiled_ws(q, k, v, out, B, H, f, h, w, d, b1, b2, tiles, iters, dtype, axis,
+                              layout, workspace, ws_bytes, stream):
+    return _lib.monarch_attn_fwd_tiled_ws(q, k, v, out, B, H, f, h, w, d, b1, b2, tiles, iters,
+                                          dtype, axis, layout, workspace, ws_bytes, stream)
 
 
 def monarch_attn_bwd_workspace_bytes(B, H, f, h, w, d, b1, b2, tiles, iters, dtype):

@@ -166,3 +166,47 @@ def monarch_attention_bnhd(q, k, v, *, f, h, w, b1, b2, tiles=1, iters=1, out=No
                                                stream),
                "monarch_attn_fwd_layout_ws")
     return out
+
+
+_AXES = {"query_rows": _lib.TILE_QUERY_ROWS, "key_columns": _lib.TILE_KEY_COLUMNS}
+_LAYOUTS = {"bhnd": _lib.BHND, "bnhd": _lib.BNHD}
+
+
+def monarch_attention_tiled(q, k, v, *, f, h, w, b1, b2, tiles=1, iters=1, axis="query_rows",
+                            layout="bhnd", out=None, workspace=None):
+    """monarch_attention with the tiles on either axis: axis="query_rows" (tiles in
+    [1, b1], every other entry point) or "key_columns" (the key columns of every
+    block split into tiles in [1, b2]; each query row's L runs over the b1*t
+    (block, key tile) super-keys).  layout "bhnd" ([B, H, N, d]) or "bnhd"
+    ([B, N, H, d])."""
+    if out is None:
+        out = torch.empty_like(q)
+    _check_tensors(q, k, v, out)
+    if q.dim() != 4:
+        raise ValueError("expected 4-D tensors")
+    if axis not in _AXES or layout not in _LAYOUTS:
+        raise ValueError("axis must be one of %s and layout one of %s" % (list(_AXES),
+                                                                          list(_LAYOUTS)))
+    if layout == "bhnd":
+        B, H, N, d = q.shape
+    else:
+        B, N, H, d = q.shape
+    if N != f * h * w:
+        raise ValueError("N = %d but f*h*w = %d" % (N, f * h * w))
+    args = (B, H, f, h, w, d, b1, b2, tiles, iters)
+    dt, ax, lay = _DTYPES[q.dtype], _AXES[axis], _LAYOUTS[layout]
+    need = _lib.monarch_attn_tiled_workspace_bytes(*args, dt, ax)
+    if need == 0:
+        _lib.check(_lib.monarch_attn_fwd_tiled_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                  out.data_ptr(), *args, dt, ax, lay, 0, 0, 0),
+                   "monarch_attn_fwd_tiled_ws")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    _lib.check(_lib.monarch_attn_fwd_tiled_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                              out.data_ptr(), *args, dt, ax, lay,
+                                              workspace.data_ptr(),
+                                              workspace.numel() * workspace.element_size(),
+                                              stream),
+               "monarch_attn_fwd_tiled_ws")
+    return out

@@ -117,8 +117,34 @@ monarch_status validate_shape(int B, int H, int f, int h, int w, int d, int b1, 
     p->Nk = p->N;
     p->b1k = b1;
     p->layout = kLayoutBHND;
+    p->key_tiles = 0;
     return MONARCH_OK;
 }
+
+namespace {
+
+// Either reading of the tiles: query rows (tiles in [1, b1]) or key columns
+// (tiles in [1, b2]); see Problem::key_tiles.
+monarch_status validate_tiled(int B, int H, int f, int h, int w, int d, int b1, int b2, int tiles,
+                              int iters, monarch_dtype dtype, monarch_tile_axis axis, Problem *p) {
+    if (axis == MONARCH_TILE_QUERY_ROWS)
+        return validate_shape(B, H, f, h, w, d, b1, b2, tiles, iters, dtype, p);
+    if (axis != MONARCH_TILE_KEY_COLUMNS) return MONARCH_ERR_INVALID_ARG;
+    monarch_status st = validate_shape(B, H, f, h, w, d, b1, b2, 1, iters, dtype, p);
+    if (st != MONARCH_OK) return st;
+    if (tiles < 1 || tiles > b2) return MONARCH_ERR_SHAPE;
+    const int64_t BHt = (int64_t)B * H * tiles;
+    if (BHt >= (1LL << 31)) return MONARCH_ERR_SHAPE;
+    if (BHt * b1 * ((b2 + 7) / 8) >= (1LL << 31) || (int64_t)B * H * b2 * ((b1 + 7) / 8) >= (1LL << 31) ||
+        BHt * b2 * ((b1 + 7) / 8) >= (1LL << 31))
+        return MONARCH_ERR_SHAPE;
+    p->tiles = tiles;
+    p->unit_end = (int)BHt;
+    p->key_tiles = 1;
+    return MONARCH_OK;
+}
+
+}  // namespace
 
 namespace {
 
@@ -265,6 +291,48 @@ monarch_status monarch_attn_fwd_layout_ws(const void *q, const void *k, const vo
         return MONARCH_ERR_INVALID_ARG;
     Problem p;
     monarch_status st = validate_shape(B, H, f, h, w, d, b1, b2, tiles, iters, dtype, &p);
+    if (st != MONARCH_OK) return st;
+    p.layout = layout == MONARCH_LAYOUT_BNHD ? kLayoutBNHD : kLayoutBHND;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        ((uintptr_t)workspace & 255u))
+        return MONARCH_ERR_ALIGN;
+    bool overflow = false;
+    const size_t need = workspace_bytes_for(p, dtype, choose_path(p, dtype), overflow);
+    if (overflow) return MONARCH_ERR_SHAPE;
+    if (ws_bytes < need) return MONARCH_ERR_NO_MEMORY;
+    return run_forward(p, dtype, q, k, v, out, workspace, (cudaStream_t)stream);
+}
+
+size_t monarch_attn_tiled_workspace_bytes(int B, int H, int f, int h, int w, int d, int b1,
+                                           int b2, int tiles, int iters, monarch_dtype dtype,
+                                           monarch_tile_axis axis) {
+    Problem p;
+    if (validate_tiled(B, H, f, h, w, d, b1, b2, tiles, iters, dtype, axis, &p) != MONARCH_OK)
+        return 0;
+    bool overflow = false;
+    const size_t n = workspace_bytes_for(p, dtype, choose_path(p, dtype), overflow);
+    return overflow ? 0 : n;
+}
+
+int monarch_attn_tiled_path(int B, int H, int f, int h, int w, int d, int b1, int b2, int tiles,
+                            int iters, monarch_dtype dtype, monarch_tile_axis axis) {
+    Problem p;
+    if (validate_tiled(B, H, f, h, w, d, b1, b2, tiles, iters, dtype, axis, &p) != MONARCH_OK)
+        return -1;
+    return choose_path(p, dtype);
+}
+
+monarch_status monarch_attn_fwd_tiled_ws(const void *q, const void *k, const void *v, void *out,
+                                         int B, int H, int f, int h, int w, int d, int b1, int b2,
+                                         int tiles, int iters, monarch_dtype dtype,
+                                         monarch_tile_axis axis, monarch_layout layout,
+                                         void *workspace, size_t ws_bytes,
+                                         monarch_stream_t stream) {
+    if (!q || !k || !v || !out || !workspace) return MONARCH_ERR_INVALID_ARG;
+    if (layout != MONARCH_LAYOUT_BHND && layout != MONARCH_LAYOUT_BNHD)
+        return MONARCH_ERR_INVALID_ARG;
+    Problem p;
+    monarch_status st = validate_tiled(B, H, f, h, w, d, b1, b2, tiles, iters, dtype, axis, &p);
     if (st != MONARCH_OK) return st;
     p.layout = layout == MONARCH_LAYOUT_BNHD ? kLayoutBNHD : kLayoutBHND;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||

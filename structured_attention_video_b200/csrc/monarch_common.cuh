@@ -49,9 +49,34 @@ struct Problem {
     int Nk, b1k;
     // layout of q, k, v and the output: kLayoutBHND or kLayoutBNHD (below)
     int layout;
+    // which axis the tiles split (the tiled parameterisation does not fix it):
+    // 0, the query rows u of every block (tile g owns R_{u',g} and the rows
+    // u in T_g); 1, the key columns v' of every block (key tile g' owns the
+    // columns [floor(g' b2/t), floor((g'+1) b2/t)), R_{u',g'} is a softmax over
+    // them, and every query row's L runs over the b1k*t (block, key tile)
+    // super-keys).  With key tiles the units are still (head, g') for the
+    // aggregated queries and the R-step; the L-step runs per head.
+    int key_tiles;
     __host__ __device__ int head_begin() const { return unit_begin / tiles; }
     __host__ __device__ int head_end() const { return (unit_end + tiles - 1) / tiles; }
 };
+
+// Query rows that unit g aggregates and whose output it writes: the rows of
+// tile g, or all b1 rows with key tiles.
+__host__ __device__ __forceinline__ int unit_row_begin(const Problem &p, int g) {
+    return p.key_tiles ? 0 : tile_begin(g, p.b1, p.tiles);
+}
+__host__ __device__ __forceinline__ int unit_row_end(const Problem &p, int g) {
+    return p.key_tiles ? p.b1 : tile_begin(g + 1, p.b1, p.tiles);
+}
+// Key columns of block u' that the R-step of tile g takes its softmax over:
+// all b2, or the key tile's own with key tiles.
+__host__ __device__ __forceinline__ int unit_col_begin(const Problem &p, int g) {
+    return p.key_tiles ? tile_begin(g, p.b2, p.tiles) : 0;
+}
+__host__ __device__ __forceinline__ int unit_col_end(const Problem &p, int g) {
+    return p.key_tiles ? tile_begin(g + 1, p.b2, p.tiles) : p.b2;
+}
 
 // Layouts of the inputs and the output: [B][H][N][d] (the tokens of a head are
 // contiguous rows) or [B][N][H][d] (the heads of a token are contiguous).

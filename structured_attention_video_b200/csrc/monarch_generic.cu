@@ -14,6 +14,11 @@
 //       and the row log-sum-exp (rounds before the last)
 //   S4  (iters > 1) qbar[g][v][u'] = sum_u L_v[u,u'] q_(u,v) / sum_u L_v[u,u'],
 //       L recomputed from the saved log-sum-exp
+// With key tiles (the other reading of the tiles: the key columns v' of every
+// block split into t tiles) S1 and S4 aggregate over all b1 query rows, the
+// R-step of key tile g' takes its softmax over the tile's columns only, and
+// the L-step of each query row runs over the t*b1k (block, key tile) rows of
+// Ktil, Z and H of its column.
 // Each warp owns one softmax row; a CTA of 8 warps shares chunks of 32 keys
 // staged in shared memory (rows padded to d+1 floats: conflict-free).
 #include "monarch_common.cuh"
@@ -49,7 +54,7 @@ __global__ void qbar_mean_kernel(const T *__restrict__ q, float *__restrict__ qb
          idx < total; idx += (int64_t)gridDim.x * blockDim.x) {
         const int64_t bhg = idx / row_elems, col = idx % row_elems;
         const int g = (int)(bhg % p.tiles), bh = (int)(bhg / p.tiles);
-        const int u0 = tile_begin(g, p.b1, p.tiles), u1 = tile_begin(g + 1, p.b1, p.tiles);
+        const int u0 = unit_row_begin(p, g), u1 = unit_row_end(p, g);
         const int64_t ts = tok_stride(p);
         const T *src = q + head_base(p, bh, p.N) + (col / p.d) * ts + col % p.d;
         float acc = 0.f;
@@ -90,13 +95,14 @@ rstep_kernel(const T *__restrict__ k, const T *__restrict__ v, const float *__re
     }
     const int64_t ts = tok_stride(p);
     const int64_t base = head_base(p, bh, p.Nk) + (int64_t)up * p.b2 * ts;
+    const int kc0 = unit_col_begin(p, g), kc1 = unit_col_end(p, g);
     float m = -INFINITY, l = 0.f, e = 0.f;
     float acck[NJ], accv[NJ];
 #pragma unroll
     for (int i = 0; i < NJ; i++) acck[i] = accv[i] = 0.f;
 
-    for (int c0 = 0; c0 < p.b2; c0 += KC) {
-        const int nk = min(KC, p.b2 - c0);
+    for (int c0 = kc0; c0 < kc1; c0 += KC) {
+        const int nk = min(KC, kc1 - c0);
         __syncthreads();
         for (int idx = threadIdx.x; idx < nk * D; idx += blockDim.x) {
             const int r = idx / D, j = idx % D;
@@ -160,31 +166,38 @@ lstep_kernel(const T *__restrict__ q, const float *__restrict__ ktil, const floa
     float *sz = sk + KC * DS;     // [KC][DS]
     float *sh = sz + KC * DS;     // [KC]
 
-    const int nug = (tile_max_rows(p.b1, p.tiles) + GW - 1) / GW;
-    int64_t bid = blockIdx.x + (int64_t)p.unit_begin * p.b2 * nug;   // from the first unit
+    // query tiles: a unit (bh, g) per grid slice; key tiles: a head per slice,
+    // its rows u over all b1 and its keys over the t key tiles
+    const int nug = (p.key_tiles ? p.b1 + GW - 1 : tile_max_rows(p.b1, p.tiles) + GW - 1) / GW;
+    const int nseg = p.key_tiles ? p.tiles : 1;
+    int64_t bid = blockIdx.x + (int64_t)(p.key_tiles ? p.head_begin() : p.unit_begin) * p.b2 * nug;
     const int ug = (int)(bid % nug);
     bid /= nug;
     const int vcol = (int)(bid % p.b2);
     bid /= p.b2;
-    const int g = (int)(bid % p.tiles);
-    const int bh = (int)(bid / p.tiles);
+    const int g = p.key_tiles ? 0 : (int)(bid % p.tiles);
+    const int bh = (int)(p.key_tiles ? bid : bid / p.tiles);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int u0 = tile_begin(g, p.b1, p.tiles), u1 = tile_begin(g + 1, p.b1, p.tiles);
+    const int u0 = unit_row_begin(p, g), u1 = unit_row_end(p, g);
     const int u = u0 + ug * GW + warp;
     const bool active = u < u1;
-    const int64_t bhg = (int64_t)bh * p.tiles + g;
     const int64_t tok = (int64_t)bh * p.N + (int64_t)u * p.b2 + vcol;   // workspace index
     const int64_t qoff = head_base(p, bh, p.N) + ((int64_t)u * p.b2 + vcol) * tok_stride(p);
 
     if (active)
         for (int j = lane; j < D; j += 32) sq[warp * D + j] = to_f32(q[qoff + j]);
-    const int64_t kbase = (bhg * p.b2 + vcol) * p.b1k;   // row of block u' = 0
     float m = -INFINITY, l = 0.f;
     float acc[NJ];
 #pragma unroll
     for (int i = 0; i < NJ; i++) acc[i] = 0.f;
 
-    for (int c0 = 0; c0 < p.b1k; c0 += KC) {
+    // chunk ch covers keys [c0, c0 + nk) of segment sg: the rows of block
+    // u' = c0 .. of (g, v), g the unit's tile or, with key tiles, key tile sg
+    const int nchunk = (p.b1k + KC - 1) / KC;
+    for (int ch = 0; ch < nseg * nchunk; ch++) {
+        const int sg = ch / nchunk, c0 = (ch % nchunk) * KC;
+        const int64_t kbase =
+            (((int64_t)bh * p.tiles + (p.key_tiles ? sg : g)) * p.b2 + vcol) * p.b1k;
         const int nk = min(KC, p.b1k - c0);
         __syncthreads();
         for (int idx = threadIdx.x; idx < nk * D; idx += blockDim.x) {
@@ -250,7 +263,7 @@ qbar_weighted_kernel(const T *__restrict__ q, const float *__restrict__ ktil,
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int up = upg * GW + warp;
     const bool active = up < p.b1k;
-    const int u0 = tile_begin(g, p.b1, p.tiles), u1 = tile_begin(g + 1, p.b1, p.tiles);
+    const int u0 = unit_row_begin(p, g), u1 = unit_row_end(p, g);
     const int64_t bhg = (int64_t)bh * p.tiles + g;
     const int64_t row = (bhg * p.b2 + vcol) * p.b1k + up;
 
@@ -331,7 +344,9 @@ cudaError_t run_generic(const Problem &p, const T *q, const T *k, const T *v, T 
         qbar_mean_kernel<T><<<mean_blocks, 256, 0, stream>>>(q, ws.qbar, p);
     }
     const unsigned r_blocks = (unsigned)(units * p.b1k * ((p.b2 + GW - 1) / GW));
-    const unsigned l_blocks = (unsigned)(units * p.b2 * ((tile_max_rows(p.b1, p.tiles) + GW - 1) / GW));
+    const unsigned l_blocks =
+        p.key_tiles ? (unsigned)((int64_t)(p.head_end() - p.head_begin()) * p.b2 * ((p.b1 + GW - 1) / GW))
+                    : (unsigned)(units * p.b2 * ((tile_max_rows(p.b1, p.tiles) + GW - 1) / GW));
     const unsigned w_blocks = (unsigned)(units * p.b2 * ((p.b1k + GW - 1) / GW));
     for (int it = 0; it < p.iters; it++) {
         const bool last = it == p.iters - 1;

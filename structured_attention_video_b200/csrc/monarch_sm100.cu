@@ -56,6 +56,16 @@ __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, const 
     return __all_sync(0xffffffffu, ok);
 }
 
+// Key rows per (q̄ row, head) slab of Ktil, Z and the entropy panels: b1k, or
+// with key-column tiles b1k rounded up to 64, so that the t key tiles of one
+// column v (q̄ rows v*t + g') form one run of t*slab keys in which every 64-key
+// half lies inside one tile.  The rows past b1k of each tile hold Ktil = Z = 0
+// and an entropy of -1e30 (tc_keypad_kernel): their L-step logits are -1e30
+// and their probabilities exactly 0.
+__host__ __device__ __forceinline__ int key_slab(const Problem &p) {
+    return p.key_tiles ? (p.b1k + 63) / 64 * 64 : p.b1k;
+}
+
 // =====================================================================
 // S1: aggregated queries
 // =====================================================================
@@ -75,10 +85,13 @@ __global__ void __launch_bounds__(128 * kQbarGroups, 2) tc_qbar_kernel(
     const int grp = threadIdx.x >> 7, tid = threadIdx.x & 127;
     // every tile of the heads that the unit range touches (the R-step reads all
     // of a head's aggregated rows, padding included)
-    const int bhg = blockIdx.x / nchunk + p.head_begin() * p.tiles;
-    const int g = bhg % p.tiles, bh = bhg / p.tiles;
+    // with key-column tiles one block per (head, chunk) aggregates all b1 rows
+    // and writes the mean to the t rows v*t + g' of column v
+    const int upb = p.key_tiles ? 1 : p.tiles;
+    const int bhg = blockIdx.x / nchunk + p.head_begin() * upb;
+    const int g = bhg % upb, bh = bhg / upb;
     const int col = (chunk * 128 + tid) * 8;
-    const int u0 = tile_begin(g, p.b1, p.tiles), u1 = tile_begin(g + 1, p.b1, p.tiles);
+    const int u0 = unit_row_begin(p, g), u1 = unit_row_end(p, g);
     // rows [r0, r1) of this group: a contiguous quarter of the tile
     const int n = u1 - u0;
     const int r0 = u0 + (grp * n) / kQbarGroups, r1 = u0 + ((grp + 1) * n) / kQbarGroups;
@@ -136,7 +149,14 @@ __global__ void __launch_bounds__(128 * kQbarGroups, 2) tc_qbar_kernel(
         uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
 #pragma unroll
         for (int i = 0; i < 4; i++) ow[i] = pack_bf16(acc[2 * i] * inv, acc[2 * i + 1] * inv);
-        *reinterpret_cast<uint4 *>(qbar + ((int64_t)bh * mpad + (int64_t)g * p.b2) * kD + col) = o;
+        if (p.key_tiles) {
+            const int v = col / kD, j = col % kD;
+            for (int gk = 0; gk < p.tiles; gk++)
+                *reinterpret_cast<uint4 *>(qbar + ((int64_t)bh * mpad + (int64_t)v * p.tiles + gk) *
+                                                      kD + j) = o;
+        } else {
+            *reinterpret_cast<uint4 *>(qbar + ((int64_t)bh * mpad + (int64_t)g * p.b2) * kD + col) = o;
+        }
     }
     if (g == 0 && grp == 0) {   // zero the padding rows [t*b2, mpad) of this head
         const int64_t pad = (int64_t)(mpad - p.tiles * p.b2) * kD;
@@ -233,6 +253,24 @@ __device__ __forceinline__ LsProblem ls_problem(const LsArgs &a, int unit) {
     unit += a.prob0;
     const int pair = unit % a.npairs;
     unit /= a.npairs;
+    if (MODE == kLsOut && p.key_tiles) {
+        // key-column tiles: (bh, v) and a pair of tiles of all b1 query rows; the
+        // keys are the t*slab rows of the q̄ rows v*t .. v*t + t - 1 of head bh
+        const int slab = key_slab(p);
+        q.v = unit % p.b2;
+        q.bh = unit / p.b2;
+        q.g = 0;
+        q.m_y = q.v;
+        q.m_first = 256 * pair;
+        q.m_z = q.bh * p.b1 + q.m_first;
+        q.m_end = p.b1;
+        q.n_y = 0;
+        q.n_z = ((q.bh * p.tiles * p.b2) + q.v * p.tiles) * slab;
+        q.nkeys = p.tiles * slab;
+        q.nch = (q.nkeys + 127) / 128;
+        q.nh = (q.nkeys + 63) / 64;
+        return q;
+    }
     q.v = unit % p.b2;
     unit /= p.b2;
     q.g = unit % p.tiles;
@@ -1012,11 +1050,19 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
 #pragma unroll
             for (int c = 0; c < B2P / 16; c++) tmem_ld16f(tS + c * 16, &x[c * 16]);
             tmem_wait_ld();
-            if (p.b2 < B2P) {   // padded key columns (uniform branch)
-                // a large finite logit, not -inf: its probability is exactly 0 and
-                // 0 * x stays finite in the entropy sum (no per-column condition)
+            if (p.key_tiles || p.b2 < B2P) {   // uniform branch
+                // columns outside [lo, hi): the padding past b2, and with key-column
+                // tiles the other tiles' columns (row r = v*t + g' of the tile stack
+                // takes key tile g').  A large finite logit, not -inf: its
+                // probability is exactly 0 and 0 * x stays finite in the entropy sum.
+                int lo = 0, hi = p.b2;
+                if (p.key_tiles) {
+                    const int gk = (mt * 128 + wq * 32 + lane) % p.tiles;
+                    lo = tile_begin(gk, p.b2, p.tiles);
+                    hi = tile_begin(gk + 1, p.b2, p.tiles);
+                }
 #pragma unroll
-                for (int col = 0; col < B2P; col++) x[col] = col < p.b2 ? x[col] : -1e30f;
+                for (int col = 0; col < B2P; col++) x[col] = col >= lo && col < hi ? x[col] : -1e30f;
             }
             // maximum with four independent chains
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -1056,7 +1102,7 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 if (a.hdirect) {
                     const int row = mt * 128 + wq * 32 + lane;
                     if (row < p.tiles * p.b2) {
-                        uint4 *dst = a.hx + (((int64_t)bh * p.tiles * p.b2 + row) * p.b1k + up) * 2;
+                        uint4 *dst = a.hx + (((int64_t)bh * p.tiles * p.b2 + row) * key_slab(p) + up) * 2;
                         dst[0] = make_uint4(pair, 0u, 0u, 0u);
                         dst[1] = make_uint4(0u, 0u, 0u, 0u);
                     }
@@ -1160,6 +1206,30 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
     }
 }
 
+// Key-column tiles: the key rows [b1k, slab) of every (head, q̄ row) slab hold
+// Ktil = Z = 0 and the entropy panel [-1e30, 0, ...], so that the L-step's logit
+// of such a row is -1e30 (its probability exactly 0) and its products stay
+// finite.  One thread per 16 bytes: 16 of Ktil, 16 of Z and 2 of the panel.
+__global__ void tc_keypad_kernel(__nv_bfloat16 *__restrict__ ktil, __nv_bfloat16 *__restrict__ z,
+                                 uint4 *__restrict__ hx, Problem p) {
+    const int slab = key_slab(p), npad = slab - p.b1k;
+    const int64_t rows = (int64_t)p.BH * p.tiles * p.b2 * npad;
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t neg = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(-1e30f));
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < rows * 34;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t pr = i / 34;
+        const int part = (int)(i % 34);
+        const int64_t row = (pr / npad) * slab + p.b1k + pr % npad;   // key row in the slabs
+        if (part < 16)
+            reinterpret_cast<uint4 *>(ktil + row * kD)[part] = zero;
+        else if (part < 32)
+            reinterpret_cast<uint4 *>(z + row * kD)[part - 16] = zero;
+        else
+            hx[row * 2 + (part - 32)] = part == 32 ? make_uint4(neg, 0u, 0u, 0u) : zero;
+    }
+}
+
 // =====================================================================
 // host side
 // =====================================================================
@@ -1217,9 +1287,12 @@ struct TcWorkspace {
     uint4 *lam;           // iters > 1: log-sum-exp panels [BH][N] rows of 32 bytes
 };
 
+// Key rows of Ktil, Z and the entropy panels over all heads and q̄ rows.
+size_t key_rows(const Problem &p) { return (size_t)p.BH * p.tiles * p.b2 * key_slab(p); }
+
 TcWorkspace carve(const Problem &p, void *base) {
     const size_t mpad = (size_t)qbar_tiles(p) * 128;
-    const size_t kz = (size_t)p.BH * p.tiles * p.Nk * kD * 2;
+    const size_t kz = key_rows(p) * kD * 2;
     char *c = (char *)base;
     TcWorkspace ws;
     ws.qbar = (__nv_bfloat16 *)c;
@@ -1229,7 +1302,7 @@ TcWorkspace carve(const Problem &p, void *base) {
     ws.z = (__nv_bfloat16 *)c;
     c += al256(kz);
     ws.hx = (uint4 *)c;
-    c += al256((size_t)p.BH * p.tiles * p.Nk * 32);
+    c += al256(key_rows(p) * 32);
     ws.qblk = nullptr;
     ws.lam = nullptr;
     if (p.iters > 1) {
@@ -1266,12 +1339,15 @@ int sm_count() {
 
 bool sm100_supports(const Problem &p, monarch_dtype dtype) {
     if (dtype != MONARCH_BF16 || p.d != kD || p.b2 > 128) return false;
+    // key-column tiles: the first iteration's kernels only (later iterations
+    // run on the generic kernels)
+    if (p.key_tiles && p.iters > 1) return false;
     // later iterations keep one slot per aggregated-query tile
     if (p.iters > 1 && qbar_tiles(p) > kMaxQbarTiles) return false;
     if (p.iters > 1 && (int64_t)p.BH * p.b1k * qbar_tiles(p) * 128 + 256 >= (1LL << 31)) return false;
     if (rstep_smem(b2_padded(p.b2), qbar_tiles(p), 1) > (uint32_t)kMaxSmem) return false;
     // TMA coordinates are 32-bit: every row index must fit
-    if ((int64_t)p.BH * p.tiles * p.Nk + 256 >= (1LL << 31)) return false;
+    if ((int64_t)key_rows(p) + 256 >= (1LL << 31)) return false;
     if ((int64_t)p.BH * p.Nk + 256 >= (1LL << 31) || (int64_t)p.BH * p.N + 256 >= (1LL << 31))
         return false;
     if ((int64_t)p.BH * qbar_tiles(p) * 128 >= (1LL << 31)) return false;
@@ -1283,8 +1359,8 @@ bool sm100_supports(const Problem &p, monarch_dtype dtype) {
 size_t sm100_workspace_bytes(const Problem &p, bool &overflow) {
     overflow = false;
     const size_t mpad = (size_t)qbar_tiles(p) * 128;
-    const size_t kz = (size_t)p.BH * p.tiles * p.Nk * kD * 2;
-    const size_t hx = (size_t)p.BH * p.tiles * p.Nk * 32;
+    const size_t kz = key_rows(p) * kD * 2;
+    const size_t hx = key_rows(p) * 32;
     size_t bytes = al256((size_t)p.BH * mpad * kD * 2) + 2 * al256(kz) + al256(hx);
     if (p.iters > 1)
         bytes += al256((size_t)p.BH * p.b1k * mpad * kD * 2) + al256((size_t)p.BH * p.N * 32);
@@ -1355,14 +1431,13 @@ cudaError_t run_rstep(const Problem &p, const TcWorkspace &ws, const void *k, co
     const uint64_t dq[2] = {(uint64_t)kD, qblk ? (uint64_t)p.BH * p.b1k * mpad : (uint64_t)p.BH * mpad};
     const uint64_t s2[1] = {kD * 2};
     const uint32_t bq[2] = {64, 128};
-    const uint64_t dst[4] = {(uint64_t)kD, (uint64_t)p.b1k, (uint64_t)p.tiles * p.b2,
-                             (uint64_t)p.BH};
-    const uint64_t sst[3] = {kD * 2, (uint64_t)p.b1k * kD * 2,
-                             (uint64_t)p.tiles * p.b2 * p.b1k * kD * 2};
+    const uint64_t slab = (uint64_t)key_slab(p);
+    const uint64_t dst[4] = {(uint64_t)kD, slab, (uint64_t)p.tiles * p.b2, (uint64_t)p.BH};
+    const uint64_t sst[3] = {kD * 2, slab * kD * 2, (uint64_t)p.tiles * p.b2 * slab * kD * 2};
     const uint32_t bst[4] = {64, 1, 32, 1};
-    // entropy panels, [bh][t*b2 rows][b1][16], stored 32 rows x 32 B per warp
-    const uint64_t dhx[4] = {16, (uint64_t)p.b1k, (uint64_t)p.tiles * p.b2, (uint64_t)p.BH};
-    const uint64_t shx[3] = {32, (uint64_t)p.b1k * 32, (uint64_t)p.tiles * p.b2 * p.b1k * 32};
+    // entropy panels, [bh][t*b2 rows][slab][16], stored 32 rows x 32 B per warp
+    const uint64_t dhx[4] = {16, slab, (uint64_t)p.tiles * p.b2, (uint64_t)p.BH};
+    const uint64_t shx[3] = {32, slab * 32, (uint64_t)p.tiles * p.b2 * slab * 32};
     const uint32_t bhx[4] = {16, 1, 32, 1};
     if (!make_map(&maps[0], qblk ? ws.qblk : ws.qbar, 2, dq, s2, bq) ||
         !map_keys(&maps[1], k, p, (uint32_t)b2p) || !map_keys(&maps[2], v, p, (uint32_t)b2p) ||
@@ -1395,7 +1470,7 @@ cudaError_t run_lstep(const Problem &p, const TcWorkspace &ws, const void *q, vo
                       cudaStream_t stream) {
     const int mpad = qbar_tiles(p) * 128;
     CUtensorMap qg, kt, zt, xp;
-    const uint64_t rows = (uint64_t)p.BH * p.tiles * p.Nk;
+    const uint64_t rows = key_rows(p);
     if (!map_queries(&qg, q, p) ||
         !map_rows(&kt, ws.ktil, rows, kD, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map_rows(&zt, ws.z, rows, kD, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -1405,10 +1480,13 @@ cudaError_t run_lstep(const Problem &p, const TcWorkspace &ws, const void *q, vo
             : !map_rows(&xp, ws.hx, rows, 16, CU_TENSOR_MAP_SWIZZLE_32B))
         return cudaErrorInvalidValue;
     // M-side rows per (g, v): the tile's queries, or (kLsAgg) the b1 Ktil rows
-    const int mrows = agg ? p.b1k : tile_max_rows(p.b1, p.tiles);
+    // (with key-column tiles: all b1 query rows of each (head, column) problem)
+    const int mrows = agg ? p.b1k : p.key_tiles ? p.b1 : tile_max_rows(p.b1, p.tiles);
     const int npairs = ((mrows + 127) / 128 + 1) / 2;
-    const int nprob = (p.unit_end - p.unit_begin) * p.b2 * npairs;
-    LsArgs a{p, mode, npairs, nprob, p.unit_begin * p.b2 * npairs, mpad, c_log2,
+    const int units = p.key_tiles ? p.head_end() - p.head_begin() : p.unit_end - p.unit_begin;
+    const int first = p.key_tiles ? p.head_begin() : p.unit_begin;
+    const int nprob = units * p.b2 * npairs;
+    LsArgs a{p, mode, npairs, nprob, first * p.b2 * npairs, mpad, c_log2,
              agg ? ws.qblk : (__nv_bfloat16 *)out, ws.lam, status, wait_limit, stall};
     const int grid = nprob < sm_count() ? nprob : sm_count();
     ProfileScope scope(mode == kLsOut ? K_TC_LSTEP : mode == kLsStat ? K_TC_LSTAT : K_TC_QAGG,
@@ -1447,9 +1525,17 @@ cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const 
     {
         const int nchunk = (p.b2 * kD / 8 + 127) / 128;
         ProfileScope scope(K_TC_QBAR, stream);
-        tc_qbar_kernel<<<(p.head_end() - p.head_begin()) * p.tiles * nchunk, 128 * kQbarGroups, 0,
+        const int upb = p.key_tiles ? 1 : p.tiles;
+        tc_qbar_kernel<<<(p.head_end() - p.head_begin()) * upb * nchunk, 128 * kQbarGroups, 0,
                          stream>>>(
             (const __nv_bfloat16 *)q, ws.qbar, p, mpad);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (key_slab(p) > p.b1k) {   // key-column tiles: the padding rows of every slab
+        const int64_t work = (int64_t)p.BH * p.tiles * p.b2 * (key_slab(p) - p.b1k) * 34;
+        const int blocks = (int)((work + 255) / 256 < 4 * 148 ? (work + 255) / 256 : 4 * 148);
+        tc_keypad_kernel<<<blocks, 256, 0, stream>>>(ws.ktil, ws.z, ws.hx, p);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

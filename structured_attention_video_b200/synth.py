@@ -87,6 +87,22 @@ class Workload:
         per_head = (4 * T + 2) * t * N * self.b2 * self.d + 4 * T * N * self.b1 * self.d
         return float(self.B * self.H * per_head)
 
+    def monarch_flops_keytiles(self) -> float:
+        """Algorithmic FLOPs of the forward pass with key-column tiles (the tiles
+        split the key columns of every block; multiply-add = 2).
+
+        Per (b, h): every iteration's R-step takes, for each block and column, the
+        logits of the aggregated query against its key tile's columns only (all t
+        tiles together: 2*N*b2*d) and Ktil = R K (2*N*b2*d); the last one also
+        forms Z = R V (2*N*b2*d).  Every iteration's L-step takes the logits of
+        each query against the t*b1 super-keys (2*t*N*b1*d) and then forms Y = L Z
+        or re-aggregates the queries (2*t*N*b1*d).  Total
+        (4T + 2)*N*b2*d + 4T*t*N*b1*d.
+        """
+        T, t, N = self.iters, self.tiles, self.N
+        per_head = (4 * T + 2) * N * self.b2 * self.d + 4 * T * t * N * self.b1 * self.d
+        return float(self.B * self.H * per_head)
+
     def backward_flops(self) -> float:
         """Algorithmic FLOPs of the backward pass of one iteration (multiply-add =
         2), without recomputing the forward's R-step.

@@ -129,3 +129,32 @@ def test_backward_workspace_and_validation():
     # a null gradient pointer
     assert _lib.monarch_attn_bwd_ws(16, 16, 16, 16, None, 16, 16, *shape, 1, _lib.F32, 256,
                                     bw, None) == 1   # MONARCH_ERR_INVALID_ARG
+
+
+def test_tiled_entry_points_validate_the_axis_and_tile_range():
+    """Key-column tiles take tiles in [1, b2] and the generic kernels; the
+    query-row axis is the default entry points' reading, bit for bit the same
+    workspace; a bad axis or range is refused before touching the device."""
+    shape = (1, 2, 3, 8, 8, 32, 24, 8)          # B, H, f, h, w, d, b1, b2
+    Q, K = _lib.TILE_QUERY_ROWS, _lib.TILE_KEY_COLUMNS
+    for t in (1, 5, 24):
+        assert (_lib.monarch_attn_tiled_workspace_bytes(*shape, t, 1, _lib.F32, Q) ==
+                _lib.monarch_attn_workspace_bytes(*shape, t, 1, _lib.F32))
+    for t in (1, 3, 8):
+        assert _lib.monarch_attn_tiled_workspace_bytes(*shape, t, 2, _lib.F32, K) > 0
+        assert _lib.monarch_attn_tiled_path(*shape, t, 1, _lib.BF16, K) == 0
+    assert _lib.monarch_attn_tiled_workspace_bytes(*shape, 9, 1, _lib.F32, K) == 0   # t > b2
+    assert _lib.monarch_attn_tiled_workspace_bytes(*shape, 0, 1, _lib.F32, K) == 0
+    assert _lib.monarch_attn_tiled_workspace_bytes(*shape, 2, 1, _lib.F32, 2) == 0   # bad axis
+    assert _lib.monarch_attn_tiled_path(*shape, 9, 1, _lib.F32, K) == -1
+    ws = _lib.monarch_attn_tiled_workspace_bytes(*shape, 3, 1, _lib.F32, K)
+    assert _lib.monarch_attn_fwd_tiled_ws(16, 16, 16, 16, *shape, 9, 1, _lib.F32, K, _lib.BHND,
+                                          256, ws, None) == 2          # MONARCH_ERR_SHAPE
+    assert _lib.monarch_attn_fwd_tiled_ws(16, 16, 16, 16, *shape, 3, 1, _lib.F32, 7, _lib.BHND,
+                                          256, ws, None) == 1          # bad axis
+    assert _lib.monarch_attn_fwd_tiled_ws(16, 16, 16, 16, *shape, 3, 1, _lib.F32, K, 5,
+                                          256, ws, None) == 1          # bad layout
+    assert _lib.monarch_attn_fwd_tiled_ws(16, 16, 16, 16, *shape, 3, 1, _lib.F32, K, _lib.BHND,
+                                          256, ws - 1, None) == 5      # workspace too small
+    assert _lib.monarch_attn_fwd_tiled_ws(16, 16, 16, 24, *shape, 3, 1, _lib.F32, K, _lib.BHND,
+                                          256, ws, None) == 3          # misaligned out

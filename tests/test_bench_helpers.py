@@ -135,3 +135,19 @@ def test_workload_config_names_the_shape_and_the_l2_policy():
     assert cfg["N"] == 75600 and cfg["b1"] == 945 and cfg["b2"] == 80 and cfg["tiles"] == 4
     assert "720p" in cfg["workload"] and "x2" in cfg["parallelism"]
     assert "L2" in cfg["l2"]
+
+
+def test_keytile_cpu_baseline_reports_the_oracle_time_and_error():
+    """The key-tile line's CPU-baseline leg: the oracle's time scaled to a whole
+    step, and the error of a device output that is the oracle's own output rounded
+    to bfloat16 (so the error is the rounding alone)."""
+    from oracle import oracle
+    wl = synth.WORKLOADS["tiny"].replace(dtype="bf16", tiles=3)
+    q, k, v = synth.make_inputs(wl)
+    y = oracle.monarch_attn_keytiles(q, k, v, wl.b1, wl.b2, wl.tiles, wl.iters)
+    bits = synth.to_device_bits(synth.round_to_dtype(y, "bf16"), "bf16")
+    rec = bench.keytile_cpu_baseline(wl, bits, 4)
+    assert rec["kind"] == "oracle" and rec["unit"] == "ms" and rec["value"] > 0
+    assert rec["cores"] >= 1
+    assert 0 < rec["rel_err"]["value"] < 4e-3
+    assert rec["rel_err"]["rows"] % wl.b1 == 0
