@@ -10,9 +10,12 @@
 //                         S = qbar K_u'^T                  (tcgen05, SMEM x SMEM)
 //                         R = rowsoftmax(s S), H = entropy (float32, per thread row)
 //                         [Z | Ktil] = R [V_u' | K_u']     (tcgen05, R from TMEM)
-//                       Z and Ktil leave through TMA stores whose 4-D tensor map
-//                       folds the Monarch permutation: row (g, v) of block u'
-//                       lands at [bh][g*b2+v][u'] (rows past t*b2 are clipped).
+//                       Z and Ktil leave through TMA stores in the R-step's own
+//                       order, [bh][u'][panel][g*b2+v][64 columns]: each warp's
+//                       32 rows of a 64-column panel are one contiguous 4 KB box
+//                       (rows past t*b2 are clipped).  The L-step gathers the
+//                       Monarch permutation back: 128 blocks u' of one row (g, v)
+//                       per 5-D box.
 //   S3 tc_lstep_kernel  per (bh, g, v) and pair of 128-query tiles: the queries
 //                       (u, v), u in T_g, come through a 3-D tensor map that
 //                       strides over b2 (P^T folded into the load); online
@@ -57,13 +60,26 @@ __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, const 
 }
 
 // Key rows per (q̄ row, head) slab of Ktil, Z and the entropy panels: b1k, or
-// with key-column tiles b1k rounded up to 64, so that the t key tiles of one
-// column v (q̄ rows v*t + g') form one run of t*slab keys in which every 64-key
-// half lies inside one tile.  The rows past b1k of each tile hold Ktil = Z = 0
-// and an entropy of -1e30 (tc_keypad_kernel): their L-step logits are -1e30
-// and their probabilities exactly 0.
+// with key-column tiles b1k rounded up to 128, so that the t key tiles of one
+// column v (q̄ rows v*t + g') form one run of t*slab keys in which every
+// 128-key chunk (one gather box) lies inside one tile.  The rows past b1k of
+// each tile hold Ktil = Z = 0 and an entropy of -1e30 (tc_keypad_kernel):
+// their L-step logits are -1e30 and their probabilities exactly 0; a problem's
+// first 64-key half always holds real keys, so the running maximum starts on one.
 __host__ __device__ __forceinline__ int key_slab(const Problem &p) {
-    return p.key_tiles ? (p.b1k + 63) / 64 * 64 : p.b1k;
+    return p.key_tiles ? (p.b1k + 127) / 128 * 128 : p.b1k;
+}
+
+// Ktil and Z are stored [bh][u'][panel][r][64] (r = q̄ row, t*b2 of them; panel =
+// 64-column half of d = 128): the R-step's natural order.  Flat key row
+// z = (bh*t*b2 + r)*slab + u' (the order the L-step walks) addresses panel pn of
+// (bh, u', r) through the 5-D map (x, r, panel, u', bh).
+__device__ __forceinline__ void kz_coords(const Problem &p, int z, int &r, int &u, int &bh) {
+    const int slab = key_slab(p), rows = p.tiles * p.b2;
+    const int rid = z / slab;
+    u = z % slab;
+    r = rid % rows;
+    bh = rid / rows;
 }
 
 // =====================================================================
@@ -312,6 +328,15 @@ __device__ __forceinline__ void ls_load_q(void *dst, const CUtensorMap *map, int
         tma_load_5d(dst, map, x, v, u0, hh, bb, bar);
 }
 
+// Panel pn of the 128 key rows z .. z + 127 (flat, see kz_coords) of Ktil or Z:
+// 128 blocks u' of one q̄ row r; blocks past the slab read zeros.
+__device__ __forceinline__ void ls_load_kz(void *dst, const CUtensorMap *map, int pn, int z,
+                                           const Problem &p, uint64_t *bar) {
+    int r, u, bh;
+    kz_coords(p, z, r, u, bh);
+    tma_load_5d(dst, map, 0, r, pn, u, bh, bar);
+}
+
 // One TMA tile load of the L-step: a 3-D gather (x, y, z) or a 2-D row box (x, z).
 __device__ __forceinline__ void ls_load(void *dst, const CUtensorMap *map, bool gather, int x,
                                         int y, int z, uint64_t *bar) {
@@ -424,8 +449,8 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                                           pr.v, pr.n_z - pr.bh * p.b1 + j * 128, pr.bh, p,
                                           k_full + sk);
                             else
-                                ls_load(sm + ls::kK + sk * kTile + pn * kPanel, &tmN, false,
-                                        pn * 64, pr.n_y, pr.n_z + j * 128, k_full + sk);
+                                ls_load_kz(sm + ls::kK + sk * kTile + pn * kPanel, &tmN, pn,
+                                           pr.n_z + j * 128, p, k_full + sk);
                         }
                         ls_load(sm + ls::kHx + sk * ls::kPanelHx, &tmX, n_gather, 0, pr.n_y,
                                 pr.n_z + j * 128, k_full + sk);
@@ -460,9 +485,9 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                             if (!n_gather)
                                 ls_load_q(sm + ls::kQ + t * kTile + pn * kPanel, &tmM, pn * 64,
                                           pr.v, pr.m_first + t * 128, pr.bh, p, q_full + t);
-                            else
-                                ls_load(sm + ls::kQ + t * kTile + pn * kPanel, &tmM, false,
-                                        pn * 64, pr.m_y, pr.m_z + t * 128, q_full + t);
+                            else   // kLsAgg: the Ktil rows are the M side
+                                ls_load_kz(sm + ls::kQ + t * kTile + pn * kPanel, &tmM, pn,
+                                           pr.m_z + t * 128, p, q_full + t);
                         }
                     }
                 }
@@ -478,8 +503,11 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                             else if (!n_gather)
                                 tma_prefetch_5d(&tmM, pn * 64, nx.v, nx.m_first + t * 128,
                                                 nx.bh % p.H, nx.bh / p.H);
-                            else
-                                tma_prefetch_2d(&tmM, pn * 64, nx.m_z + t * 128);
+                            else {
+                                int r, u, bh;
+                                kz_coords(p, nx.m_z + t * 128, r, u, bh);
+                                tma_prefetch_5d(&tmM, 0, r, pn, u, bh);
+                            }
                         }
                 }
                 for (int j = 0; values && j < pr.nch; j++) {
@@ -496,8 +524,8 @@ tc_lstep_kernel(const __grid_constant__ CUtensorMap tmM, const __grid_constant__
                                           pr.v, pr.n_z - pr.bh * p.b1 + j * 128, pr.bh, p,
                                           z_full + st);
                             else
-                                ls_load(sm + ls::kZ + st * kTile + pn * kPanel, &tmV, false,
-                                        pn * 64, pr.n_y, pr.n_z + j * 128, z_full + st);
+                                ls_load_kz(sm + ls::kZ + st * kTile + pn * kPanel, &tmV, pn,
+                                           pr.n_z + j * 128, p, z_full + st);
                         }
                     }
                     issued_z[st]++;
@@ -1189,8 +1217,8 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_4d(part == 0 ? &tmZs : &tmKs, stg + pn * 4096, pn * 64, up,
-                                     mt * 128 + wq * 32, bh);
+                        tma_store_5d(part == 0 ? &tmZs : &tmKs, stg + pn * 4096, 0,
+                                     mt * 128 + wq * 32, pn, up, bh);
                         tma_store_commit();
                     }
                 }
@@ -1206,10 +1234,11 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
     }
 }
 
-// Key-column tiles: the key rows [b1k, slab) of every (head, q̄ row) slab hold
+// Key-column tiles: the key rows u' in [b1k, slab) of every (head, q̄ row) hold
 // Ktil = Z = 0 and the entropy panel [-1e30, 0, ...], so that the L-step's logit
 // of such a row is -1e30 (its probability exactly 0) and its products stay
-// finite.  One thread per 16 bytes: 16 of Ktil, 16 of Z and 2 of the panel.
+// finite.  One thread per 16 bytes: 16 of Ktil, 16 of Z (8 per 64-column panel
+// of the [bh][u'][panel][r][64] layout) and 2 of the panel row [bh][r][slab].
 __global__ void tc_keypad_kernel(__nv_bfloat16 *__restrict__ ktil, __nv_bfloat16 *__restrict__ z,
                                  uint4 *__restrict__ hx, Problem p) {
     const int slab = key_slab(p), npad = slab - p.b1k;
@@ -1220,13 +1249,17 @@ __global__ void tc_keypad_kernel(__nv_bfloat16 *__restrict__ ktil, __nv_bfloat16
          i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t pr = i / 34;
         const int part = (int)(i % 34);
-        const int64_t row = (pr / npad) * slab + p.b1k + pr % npad;   // key row in the slabs
-        if (part < 16)
-            reinterpret_cast<uint4 *>(ktil + row * kD)[part] = zero;
-        else if (part < 32)
-            reinterpret_cast<uint4 *>(z + row * kD)[part - 16] = zero;
-        else
-            hx[row * 2 + (part - 32)] = part == 32 ? make_uint4(neg, 0u, 0u, 0u) : zero;
+        const int64_t rid = pr / npad;                        // bh * t * b2 + r
+        const int up = p.b1k + (int)(pr % npad);              // a padding block row
+        const int64_t rows = (int64_t)p.tiles * p.b2;
+        const int64_t bh = rid / rows, r = rid % rows;
+        if (part < 32) {
+            const int pn = (part & 15) >> 3, c = part & 7;  // panel, 16-byte chunk
+            const int64_t off = (((bh * slab + up) * 2 + pn) * rows + r) * 64;
+            reinterpret_cast<uint4 *>((part < 16 ? ktil : z) + off)[c] = zero;
+        } else {
+            hx[(rid * slab + up) * 2 + (part - 32)] = part == 32 ? make_uint4(neg, 0u, 0u, 0u) : zero;
+        }
     }
 }
 
@@ -1431,17 +1464,18 @@ cudaError_t run_rstep(const Problem &p, const TcWorkspace &ws, const void *k, co
     const uint64_t dq[2] = {(uint64_t)kD, qblk ? (uint64_t)p.BH * p.b1k * mpad : (uint64_t)p.BH * mpad};
     const uint64_t s2[1] = {kD * 2};
     const uint32_t bq[2] = {64, 128};
-    const uint64_t slab = (uint64_t)key_slab(p);
-    const uint64_t dst[4] = {(uint64_t)kD, slab, (uint64_t)p.tiles * p.b2, (uint64_t)p.BH};
-    const uint64_t sst[3] = {kD * 2, slab * kD * 2, (uint64_t)p.tiles * p.b2 * slab * kD * 2};
-    const uint32_t bst[4] = {64, 1, 32, 1};
+    const uint64_t slab = (uint64_t)key_slab(p), rr = (uint64_t)p.tiles * p.b2;
+    // Ktil and Z, [bh][u'][panel][r][64]: (x, r, panel, u', bh), one warp's 32 rows
+    const uint64_t dst[5] = {64, rr, 2, slab, (uint64_t)p.BH};
+    const uint64_t sst[4] = {128, rr * 128, 2 * rr * 128, slab * 2 * rr * 128};
+    const uint32_t bst[5] = {64, 32, 1, 1, 1};
     // entropy panels, [bh][t*b2 rows][slab][16], stored 32 rows x 32 B per warp
     const uint64_t dhx[4] = {16, slab, (uint64_t)p.tiles * p.b2, (uint64_t)p.BH};
     const uint64_t shx[3] = {32, slab * 32, (uint64_t)p.tiles * p.b2 * slab * 32};
     const uint32_t bhx[4] = {16, 1, 32, 1};
     if (!make_map(&maps[0], qblk ? ws.qblk : ws.qbar, 2, dq, s2, bq) ||
         !map_keys(&maps[1], k, p, (uint32_t)b2p) || !map_keys(&maps[2], v, p, (uint32_t)b2p) ||
-        !make_map(&maps[3], ws.z, 4, dst, sst, bst) || !make_map(&maps[4], ws.ktil, 4, dst, sst, bst) ||
+        !make_map(&maps[3], ws.z, 5, dst, sst, bst) || !make_map(&maps[4], ws.ktil, 5, dst, sst, bst) ||
         !make_map(&maps[5], ws.hx, 4, dhx, shx, bhx, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     const int total = (p.head_end() - p.head_begin()) * p.b1k;
@@ -1471,9 +1505,13 @@ cudaError_t run_lstep(const Problem &p, const TcWorkspace &ws, const void *q, vo
     const int mpad = qbar_tiles(p) * 128;
     CUtensorMap qg, kt, zt, xp;
     const uint64_t rows = key_rows(p);
-    if (!map_queries(&qg, q, p) ||
-        !map_rows(&kt, ws.ktil, rows, kD, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map_rows(&zt, ws.z, rows, kD, CU_TENSOR_MAP_SWIZZLE_128B))
+    // Ktil and Z gathered from [bh][u'][panel][r][64]: 128 blocks u' of one row r
+    const uint64_t rr = (uint64_t)p.tiles * p.b2, slab = (uint64_t)key_slab(p);
+    const uint64_t dkz[5] = {64, rr, 2, slab, (uint64_t)p.BH};
+    const uint64_t skz[4] = {128, rr * 128, 2 * rr * 128, slab * 2 * rr * 128};
+    const uint32_t bkz[5] = {64, 1, 1, 128, 1};
+    if (!map_queries(&qg, q, p) || !make_map(&kt, ws.ktil, 5, dkz, skz, bkz) ||
+        !make_map(&zt, ws.z, 5, dkz, skz, bkz))
         return cudaErrorInvalidValue;
     const bool agg = mode == kLsAgg;
     if (agg ? !map_gather(&xp, ws.lam, p, 16, CU_TENSOR_MAP_SWIZZLE_32B)

@@ -161,6 +161,14 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, const void 
         "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z), "r"(w)
         : "memory");
 }
+__device__ __forceinline__ void tma_store_5d(const CUtensorMap *map, const void *src, int x, int y,
+                                             int z, int w, int u) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5, %6}], [%1];" ::
+            "l"(reinterpret_cast<uint64_t>(map)),
+        "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(u)
+        : "memory");
+}
 __device__ __forceinline__ void tma_store_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
