@@ -60,14 +60,15 @@ __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, const 
 }
 
 // Key rows per (q̄ row, head) slab of Ktil, Z and the entropy panels: b1k, or
-// with key-column tiles b1k rounded up to 128, so that the t key tiles of one
-// column v (q̄ rows v*t + g') form one run of t*slab keys in which every
-// 128-key chunk (one gather box) lies inside one tile.  The rows past b1k of
-// each tile hold Ktil = Z = 0 and an entropy of -1e30 (tc_keypad_kernel):
-// their L-step logits are -1e30 and their probabilities exactly 0; a problem's
-// first 64-key half always holds real keys, so the running maximum starts on one.
+// with key-column tiles b1k rounded up to 64, so that the t key tiles of one
+// column v (q̄ rows v*t + g') form one run of t*slab keys in which every 64-key
+// half (one gather box with key-column tiles) lies inside one tile.  The rows
+// past b1k of each tile hold Ktil = Z = 0 and an entropy of -1e30
+// (tc_keypad_kernel): their L-step logits are -1e30 and their probabilities
+// exactly 0; a problem's first half always holds real keys, so the running
+// maximum starts on one.
 __host__ __device__ __forceinline__ int key_slab(const Problem &p) {
-    return p.key_tiles ? (p.b1k + 127) / 128 * 128 : p.b1k;
+    return p.key_tiles ? (p.b1k + 63) / 64 * 64 : p.b1k;
 }
 
 // Ktil and Z are stored [bh][u'][panel][r][64] (r = q̄ row, t*b2 of them; panel =
@@ -329,12 +330,18 @@ __device__ __forceinline__ void ls_load_q(void *dst, const CUtensorMap *map, int
 }
 
 // Panel pn of the 128 key rows z .. z + 127 (flat, see kz_coords) of Ktil or Z:
-// 128 blocks u' of one q̄ row r; blocks past the slab read zeros.
+// 128 blocks u' of one q̄ row r (blocks past the slab read zeros), or with
+// key-column tiles two boxes of 64, each inside one key tile (a 64-row box
+// lands 8 KB on, where the 128-byte swizzle pattern repeats).
 __device__ __forceinline__ void ls_load_kz(void *dst, const CUtensorMap *map, int pn, int z,
                                            const Problem &p, uint64_t *bar) {
     int r, u, bh;
     kz_coords(p, z, r, u, bh);
     tma_load_5d(dst, map, 0, r, pn, u, bh, bar);
+    if (p.key_tiles) {
+        kz_coords(p, z + 64, r, u, bh);
+        tma_load_5d(static_cast<uint8_t *>(dst) + 64 * 128, map, 0, r, pn, u, bh, bar);
+    }
 }
 
 // One TMA tile load of the L-step: a 3-D gather (x, y, z) or a 2-D row box (x, z).
@@ -1084,10 +1091,10 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 // takes key tile g').  A large finite logit, not -inf: its
                 // probability is exactly 0 and 0 * x stays finite in the entropy sum.
                 int lo = 0, hi = p.b2;
-                if (p.key_tiles) {
+                if (p.key_tiles) {   // t <= b2 <= 128: the products fit in 32 bits
                     const int gk = (mt * 128 + wq * 32 + lane) % p.tiles;
-                    lo = tile_begin(gk, p.b2, p.tiles);
-                    hi = tile_begin(gk + 1, p.b2, p.tiles);
+                    lo = gk * p.b2 / p.tiles;
+                    hi = (gk + 1) * p.b2 / p.tiles;
                 }
 #pragma unroll
                 for (int col = 0; col < B2P; col++) x[col] = col >= lo && col < hi ? x[col] : -1e30f;
@@ -1509,7 +1516,7 @@ cudaError_t run_lstep(const Problem &p, const TcWorkspace &ws, const void *q, vo
     const uint64_t rr = (uint64_t)p.tiles * p.b2, slab = (uint64_t)key_slab(p);
     const uint64_t dkz[5] = {64, rr, 2, slab, (uint64_t)p.BH};
     const uint64_t skz[4] = {128, rr * 128, 2 * rr * 128, slab * 2 * rr * 128};
-    const uint32_t bkz[5] = {64, 1, 1, 128, 1};
+    const uint32_t bkz[5] = {64, 1, 1, p.key_tiles ? 64u : 128u, 1};
     if (!map_queries(&qg, q, p) || !make_map(&kt, ws.ktil, 5, dkz, skz, bkz) ||
         !make_map(&zt, ws.z, 5, dkz, skz, bkz))
         return cudaErrorInvalidValue;
