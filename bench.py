@@ -426,19 +426,23 @@ def dense_rows_error(wl: synth.Workload, q, k, v, out, heads, rows_per_head: int
     return float(np.sqrt(num / den))
 
 
-def time_forward(wl: synth.Workload, q, k, v, out, steps: int, warmup: int, flush, stream):
-    """Per-step device times (ms) of monarch_attn_fwd_ws on resident inputs."""
+def time_forward(wl: synth.Workload, q, k, v, out, steps: int, warmup: int, flush, stream,
+                 axis: int = 0):
+    """Per-step device times (ms) of monarch_attn_fwd_tiled_ws on resident inputs, with
+    the tiles on the query rows (axis 0, monarch_attn_fwd_ws's reading) or the key
+    columns (axis 1)."""
     import torch
     from structured_attention_video_b200 import _lib
     sargs = (wl.B, wl.H, wl.f, wl.h, wl.w, wl.d, wl.b1, wl.b2, wl.tiles, wl.iters)
-    ws_bytes = _lib.monarch_attn_workspace_bytes(*sargs, _lib.BF16)
+    ws_bytes = _lib.monarch_attn_tiled_workspace_bytes(*sargs, _lib.BF16, axis)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     sh = stream.cuda_stream
 
     def step():
-        _lib.check(_lib.monarch_attn_fwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                            out.data_ptr(), *sargs, _lib.BF16, ws.data_ptr(),
-                                            ws_bytes, sh), "monarch_attn_fwd_ws")
+        _lib.check(_lib.monarch_attn_fwd_tiled_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                  out.data_ptr(), *sargs, _lib.BF16, axis,
+                                                  _lib.BHND, ws.data_ptr(), ws_bytes, sh),
+                   "monarch_attn_fwd_tiled_ws")
     for _ in range(warmup):
         flush.zero_()
         step()
@@ -453,7 +457,7 @@ def time_forward(wl: synth.Workload, q, k, v, out, steps: int, warmup: int, flus
         torch.cuda.synchronize()
         times.append(a.elapsed_time(b))
     _lib.check(_lib.monarch_last_device_status(sh), "device status (sweep)")
-    return times, _lib.monarch_attn_path(*sargs, _lib.BF16)
+    return times, _lib.monarch_attn_tiled_path(*sargs, _lib.BF16, axis)
 
 
 def run_backward(args, wl: synth.Workload) -> None:
@@ -634,8 +638,11 @@ def run_keytiles(args, wl: synth.Workload) -> None:
         "gpu": torch.cuda.get_device_name(0)}), flush=True)
 
 
+# (workload, swept key, values, heads of the dense check): "key_tiles" sweeps the tile
+# count with the tiles on the key columns (t = b2 = 52 is exact attention)
 SWEEPS = (("480p_full", "tiles", (1, 2, 4, 8), None),
-          ("14b", "iters", (1, 2, 5, 10), (0, 13, 27, 40, 53, 79)))
+          ("14b", "iters", (1, 2, 5, 10), (0, 13, 27, 40, 53, 79)),
+          ("480p_full", "key_tiles", (1, 2, 4, 8, 52), None))
 
 
 def run_sweeps(args) -> None:
@@ -661,16 +668,21 @@ def run_sweeps(args) -> None:
         out = torch.empty_like(q)
         bhs = list(heads) if heads else list(range(wl0.B * wl0.H))
         for val in values:
-            wl = wl0.replace(**{key: val})
+            keys = key == "key_tiles"
+            wl = wl0.replace(**{"tiles" if keys else key: val})
             steps = max(3, args.sweep_steps // max(1, wl.iters))
-            times, path = time_forward(wl, q, k, v, out, steps, 3, flush, stream)
+            times, path = time_forward(wl, q, k, v, out, steps, 3, flush, stream,
+                                       axis=1 if keys else 0)
             ms = float(np.median(times))
-            flops, io = wl.monarch_flops(), wl.io_bytes()
+            flops = wl.monarch_flops_keytiles() if keys else wl.monarch_flops()
+            io = wl.io_bytes()
             roof_ms = max(flops / (peaks["bf16_tflops"] * 1e12),
                           io / (peaks["hbm_gbs"] * 1e9)) * 1e3
             err = dense_rows_error(wl, q, k, v, out, bhs, args.sweep_rows, seed=val)
             records.append({
-                "workload": workload_config(wl, 1)["workload"], key: val, "ms_median": ms,
+                "workload": workload_config(wl, 1)["workload"]
+                            + (" (tiles on the key columns)" if keys else ""),
+                key: val, "ms_median": ms,
                 "steps": steps, "monarch_gflop": flops / 1e9,
                 "monarch_tflops": flops / (ms * 1e-3) / 1e12,
                 "path_roofline_frac": roof_ms / ms,

@@ -167,3 +167,18 @@ def test_key_tiles_tensor_core_whole_output(B, H, f, h, w, b1, tiles):
     ref = oracle.monarch_attn_keytiles(q64, k64, v64, b1, b2, tiles, 1)
     assert np.isfinite(got).all()
     assert rel_fro(got, ref) <= TOL["bf16"]
+
+
+def test_chunk_480p_key_tiles_two_iterations_whole_output():
+    """Later iterations with key-column tiles run on the generic kernels: the 480p
+    chunk with four key tiles and two iterations, every output row against the
+    oracle."""
+    wl = synth.WORKLOADS["480p_chunk"].replace(tiles=4, iters=2)
+    assert _lib.monarch_attn_tiled_path(wl.B, wl.H, wl.f, wl.h, wl.w, wl.d, wl.b1, wl.b2, 4, 2,
+                                        _lib.BF16, _lib.TILE_KEY_COLUMNS) == 0
+    q, k, v = device_inputs(wl)
+    got = from_torch(run_keytiles(wl, q, k, v), wl.dtype)[0]
+    q64, k64, v64 = synth.make_inputs(wl)
+    ref = oracle.monarch_attn_keytiles(q64[0], k64[0], v64[0], wl.b1, wl.b2, 4, 2)
+    assert np.isfinite(got).all()
+    assert rel_fro(got, ref) <= TOL["bf16"]
