@@ -94,7 +94,8 @@ __device__ __forceinline__ void kz_coords(const Problem &p, int z, int &r, int &
 // memory in a fixed order.
 constexpr int kQbarGroups = 4;
 __global__ void __launch_bounds__(128 * kQbarGroups, 2) tc_qbar_kernel(
-    const __nv_bfloat16 *__restrict__ q, __nv_bfloat16 *__restrict__ qbar, Problem p, int mpad) {
+    const __nv_bfloat16 *__restrict__ q, __nv_bfloat16 *__restrict__ qbar, Problem p, int mpad,
+    int pack) {
     __shared__ float part[kQbarGroups - 1][8][128];
     const int row_elems = p.b2 * kD;
     const int nchunk = (row_elems / 8 + 127) / 128;
@@ -166,20 +167,32 @@ __global__ void __launch_bounds__(128 * kQbarGroups, 2) tc_qbar_kernel(
         uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
 #pragma unroll
         for (int i = 0; i < 4; i++) ow[i] = pack_bf16(acc[2 * i] * inv, acc[2 * i + 1] * inv);
-        if (p.key_tiles) {
-            const int v = col / kD, j = col % kD;
-            for (int gk = 0; gk < p.tiles; gk++)
-                *reinterpret_cast<uint4 *>(qbar + ((int64_t)bh * mpad + (int64_t)v * p.tiles + gk) *
-                                                      kD + j) = o;
-        } else {
-            *reinterpret_cast<uint4 *>(qbar + ((int64_t)bh * mpad + (int64_t)g * p.b2) * kD + col) = o;
+        // the R-step's packed tile (pack > 1) repeats the rows in each segment of
+        // 128 / pack rows
+        const int pseg = 128 / pack;
+        for (int sg = 0; sg < pack; sg++) {
+            __nv_bfloat16 *seg = qbar + ((int64_t)bh * mpad + (int64_t)sg * pseg) * kD;
+            if (p.key_tiles) {
+                const int v = col / kD, j = col % kD;
+                for (int gk = 0; gk < p.tiles; gk++)
+                    *reinterpret_cast<uint4 *>(seg + ((int64_t)v * p.tiles + gk) * kD + j) = o;
+            } else {
+                *reinterpret_cast<uint4 *>(seg + (int64_t)g * p.b2 * kD + col) = o;
+            }
         }
     }
-    if (g == 0 && grp == 0) {   // zero the padding rows [t*b2, mpad) of this head
-        const int64_t pad = (int64_t)(mpad - p.tiles * p.b2) * kD;
-        __nv_bfloat16 *base = qbar + ((int64_t)bh * mpad + (int64_t)p.tiles * p.b2) * kD;
-        for (int64_t e = col; e < pad; e += (int64_t)nchunk * 128 * 8)
-            *reinterpret_cast<uint4 *>(base + e) = make_uint4(0, 0, 0, 0);
+    if (g == 0 && grp == 0) {
+        // zero the padding rows of this head: [t*b2, mpad), or [t*b2, 128 / pack) of
+        // every segment of a packed tile
+        const int nseg = pack > 1 ? pack : 1;
+        const int seglen = pack > 1 ? 128 / pack : mpad;
+        for (int sg = 0; sg < nseg; sg++) {
+            const int64_t pad = (int64_t)(seglen - p.tiles * p.b2) * kD;
+            __nv_bfloat16 *base =
+                qbar + ((int64_t)bh * mpad + (int64_t)sg * seglen + (int64_t)p.tiles * p.b2) * kD;
+            for (int64_t e = col; e < pad; e += (int64_t)nchunk * 128 * 8)
+                *reinterpret_cast<uint4 *>(base + e) = make_uint4(0, 0, 0, 0);
+        }
     }
 }
 
@@ -860,6 +873,12 @@ struct RsArgs {
     int *status;
     long long limit;
     int stall;           // test hook: the MMA warp first waits on a barrier nothing completes
+    // blocks per item (1, 2 or 4): when the t*b2 aggregated rows fill at most a half
+    // (a quarter) of the 128-row tile, the tile holds `pack` copies of them in
+    // segments of 128/pack rows, and one item covers `pack` consecutive blocks u':
+    // segment s meets the keys of block u' + s (a block-diagonal mask on the logits)
+    int pack;
+    int gph;             // items (groups of `pack` blocks) per head
 };
 constexpr int kMaxQbarTiles = 4;   // slots of the per-block aggregated-query ring
 
@@ -869,16 +888,19 @@ struct RsLayout {
     static constexpr uint32_t kVOff = 2 * B2P * 128;    // V inside a stage
     static constexpr uint32_t kPanelKV = B2P * 128;
     __host__ __device__ static uint32_t kv(int nmt) { return (uint32_t)nmt * kTile; }
-    __host__ __device__ static uint32_t stg(int nmt) { return kv(nmt) + 2 * kStage; }
+    // two stages, each the K and V panels of `pack` blocks
+    __host__ __device__ static uint32_t stg(int nmt, int pack) {
+        return kv(nmt) + 2 * kStage * (uint32_t)pack;
+    }
     // entropy-panel staging of the softmax warps: 4 warps x 32 rows x 32 B, when
     // it fits (hdirect = 0); otherwise each softmax thread stores its panel row
     // with plain stores (hdirect = 1, no staging)
-    __host__ __device__ static uint32_t hstg(int nmt) { return stg(nmt) + 4 * 8192; }
-    __host__ __device__ static uint32_t bar(int nmt, int hdirect) {
-        return hstg(nmt) + (hdirect ? 0 : 4 * 1024);
+    __host__ __device__ static uint32_t hstg(int nmt, int pack) { return stg(nmt, pack) + 4 * 8192; }
+    __host__ __device__ static uint32_t bar(int nmt, int hdirect, int pack) {
+        return hstg(nmt, pack) + (hdirect ? 0 : 4 * 1024);
     }
-    __host__ __device__ static uint32_t smem(int nmt, int hdirect) {
-        return bar(nmt, hdirect) + 256 + 1024;
+    __host__ __device__ static uint32_t smem(int nmt, int hdirect, int pack) {
+        return bar(nmt, hdirect, pack) + 256 + 1024;
     }
 };
 
@@ -892,7 +914,7 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     const int nmt = a.nmt;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::bar(nmt, a.hdirect));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::bar(nmt, a.hdirect, a.pack));
     uint64_t *q_full = bars + 0;
     uint64_t *q_empty = bars + 1;
     uint64_t *kv_full = bars + 2;    // [2]
@@ -911,9 +933,11 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
 
     const Problem &p = a.p;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // (head, block) items of the heads that the unit range touches
-    const int total = p.head_end() * p.b1k;
-    const int first = p.head_begin() * p.b1k + blockIdx.x * a.bpc;
+    // (head, group of `pack` blocks) items of the heads that the unit range touches
+    const int pack = a.pack, pseg = 128 / pack;
+    const uint32_t kstage = L::kStage * pack, kpanel = L::kPanelKV * pack, kvoff = L::kVOff * pack;
+    const int total = p.head_end() * a.gph;
+    const int first = p.head_begin() * a.gph + blockIdx.x * a.bpc;
     const int nblk = min(a.bpc, total - first);
     const int nitems = nblk * nmt;
 
@@ -951,7 +975,7 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
             int heads = 0, cur = -1, issued[2] = {0, 0}, qissued[kMaxQbarTiles] = {0, 0, 0, 0};
             bool ok = true;
             for (int ib = 0; ib < nblk && ok; ib++) {
-                const int fb = first + ib, bh = fb / p.b1k, up = fb % p.b1k;
+                const int fb = first + ib, bh = fb / a.gph, up = (fb % a.gph) * pack;
                 if (a.qblk) {
                     // slot mt takes tile mt of this block once the S MMA of the
                     // previous block's tile mt is done
@@ -979,17 +1003,23 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 }
                 const int st = ib & 1;
                 if (ib >= 2 && !wait_phase(kv_empty + st, ((ib >> 1) - 1) & 1, w)) break;
-                uint8_t *stage = sm + L::kv(nmt) + st * L::kStage;
-                mbar_expect_tx(kv_full + st, L::kStage);
-                // the block's b2 tokens of head bh: (x, token, head, batch), or
-                // (x, head, token, batch) for [B][N][H][d] (increasing strides)
+                uint8_t *stage = sm + L::kv(nmt) + st * kstage;
+                mbar_expect_tx(kv_full + st, kstage);
+                // the b2 tokens of each block of the group, head bh: (x, token, head,
+                // batch), or (x, head, token, batch) for [B][N][H][d] (increasing
+                // strides); block s at row s*B2P of each panel.  A block past b1k
+                // (the head's last group) reads zeros: every row stays finite.
                 const bool bnhd = p.layout == kLayoutBNHD;
-                const int tok0 = up * p.b2, hh = bh % p.H, bb = bh / p.H;
-                const int c1 = bnhd ? hh : tok0, c2 = bnhd ? tok0 : hh;
-                for (int pn = 0; pn < 2; pn++) {
-                    tma_load_4d(stage + pn * L::kPanelKV, &tmK, pn * 64, c1, c2, bb, kv_full + st);
-                    tma_load_4d(stage + L::kVOff + pn * L::kPanelKV, &tmV, pn * 64, c1, c2, bb,
-                                kv_full + st);
+                const int hh = bh % p.H, bb = bh / p.H;
+                for (int sg = 0; sg < pack; sg++) {
+                    const int tok0 = (up + sg) * p.b2;
+                    const int c1 = bnhd ? hh : tok0, c2 = bnhd ? tok0 : hh;
+                    for (int pn = 0; pn < 2; pn++) {
+                        tma_load_4d(stage + pn * kpanel + sg * L::kPanelKV, &tmK, pn * 64, c1, c2,
+                                    bb, kv_full + st);
+                        tma_load_4d(stage + kvoff + pn * kpanel + sg * L::kPanelKV, &tmV, pn * 64,
+                                    c1, c2, bb, kv_full + st);
+                    }
                 }
                 issued[st]++;
             }
@@ -1005,21 +1035,21 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
         // ---------------- MMA issuer: the whole warp runs the loop, one elected
         // lane issues each MMA (see mma_ss_warp)
         {
-            constexpr uint32_t id1 = idesc_bf16(128, B2P, 0, 0);
+            const uint32_t id1 = idesc_bf16(128, B2P * pack, 0, 0);
             constexpr uint32_t id2 = idesc_bf16(128, 128, 0, 1);
             const uint64_t dQ = smem_desc_sw128(smem_u32(sm), 16, 1024);
             const uint64_t dK = smem_desc_sw128(smem_u32(sm + L::kv(nmt)), 16, 1024);
-            const uint64_t dV = smem_desc_sw128(smem_u32(sm + L::kv(nmt)), L::kPanelKV, 1024);
+            const uint64_t dV = smem_desc_sw128(smem_u32(sm + L::kv(nmt)), kpanel, 1024);
             int heads = 0;
             // fault injection: a wait that can only give up (bounded, then abort)
             bool ok = !a.stall || spin_warp(stall_bar, 0, w);
             // S = qbar_mt K_u'^T for item i into S buffer i & 1
             auto gemm1 = [&](int i) -> bool {
                 const int ib = i / nmt, mt = i % nmt;
-                const int fb = first + ib, bh = fb / p.b1k;
+                const int fb = first + ib, bh = fb / a.gph;
                 if (a.qblk) {
                     if (!wait_warp(qs_full + mt, ib & 1, w)) return false;
-                } else if (mt == 0 && (ib == 0 || (fb - 1) / p.b1k != bh)) {
+                } else if (mt == 0 && (ib == 0 || (fb - 1) / a.gph != bh)) {
                     if (!wait_warp(q_full, heads & 1, w)) return false;
                     heads++;
                 }
@@ -1027,17 +1057,17 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 if (i >= 2 && !wait_warp(s_free + (i & 1), ((i >> 1) - 1) & 1, w)) return false;
                 tc_fence_after();
                 const uint64_t a0 = desc_plus(dQ, mt * kTile);
-                const uint64_t b0 = desc_plus(dK, (ib & 1) * L::kStage);
+                const uint64_t b0 = desc_plus(dK, (ib & 1) * kstage);
 #pragma unroll
                 for (int kk = 0; kk < 8; kk++)
                     mma_ss_warp(tmem + (i & 1) * 128,
                            desc_plus(a0, (kk >> 2) * kPanel + (kk & 3) * 32),
-                           desc_plus(b0, (kk >> 2) * L::kPanelKV + (kk & 3) * 32), id1, kk > 0);
+                           desc_plus(b0, (kk >> 2) * kpanel + (kk & 3) * 32), id1, kk > 0);
                 mma_commit_warp(s_full + (i & 1));
                 if (a.qblk) {
                     mma_commit_warp(qs_empty + mt);   // slot mt may take the next block's tile
                 } else {
-                    const bool head_ends = (ib == nblk - 1) || ((fb + 1) / p.b1k != bh);
+                    const bool head_ends = (ib == nblk - 1) || ((fb + 1) / a.gph != bh);
                     if (mt == nmt - 1 && head_ends) mma_commit_warp(q_empty);
                 }
                 return true;
@@ -1050,18 +1080,18 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 tc_fence_after();
                 const uint32_t pa = tmem + (i & 1) * 128;
                 // 0: Z = R V, 1: Ktil = R K
-                const uint64_t bz = desc_plus(dV, (ib & 1) * L::kStage + L::kVOff);
-                const uint64_t bk = desc_plus(dV, (ib & 1) * L::kStage);
+                const uint64_t bz = desc_plus(dV, (ib & 1) * kstage + kvoff);
+                const uint64_t bk = desc_plus(dV, (ib & 1) * kstage);
                 if (i > 0 && !wait_warp(o_empty + 0, (i - 1) & 1, w)) break;
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < B2P / 16; kk++)
+                // K = pack * B2P: the packed blocks' P columns (zero outside a row's
+                // own segment) against their V (then K) rows
+                for (int kk = 0; kk < (B2P / 16) * pack; kk++)
                     mma_ts_warp(tmem + 256, pa + kk * 8, desc_plus(bz, kk * 2048), id2, kk > 0 ? 1u : 0u);
                 mma_commit_warp(o_full + 0);
                 if (i > 0 && !wait_warp(o_empty + 1, (i - 1) & 1, w)) break;
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < B2P / 16; kk++)
+                for (int kk = 0; kk < (B2P / 16) * pack; kk++)
                     mma_ts_warp(tmem + 384, pa + kk * 8, desc_plus(bk, kk * 2048), id2, kk > 0 ? 1u : 0u);
                 mma_commit_warp(o_full + 1);
                 mma_commit_warp(s_free + (i & 1));
@@ -1074,13 +1104,19 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
         // ---------------- softmax: R rows, entropy, normalised P back to TMEM (bf16)
         const int wq = warp & 3;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        // this thread's row: segment sg of the tile (block up + sg of the group) and
+        // its aggregated-query row qrow (packed tiles: every segment repeats rows
+        // 0 .. pseg - 1; otherwise mt * 128 + the tile row)
+        const int trow = wq * 32 + lane, sg = trow / pseg;
         for (int i = 0; i < nitems; i++) {
             const int ib = i / nmt, mt = i % nmt;
-            const int fb = first + ib, bh = fb / p.b1k, up = fb % p.b1k;
+            const int fb = first + ib, bh = fb / a.gph, up = (fb % a.gph) * pack;
+            const int qrow = mt * 128 + trow % pseg;
             if (!wait_warp(s_full + (i & 1), (i >> 1) & 1, w)) break;
             tc_fence_after();
-            const uint32_t tS = tmem + lane_off + (i & 1) * 128;
-            // the row's B2P logits: all TMEM loads in flight together, one wait
+            const uint32_t tS = tmem + lane_off + (i & 1) * 128 + sg * B2P;
+            // the row's B2P logits (its segment's columns): all TMEM loads in flight
+            // together, one wait
             float x[B2P];
 #pragma unroll
             for (int c = 0; c < B2P / 16; c++) tmem_ld16f(tS + c * 16, &x[c * 16]);
@@ -1092,7 +1128,7 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 // probability is exactly 0 and 0 * x stays finite in the entropy sum.
                 int lo = 0, hi = p.b2;
                 if (p.key_tiles) {   // t <= b2 <= 128: the products fit in 32 bits
-                    const int gk = (mt * 128 + wq * 32 + lane) % p.tiles;
+                    const int gk = qrow % p.tiles;
                     lo = gk * p.b2 / p.tiles;
                     hi = (gk + 1) * p.b2 / p.tiles;
                 }
@@ -1135,9 +1171,9 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 const uint32_t pair = (uint32_t)__bfloat16_as_ushort(hi) |
                                       ((uint32_t)__bfloat16_as_ushort(lo) << 16);
                 if (a.hdirect) {
-                    const int row = mt * 128 + wq * 32 + lane;
-                    if (row < p.tiles * p.b2) {
-                        uint4 *dst = a.hx + (((int64_t)bh * p.tiles * p.b2 + row) * key_slab(p) + up) * 2;
+                    const int row = qrow;
+                    if (row < p.tiles * p.b2 && up + sg < p.b1k) {
+                        uint4 *dst = a.hx + (((int64_t)bh * p.tiles * p.b2 + row) * key_slab(p) + up + sg) * 2;
                         dst[0] = make_uint4(pair, 0u, 0u, 0u);
                         dst[1] = make_uint4(0u, 0u, 0u, 0u);
                     }
@@ -1145,20 +1181,23 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                     // the warp's 32 panel rows (32 B each) leave in one TMA store,
                     // which clips the rows past t*b2; the previous item's store must
                     // have finished reading the staging first
-                    uint8_t *hs = sm + L::hstg(nmt) + wq * 1024;
+                    uint8_t *hs = sm + L::hstg(nmt, pack) + wq * 1024;
                     if (lane == 0) tma_store_wait_read_all();
                     __syncwarp();
                     *reinterpret_cast<uint4 *>(hs + lane * 32) = make_uint4(pair, 0u, 0u, 0u);
                     *reinterpret_cast<uint4 *>(hs + lane * 32 + 16) = make_uint4(0u, 0u, 0u, 0u);
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) {
-                        tma_store_4d(&tmHs, hs, 0, up, mt * 128 + wq * 32, bh);
+                    if (lane == 0) {   // the warp's 32 rows lie in one segment
+                        tma_store_4d(&tmHs, hs, 0, up + sg, mt * 128 + (wq * 32) % pseg, bh);
                         tma_store_commit();
                     }
                 }
             }
             const uint64_t inv2 = f2_pack(inv, inv);
+            // P of the PV MMA: K = pack * B2P bfloat16 values, packed in pairs from
+            // the buffer's first column; this row's segment holds R, the others zero
+            const uint32_t tP = tmem + lane_off + (i & 1) * 128;
 #pragma unroll
             for (int c = 0; c < B2P / 16; c++) {
                 uint32_t pk[8];
@@ -1168,7 +1207,14 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                     f2_unpack(f2_mul(pp[c * 8 + k], inv2), p0, p1);
                     pk[k] = pack_bf16(p0, p1);
                 }
-                tmem_st8(tS + c * 8, pk);
+                tmem_st8(tP + sg * (B2P / 2) + c * 8, pk);
+            }
+            if (pack > 1) {
+                uint32_t zk[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                for (int s2 = 0; s2 < pack; s2++)
+                    if (s2 != sg)
+#pragma unroll
+                        for (int c = 0; c < B2P / 16; c++) tmem_st8(tP + s2 * (B2P / 2) + c * 8, zk);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -1179,11 +1225,14 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
         // ---------------- epilogue: Z and Ktil rows -> bf16 -> staging -> TMA store
         const int wq = warp & 3;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-        uint8_t *stg = sm + L::stg(nmt) + wq * 8192;   // 2 panels x 32 rows x 128 B
+        uint8_t *stg = sm + L::stg(nmt, pack) + wq * 8192;   // 2 panels x 32 rows x 128 B
+        // the warp's 32 rows: segment sgw (block up + sgw), aggregated-query rows
+        // from mt * 128 + r0w
+        const int sgw = (wq * 32) / pseg, r0w = (wq * 32) % pseg;
         bool ok = true;
         for (int i = 0; ok && i < nitems; i++) {
             const int ib = i / nmt, mt = i % nmt;
-            const int fb = first + ib, bh = fb / p.b1k, up = fb % p.b1k;
+            const int fb = first + ib, bh = fb / a.gph, up = (fb % a.gph) * pack;
             for (int part = 0; part < 2; part++) {
                 if (!wait_warp(o_full + part, i & 1, w)) {
                     ok = false;
@@ -1225,7 +1274,7 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                     __syncwarp();
                     if (lane == 0) {
                         tma_store_5d(part == 0 ? &tmZs : &tmKs, stg + pn * 4096, 0,
-                                     mt * 128 + wq * 32, pn, up, bh);
+                                     mt * 128 + r0w, pn, up + sgw, bh);
                         tma_store_commit();
                     }
                 }
@@ -1309,15 +1358,26 @@ int b2_padded(int b2) { return (b2 + 15) / 16 * 16; }
 int qbar_tiles(const Problem &p) { return (p.tiles * p.b2 + 127) / 128; }
 size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-uint32_t rstep_smem(int b2p, int nmt, int hdirect) {
+uint32_t rstep_smem(int b2p, int nmt, int hdirect, int pack = 1) {
     switch (b2p) {
 #define MONARCH_RS_CASE(V) \
-    case V: return RsLayout<V>::smem(nmt, hdirect);
+    case V: return RsLayout<V>::smem(nmt, hdirect, pack);
         MONARCH_RS_CASE(16) MONARCH_RS_CASE(32) MONARCH_RS_CASE(48) MONARCH_RS_CASE(64)
         MONARCH_RS_CASE(80) MONARCH_RS_CASE(96) MONARCH_RS_CASE(112) MONARCH_RS_CASE(128)
 #undef MONARCH_RS_CASE
     }
     return 0xFFFFFFFFu;
+}
+
+// Blocks per R-step item with the shared aggregated queries of the first
+// iteration: 4 (2) when the t*b2 rows fit in a quarter (half) of the 128-row tile
+// and the stages of that many blocks fit in shared memory, else 1.  (t*b2 <= 64
+// implies b2 <= 64, so pack * B2P <= 128: the logits of a group fit one S buffer.)
+int rstep_pack(const Problem &p) {
+    const int rows = p.tiles * p.b2, b2p = b2_padded(p.b2);
+    int pack = rows <= 32 ? 4 : rows <= 64 ? 2 : 1;
+    while (pack > 1 && rstep_smem(b2p, 1, 1, pack) > (uint32_t)kMaxSmem) pack /= 2;
+    return pack;
 }
 
 struct TcWorkspace {
@@ -1360,7 +1420,7 @@ cudaError_t set_smem(K kernel, uint32_t bytes) {
 
 template <int B2P>
 cudaError_t launch_rstep(const CUtensorMap *maps, const RsArgs &a, int grid, cudaStream_t s) {
-    const uint32_t smem = RsLayout<B2P>::smem(a.nmt, a.hdirect);
+    const uint32_t smem = RsLayout<B2P>::smem(a.nmt, a.hdirect, a.pack);
     cudaError_t e = set_smem(tc_rstep_kernel<B2P>, smem);
     if (e != cudaSuccess) return e;
     tc_rstep_kernel<B2P><<<grid, 384, smem, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
@@ -1485,13 +1545,15 @@ cudaError_t run_rstep(const Problem &p, const TcWorkspace &ws, const void *k, co
         !make_map(&maps[3], ws.z, 5, dst, sst, bst) || !make_map(&maps[4], ws.ktil, 5, dst, sst, bst) ||
         !make_map(&maps[5], ws.hx, 4, dhx, shx, bhx, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    const int total = (p.head_end() - p.head_begin()) * p.b1k;
+    const int pack = qblk ? 1 : rstep_pack(p);
+    const int gph = (p.b1k + pack - 1) / pack;
+    const int total = (p.head_end() - p.head_begin()) * gph;
     const int sms = sm_count();
     const int bpc = (total + sms - 1) / sms;
     const int grid = (total + bpc - 1) / bpc;
-    const int hdirect = rstep_smem(b2p, nmt, 0) > (uint32_t)kMaxSmem ? 1 : 0;
+    const int hdirect = rstep_smem(b2p, nmt, 0, pack) > (uint32_t)kMaxSmem ? 1 : 0;
     RsArgs a{p, nmt, mpad, bpc, c_log2, 1.f / c_log2, qblk, hdirect, ws.hx, status, wait_limit,
-             stall};
+             stall, pack, gph};
     ProfileScope scope(K_TC_RSTEP, stream);
     switch (b2p) {
         case 16: return launch_rstep<16>(maps, a, grid, stream);
@@ -1573,7 +1635,7 @@ cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const 
         const int upb = p.key_tiles ? 1 : p.tiles;
         tc_qbar_kernel<<<(p.head_end() - p.head_begin()) * upb * nchunk, 128 * kQbarGroups, 0,
                          stream>>>(
-            (const __nv_bfloat16 *)q, ws.qbar, p, mpad);
+            (const __nv_bfloat16 *)q, ws.qbar, p, mpad, rstep_pack(p));
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

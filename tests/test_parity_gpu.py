@@ -104,6 +104,11 @@ TC_EDGES = [
     (10, 100, 16, 1000, 16, 1),  # 1000 query rows per tile: four pairs of query tiles
     (1, 65, 4, 65, 4, 2),        # 65 keys: a second 64-key half with one valid key
     (1, 129, 8, 129, 8, 3),      # 129 keys: the last 128-key chunk has a single half
+    # packed R-step tiles (t*b2 <= 64: two or four blocks per 128-row tile), with a
+    # head's last group of blocks only partly inside the head
+    (1, 9, 16, 9, 16, 1),        # 16 rows: four blocks per tile, 9 blocks = 4 + 4 + 1
+    (1, 7, 52, 7, 52, 1),        # 52 rows: two blocks per tile, 7 blocks = 2 + 2 + 2 + 1
+    (3, 5, 20, 15, 20, 3),       # 60 rows (three tiles of 20): two blocks per tile, 15 blocks
 ]
 
 
