@@ -436,7 +436,7 @@ size_t monarch_attn_bwd_workspace_bytes(int B, int H, int f, int h, int w, int d
         iters != 1)
         return 0;
     bool overflow = false;
-    const size_t n = backward_workspace_bytes(p, overflow);
+    const size_t n = backward_workspace_bytes(p, dtype, overflow);
     return overflow ? 0 : n;
 }
 
@@ -454,11 +454,12 @@ monarch_status monarch_attn_bwd_ws(const void *q, const void *k, const void *v, 
         !aligned16(dk) || !aligned16(dv) || ((uintptr_t)workspace & 255u))
         return MONARCH_ERR_ALIGN;
     bool overflow = false;
-    const size_t need = backward_workspace_bytes(p, overflow);
+    const size_t need = backward_workspace_bytes(p, dtype, overflow);
     if (overflow) return MONARCH_ERR_SHAPE;
     if (ws_bytes < need) return MONARCH_ERR_NO_MEMORY;
-    return generic_backward(p, dtype, q, k, v, dy, dq, dk, dv, workspace,
-                            (cudaStream_t)stream) == cudaSuccess
+    int *status = status_word_on_current_device();
+    return generic_backward(p, dtype, q, k, v, dy, dq, dk, dv, workspace, status,
+                            g_wait_limit.load(), (cudaStream_t)stream) == cudaSuccess
                ? MONARCH_OK
                : MONARCH_ERR_CUDA;
 }

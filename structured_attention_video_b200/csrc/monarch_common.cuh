@@ -200,6 +200,9 @@ size_t generic_workspace_bytes(const Problem &p, bool &overflow);
 GenericWorkspace generic_workspace_carve(const Problem &p, void *base);
 // S1 and the first R-step only (qbar, Ktil, Z, H into the workspace), for the
 // backward pass of one iteration.
+// S1 only: the float32 aggregated queries into ws.qbar.
+cudaError_t generic_qbar_only(const Problem &p, monarch_dtype dtype, const void *q,
+                              const GenericWorkspace &ws, cudaStream_t stream);
 cudaError_t generic_rstep_only(const Problem &p, monarch_dtype dtype, const void *q,
                                const void *k, const void *v, const GenericWorkspace &ws,
                                cudaStream_t stream);
@@ -213,10 +216,13 @@ struct BwdWorkspace {
     float *lsea, *ea, *rho;   // [BH][t][b2][b1k]  per R row: lse(a), E_R[a], sum R dR
     float *dqbar;         // [BH][t][b2][d]
 };
-size_t backward_workspace_bytes(const Problem &p, bool &overflow);
+size_t backward_workspace_bytes(const Problem &p, monarch_dtype dtype, bool &overflow);
+// status/wait_limit: the device status word and the poll limit of the bounded
+// waits (the tensor-core L-step side runs when `status` is given and it applies)
 cudaError_t generic_backward(const Problem &p, monarch_dtype dtype, const void *q, const void *k,
                              const void *v, const void *dy, void *dq, void *dk, void *dv,
-                             void *workspace, cudaStream_t stream);
+                             void *workspace, int *status, long long wait_limit,
+                             cudaStream_t stream);
 cudaError_t generic_forward(const Problem &p, monarch_dtype dtype, const void *q, const void *k,
                             const void *v, void *out, const GenericWorkspace &ws,
                             cudaStream_t stream);

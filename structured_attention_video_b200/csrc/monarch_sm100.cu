@@ -879,6 +879,10 @@ struct RsArgs {
     // segment s meets the keys of block u' + s (a block-diagonal mask on the logits)
     int pack;
     int gph;             // items (groups of `pack` blocks) per head
+    // 1: R enters [Z | Ktil] = R [V | K] as two bfloat16 parts, R_hi + R_lo with
+    // R_lo = R - R_hi rounded again (R to about 2^-16), in two passes of the TS
+    // MMAs (the backward's recompute of the forward uses it)
+    int split;
 };
 constexpr int kMaxQbarTiles = 4;   // slots of the per-block aggregated-query ring
 
@@ -1086,13 +1090,19 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 tc_fence_after();
                 // K = pack * B2P: the packed blocks' P columns (zero outside a row's
                 // own segment) against their V (then K) rows
-                for (int kk = 0; kk < (B2P / 16) * pack; kk++)
-                    mma_ts_warp(tmem + 256, pa + kk * 8, desc_plus(bz, kk * 2048), id2, kk > 0 ? 1u : 0u);
+                // with split R the low parts follow the high ones, nks * 8 columns on
+                const int nks = (B2P / 16) * pack, passes = a.split ? 2 : 1;
+                for (int ps = 0; ps < passes; ps++)
+                    for (int kk = 0; kk < nks; kk++)
+                        mma_ts_warp(tmem + 256, pa + (ps * nks + kk) * 8, desc_plus(bz, kk * 2048),
+                                    id2, (ps > 0 || kk > 0) ? 1u : 0u);
                 mma_commit_warp(o_full + 0);
                 if (i > 0 && !wait_warp(o_empty + 1, (i - 1) & 1, w)) break;
                 tc_fence_after();
-                for (int kk = 0; kk < (B2P / 16) * pack; kk++)
-                    mma_ts_warp(tmem + 384, pa + kk * 8, desc_plus(bk, kk * 2048), id2, kk > 0 ? 1u : 0u);
+                for (int ps = 0; ps < passes; ps++)
+                    for (int kk = 0; kk < nks; kk++)
+                        mma_ts_warp(tmem + 384, pa + (ps * nks + kk) * 8, desc_plus(bk, kk * 2048),
+                                    id2, (ps > 0 || kk > 0) ? 1u : 0u);
                 mma_commit_warp(o_full + 1);
                 mma_commit_warp(s_free + (i & 1));
                 if (mt == nmt - 1) mma_commit_warp(kv_empty + (ib & 1));
@@ -1198,23 +1208,30 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
             // P of the PV MMA: K = pack * B2P bfloat16 values, packed in pairs from
             // the buffer's first column; this row's segment holds R, the others zero
             const uint32_t tP = tmem + lane_off + (i & 1) * 128;
+            const uint32_t lo_off = (uint32_t)(pack * (B2P / 2));   // split R: the low parts
 #pragma unroll
             for (int c = 0; c < B2P / 16; c++) {
-                uint32_t pk[8];
+                uint32_t pk[8], pl[8];
 #pragma unroll
                 for (int k = 0; k < 8; k++) {
                     float p0, p1;
                     f2_unpack(f2_mul(pp[c * 8 + k], inv2), p0, p1);
                     pk[k] = pack_bf16(p0, p1);
+                    pl[k] = pack_bf16(p0 - __uint_as_float(pk[k] << 16),
+                                      p1 - __uint_as_float(pk[k] & 0xFFFF0000u));
                 }
                 tmem_st8(tP + sg * (B2P / 2) + c * 8, pk);
+                if (a.split) tmem_st8(tP + lo_off + sg * (B2P / 2) + c * 8, pl);
             }
             if (pack > 1) {
                 uint32_t zk[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
                 for (int s2 = 0; s2 < pack; s2++)
                     if (s2 != sg)
 #pragma unroll
-                        for (int c = 0; c < B2P / 16; c++) tmem_st8(tP + s2 * (B2P / 2) + c * 8, zk);
+                        for (int c = 0; c < B2P / 16; c++) {
+                            tmem_st8(tP + s2 * (B2P / 2) + c * 8, zk);
+                            if (a.split) tmem_st8(tP + lo_off + s2 * (B2P / 2) + c * 8, zk);
+                        }
             }
             tmem_wait_st();
             tc_fence_before();
@@ -1316,6 +1333,395 @@ __global__ void tc_keypad_kernel(__nv_bfloat16 *__restrict__ ktil, __nv_bfloat16
         } else {
             hx[(rid * slab + up) * 2 + (part - 32)] = part == 32 ? make_uint4(neg, 0u, 0u, 0u) : zero;
         }
+    }
+}
+
+// =====================================================================
+// Backward of the L-step and the output on the tensor cores (bfloat16, d = 128,
+// query-row tiles, one iteration).  Per (head, tile g, column v) problem, with
+// the forward's row statistic lam (S units, S = q.Ktil raw) and delta = dy.y:
+//   L = 2^((S + H' - lam) c_log2) (the L-step's probabilities), dP = dy.Z,
+//   dS = L (dP - delta)  (the gradient of the natural logits s q.Ktil + H),
+//   dZ = L^T dy,  dKtil = s dS^T q,  dH = sum over the tile's queries of dS,
+//   dq (the L-step's part) = s dS Ktil.
+// Two kernels, one 128-thread CTA per unit, one MMA stage at a time: the two
+// logit products go to tensor memory, the threads overwrite them in place with
+// the bfloat16 pairs of L and dS, and the accumulating products read those as
+// their tensor-memory A operand.
+//   tc_bwd_dkz_kernel: unit (bh, g, v, 128-key block); the key block's Ktil and Z
+//     (M side) against each 128-query tile of the tile (N side): S^T, dP^T, then
+//     dZ += L^T dy and dKtil += dS^T q over the query tiles; dH per key row.
+//   tc_bwd_dq_kernel<0>: unit (bh, g, v, 128-query tile); the queries and dy (M
+//     side) against each 128-key block: S, dP, and delta = sum L dP per query row
+//     (= dy.y, from the same products that form dS, so that every dS row sums to
+//     zero up to rounding).
+//   tc_bwd_dq_kernel<1>: the same units, then dq += dS Ktil over the blocks.
+// Every wait is bounded; on a time-out the CTA records MONARCH_ERR_TIMEOUT,
+// drains its own copies and MMAs, frees its tensor memory and returns.
+// =====================================================================
+namespace lb {
+constexpr uint32_t kT0 = 0, kT1 = kTile, kT2 = 2 * kTile, kT3 = 3 * kTile;   // four 128 x 128 tiles
+constexpr uint32_t kVec = 4 * kTile;             // 2 x 128 floats
+constexpr uint32_t kBar = kVec + 2 * 512;
+constexpr uint32_t kSmem = kBar + 64 + 1024;     // + slack to align the base to 1024
+}  // namespace lb
+
+struct LbArgs {
+    Problem p;
+    const uint4 *hx;        // entropy panels, one 32-byte row [H'_hi, H'_lo, 0...] per key row
+    const uint4 *lam;       // row statistics, one 32-byte row [-lam_hi, -lam_lo, 0...] per query
+    float *delta;           // [BH][N]: dy.y (written by tc_bwd_dq_kernel<0>)
+    float *dkt, *dz, *dh;   // [BH][t][b2][b1k] (x d): dKtil, dZ, dH
+    float *dql;             // [BH][N][d]: the L-step's part of dq
+    float c_log2;
+    int nkb;                // 128-key blocks per problem
+    int nqt;                // 128-query tiles per problem (of the largest tile)
+    int *status;
+    long long limit;
+};
+
+__device__ __forceinline__ float pair_sum(uint32_t pr) {   // hi + lo of a bfloat16 pair
+    return __uint_as_float(pr << 16) + __uint_as_float(pr & 0xFFFF0000u);
+}
+
+// Block-wide bounded wait: every thread polls, the CTA takes one decision.
+__device__ __forceinline__ bool wait_block(uint64_t *bar, uint32_t parity, const WaitCtx &w) {
+    const bool ok = wait_phase(bar, parity, w);
+    return __syncthreads_and(ok) != 0;
+}
+
+__global__ void __launch_bounds__(128, 1)
+tc_bwd_dkz_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDy,
+                  const __grid_constant__ CUtensorMap tmKt, const __grid_constant__ CUtensorMap tmZ,
+                  LbArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = align1024(smem_raw);
+    const Problem &p = a.p;
+    uint64_t *ld_bar = reinterpret_cast<uint64_t *>(sm + lb::kBar);
+    uint64_t *mma_bar = ld_bar + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ld_bar + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(ld_bar + 3);
+    float *lq = reinterpret_cast<float *>(sm + lb::kVec);   // lam of the query tile
+    float *dq_s = lq + 128;                                  // delta of the query tile
+    const int warp = threadIdx.x >> 5, j = threadIdx.x;
+
+    int unit = blockIdx.x;
+    const int kb = unit % a.nkb;
+    unit /= a.nkb;
+    const int v = unit % p.b2;
+    unit /= p.b2;
+    const int g = unit % p.tiles, bh = unit / p.tiles;
+    const int u_lo = tile_begin(g, p.b1, p.tiles), u_hi = tile_begin(g + 1, p.b1, p.tiles);
+    const int64_t krow0 = (((int64_t)bh * p.tiles + g) * p.b2 + v) * p.b1k + (int64_t)kb * 128;
+    const int nkv = min(128, p.b1k - kb * 128);
+    const int nqt = (u_hi - u_lo + 127) / 128;
+
+    if (threadIdx.x == 0) {
+        mbar_init(ld_bar, 1);
+        mbar_init(mma_bar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);   // this warp's lanes
+    const WaitCtx w{a.limit, a.status, abort_flag};
+    uint32_t ld_issued = 0, ld_done = 0, mma_issued = 0, mma_done = 0;
+
+    // the key block: Ktil and Z rows (128 blocks u' of row (g, v); past b1k: zeros)
+    if (threadIdx.x == 0) {
+        mbar_expect_tx(ld_bar, 2 * kTile);
+        for (int pn = 0; pn < 2; pn++) {
+            ls_load_kz(sm + lb::kT0 + pn * kPanel, &tmKt, pn, (int)krow0, p, ld_bar);
+            ls_load_kz(sm + lb::kT1 + pn * kPanel, &tmZ, pn, (int)krow0, p, ld_bar);
+        }
+    }
+    ld_issued++;
+    const bool key_ok = j < nkv;
+    const float hj = key_ok ? pair_sum(a.hx[(krow0 + j) * 2].x) : 0.f;
+    bool ok = wait_block(ld_bar, ld_done & 1, w);
+    if (ok) ld_done++;
+
+    const uint64_t dKt = smem_desc_sw128(smem_u32(sm + lb::kT0), 16, 1024);
+    const uint64_t dZk = smem_desc_sw128(smem_u32(sm + lb::kT1), 16, 1024);
+    const uint64_t dQk = smem_desc_sw128(smem_u32(sm + lb::kT2), 16, 1024);
+    const uint64_t dYk = smem_desc_sw128(smem_u32(sm + lb::kT3), 16, 1024);
+    const uint64_t dQm = smem_desc_sw128(smem_u32(sm + lb::kT2), kPanel, 1024);
+    const uint64_t dYm = smem_desc_sw128(smem_u32(sm + lb::kT3), kPanel, 1024);
+    constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0), idO = idesc_bf16(128, 128, 0, 1);
+    float dh_acc = 0.f;
+    for (int c = 0; ok && c < nqt; c++) {
+        const int u0 = u_lo + 128 * c, nqc = min(128, u_hi - u0);
+        if (threadIdx.x == 0) {
+            mbar_expect_tx(ld_bar, 2 * kTile);
+            for (int pn = 0; pn < 2; pn++) {
+                ls_load_q(sm + lb::kT2 + pn * kPanel, &tmQ, pn * 64, v, u0, bh, p, ld_bar);
+                ls_load_q(sm + lb::kT3 + pn * kPanel, &tmDy, pn * 64, v, u0, bh, p, ld_bar);
+            }
+        }
+        ld_issued++;
+        {   // the query tile's lam and delta (read after the block-wide wait below)
+            float lm = 0.f, dl = 0.f;
+            if (j < nqc) {
+                const int64_t tok = (int64_t)bh * p.N + (int64_t)(u0 + j) * p.b2 + v;
+                lm = -pair_sum(a.lam[tok * 2].x);
+                dl = a.delta[tok];
+            }
+            lq[j] = lm;
+            dq_s[j] = dl;
+        }
+        if (!(ok = wait_block(ld_bar, ld_done & 1, w))) break;
+        ld_done++;
+        if (warp == 0) {
+            tc_fence_after();
+            mma8_ss_k128(tmem, dKt, dQk, idS, 0u);          // S^T = Ktil q^T
+            mma8_ss_k128(tmem + 128, dZk, dYk, idS, 0u);    // dP^T = Z dy^T
+            mma_commit_warp(mma_bar);
+        }
+        mma_issued++;
+        if (!(ok = wait_block(mma_bar, mma_done & 1, w))) break;
+        mma_done++;
+        tc_fence_after();
+        // L^T and dS^T of this key row over the tile's queries, packed in place
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ch++) {
+            float s[32], d[32];
+            tmem_ld32f(tl + ch * 32, s);
+            tmem_ld32f(tl + 128 + ch * 32, d);
+            tmem_wait_ld();
+            uint32_t pk[16], dk[16];
+#pragma unroll
+            for (int k = 0; k < 32; k += 2) {
+                float pv[2], dv[2];
+#pragma unroll
+                for (int e = 0; e < 2; e++) {
+                    const int i = ch * 32 + k + e;
+                    const float pr = (key_ok && i < nqc)
+                                         ? fast_exp2((s[k + e] + hj - lq[i]) * a.c_log2) : 0.f;
+                    const float ds = pr * (d[k + e] - dq_s[i]);
+                    dh_acc += ds;
+                    pv[e] = pr;
+                    dv[e] = ds;
+                }
+                pk[k / 2] = pack_bf16(pv[0], pv[1]);
+                dk[k / 2] = pack_bf16(dv[0], dv[1]);
+            }
+            const uint32_t(&pk0)[8] = *reinterpret_cast<const uint32_t(*)[8]>(&pk[0]);
+            const uint32_t(&pk1)[8] = *reinterpret_cast<const uint32_t(*)[8]>(&pk[8]);
+            const uint32_t(&dk0)[8] = *reinterpret_cast<const uint32_t(*)[8]>(&dk[0]);
+            const uint32_t(&dk1)[8] = *reinterpret_cast<const uint32_t(*)[8]>(&dk[8]);
+            tmem_st8(tl + ch * 16, pk0);
+            tmem_st8(tl + ch * 16 + 8, pk1);
+            tmem_st8(tl + 128 + ch * 16, dk0);
+            tmem_st8(tl + 128 + ch * 16 + 8, dk1);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 0) {
+            tc_fence_after();
+            mma8_ts_mn128(tmem + 256, tmem, dYm, idO, c > 0 ? 1u : 0u);        // dZ += L^T dy
+            mma8_ts_mn128(tmem + 384, tmem + 128, dQm, idO, c > 0 ? 1u : 0u);  // += dS^T q
+            mma_commit_warp(mma_bar);
+        }
+        mma_issued++;
+        if (!(ok = wait_block(mma_bar, mma_done & 1, w))) break;
+        mma_done++;
+        tc_fence_after();
+    }
+    if (ok && nqt > 0) {
+        const int64_t krow = krow0 + j;
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ch++) {
+            float z[32], kt[32];
+            tmem_ld32f(tl + 256 + ch * 32, z);
+            tmem_ld32f(tl + 384 + ch * 32, kt);
+            tmem_wait_ld();
+            if (key_ok) {
+                float4 *oz = reinterpret_cast<float4 *>(a.dz + krow * kD + ch * 32);
+                float4 *ok4 = reinterpret_cast<float4 *>(a.dkt + krow * kD + ch * 32);
+#pragma unroll
+                for (int e = 0; e < 8; e++) {
+                    oz[e] = make_float4(z[4 * e], z[4 * e + 1], z[4 * e + 2], z[4 * e + 3]);
+                    ok4[e] = make_float4(kt[4 * e] * p.scale, kt[4 * e + 1] * p.scale,
+                                         kt[4 * e + 2] * p.scale, kt[4 * e + 3] * p.scale);
+                }
+            }
+        }
+        if (key_ok) a.dh[krow] = dh_acc;
+    }
+    // drain this CTA's own copies and MMAs before its tensor memory is freed
+    if (threadIdx.x == 0 && ld_issued > ld_done)
+        wait_phase_cleanup(ld_bar, (ld_issued - 1) & 1, kCleanupPolls);
+    if (warp == 0 && mma_issued > mma_done)
+        wait_phase_cleanup(mma_bar, (mma_issued - 1) & 1, kCleanupPolls);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(128, 1)
+tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDy,
+                 const __grid_constant__ CUtensorMap tmKt, const __grid_constant__ CUtensorMap tmZ,
+                 LbArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = align1024(smem_raw);
+    const Problem &p = a.p;
+    uint64_t *ld_bar = reinterpret_cast<uint64_t *>(sm + lb::kBar);
+    uint64_t *mma_bar = ld_bar + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ld_bar + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(ld_bar + 3);
+    float *hk = reinterpret_cast<float *>(sm + lb::kVec);   // H' of the key block
+    const int warp = threadIdx.x >> 5, j = threadIdx.x;
+
+    int unit = blockIdx.x;
+    const int c = unit % a.nqt;
+    unit /= a.nqt;
+    const int v = unit % p.b2;
+    unit /= p.b2;
+    const int g = unit % p.tiles, bh = unit / p.tiles;
+    const int u_lo = tile_begin(g, p.b1, p.tiles), u_hi = tile_begin(g + 1, p.b1, p.tiles);
+    const int u0 = u_lo + 128 * c, nqc = min(128, u_hi - u0);
+    if (nqc <= 0) return;   // a tile shorter than the longest one: no query tile c (uniform)
+    const int64_t slab0 = (((int64_t)bh * p.tiles + g) * p.b2 + v) * p.b1k;
+    const int64_t tok = (int64_t)bh * p.N + (int64_t)(u0 + j) * p.b2 + v;
+    const bool row_ok = j < nqc;
+    const float lam = row_ok ? -pair_sum(a.lam[tok * 2].x) : 0.f;
+    const float dlt = (MODE == 1 && row_ok) ? a.delta[tok] : 0.f;
+    float dsum = 0.f;   // MODE 0: sum over the keys of L dP
+
+    if (threadIdx.x == 0) {
+        mbar_init(ld_bar, 1);
+        mbar_init(mma_bar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const WaitCtx w{a.limit, a.status, abort_flag};
+    uint32_t ld_issued = 0, ld_done = 0, mma_issued = 0, mma_done = 0;
+
+    if (threadIdx.x == 0) {   // the query tile and its dy rows
+        mbar_expect_tx(ld_bar, 2 * kTile);
+        for (int pn = 0; pn < 2; pn++) {
+            ls_load_q(sm + lb::kT0 + pn * kPanel, &tmQ, pn * 64, v, u0, bh, p, ld_bar);
+            ls_load_q(sm + lb::kT1 + pn * kPanel, &tmDy, pn * 64, v, u0, bh, p, ld_bar);
+        }
+    }
+    ld_issued++;
+    bool ok = wait_block(ld_bar, ld_done & 1, w);
+    if (ok) ld_done++;
+
+    const uint64_t dQk = smem_desc_sw128(smem_u32(sm + lb::kT0), 16, 1024);
+    const uint64_t dYk = smem_desc_sw128(smem_u32(sm + lb::kT1), 16, 1024);
+    const uint64_t dKt = smem_desc_sw128(smem_u32(sm + lb::kT2), 16, 1024);
+    const uint64_t dZk = smem_desc_sw128(smem_u32(sm + lb::kT3), 16, 1024);
+    const uint64_t dKm = smem_desc_sw128(smem_u32(sm + lb::kT2), kPanel, 1024);
+    constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0), idO = idesc_bf16(128, 128, 0, 1);
+    for (int kb = 0; ok && kb < a.nkb; kb++) {
+        const int nkv = min(128, p.b1k - kb * 128);
+        if (threadIdx.x == 0) {
+            mbar_expect_tx(ld_bar, 2 * kTile);
+            for (int pn = 0; pn < 2; pn++) {
+                ls_load_kz(sm + lb::kT2 + pn * kPanel, &tmKt, pn, (int)(slab0 + kb * 128), p, ld_bar);
+                ls_load_kz(sm + lb::kT3 + pn * kPanel, &tmZ, pn, (int)(slab0 + kb * 128), p, ld_bar);
+            }
+        }
+        ld_issued++;
+        hk[j] = j < nkv ? pair_sum(a.hx[(slab0 + kb * 128 + j) * 2].x) : 0.f;
+        if (!(ok = wait_block(ld_bar, ld_done & 1, w))) break;
+        ld_done++;
+        if (warp == 0) {
+            tc_fence_after();
+            mma8_ss_k128(tmem, dQk, dKt, idS, 0u);          // S = q Ktil^T
+            mma8_ss_k128(tmem + 128, dYk, dZk, idS, 0u);    // dP = dy Z^T
+            mma_commit_warp(mma_bar);
+        }
+        mma_issued++;
+        if (!(ok = wait_block(mma_bar, mma_done & 1, w))) break;
+        mma_done++;
+        tc_fence_after();
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ch++) {
+            float s[32], d[32];
+            tmem_ld32f(tl + ch * 32, s);
+            tmem_ld32f(tl + 128 + ch * 32, d);
+            tmem_wait_ld();
+            uint32_t dk[16];
+#pragma unroll
+            for (int k = 0; k < 32; k += 2) {
+                float dv[2];
+#pragma unroll
+                for (int e = 0; e < 2; e++) {
+                    const int key = ch * 32 + k + e;
+                    const float pr = (row_ok && key < nkv)
+                                         ? fast_exp2((s[k + e] + hk[key] - lam) * a.c_log2) : 0.f;
+                    if (MODE == 0) dsum = fmaf(pr, d[k + e], dsum);
+                    dv[e] = pr * (d[k + e] - dlt);
+                }
+                dk[k / 2] = pack_bf16(dv[0], dv[1]);
+            }
+            if (MODE == 1) {
+                const uint32_t(&dk0)[8] = *reinterpret_cast<const uint32_t(*)[8]>(&dk[0]);
+                const uint32_t(&dk1)[8] = *reinterpret_cast<const uint32_t(*)[8]>(&dk[8]);
+                tmem_st8(tl + ch * 16, dk0);
+                tmem_st8(tl + ch * 16 + 8, dk1);
+            }
+        }
+        if (MODE == 0) {   // the next block's S and dP may overwrite this block's
+            tc_fence_before();
+            __syncthreads();
+            continue;
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 0) {
+            tc_fence_after();
+            mma8_ts_mn128(tmem + 256, tmem, dKm, idO, kb > 0 ? 1u : 0u);   // dq' += dS Ktil
+            mma_commit_warp(mma_bar);
+        }
+        mma_issued++;
+        if (!(ok = wait_block(mma_bar, mma_done & 1, w))) break;
+        mma_done++;
+        tc_fence_after();
+    }
+    if (ok && MODE == 0 && row_ok) a.delta[tok] = dsum;
+    if (ok && MODE == 1) {
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ch++) {
+            float o[32];
+            tmem_ld32f(tl + 256 + ch * 32, o);
+            tmem_wait_ld();
+            if (row_ok) {
+                float4 *dst = reinterpret_cast<float4 *>(a.dql + tok * kD + ch * 32);
+#pragma unroll
+                for (int e = 0; e < 8; e++)
+                    dst[e] = make_float4(o[4 * e] * p.scale, o[4 * e + 1] * p.scale,
+                                         o[4 * e + 2] * p.scale, o[4 * e + 3] * p.scale);
+            }
+        }
+    }
+    if (threadIdx.x == 0 && ld_issued > ld_done)
+        wait_phase_cleanup(ld_bar, (ld_issued - 1) & 1, kCleanupPolls);
+    if (warp == 0 && mma_issued > mma_done)
+        wait_phase_cleanup(mma_bar, (mma_issued - 1) & 1, kCleanupPolls);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -1525,7 +1931,7 @@ bool map_queries(CUtensorMap *m, const void *base, const Problem &p) {
 
 cudaError_t run_rstep(const Problem &p, const TcWorkspace &ws, const void *k, const void *v,
                       int qblk, float c_log2, int *status, long long wait_limit, int stall,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, int split = 0) {
     const int nmt = qbar_tiles(p), mpad = nmt * 128, b2p = b2_padded(p.b2);
     CUtensorMap maps[6];
     const uint64_t dq[2] = {(uint64_t)kD, qblk ? (uint64_t)p.BH * p.b1k * mpad : (uint64_t)p.BH * mpad};
@@ -1553,7 +1959,7 @@ cudaError_t run_rstep(const Problem &p, const TcWorkspace &ws, const void *k, co
     const int grid = (total + bpc - 1) / bpc;
     const int hdirect = rstep_smem(b2p, nmt, 0, pack) > (uint32_t)kMaxSmem ? 1 : 0;
     RsArgs a{p, nmt, mpad, bpc, c_log2, 1.f / c_log2, qblk, hdirect, ws.hx, status, wait_limit,
-             stall, pack, gph};
+             stall, pack, gph, split};
     ProfileScope scope(K_TC_RSTEP, stream);
     switch (b2p) {
         case 16: return launch_rstep<16>(maps, a, grid, stream);
@@ -1621,22 +2027,28 @@ cudaError_t run_lstep(const Problem &p, const TcWorkspace &ws, const void *q, vo
 
 }  // namespace
 
+namespace {
+
+// S1: the first R-step's aggregated queries (uniform L: plain means).
+cudaError_t run_qbar(const Problem &p, const void *q, const TcWorkspace &ws, cudaStream_t stream) {
+    const int nchunk = (p.b2 * kD / 8 + 127) / 128;
+    ProfileScope scope(K_TC_QBAR, stream);
+    const int upb = p.key_tiles ? 1 : p.tiles;
+    tc_qbar_kernel<<<(p.head_end() - p.head_begin()) * upb * nchunk, 128 * kQbarGroups, 0,
+                     stream>>>((const __nv_bfloat16 *)q, ws.qbar, p, qbar_tiles(p) * 128,
+                               rstep_pack(p));
+    return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const void *v,
                           void *out, void *workspace, int *status, long long wait_limit,
                           int stall, cudaStream_t stream) {
     const TcWorkspace ws = carve(p, workspace);
-    const int mpad = qbar_tiles(p) * 128;
     const float c_log2 = p.scale * kLog2e;
-
-    // S1: the first R-step's aggregated queries (uniform L: plain means)
     {
-        const int nchunk = (p.b2 * kD / 8 + 127) / 128;
-        ProfileScope scope(K_TC_QBAR, stream);
-        const int upb = p.key_tiles ? 1 : p.tiles;
-        tc_qbar_kernel<<<(p.head_end() - p.head_begin()) * upb * nchunk, 128 * kQbarGroups, 0,
-                         stream>>>(
-            (const __nv_bfloat16 *)q, ws.qbar, p, mpad, rstep_pack(p));
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = run_qbar(p, q, ws, stream);
         if (e != cudaSuccess) return e;
     }
     if (key_slab(p) > p.b1k) {   // key-column tiles: the padding rows of every slab
@@ -1659,6 +2071,55 @@ cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const 
     if (e == cudaSuccess)
         e = run_lstep(p, ws, q, out, kLsOut, c_log2, status, wait_limit, stall, stream);
     return e;
+}
+
+bool sm100_backward_supports(const Problem &p, monarch_dtype dtype) {
+    return p.iters == 1 && !p.key_tiles && p.layout == kLayoutBHND && p.b1k == p.b1 &&
+           p.unit_begin == 0 && p.unit_end == p.BH * p.tiles && sm100_supports(p, dtype);
+}
+
+size_t sm100_backward_workspace_bytes(const Problem &p, bool &overflow) {
+    const size_t fw = sm100_workspace_bytes(p, overflow);
+    const size_t nq = (size_t)p.BH * p.N;
+    return al256(fw) + al256(nq * 32);
+}
+
+cudaError_t sm100_backward_lstep(const Problem &p, const void *q, const void *k, const void *v,
+                                 const void *dy, void *workspace, float *delta, float *dkt,
+                                 float *dz, float *dh, float *dql, int *status,
+                                 long long wait_limit, cudaStream_t stream) {
+    bool overflow = false;
+    TcWorkspace ws = carve(p, workspace);
+    char *extra = (char *)workspace + al256(sm100_workspace_bytes(p, overflow));
+    ws.lam = (uint4 *)extra;   // [BH][N] rows of 32 bytes
+    const float c_log2 = p.scale * kLog2e;
+    // the forward on the tensor cores: q̄, the R-step (Ktil, Z, entropy panels), the
+    // L-step's row statistics lam and its output y
+    cudaError_t e = run_qbar(p, q, ws, stream);
+    if (e == cudaSuccess)   // R in two bfloat16 parts: Ktil and Z to about 2^-16 before storage
+        e = run_rstep(p, ws, k, v, 0, c_log2, status, wait_limit, 0, stream, 1);
+    if (e == cudaSuccess) e = run_lstep(p, ws, q, nullptr, kLsStat, c_log2, status, wait_limit, 0, stream);
+    if (e != cudaSuccess) return e;
+    CUtensorMap mq, mdy, mkt, mz;
+    const uint64_t rr = (uint64_t)p.tiles * p.b2, slab = (uint64_t)key_slab(p);
+    const uint64_t dkz[5] = {64, rr, 2, slab, (uint64_t)p.BH};
+    const uint64_t skz[4] = {128, rr * 128, 2 * rr * 128, slab * 2 * rr * 128};
+    const uint32_t bkz[5] = {64, 1, 1, 128, 1};
+    if (!map_queries(&mq, q, p) || !map_queries(&mdy, dy, p) ||
+        !make_map(&mkt, ws.ktil, 5, dkz, skz, bkz) || !make_map(&mz, ws.z, 5, dkz, skz, bkz))
+        return cudaErrorInvalidValue;
+    if ((e = set_smem(tc_bwd_dkz_kernel, lb::kSmem)) != cudaSuccess ||
+        (e = set_smem(tc_bwd_dq_kernel<0>, lb::kSmem)) != cudaSuccess ||
+        (e = set_smem(tc_bwd_dq_kernel<1>, lb::kSmem)) != cudaSuccess)
+        return e;
+    LbArgs a{p, ws.hx, ws.lam, delta, dkt, dz, dh, dql, c_log2, (p.b1k + 127) / 128,
+             (tile_max_rows(p.b1, p.tiles) + 127) / 128, status, wait_limit};
+    const int64_t probs = (int64_t)p.BH * p.tiles * p.b2;
+    ProfileScope scope(K_BWD_L, stream);
+    tc_bwd_dq_kernel<0><<<(unsigned)(probs * a.nqt), 128, lb::kSmem, stream>>>(mq, mdy, mkt, mz, a);
+    tc_bwd_dkz_kernel<<<(unsigned)(probs * a.nkb), 128, lb::kSmem, stream>>>(mq, mdy, mkt, mz, a);
+    tc_bwd_dq_kernel<1><<<(unsigned)(probs * a.nqt), 128, lb::kSmem, stream>>>(mq, mdy, mkt, mz, a);
+    return cudaGetLastError();
 }
 
 }  // namespace monarch
