@@ -18,7 +18,8 @@
 //     dv_(u',v') += sum_(g,v) R dZ
 //   Aggregation: dq_(u,v) += dqbar[g][v] / |T_g|.
 //
-// SIMT kernels with float32 arithmetic for every supported shape and dtype.
+// SIMT kernels with float32 arithmetic for every supported shape and dtype
+// (bfloat16 with d = 128 takes the tensor-core backward of monarch_sm100.cu).
 // Each gradient element is written by exactly one warp (no atomics): the
 // kernels are deterministic.  One warp per row; a CTA of GW warps shares chunks
 // of KC rows staged in shared memory (rows padded to d+1 floats).
@@ -566,12 +567,10 @@ cudaError_t smem_opt_in(K kernel, size_t bytes) {
                : cudaSuccess;
 }
 
-// lside = false: the L-step's gradients (dql, dkt, dz, dh) are already in the
-// workspace (the tensor-core kernels computed them); only the R-step side runs.
 template <typename T, int D>
 cudaError_t run_backward(const Problem &p, const T *q, const T *k, const T *v, const T *dy,
                          T *dq, T *dk, T *dv, const GenericWorkspace &fw, const BwdWorkspace &bw,
-                         bool lside, cudaStream_t stream) {
+                         cudaStream_t stream) {
     constexpr int DS = D + 1;
     const size_t sm_ls = (GW * D + 2 * KC * DS + KC) * sizeof(float);
     const size_t sm_ldq = (2 * GW * D + 2 * KC * DS + KC) * sizeof(float);
@@ -593,7 +592,7 @@ cudaError_t run_backward(const Problem &p, const T *q, const T *k, const T *v, c
     const unsigned rs_blocks = (unsigned)(units * p.b1k * ((p.b2 + GW - 1) / GW));
     const unsigned rq_blocks = (unsigned)(units * ((p.b2 + GW - 1) / GW));
     const unsigned kv_blocks = (unsigned)((int64_t)p.BH * p.b1k * ((p.b2 + GW - 1) / GW));
-    if (lside) {
+    {
         ProfileScope scope(K_BWD_L, stream);
         bwd_lstats_kernel<T, D><<<q_blocks, GW * 32, sm_ls, stream>>>(
             q, dy, fw.ktil, fw.z, fw.hent, bw.lse, bw.delta, p);
@@ -620,27 +619,15 @@ cudaError_t run_backward(const Problem &p, const T *q, const T *k, const T *v, c
 template <typename T>
 cudaError_t dispatch_bwd(const Problem &p, const void *q, const void *k, const void *v,
                          const void *dy, void *dq, void *dk, void *dv,
-                         const GenericWorkspace &fw, const BwdWorkspace &bw, bool lside,
-                         cudaStream_t s) {
+                         const GenericWorkspace &fw, const BwdWorkspace &bw, cudaStream_t s) {
     const T *qq = (const T *)q, *kk = (const T *)k, *vv = (const T *)v, *gg = (const T *)dy;
     T *a = (T *)dq, *b = (T *)dk, *c = (T *)dv;
     switch (p.d) {
-        case 32: return run_backward<T, 32>(p, qq, kk, vv, gg, a, b, c, fw, bw, lside, s);
-        case 64: return run_backward<T, 64>(p, qq, kk, vv, gg, a, b, c, fw, bw, lside, s);
-        case 128: return run_backward<T, 128>(p, qq, kk, vv, gg, a, b, c, fw, bw, lside, s);
+        case 32: return run_backward<T, 32>(p, qq, kk, vv, gg, a, b, c, fw, bw, s);
+        case 64: return run_backward<T, 64>(p, qq, kk, vv, gg, a, b, c, fw, bw, s);
+        case 128: return run_backward<T, 128>(p, qq, kk, vv, gg, a, b, c, fw, bw, s);
         default: return cudaErrorInvalidValue;
     }
-}
-
-// The forward quantities the backward keeps in the generic layout: everything
-// (generic L-step side), or only the float32 aggregated queries (the tensor-core
-// L-step side, whose own forward intermediates follow the backward's arrays).
-size_t fwd_part_bytes(const Problem &p, bool tc, bool &overflow) {
-    if (tc) {
-        overflow = false;
-        return a256((size_t)p.BH * p.tiles * p.b2 * p.d * 4);
-    }
-    return generic_workspace_bytes(p, overflow);
 }
 
 size_t bwd_arrays_bytes(const Problem &p) {
@@ -654,28 +641,16 @@ size_t bwd_arrays_bytes(const Problem &p) {
 }  // namespace
 
 size_t backward_workspace_bytes(const Problem &p, monarch_dtype dtype, bool &overflow) {
-    const bool tc = sm100_backward_supports(p, dtype);
-    const size_t fwd = fwd_part_bytes(p, tc, overflow);
+    if (sm100_backward_supports(p, dtype)) return sm100_backward_workspace_bytes(p, overflow);
+    const size_t fwd = generic_workspace_bytes(p, overflow);
     if (overflow) return 0;
-    size_t extra = 0;
-    if (tc) {
-        extra = sm100_backward_workspace_bytes(p, overflow);
-        if (overflow) return 0;
-    }
-    return fwd + bwd_arrays_bytes(p) + extra;
+    return fwd + bwd_arrays_bytes(p);
 }
 
-BwdWorkspace backward_workspace_carve(const Problem &p, bool tc, void *base, GenericWorkspace &fw,
-                                      void **tc_base) {
+BwdWorkspace backward_workspace_carve(const Problem &p, void *base, GenericWorkspace &fw) {
     bool overflow = false;
-    if (tc) {
-        fw = GenericWorkspace{};
-        fw.qbar = (float *)base;
-    } else {
-        fw = generic_workspace_carve(p, base);
-    }
-    char *c = (char *)base + fwd_part_bytes(p, tc, overflow);
-    *tc_base = tc ? c + bwd_arrays_bytes(p) : nullptr;
+    fw = generic_workspace_carve(p, base);
+    char *c = (char *)base + generic_workspace_bytes(p, overflow);
     const size_t td = (size_t)p.BH * p.tiles * p.Nk * p.d;
     const size_t tr = (size_t)p.BH * p.tiles * p.Nk;
     const size_t nq = (size_t)p.BH * p.N;
@@ -698,27 +673,18 @@ cudaError_t generic_backward(const Problem &p, monarch_dtype dtype, const void *
                              void *workspace, int *status, long long wait_limit,
                              cudaStream_t stream) {
     // the workspace was sized for the same choice (backward_workspace_bytes)
-    const bool tc = sm100_backward_supports(p, dtype);
-    if (tc && status == nullptr) return cudaErrorInvalidValue;
-    GenericWorkspace fw;
-    void *tc_ws = nullptr;
-    BwdWorkspace bw = backward_workspace_carve(p, tc, workspace, fw, &tc_ws);
-    cudaError_t e;
-    if (tc) {
-        // the L-step side on the tensor cores (its own forward intermediates), and
-        // the float32 aggregated queries that the R-step side reads
-        e = generic_qbar_only(p, dtype, q, fw, stream);
-        if (e == cudaSuccess)
-            e = sm100_backward_lstep(p, q, k, v, dy, tc_ws, bw.delta, bw.dkt, bw.dz, bw.dh,
-                                     bw.dql, status, wait_limit, stream);
-    } else {
-        // the forward quantities the backward reads: qbar, Ktil, Z and H of the R-step
-        e = generic_rstep_only(p, dtype, q, k, v, fw, stream);
+    if (sm100_backward_supports(p, dtype)) {
+        if (status == nullptr) return cudaErrorInvalidValue;
+        return sm100_backward(p, q, k, v, dy, dq, dk, dv, workspace, status, wait_limit, stream);
     }
+    GenericWorkspace fw;
+    BwdWorkspace bw = backward_workspace_carve(p, workspace, fw);
+    // the forward quantities the backward reads: qbar, Ktil, Z and H of the R-step
+    cudaError_t e = generic_rstep_only(p, dtype, q, k, v, fw, stream);
     if (e != cudaSuccess) return e;
     if (dtype == MONARCH_F32)
-        return dispatch_bwd<float>(p, q, k, v, dy, dq, dk, dv, fw, bw, !tc, stream);
-    return dispatch_bwd<__nv_bfloat16>(p, q, k, v, dy, dq, dk, dv, fw, bw, !tc, stream);
+        return dispatch_bwd<float>(p, q, k, v, dy, dq, dk, dv, fw, bw, stream);
+    return dispatch_bwd<__nv_bfloat16>(p, q, k, v, dy, dq, dk, dv, fw, bw, stream);
 }
 
 }  // namespace monarch

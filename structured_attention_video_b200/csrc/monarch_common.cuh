@@ -200,9 +200,6 @@ size_t generic_workspace_bytes(const Problem &p, bool &overflow);
 GenericWorkspace generic_workspace_carve(const Problem &p, void *base);
 // S1 and the first R-step only (qbar, Ktil, Z, H into the workspace), for the
 // backward pass of one iteration.
-// S1 only: the float32 aggregated queries into ws.qbar.
-cudaError_t generic_qbar_only(const Problem &p, monarch_dtype dtype, const void *q,
-                              const GenericWorkspace &ws, cudaStream_t stream);
 cudaError_t generic_rstep_only(const Problem &p, monarch_dtype dtype, const void *q,
                                const void *k, const void *v, const GenericWorkspace &ws,
                                cudaStream_t stream);

@@ -438,19 +438,6 @@ cudaError_t generic_forward(const Problem &p, monarch_dtype dtype, const void *q
     return dispatch_d<__nv_bfloat16>(p, q, k, v, out, ws, stream);
 }
 
-cudaError_t generic_qbar_only(const Problem &p, monarch_dtype dtype, const void *q,
-                              const GenericWorkspace &ws, cudaStream_t stream) {
-    const int64_t nmean = (int64_t)(p.unit_end - p.unit_begin) * p.b2 * p.d;
-    const int blocks = (int)((nmean + 255) / 256 < 148 * 64 ? (nmean + 255) / 256 : 148 * 64);
-    ProfileScope scope(K_QBAR_MEAN, stream);
-    if (dtype == MONARCH_F32)
-        qbar_mean_kernel<float><<<blocks, 256, 0, stream>>>((const float *)q, ws.qbar, p);
-    else
-        qbar_mean_kernel<__nv_bfloat16><<<blocks, 256, 0, stream>>>((const __nv_bfloat16 *)q,
-                                                                    ws.qbar, p);
-    return cudaGetLastError();
-}
-
 cudaError_t generic_rstep_only(const Problem &p, monarch_dtype dtype, const void *q,
                                const void *k, const void *v, const GenericWorkspace &ws,
                                cudaStream_t stream) {

@@ -15,18 +15,18 @@ cudaError_t sm100_forward(const Problem &p, const void *q, const void *k, const 
                           void *out, void *workspace, int *status, long long wait_limit,
                           int stall, cudaStream_t stream);
 
-// The backward of the L-step and the output on the tensor cores: bfloat16,
-// d = 128, [B][H][N][d], self-attention, query-row tiles, one iteration.
+// The backward pass on the tensor cores: bfloat16, d = 128, [B][H][N][d],
+// self-attention, query-row tiles, one iteration.
 bool sm100_backward_supports(const Problem &p, monarch_dtype dtype);
-// Its workspace: the forward's tensor-core intermediates and the row statistics.
+// Its workspace: the forward's tensor-core intermediates, the row statistics and
+// the intermediate gradients.
 size_t sm100_backward_workspace_bytes(const Problem &p, bool &overflow);
-// Runs the forward's q̄, R-step (R in two bfloat16 parts) and the L-step's row
-// statistics on the tensor cores, then delta = dy.y (as sum L dP), the gradients
-// dKtil, dZ, dH (float32, [BH][t][b2][b1] rows) and the L-step's part of dq
-// (float32 [BH][N][d]).
-cudaError_t sm100_backward_lstep(const Problem &p, const void *q, const void *k, const void *v,
-                                 const void *dy, void *workspace, float *delta, float *dkt,
-                                 float *dz, float *dh, float *dql, int *status,
-                                 long long wait_limit, cudaStream_t stream);
+// The forward's q̄, R-step (R in two bfloat16 parts) and L-step row statistics on
+// the tensor cores; then the L-step side (delta as sum L dP, dKtil, dZ, dH, the
+// L-step's part of dq) and the R-step side (dk, dv, the partial sums of dq̄), and
+// dq = dq_L + dq̄ / |T_g|.  dq, dk, dv: bfloat16 [B][H][N][d].
+cudaError_t sm100_backward(const Problem &p, const void *q, const void *k, const void *v,
+                           const void *dy, void *dq, void *dk, void *dv, void *workspace,
+                           int *status, long long wait_limit, cudaStream_t stream);
 
 }  // namespace monarch
