@@ -284,11 +284,14 @@ MONARCH_API monarch_status monarch_attn_fwd_kv_ws(const void *q, const void *k, 
  * aggregation (qbar = mean of the tile's queries).
  *   q, k, v, dy   device pointers, [B][H][N][d] in `dtype`, read only.
  *   dq, dk, dv    device pointers, [B][H][N][d] in `dtype`, fully overwritten.
- * Other arguments as monarch_attn_fwd.  The generic float32 kernels run for every
- * supported shape and dtype (recomputing the forward's R-step); each gradient
- * element is written by one warp, so results are deterministic.  The workspace
+ * Other arguments as monarch_attn_fwd.  Where the forward takes the tensor-core
+ * kernels (bfloat16, d = 128; monarch_attn_path = 1) the backward does too: it
+ * recomputes the forward's intermediates on the tensor cores and forms every
+ * gradient with tcgen05 products (bfloat16 operands, float32 accumulation).  Every
+ * other shape and dtype runs on generic float32 kernels.  Both are deterministic
+ * (no atomics; reductions in a fixed order).  The workspace
  * (monarch_attn_bwd_workspace_bytes, 0 if the arguments fail validation or
- * iters != 1) holds the forward intermediates and the backward's, all float32.
+ * iters != 1) holds the forward intermediates and the backward's.
  * monarch_attn_bwd takes it with cudaMallocAsync on `stream`; monarch_attn_bwd_ws
  * uses the caller's (256-byte aligned; MONARCH_ERR_NO_MEMORY if too small).
  * Source: the pages print no backward; they finetune through the attention
