@@ -838,7 +838,9 @@ struct RsLayout {
     }
 };
 
-template <int B2P>
+// SPLIT (the backward's recompute): R enters the TS products as R_hi + R_lo.  A
+// template parameter, so that the forward's kernel carries none of it.
+template <int B2P, int SPLIT>
 __global__ void __launch_bounds__(384, 1)
 tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmZs,
@@ -1020,19 +1022,23 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 tc_fence_after();
                 // K = pack * B2P: the packed blocks' P columns (zero outside a row's
                 // own segment) against their V (then K) rows
-                // with split R the low parts follow the high ones, nks * 8 columns on
-                const int nks = (B2P / 16) * pack, passes = a.split ? 2 : 1;
-                for (int ps = 0; ps < passes; ps++)
+                for (int kk = 0; kk < (B2P / 16) * pack; kk++)
+                    mma_ts_warp(tmem + 256, pa + kk * 8, desc_plus(bz, kk * 2048), id2, kk > 0 ? 1u : 0u);
+                if constexpr (SPLIT != 0) {   // the low parts, (B2P / 16) * pack * 8 columns on
+                    const int nks = (B2P / 16) * pack;
                     for (int kk = 0; kk < nks; kk++)
-                        mma_ts_warp(tmem + 256, pa + (ps * nks + kk) * 8, desc_plus(bz, kk * 2048),
-                                    id2, (ps > 0 || kk > 0) ? 1u : 0u);
+                        mma_ts_warp(tmem + 256, pa + (nks + kk) * 8, desc_plus(bz, kk * 2048), id2, 1u);
+                }
                 mma_commit_warp(o_full + 0);
                 if (i > 0 && !wait_warp(o_empty + 1, (i - 1) & 1, w)) break;
                 tc_fence_after();
-                for (int ps = 0; ps < passes; ps++)
+                for (int kk = 0; kk < (B2P / 16) * pack; kk++)
+                    mma_ts_warp(tmem + 384, pa + kk * 8, desc_plus(bk, kk * 2048), id2, kk > 0 ? 1u : 0u);
+                if constexpr (SPLIT != 0) {
+                    const int nks = (B2P / 16) * pack;
                     for (int kk = 0; kk < nks; kk++)
-                        mma_ts_warp(tmem + 384, pa + (ps * nks + kk) * 8, desc_plus(bk, kk * 2048),
-                                    id2, (ps > 0 || kk > 0) ? 1u : 0u);
+                        mma_ts_warp(tmem + 384, pa + (nks + kk) * 8, desc_plus(bk, kk * 2048), id2, 1u);
+                }
                 mma_commit_warp(o_full + 1);
                 mma_commit_warp(s_free + (i & 1));
                 if (mt == nmt - 1) mma_commit_warp(kv_empty + (ib & 1));
@@ -1138,25 +1144,29 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
             // P of the PV MMA: K = pack * B2P bfloat16 values, packed in pairs from
             // the buffer's first column; this row's segment holds R, the others zero
             const uint32_t tP = tmem + lane_off + (i & 1) * 128;
-            const uint32_t lo_off = (uint32_t)(pack * (B2P / 2));   // split R: the low parts
 #pragma unroll
             for (int c = 0; c < B2P / 16; c++) {
                 uint32_t pk[8];
-                float pf[16];
+                if constexpr (SPLIT == 0) {
 #pragma unroll
-                for (int k = 0; k < 8; k++) {
-                    f2_unpack(f2_mul(pp[c * 8 + k], inv2), pf[2 * k], pf[2 * k + 1]);
-                    pk[k] = pack_bf16(pf[2 * k], pf[2 * k + 1]);
-                }
-                tmem_st8(tP + sg * (B2P / 2) + c * 8, pk);
-                if (a.split) {   // R_lo = R - R_hi, rounded again
+                    for (int k = 0; k < 8; k++) {
+                        float p0, p1;
+                        f2_unpack(f2_mul(pp[c * 8 + k], inv2), p0, p1);
+                        pk[k] = pack_bf16(p0, p1);
+                    }
+                } else {   // R_lo = R - R_hi, rounded again, pack * B2P / 2 columns on
                     uint32_t pl[8];
 #pragma unroll
-                    for (int k = 0; k < 8; k++)
-                        pl[k] = pack_bf16(pf[2 * k] - __uint_as_float(pk[k] << 16),
-                                          pf[2 * k + 1] - __uint_as_float(pk[k] & 0xFFFF0000u));
-                    tmem_st8(tP + lo_off + sg * (B2P / 2) + c * 8, pl);
+                    for (int k = 0; k < 8; k++) {
+                        float p0, p1;
+                        f2_unpack(f2_mul(pp[c * 8 + k], inv2), p0, p1);
+                        pk[k] = pack_bf16(p0, p1);
+                        pl[k] = pack_bf16(p0 - __uint_as_float(pk[k] << 16),
+                                          p1 - __uint_as_float(pk[k] & 0xFFFF0000u));
+                    }
+                    tmem_st8(tP + pack * (B2P / 2) + sg * (B2P / 2) + c * 8, pl);
                 }
+                tmem_st8(tP + sg * (B2P / 2) + c * 8, pk);
             }
             if (pack > 1) {
                 uint32_t zk[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
@@ -1165,7 +1175,8 @@ tc_rstep_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
 #pragma unroll
                         for (int c = 0; c < B2P / 16; c++) {
                             tmem_st8(tP + s2 * (B2P / 2) + c * 8, zk);
-                            if (a.split) tmem_st8(tP + lo_off + s2 * (B2P / 2) + c * 8, zk);
+                            if constexpr (SPLIT != 0)
+                                tmem_st8(tP + pack * (B2P / 2) + s2 * (B2P / 2) + c * 8, zk);
                         }
             }
             tmem_wait_st();
@@ -1357,10 +1368,17 @@ TcWorkspace carve(const Problem &p, void *base) {
 template <int B2P>
 cudaError_t launch_rstep(const CUtensorMap *maps, const RsArgs &a, int grid, cudaStream_t s) {
     const uint32_t smem = RsLayout<B2P>::smem(a.nmt, a.hdirect, a.pack);
-    cudaError_t e = set_smem(tc_rstep_kernel<B2P>, smem);
-    if (e != cudaSuccess) return e;
-    tc_rstep_kernel<B2P><<<grid, 384, smem, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
-                                                   maps[5], a);
+    if (a.split) {
+        cudaError_t e = set_smem(tc_rstep_kernel<B2P, 1>, smem);
+        if (e != cudaSuccess) return e;
+        tc_rstep_kernel<B2P, 1><<<grid, 384, smem, s>>>(maps[0], maps[1], maps[2], maps[3],
+                                                          maps[4], maps[5], a);
+    } else {
+        cudaError_t e = set_smem(tc_rstep_kernel<B2P, 0>, smem);
+        if (e != cudaSuccess) return e;
+        tc_rstep_kernel<B2P, 0><<<grid, 384, smem, s>>>(maps[0], maps[1], maps[2], maps[3],
+                                                          maps[4], maps[5], a);
+    }
     return cudaGetLastError();
 }
 
