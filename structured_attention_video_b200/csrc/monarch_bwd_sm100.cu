@@ -39,10 +39,13 @@ using namespace tcs;
 // drains its own copies and MMAs, frees its tensor memory and returns.
 // =====================================================================
 namespace lb {
-constexpr uint32_t kT0 = 0, kT1 = kTile, kT2 = 2 * kTile, kT3 = 3 * kTile;   // four 128 x 128 tiles
-constexpr uint32_t kVec = 4 * kTile;             // 2 x 128 floats
-constexpr uint32_t kBar = kVec + 2 * 512;
-constexpr uint32_t kSmem = kBar + 64 + 1024;     // + slack to align the base to 1024
+// six 128 x 128 bfloat16 tiles: the operands loaded once (T0, T1) and two buffers of
+// the ones loaded per step (T2, T3 and T4, T5), so that step i + 1's copies overlap
+// step i's products and elementwise work
+__host__ __device__ constexpr uint32_t tile(int i) { return (uint32_t)i * kTile; }
+constexpr uint32_t kVec = 6 * kTile;             // 4 x 128 floats
+constexpr uint32_t kBar = kVec + 4 * 512;
+constexpr uint32_t kSmem = kBar + 128 + 1024;    // + slack to align the base to 1024
 }  // namespace lb
 
 struct LbArgs {
@@ -79,12 +82,12 @@ tc_bwd_dkz_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     const Problem &p = a.p;
-    uint64_t *ld_bar = reinterpret_cast<uint64_t *>(sm + lb::kBar);
-    uint64_t *mma_bar = ld_bar + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ld_bar + 2);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(ld_bar + 3);
-    float *lq = reinterpret_cast<float *>(sm + lb::kVec);   // lam of the query tile
-    float *dq_s = lq + 128;                                  // delta of the query tile
+    uint64_t *kz_bar = reinterpret_cast<uint64_t *>(sm + lb::kBar);
+    uint64_t *qb_bar = kz_bar + 1;    // [2]: query tile buffers
+    uint64_t *mma_bar = kz_bar + 3;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(kz_bar + 4);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(kz_bar + 5);
+    float *vec = reinterpret_cast<float *>(sm + lb::kVec);   // [buffer][lam | delta][128]
     const int warp = threadIdx.x >> 5, j = threadIdx.x;
 
     int unit = blockIdx.x;
@@ -99,8 +102,7 @@ tc_bwd_dkz_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const int nqt = (u_hi - u_lo + 127) / 128;
 
     if (threadIdx.x == 0) {
-        mbar_init(ld_bar, 1);
-        mbar_init(mma_bar, 1);
+        for (int i = 0; i < 4; i++) mbar_init(kz_bar + i, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -111,56 +113,63 @@ tc_bwd_dkz_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const uint32_t tmem = *tmem_slot;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);   // this warp's lanes
     const WaitCtx w{a.limit, a.status, abort_flag};
-    uint32_t ld_issued = 0, ld_done = 0, mma_issued = 0, mma_done = 0;
+    uint32_t kz_issued = 0, kz_done = 0, mma_issued = 0, mma_done = 0;
+    uint32_t qb_issued[2] = {0, 0}, qb_done[2] = {0, 0};
 
-    // the key block: Ktil and Z rows (128 blocks u' of row (g, v); past b1k: zeros)
+    // query tile cc into buffer b: its q and dy rows (thread 0), its lam and delta
+    auto stage_q = [&](int cc, int b) {
+        const int u0 = u_lo + 128 * cc, nqc = min(128, u_hi - u0);
+        if (threadIdx.x == 0) {
+            mbar_expect_tx(qb_bar + b, 2 * kTile);
+            for (int pn = 0; pn < 2; pn++) {
+                ls_load_q(sm + lb::tile(2 + 2 * b) + pn * kPanel, &tmQ, pn * 64, v, u0, bh, p,
+                          qb_bar + b);
+                ls_load_q(sm + lb::tile(3 + 2 * b) + pn * kPanel, &tmDy, pn * 64, v, u0, bh, p,
+                          qb_bar + b);
+            }
+        }
+        qb_issued[b]++;
+        float lm = 0.f, dl = 0.f;
+        if (j < nqc) {
+            const int64_t tok = (int64_t)bh * p.N + (int64_t)(u0 + j) * p.b2 + v;
+            lm = -pair_sum(a.lam[tok * 2].x);
+            dl = a.delta[tok];
+        }
+        vec[b * 256 + j] = lm;
+        vec[b * 256 + 128 + j] = dl;
+    };
+
+    // the key block: Ktil and Z rows (128 blocks u' of row (g, v); past b1k: zeros),
+    // then the first two query tiles
     if (threadIdx.x == 0) {
-        mbar_expect_tx(ld_bar, 2 * kTile);
+        mbar_expect_tx(kz_bar, 2 * kTile);
         for (int pn = 0; pn < 2; pn++) {
-            ls_load_kz(sm + lb::kT0 + pn * kPanel, &tmKt, pn, (int)krow0, p, ld_bar);
-            ls_load_kz(sm + lb::kT1 + pn * kPanel, &tmZ, pn, (int)krow0, p, ld_bar);
+            ls_load_kz(sm + lb::tile(0) + pn * kPanel, &tmKt, pn, (int)krow0, p, kz_bar);
+            ls_load_kz(sm + lb::tile(1) + pn * kPanel, &tmZ, pn, (int)krow0, p, kz_bar);
         }
     }
-    ld_issued++;
+    kz_issued++;
+    stage_q(0, 0);
+    if (nqt > 1) stage_q(1, 1);
     const bool key_ok = j < nkv;
     const float hj = key_ok ? pair_sum(a.hx[(krow0 + j) * 2].x) : 0.f;
-    bool ok = wait_block(ld_bar, ld_done & 1, w);
-    if (ok) ld_done++;
+    bool ok = wait_block(kz_bar, 0, w);
+    if (ok) kz_done++;
 
-    const uint64_t dKt = smem_desc_sw128(smem_u32(sm + lb::kT0), 16, 1024);
-    const uint64_t dZk = smem_desc_sw128(smem_u32(sm + lb::kT1), 16, 1024);
-    const uint64_t dQk = smem_desc_sw128(smem_u32(sm + lb::kT2), 16, 1024);
-    const uint64_t dYk = smem_desc_sw128(smem_u32(sm + lb::kT3), 16, 1024);
-    const uint64_t dQm = smem_desc_sw128(smem_u32(sm + lb::kT2), kPanel, 1024);
-    const uint64_t dYm = smem_desc_sw128(smem_u32(sm + lb::kT3), kPanel, 1024);
+    const uint64_t dKt = smem_desc_sw128(smem_u32(sm + lb::tile(0)), 16, 1024);
+    const uint64_t dZk = smem_desc_sw128(smem_u32(sm + lb::tile(1)), 16, 1024);
     constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0), idO = idesc_bf16(128, 128, 0, 1);
     float dh_acc = 0.f;
     for (int c = 0; ok && c < nqt; c++) {
-        const int u0 = u_lo + 128 * c, nqc = min(128, u_hi - u0);
-        if (threadIdx.x == 0) {
-            mbar_expect_tx(ld_bar, 2 * kTile);
-            for (int pn = 0; pn < 2; pn++) {
-                ls_load_q(sm + lb::kT2 + pn * kPanel, &tmQ, pn * 64, v, u0, bh, p, ld_bar);
-                ls_load_q(sm + lb::kT3 + pn * kPanel, &tmDy, pn * 64, v, u0, bh, p, ld_bar);
-            }
-        }
-        ld_issued++;
-        {   // the query tile's lam and delta (read after the block-wide wait below)
-            float lm = 0.f, dl = 0.f;
-            if (j < nqc) {
-                const int64_t tok = (int64_t)bh * p.N + (int64_t)(u0 + j) * p.b2 + v;
-                lm = -pair_sum(a.lam[tok * 2].x);
-                dl = a.delta[tok];
-            }
-            lq[j] = lm;
-            dq_s[j] = dl;
-        }
-        if (!(ok = wait_block(ld_bar, ld_done & 1, w))) break;
-        ld_done++;
+        const int b = c & 1, nqc = min(128, u_hi - (u_lo + 128 * c));
+        const float *lq = vec + b * 256, *dq_s = vec + b * 256 + 128;
+        const uint32_t tq = smem_u32(sm + lb::tile(2 + 2 * b)), ty = smem_u32(sm + lb::tile(3 + 2 * b));
+        if (!(ok = wait_block(qb_bar + b, (c >> 1) & 1, w))) break;
+        qb_done[b]++;
         if (warp == 0) {
             tc_fence_after();
-            mma8_ss_k128(tmem, dKt, dQk, idS, 0u);          // S^T = Ktil q^T
-            mma8_ss_k128(tmem + 128, dZk, dYk, idS, 0u);    // dP^T = Z dy^T
+            mma8_ss_k128(tmem, dKt, smem_desc_sw128(tq, 16, 1024), idS, 0u);          // S^T = Ktil q^T
+            mma8_ss_k128(tmem + 128, dZk, smem_desc_sw128(ty, 16, 1024), idS, 0u);    // dP^T = Z dy^T
             mma_commit_warp(mma_bar);
         }
         mma_issued++;
@@ -205,14 +214,17 @@ tc_bwd_dkz_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         __syncthreads();
         if (warp == 0) {
             tc_fence_after();
-            mma8_ts_mn128(tmem + 256, tmem, dYm, idO, c > 0 ? 1u : 0u);        // dZ += L^T dy
-            mma8_ts_mn128(tmem + 384, tmem + 128, dQm, idO, c > 0 ? 1u : 0u);  // += dS^T q
+            mma8_ts_mn128(tmem + 256, tmem, smem_desc_sw128(ty, kPanel, 1024), idO,
+                          c > 0 ? 1u : 0u);                                        // dZ += L^T dy
+            mma8_ts_mn128(tmem + 384, tmem + 128, smem_desc_sw128(tq, kPanel, 1024), idO,
+                          c > 0 ? 1u : 0u);                                        // += dS^T q
             mma_commit_warp(mma_bar);
         }
         mma_issued++;
         if (!(ok = wait_block(mma_bar, mma_done & 1, w))) break;
         mma_done++;
         tc_fence_after();
+        if (c + 2 < nqt) stage_q(c + 2, b);   // buffer b is free again
     }
     if (ok && nqt > 0) {
         // key row u' of q̄ row r = g*b2 + v: 32 columns per chunk, two chunks per panel
@@ -244,8 +256,12 @@ tc_bwd_dkz_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         if (key_ok) a.dhr[((int64_t)bh * p.b1k + up) * rr + r] = dh_acc;
     }
     // drain this CTA's own copies and MMAs before its tensor memory is freed
-    if (threadIdx.x == 0 && ld_issued > ld_done)
-        wait_phase_cleanup(ld_bar, (ld_issued - 1) & 1, kCleanupPolls);
+    if (threadIdx.x == 0) {
+        if (kz_issued > kz_done) wait_phase_cleanup(kz_bar, 0, kCleanupPolls);
+        for (int b = 0; b < 2; b++)
+            if (qb_issued[b] > qb_done[b])
+                wait_phase_cleanup(qb_bar + b, (qb_issued[b] - 1) & 1, kCleanupPolls);
+    }
     if (warp == 0 && mma_issued > mma_done)
         wait_phase_cleanup(mma_bar, (mma_issued - 1) & 1, kCleanupPolls);
     tc_fence_before();
@@ -264,11 +280,12 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     const Problem &p = a.p;
-    uint64_t *ld_bar = reinterpret_cast<uint64_t *>(sm + lb::kBar);
-    uint64_t *mma_bar = ld_bar + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ld_bar + 2);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(ld_bar + 3);
-    float *hk = reinterpret_cast<float *>(sm + lb::kVec);   // H' of the key block
+    uint64_t *q_bar = reinterpret_cast<uint64_t *>(sm + lb::kBar);
+    uint64_t *kb_bar = q_bar + 1;     // [2]: key block buffers
+    uint64_t *mma_bar = q_bar + 3;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(q_bar + 4);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(q_bar + 5);
+    float *hk = reinterpret_cast<float *>(sm + lb::kVec);   // [buffer][128]: H' of the block
     const int warp = threadIdx.x >> 5, j = threadIdx.x;
 
     int unit = blockIdx.x;
@@ -288,8 +305,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     float dsum = 0.f;   // MODE 0: sum over the keys of L dP
 
     if (threadIdx.x == 0) {
-        mbar_init(ld_bar, 1);
-        mbar_init(mma_bar, 1);
+        for (int i = 0; i < 4; i++) mbar_init(q_bar + i, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -300,42 +316,52 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint32_t tmem = *tmem_slot;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
     const WaitCtx w{a.limit, a.status, abort_flag};
-    uint32_t ld_issued = 0, ld_done = 0, mma_issued = 0, mma_done = 0;
+    uint32_t q_issued = 0, q_done = 0, mma_issued = 0, mma_done = 0;
+    uint32_t kb_issued[2] = {0, 0}, kb_done[2] = {0, 0};
 
-    if (threadIdx.x == 0) {   // the query tile and its dy rows
-        mbar_expect_tx(ld_bar, 2 * kTile);
-        for (int pn = 0; pn < 2; pn++) {
-            ls_load_q(sm + lb::kT0 + pn * kPanel, &tmQ, pn * 64, v, u0, bh, p, ld_bar);
-            ls_load_q(sm + lb::kT1 + pn * kPanel, &tmDy, pn * 64, v, u0, bh, p, ld_bar);
-        }
-    }
-    ld_issued++;
-    bool ok = wait_block(ld_bar, ld_done & 1, w);
-    if (ok) ld_done++;
-
-    const uint64_t dQk = smem_desc_sw128(smem_u32(sm + lb::kT0), 16, 1024);
-    const uint64_t dYk = smem_desc_sw128(smem_u32(sm + lb::kT1), 16, 1024);
-    const uint64_t dKt = smem_desc_sw128(smem_u32(sm + lb::kT2), 16, 1024);
-    const uint64_t dZk = smem_desc_sw128(smem_u32(sm + lb::kT3), 16, 1024);
-    const uint64_t dKm = smem_desc_sw128(smem_u32(sm + lb::kT2), kPanel, 1024);
-    constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0), idO = idesc_bf16(128, 128, 0, 1);
-    for (int kb = 0; ok && kb < a.nkb; kb++) {
-        const int nkv = min(128, p.b1k - kb * 128);
+    // key block kk into buffer b: its Ktil and Z rows (thread 0) and its entropies
+    auto stage_k = [&](int kk, int b) {
         if (threadIdx.x == 0) {
-            mbar_expect_tx(ld_bar, 2 * kTile);
+            mbar_expect_tx(kb_bar + b, 2 * kTile);
             for (int pn = 0; pn < 2; pn++) {
-                ls_load_kz(sm + lb::kT2 + pn * kPanel, &tmKt, pn, (int)(slab0 + kb * 128), p, ld_bar);
-                ls_load_kz(sm + lb::kT3 + pn * kPanel, &tmZ, pn, (int)(slab0 + kb * 128), p, ld_bar);
+                ls_load_kz(sm + lb::tile(2 + 2 * b) + pn * kPanel, &tmKt, pn,
+                           (int)(slab0 + kk * 128), p, kb_bar + b);
+                ls_load_kz(sm + lb::tile(3 + 2 * b) + pn * kPanel, &tmZ, pn,
+                           (int)(slab0 + kk * 128), p, kb_bar + b);
             }
         }
-        ld_issued++;
-        hk[j] = j < nkv ? pair_sum(a.hx[(slab0 + kb * 128 + j) * 2].x) : 0.f;
-        if (!(ok = wait_block(ld_bar, ld_done & 1, w))) break;
-        ld_done++;
+        kb_issued[b]++;
+        const int nkv = min(128, p.b1k - kk * 128);
+        hk[b * 128 + j] = j < nkv ? pair_sum(a.hx[(slab0 + kk * 128 + j) * 2].x) : 0.f;
+    };
+
+    if (threadIdx.x == 0) {   // the query tile and its dy rows
+        mbar_expect_tx(q_bar, 2 * kTile);
+        for (int pn = 0; pn < 2; pn++) {
+            ls_load_q(sm + lb::tile(0) + pn * kPanel, &tmQ, pn * 64, v, u0, bh, p, q_bar);
+            ls_load_q(sm + lb::tile(1) + pn * kPanel, &tmDy, pn * 64, v, u0, bh, p, q_bar);
+        }
+    }
+    q_issued++;
+    stage_k(0, 0);
+    bool ok = wait_block(q_bar, 0, w);
+    if (ok) q_done++;
+
+    const uint64_t dQk = smem_desc_sw128(smem_u32(sm + lb::tile(0)), 16, 1024);
+    const uint64_t dYk = smem_desc_sw128(smem_u32(sm + lb::tile(1)), 16, 1024);
+    constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0), idO = idesc_bf16(128, 128, 0, 1);
+    for (int kb = 0; ok && kb < a.nkb; kb++) {
+        const int b = kb & 1, nkv = min(128, p.b1k - kb * 128);
+        // the next block into the other buffer: its last reader, block kb - 1, is done
+        if (kb + 1 < a.nkb) stage_k(kb + 1, b ^ 1);
+        const float *hkb = hk + b * 128;
+        const uint32_t tk = smem_u32(sm + lb::tile(2 + 2 * b)), tz = smem_u32(sm + lb::tile(3 + 2 * b));
+        if (!(ok = wait_block(kb_bar + b, (kb >> 1) & 1, w))) break;
+        kb_done[b]++;
         if (warp == 0) {
             tc_fence_after();
-            mma8_ss_k128(tmem, dQk, dKt, idS, 0u);          // S = q Ktil^T
-            mma8_ss_k128(tmem + 128, dYk, dZk, idS, 0u);    // dP = dy Z^T
+            mma8_ss_k128(tmem, dQk, smem_desc_sw128(tk, 16, 1024), idS, 0u);          // S = q Ktil^T
+            mma8_ss_k128(tmem + 128, dYk, smem_desc_sw128(tz, 16, 1024), idS, 0u);    // dP = dy Z^T
             mma_commit_warp(mma_bar);
         }
         mma_issued++;
@@ -356,7 +382,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 for (int e = 0; e < 2; e++) {
                     const int key = ch * 32 + k + e;
                     const float pr = (row_ok && key < nkv)
-                                         ? fast_exp2((s[k + e] + hk[key] - lam) * a.c_log2) : 0.f;
+                                         ? fast_exp2((s[k + e] + hkb[key] - lam) * a.c_log2) : 0.f;
                     if (MODE == 0) dsum = fmaf(pr, d[k + e], dsum);
                     dv[e] = pr * (d[k + e] - dlt);
                 }
@@ -379,7 +405,8 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         __syncthreads();
         if (warp == 0) {
             tc_fence_after();
-            mma8_ts_mn128(tmem + 256, tmem, dKm, idO, kb > 0 ? 1u : 0u);   // dq' += dS Ktil
+            mma8_ts_mn128(tmem + 256, tmem, smem_desc_sw128(tk, kPanel, 1024), idO,
+                          kb > 0 ? 1u : 0u);   // dq' += dS Ktil
             mma_commit_warp(mma_bar);
         }
         mma_issued++;
@@ -403,8 +430,12 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             }
         }
     }
-    if (threadIdx.x == 0 && ld_issued > ld_done)
-        wait_phase_cleanup(ld_bar, (ld_issued - 1) & 1, kCleanupPolls);
+    if (threadIdx.x == 0) {
+        if (q_issued > q_done) wait_phase_cleanup(q_bar, 0, kCleanupPolls);
+        for (int b = 0; b < 2; b++)
+            if (kb_issued[b] > kb_done[b])
+                wait_phase_cleanup(kb_bar + b, (kb_issued[b] - 1) & 1, kCleanupPolls);
+    }
     if (warp == 0 && mma_issued > mma_done)
         wait_phase_cleanup(mma_bar, (mma_issued - 1) & 1, kCleanupPolls);
     tc_fence_before();
