@@ -43,8 +43,8 @@ namespace lb {
 // the ones loaded per step (T2, T3 and T4, T5), so that step i + 1's copies overlap
 // step i's products and elementwise work
 __host__ __device__ constexpr uint32_t tile(int i) { return (uint32_t)i * kTile; }
-constexpr uint32_t kVec = 6 * kTile;             // 4 x 128 floats
-constexpr uint32_t kBar = kVec + 4 * 512;
+constexpr uint32_t kVec = 6 * kTile;             // 8 x 128 floats
+constexpr uint32_t kBar = kVec + 8 * 512;
 constexpr uint32_t kSmem = kBar + 128 + 1024;    // + slack to align the base to 1024
 }  // namespace lb
 
@@ -75,7 +75,7 @@ __device__ __forceinline__ bool wait_block(uint64_t *bar, uint32_t parity, const
     return __syncthreads_and(ok) != 0;
 }
 
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
 tc_bwd_dkz_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDy,
                   const __grid_constant__ CUtensorMap tmKt, const __grid_constant__ CUtensorMap tmZ,
                   LbArgs a) {
@@ -88,7 +88,10 @@ tc_bwd_dkz_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(kz_bar + 4);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(kz_bar + 5);
     float *vec = reinterpret_cast<float *>(sm + lb::kVec);   // [buffer][lam | delta][128]
-    const int warp = threadIdx.x >> 5, j = threadIdx.x;
+    float *dh_part = vec + 512;                               // [128]: the second half's dH
+    // two warps per group of 32 TMEM lanes: thread (j, half) takes key row j and the
+    // half's 64 query columns (chunks 2*half, 2*half + 1)
+    const int warp = threadIdx.x >> 5, j = (warp & 3) * 32 + (threadIdx.x & 31), half = warp >> 2;
 
     int unit = blockIdx.x;
     const int kb = unit % a.nkb;
@@ -111,7 +114,7 @@ tc_bwd_dkz_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);   // this warp's lanes
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);   // this warp's lanes
     const WaitCtx w{a.limit, a.status, abort_flag};
     uint32_t kz_issued = 0, kz_done = 0, mma_issued = 0, mma_done = 0;
     uint32_t qb_issued[2] = {0, 0}, qb_done[2] = {0, 0};
@@ -129,14 +132,17 @@ tc_bwd_dkz_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             }
         }
         qb_issued[b]++;
-        float lm = 0.f, dl = 0.f;
-        if (j < nqc) {
-            const int64_t tok = (int64_t)bh * p.N + (int64_t)(u0 + j) * p.b2 + v;
-            lm = -pair_sum(a.lam[tok * 2].x);
-            dl = a.delta[tok];
+        const int i = threadIdx.x;
+        if (i < 128) {
+            float lm = 0.f, dl = 0.f;
+            if (i < nqc) {
+                const int64_t tok = (int64_t)bh * p.N + (int64_t)(u0 + i) * p.b2 + v;
+                lm = -pair_sum(a.lam[tok * 2].x);
+                dl = a.delta[tok];
+            }
+            vec[b * 256 + i] = lm;
+            vec[b * 256 + 128 + i] = dl;
         }
-        vec[b * 256 + j] = lm;
-        vec[b * 256 + 128 + j] = dl;
     };
 
     // the key block: Ktil and Z rows (128 blocks u' of row (g, v); past b1k: zeros),
@@ -176,13 +182,20 @@ tc_bwd_dkz_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         if (!(ok = wait_block(mma_bar, mma_done & 1, w))) break;
         mma_done++;
         tc_fence_after();
-        // L^T and dS^T of this key row over the tile's queries, packed in place
-#pragma unroll 1
-        for (int ch = 0; ch < 4; ch++) {
-            float s[32], d[32];
-            tmem_ld32f(tl + ch * 32, s);
-            tmem_ld32f(tl + 128 + ch * 32, d);
-            tmem_wait_ld();
+        // L^T and dS^T of this key row over the half's queries, packed in place: both
+        // halves read all of their S^T and dP^T columns before either writes (the
+        // packed pairs of the upper half land on columns the lower half reads)
+        float sv[64], dv64[64];
+        tmem_ld32f(tl + 64 * half, sv);
+        tmem_ld32f(tl + 64 * half + 32, sv + 32);
+        tmem_ld32f(tl + 128 + 64 * half, dv64);
+        tmem_ld32f(tl + 128 + 64 * half + 32, dv64 + 32);
+        tmem_wait_ld();
+        __syncthreads();
+#pragma unroll
+        for (int cc = 0; cc < 2; cc++) {
+            const int ch = 2 * half + cc;
+            const float *s = sv + 32 * cc, *d = dv64 + 32 * cc;
             uint32_t pk[16], dk[16];
 #pragma unroll
             for (int k = 0; k < 32; k += 2) {
@@ -226,12 +239,15 @@ tc_bwd_dkz_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         tc_fence_after();
         if (c + 2 < nqt) stage_q(c + 2, b);   // buffer b is free again
     }
+    if (half == 1) dh_part[j] = dh_acc;
+    __syncthreads();
     if (ok && nqt > 0) {
         // key row u' of q̄ row r = g*b2 + v: 32 columns per chunk, two chunks per panel
+        // (the half's panel)
         const int up = kb * 128 + j, r = g * p.b2 + v, rr = p.tiles * p.b2;
         const int64_t rowbase = ((int64_t)bh * p.b1k + up) * 2;   // panel 0 of (bh, u')
 #pragma unroll 1
-        for (int ch = 0; ch < 4; ch++) {
+        for (int ch = 2 * half; ch < 2 * half + 2; ch++) {
             float z[32], kt[32];
             tmem_ld32f(tl + 256 + ch * 32, z);
             tmem_ld32f(tl + 384 + ch * 32, kt);
@@ -253,7 +269,7 @@ tc_bwd_dkz_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 }
             }
         }
-        if (key_ok) a.dhr[((int64_t)bh * p.b1k + up) * rr + r] = dh_acc;
+        if (key_ok && half == 0) a.dhr[((int64_t)bh * p.b1k + up) * rr + r] = dh_acc + dh_part[j];
     }
     // drain this CTA's own copies and MMAs before its tensor memory is freed
     if (threadIdx.x == 0) {
@@ -273,7 +289,7 @@ tc_bwd_dkz_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
 tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDy,
                  const __grid_constant__ CUtensorMap tmKt, const __grid_constant__ CUtensorMap tmZ,
                  LbArgs a) {
@@ -286,7 +302,10 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(q_bar + 4);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(q_bar + 5);
     float *hk = reinterpret_cast<float *>(sm + lb::kVec);   // [buffer][128]: H' of the block
-    const int warp = threadIdx.x >> 5, j = threadIdx.x;
+    float *ds_part = hk + 256;                               // [128]: the second half's delta
+    // two warps per group of 32 TMEM lanes: thread (j, half) takes query row j and the
+    // half's 64 key columns (chunks 2*half, 2*half + 1)
+    const int warp = threadIdx.x >> 5, j = (warp & 3) * 32 + (threadIdx.x & 31), half = warp >> 2;
 
     int unit = blockIdx.x;
     const int c = unit % a.nqt;
@@ -314,7 +333,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const WaitCtx w{a.limit, a.status, abort_flag};
     uint32_t q_issued = 0, q_done = 0, mma_issued = 0, mma_done = 0;
     uint32_t kb_issued[2] = {0, 0}, kb_done[2] = {0, 0};
@@ -331,8 +350,8 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             }
         }
         kb_issued[b]++;
-        const int nkv = min(128, p.b1k - kk * 128);
-        hk[b * 128 + j] = j < nkv ? pair_sum(a.hx[(slab0 + kk * 128 + j) * 2].x) : 0.f;
+        const int nkv = min(128, p.b1k - kk * 128), i = threadIdx.x;
+        if (i < 128) hk[b * 128 + i] = i < nkv ? pair_sum(a.hx[(slab0 + kk * 128 + i) * 2].x) : 0.f;
     };
 
     if (threadIdx.x == 0) {   // the query tile and its dy rows
@@ -368,12 +387,19 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (!(ok = wait_block(mma_bar, mma_done & 1, w))) break;
         mma_done++;
         tc_fence_after();
-#pragma unroll 1
-        for (int ch = 0; ch < 4; ch++) {
-            float s[32], d[32];
-            tmem_ld32f(tl + ch * 32, s);
-            tmem_ld32f(tl + 128 + ch * 32, d);
-            tmem_wait_ld();
+        // both halves read all of their S and dP columns before either writes dS over
+        // S (the upper half's packed pairs land on columns the lower half reads)
+        float sv[64], dv64[64];
+        tmem_ld32f(tl + 64 * half, sv);
+        tmem_ld32f(tl + 64 * half + 32, sv + 32);
+        tmem_ld32f(tl + 128 + 64 * half, dv64);
+        tmem_ld32f(tl + 128 + 64 * half + 32, dv64 + 32);
+        tmem_wait_ld();
+        if (MODE == 1) __syncthreads();
+#pragma unroll
+        for (int cc = 0; cc < 2; cc++) {
+            const int ch = 2 * half + cc;
+            const float *s = sv + 32 * cc, *d = dv64 + 32 * cc;
             uint32_t dk[16];
 #pragma unroll
             for (int k = 0; k < 32; k += 2) {
@@ -414,10 +440,14 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         mma_done++;
         tc_fence_after();
     }
-    if (ok && MODE == 0 && row_ok) a.delta[tok] = dsum;
+    if (MODE == 0) {
+        if (half == 1) ds_part[j] = dsum;
+        __syncthreads();
+        if (ok && row_ok && half == 0) a.delta[tok] = dsum + ds_part[j];
+    }
     if (ok && MODE == 1) {
 #pragma unroll 1
-        for (int ch = 0; ch < 4; ch++) {
+        for (int ch = 2 * half; ch < 2 * half + 2; ch++) {
             float o[32];
             tmem_ld32f(tl + 256 + ch * 32, o);
             tmem_wait_ld();
@@ -931,9 +961,9 @@ cudaError_t sm100_backward(const Problem &p, const void *q, const void *k, const
     const int64_t probs = (int64_t)p.BH * p.tiles * p.b2;
     {
         ProfileScope scope(K_BWD_L, stream);
-        tc_bwd_dq_kernel<0><<<(unsigned)(probs * la.nqt), 128, lb::kSmem, stream>>>(mq, mdy, mkt, mz, la);
-        tc_bwd_dkz_kernel<<<(unsigned)(probs * la.nkb), 128, lb::kSmem, stream>>>(mq, mdy, mkt, mz, la);
-        tc_bwd_dq_kernel<1><<<(unsigned)(probs * la.nqt), 128, lb::kSmem, stream>>>(mq, mdy, mkt, mz, la);
+        tc_bwd_dq_kernel<0><<<(unsigned)(probs * la.nqt), 256, lb::kSmem, stream>>>(mq, mdy, mkt, mz, la);
+        tc_bwd_dkz_kernel<<<(unsigned)(probs * la.nkb), 256, lb::kSmem, stream>>>(mq, mdy, mkt, mz, la);
+        tc_bwd_dq_kernel<1><<<(unsigned)(probs * la.nqt), 256, lb::kSmem, stream>>>(mq, mdy, mkt, mz, la);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     RbArgs ra{p, mpad, w.dhr, w.da, (__nv_bfloat16 *)dk, (__nv_bfloat16 *)dv, w.part, w.nmt, w.nch,
