@@ -383,7 +383,7 @@ MONARCH_API int monarch_debug_inject_stall(int on);
 
 /*
  * Benchmark hook: per-kernel timing.  While enabled (on != 0), every kernel
- * launch of the forward pass is bracketed by CUDA events recorded on its launch
+ * launch of the forward and backward passes is bracketed by CUDA events recorded on its launch
  * stream; the launches themselves are unchanged.  Disabling keeps the counters.
  * Source: no counterpart in the pages (a measurement facility).
  */

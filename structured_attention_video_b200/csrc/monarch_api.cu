@@ -617,7 +617,9 @@ const char *monarch_profile_kernel_name(int k) {
                                          "tc_qbar_kernel",       "tc_rstep_kernel",
                                          "tc_lstep_kernel",      "tc_lstat_kernel",
                                          "tc_qagg_kernel", "bwd_lstep_kernels",
-                                         "bwd_rstep_kernels"};
+                                         "bwd_rstep_kernels",    "tc_bwd_dq_kernel<0>",
+                                         "tc_bwd_dkz_kernel",    "tc_bwd_dq_kernel<1>",
+                                         "tc_bwd_r_kernel",      "tc_bwd_dqbar+combine"};
     return (k >= 0 && k < K_COUNT) ? names[k] : nullptr;
 }
 

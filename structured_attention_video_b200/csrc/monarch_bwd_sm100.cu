@@ -369,6 +369,56 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint64_t dQk = smem_desc_sw128(smem_u32(sm + lb::tile(0)), 16, 1024);
     const uint64_t dYk = smem_desc_sw128(smem_u32(sm + lb::tile(1)), 16, 1024);
     constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0), idO = idesc_bf16(128, 128, 0, 1);
+    if constexpr (MODE == 0) {
+        // delta needs no accumulator: the products of block kb + 1 go to the other 256
+        // columns of tensor memory while the threads work on block kb
+        if (a.nkb > 1) stage_k(1, 1);
+        auto issue = [&](int kb) {   // warp 0
+            const int b = kb & 1;
+            const uint32_t tk = smem_u32(sm + lb::tile(2 + 2 * b)), tz = smem_u32(sm + lb::tile(3 + 2 * b));
+            tc_fence_after();
+            mma8_ss_k128(tmem + 256 * b, dQk, smem_desc_sw128(tk, 16, 1024), idS, 0u);         // S = q Ktil^T
+            mma8_ss_k128(tmem + 256 * b + 128, dYk, smem_desc_sw128(tz, 16, 1024), idS, 0u);   // dP = dy Z^T
+            mma_commit_warp(mma_bar);
+        };
+        if (ok && a.nkb > 0 && (ok = wait_block(kb_bar, 0, w))) {
+            kb_done[0]++;
+            if (warp == 0) issue(0);
+            mma_issued++;
+        }
+        for (int kb = 0; ok && kb < a.nkb; kb++) {
+            const int b = kb & 1, nkv = min(128, p.b1k - kb * 128);
+            if (!(ok = wait_block(mma_bar, mma_done & 1, w))) break;
+            mma_done++;
+            if (kb + 1 < a.nkb) {   // block kb + 1, loaded during the previous step
+                if (!(ok = wait_block(kb_bar + (b ^ 1), ((kb + 1) >> 1) & 1, w))) break;
+                kb_done[b ^ 1]++;
+                if (warp == 0) issue(kb + 1);
+                mma_issued++;
+            }
+            tc_fence_after();
+            const float *hkb = hk + b * 128;
+            const uint32_t tb = tl + 256 * b + 64 * half;
+            float sv[64], dv64[64];
+            tmem_ld32f(tb, sv);
+            tmem_ld32f(tb + 32, sv + 32);
+            tmem_ld32f(tb + 128, dv64);
+            tmem_ld32f(tb + 160, dv64 + 32);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 64; k++) {
+                const int key = 64 * half + k;
+                const float pr = (row_ok && key < nkv)
+                                     ? fast_exp2((sv[k] + hkb[key] - lam) * a.c_log2) : 0.f;
+                dsum = fmaf(pr, dv64[k], dsum);
+            }
+            // every thread is done with block kb's columns and entropies: the products
+            // of block kb + 2 may overwrite the columns, and buffer b takes its rows
+            tc_fence_before();
+            __syncthreads();
+            if (kb + 2 < a.nkb) stage_k(kb + 2, b);
+        }
+    } else {
     for (int kb = 0; ok && kb < a.nkb; kb++) {
         const int b = kb & 1, nkv = min(128, p.b1k - kb * 128);
         // the next block into the other buffer: its last reader, block kb - 1, is done
@@ -395,7 +445,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tmem_ld32f(tl + 128 + 64 * half, dv64);
         tmem_ld32f(tl + 128 + 64 * half + 32, dv64 + 32);
         tmem_wait_ld();
-        if (MODE == 1) __syncthreads();
+        __syncthreads();
 #pragma unroll
         for (int cc = 0; cc < 2; cc++) {
             const int ch = 2 * half + cc;
@@ -409,22 +459,14 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     const int key = ch * 32 + k + e;
                     const float pr = (row_ok && key < nkv)
                                          ? fast_exp2((s[k + e] + hkb[key] - lam) * a.c_log2) : 0.f;
-                    if (MODE == 0) dsum = fmaf(pr, d[k + e], dsum);
                     dv[e] = pr * (d[k + e] - dlt);
                 }
                 dk[k / 2] = pack_bf16(dv[0], dv[1]);
             }
-            if (MODE == 1) {
-                const uint32_t(&dk0)[8] = *reinterpret_cast<const uint32_t(*)[8]>(&dk[0]);
-                const uint32_t(&dk1)[8] = *reinterpret_cast<const uint32_t(*)[8]>(&dk[8]);
-                tmem_st8(tl + ch * 16, dk0);
-                tmem_st8(tl + ch * 16 + 8, dk1);
-            }
-        }
-        if (MODE == 0) {   // the next block's S and dP may overwrite this block's
-            tc_fence_before();
-            __syncthreads();
-            continue;
+            const uint32_t(&dk0)[8] = *reinterpret_cast<const uint32_t(*)[8]>(&dk[0]);
+            const uint32_t(&dk1)[8] = *reinterpret_cast<const uint32_t(*)[8]>(&dk[8]);
+            tmem_st8(tl + ch * 16, dk0);
+            tmem_st8(tl + ch * 16 + 8, dk1);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -439,6 +481,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (!(ok = wait_block(mma_bar, mma_done & 1, w))) break;
         mma_done++;
         tc_fence_after();
+    }
     }
     if (MODE == 0) {
         if (half == 1) ds_part[j] = dsum;
@@ -483,10 +526,12 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 //   da = R (dR - sum R dR) - dH R (a - sum R a)   (dH/da = -R (a - E_R[a])),
 //   dk = s da^T q̄ + R^T dKtil,  dv = R^T dZ  (complete in the CTA: the block's keys),
 //   dq̄ = s sum over u' of da K  (tc_bwd_dqbar_kernel, over the blocks in chunks).
-// tc_bwd_r_kernel: the logits and dR as tcgen05 products into tensor memory; one
-// thread per row forms R and s*da, writes them as bfloat16 [row][key] tiles (the
-// MN-major A operands of dk and dv, keys along M) and s*da to global memory; dk
-// and dv accumulate in tensor memory over the row tiles.
+// tc_bwd_r_kernel: the logits and dR as tcgen05 products into tensor memory; two
+// threads per row (warps w and w + 4 share a group of 32 TMEM lanes, each with
+// half of the key chunks, their row sums met in shared memory) form R and s*da,
+// write them as bfloat16 [row][key] tiles (the MN-major A operands of dk and dv,
+// keys along M) and s*da to global memory; dk and dv accumulate in tensor memory
+// over the row tiles.
 // =====================================================================
 namespace rb {
 constexpr uint32_t kQ = 0;              // q̄ row tile (K-major for the logits, MN-major for dk)
@@ -518,7 +563,7 @@ __device__ __forceinline__ uint32_t sw128(int r, int c) {
 }
 
 template <int B2P>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
 tc_bwd_r_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDK,
                 const __grid_constant__ CUtensorMap tmDZ, RbArgs a) {
@@ -529,10 +574,15 @@ tc_bwd_r_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
     uint64_t *mma_bar = ld_bar + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ld_bar + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(ld_bar + 3);
-    const int warp = threadIdx.x >> 5, r = threadIdx.x;
+    const int warp = threadIdx.x >> 5, r = (warp & 3) * 32 + (threadIdx.x & 31), half = warp >> 2;
     const int bh = blockIdx.x / p.b1k, up = blockIdx.x % p.b1k;
     const int rr = p.tiles * p.b2;
     constexpr uint32_t kPanelKV = B2P * 128;
+    // the row's 16-key chunks: the first kC0 to half 0, the rest to half 1
+    constexpr int kC = B2P / 16, kC0 = (kC + 1) / 2;
+    const int nck = half ? kC - kC0 : kC0, kbase = half ? kC0 * 16 : 0;
+    // the two halves' row sums (max, sum, E, rho), in the s*da tile before it is written
+    float *red = reinterpret_cast<float *>(sm + rb::kDA);
 
     if (threadIdx.x == 0) {
         mbar_init(ld_bar, 1);
@@ -545,7 +595,7 @@ tc_bwd_r_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const WaitCtx w{a.limit, a.status, abort_flag};
     uint32_t ld_issued = 0, ld_done = 0, mma_issued = 0, mma_done = 0;
 
@@ -610,51 +660,66 @@ tc_bwd_r_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
         if (!(ok = wait_block(mma_bar, mma_done & 1, w))) break;
         mma_done++;
         tc_fence_after();
-        // this row: R and s*da over the block's keys (x: the natural logits s*a,
+        // this row: R and s*da over this half's keys (x: the natural logits s*a,
         // y: dR; R is recomputed from x where it is needed, to keep two arrays)
-        float x[B2P], y[B2P];
+        float x[kC0 * 16], y[kC0 * 16];
 #pragma unroll
-        for (int cc = 0; cc < B2P / 16; cc++) {
-            tmem_ld16f(tl + cc * 16, &x[cc * 16]);
-            tmem_ld16f(tl + 128 + cc * 16, &y[cc * 16]);
-        }
+        for (int cc = 0; cc < kC0; cc++)
+            if (cc < nck) {
+                tmem_ld16f(tl + kbase + cc * 16, &x[cc * 16]);
+                tmem_ld16f(tl + 128 + kbase + cc * 16, &y[cc * 16]);
+            }
         tmem_wait_ld();
         float mx = -INFINITY;
 #pragma unroll
-        for (int k = 0; k < B2P; k++) {
-            x[k] = k < p.b2 ? x[k] * p.scale : 0.f;
-            y[k] = k < p.b2 ? y[k] : 0.f;
-            mx = k < p.b2 ? fmaxf(mx, x[k]) : mx;
+        for (int k = 0; k < kC0 * 16; k++) {
+            const bool kv = k < nck * 16 && kbase + k < p.b2;
+            x[k] = kv ? x[k] * p.scale : 0.f;
+            y[k] = kv ? y[k] : 0.f;
+            mx = kv ? fmaxf(mx, x[k]) : mx;
         }
+        red[half * 128 + r] = mx;
+        __syncthreads();
+        mx = fmaxf(mx, red[(half ^ 1) * 128 + r]);
         float l = 0.f;
 #pragma unroll
-        for (int k = 0; k < B2P; k++) l += k < p.b2 ? fast_exp2((x[k] - mx) * kLog2e) : 0.f;
+        for (int k = 0; k < kC0 * 16; k++)
+            l += (k < nck * 16 && kbase + k < p.b2) ? fast_exp2((x[k] - mx) * kLog2e) : 0.f;
+        red[256 + half * 128 + r] = l;
+        __syncthreads();
+        l += red[256 + (half ^ 1) * 128 + r];   // the same sum in both halves (a + b = b + a)
         const float inv = 1.f / l;
         float E = 0.f, rho = 0.f;
 #pragma unroll
-        for (int k = 0; k < B2P; k++) {
-            const float rk = k < p.b2 ? fast_exp2((x[k] - mx) * kLog2e) * inv : 0.f;
+        for (int k = 0; k < kC0 * 16; k++) {
+            const float rk = (k < nck * 16 && kbase + k < p.b2) ? fast_exp2((x[k] - mx) * kLog2e) * inv : 0.f;
             E = fmaf(rk, x[k], E);
             rho = fmaf(rk, y[k], rho);
         }
+        red[512 + half * 128 + r] = E;
+        red[768 + half * 128 + r] = rho;
+        __syncthreads();
+        E += red[512 + (half ^ 1) * 128 + r];
+        rho += red[768 + (half ^ 1) * 128 + r];
+        __syncthreads();   // the sums are read before the s*da tile is written over them
         // s*da and R as bfloat16 [row][key] tiles; s*da also to global memory
         __nv_bfloat16 *dag = a.da + (((int64_t)bh * p.b1k + up) * 2 * rr + rg) * 64;
 #pragma unroll
-        for (int pn = 0; pn < 2; pn++) {
-#pragma unroll
-            for (int ch = 0; ch < 8; ch++) {
+        for (int lc = 0; lc < 2 * kC0; lc++) {   // this half's 8-key chunks
+            if (lc < 2 * nck) {
+                const int key0 = kbase + 8 * lc, pn = key0 >> 6, ch = (key0 & 63) >> 3;
                 uint32_t dw[4], rw[4];
 #pragma unroll
                 for (int e = 0; e < 4; e++) {
-                    const int k0 = pn * 64 + ch * 8 + 2 * e;
+                    const int k = 8 * lc + 2 * e;
                     float d0 = 0.f, d1 = 0.f, r0 = 0.f, r1 = 0.f;
-                    if (k0 < B2P && k0 < p.b2 && row_ok) {
-                        r0 = fast_exp2((x[k0] - mx) * kLog2e) * inv;
-                        d0 = p.scale * (r0 * (y[k0] - rho) - dh * r0 * (x[k0] - E));
+                    if (row_ok && key0 + 2 * e < p.b2) {
+                        r0 = fast_exp2((x[k] - mx) * kLog2e) * inv;
+                        d0 = p.scale * (r0 * (y[k] - rho) - dh * r0 * (x[k] - E));
                     }
-                    if (k0 + 1 < B2P && k0 + 1 < p.b2 && row_ok) {
-                        r1 = fast_exp2((x[k0 + 1] - mx) * kLog2e) * inv;
-                        d1 = p.scale * (r1 * (y[k0 + 1] - rho) - dh * r1 * (x[k0 + 1] - E));
+                    if (row_ok && key0 + 2 * e + 1 < p.b2) {
+                        r1 = fast_exp2((x[k + 1] - mx) * kLog2e) * inv;
+                        d1 = p.scale * (r1 * (y[k + 1] - rho) - dh * r1 * (x[k + 1] - E));
                     }
                     dw[e] = pack_bf16(d0, d1);
                     rw[e] = pack_bf16(r0, r1);
@@ -663,8 +728,16 @@ tc_bwd_r_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
                 const uint4 rv4 = make_uint4(rw[0], rw[1], rw[2], rw[3]);
                 *reinterpret_cast<uint4 *>(sm + rb::kDA + pn * kPanel + sw128(r, ch)) = dv4;
                 *reinterpret_cast<uint4 *>(sm + rb::kR + pn * kPanel + sw128(r, ch)) = rv4;
-                if (row_ok && pn * 64 < B2P)
-                    reinterpret_cast<uint4 *>(dag + (int64_t)pn * rr * 64)[ch] = dv4;
+                if (row_ok) reinterpret_cast<uint4 *>(dag + (int64_t)pn * rr * 64)[ch] = dv4;
+            }
+        }
+        if (half == 1) {   // keys B2P..127 of the tiles (and of s*da's last panel): zeros
+            const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+            for (int key0 = B2P; key0 < 128; key0 += 8) {
+                const int pn = key0 >> 6, ch = (key0 & 63) >> 3;
+                *reinterpret_cast<uint4 *>(sm + rb::kDA + pn * kPanel + sw128(r, ch)) = z4;
+                *reinterpret_cast<uint4 *>(sm + rb::kR + pn * kPanel + sw128(r, ch)) = z4;
+                if (row_ok && pn * 64 < B2P) reinterpret_cast<uint4 *>(dag + (int64_t)pn * rr * 64)[ch] = z4;
             }
         }
         fence_proxy_async_smem();
@@ -691,11 +764,11 @@ tc_bwd_r_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
         mma_done++;
         tc_fence_after();
     }
-    if (ok) {   // thread m: key m of the block
+    if (ok) {   // thread (m, half): key m of the block, the half's 64 columns
         const bool key_ok = r < p.b2;
         const int64_t tok = (int64_t)bh * p.N + (int64_t)up * p.b2 + r;
 #pragma unroll 1
-        for (int ch = 0; ch < 4; ch++) {
+        for (int ch = 2 * half; ch < 2 * half + 2; ch++) {
             float o[32], u[32];
             tmem_ld32f(tl + 256 + ch * 32, o);
             tmem_ld32f(tl + 384 + ch * 32, u);
@@ -902,14 +975,20 @@ size_t bw_tc_layout(const Problem &p, void *base, BwTc *out) {
     return total;
 }
 
+// stage 0: tc_bwd_r_kernel (dk, dv, s*da); stage 1: tc_bwd_dqbar_kernel (dq̄ partial sums)
 template <int B2P>
-cudaError_t launch_bwd_r(const CUtensorMap *m, const RbArgs &a, cudaStream_t s) {
-    cudaError_t e = set_smem(tc_bwd_r_kernel<B2P>, rb::kSmem);
-    if (e == cudaSuccess) e = set_smem(tc_bwd_dqbar_kernel<B2P>, rb::kSmemQ);
-    if (e != cudaSuccess) return e;
-    tc_bwd_r_kernel<B2P><<<(unsigned)(a.p.BH * a.p.b1k), 128, rb::kSmem, s>>>(m[0], m[1], m[2], m[3],
-                                                                           m[4], a);
-    tc_bwd_dqbar_kernel<B2P><<<(unsigned)(a.p.BH * a.nmt * a.nch), 128, rb::kSmemQ, s>>>(m[5], m[1], a);
+cudaError_t launch_bwd_r(const CUtensorMap *m, const RbArgs &a, int stage, cudaStream_t s) {
+    if (stage == 0) {
+        const cudaError_t e = set_smem(tc_bwd_r_kernel<B2P>, rb::kSmem);
+        if (e != cudaSuccess) return e;
+        tc_bwd_r_kernel<B2P><<<(unsigned)(a.p.BH * a.p.b1k), 256, rb::kSmem, s>>>(m[0], m[1], m[2],
+                                                                               m[3], m[4], a);
+    } else {
+        const cudaError_t e = set_smem(tc_bwd_dqbar_kernel<B2P>, rb::kSmemQ);
+        if (e != cudaSuccess) return e;
+        tc_bwd_dqbar_kernel<B2P><<<(unsigned)(a.p.BH * a.nmt * a.nch), 128, rb::kSmemQ, s>>>(m[5], m[1],
+                                                                                          a);
+    }
     return cudaGetLastError();
 }
 
@@ -960,27 +1039,39 @@ cudaError_t sm100_backward(const Problem &p, const void *q, const void *k, const
               (tile_max_rows(p.b1, p.tiles) + 127) / 128, status, wait_limit};
     const int64_t probs = (int64_t)p.BH * p.tiles * p.b2;
     {
-        ProfileScope scope(K_BWD_L, stream);
+        ProfileScope scope(K_TC_BWD_DELTA, stream);
         tc_bwd_dq_kernel<0><<<(unsigned)(probs * la.nqt), 256, lb::kSmem, stream>>>(mq, mdy, mkt, mz, la);
-        tc_bwd_dkz_kernel<<<(unsigned)(probs * la.nkb), 256, lb::kSmem, stream>>>(mq, mdy, mkt, mz, la);
-        tc_bwd_dq_kernel<1><<<(unsigned)(probs * la.nqt), 256, lb::kSmem, stream>>>(mq, mdy, mkt, mz, la);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
+    {
+        ProfileScope scope(K_TC_BWD_DKZ, stream);
+        tc_bwd_dkz_kernel<<<(unsigned)(probs * la.nkb), 256, lb::kSmem, stream>>>(mq, mdy, mkt, mz, la);
+    }
+    {
+        ProfileScope scope(K_TC_BWD_DQ, stream);
+        tc_bwd_dq_kernel<1><<<(unsigned)(probs * la.nqt), 256, lb::kSmem, stream>>>(mq, mdy, mkt, mz, la);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     RbArgs ra{p, mpad, w.dhr, w.da, (__nv_bfloat16 *)dk, (__nv_bfloat16 *)dv, w.part, w.nmt, w.nch,
               w.upc, status, wait_limit};
-    ProfileScope scope(K_BWD_R, stream);
-    switch (b2p) {
-        case 16: e = launch_bwd_r<16>(rm, ra, stream); break;
-        case 32: e = launch_bwd_r<32>(rm, ra, stream); break;
-        case 48: e = launch_bwd_r<48>(rm, ra, stream); break;
-        case 64: e = launch_bwd_r<64>(rm, ra, stream); break;
-        case 80: e = launch_bwd_r<80>(rm, ra, stream); break;
-        case 96: e = launch_bwd_r<96>(rm, ra, stream); break;
-        case 112: e = launch_bwd_r<112>(rm, ra, stream); break;
-        case 128: e = launch_bwd_r<128>(rm, ra, stream); break;
-        default: return cudaErrorInvalidValue;
+    auto launch_r = [&](int stage) -> cudaError_t {
+        switch (b2p) {
+            case 16: return launch_bwd_r<16>(rm, ra, stage, stream);
+            case 32: return launch_bwd_r<32>(rm, ra, stage, stream);
+            case 48: return launch_bwd_r<48>(rm, ra, stage, stream);
+            case 64: return launch_bwd_r<64>(rm, ra, stage, stream);
+            case 80: return launch_bwd_r<80>(rm, ra, stage, stream);
+            case 96: return launch_bwd_r<96>(rm, ra, stage, stream);
+            case 112: return launch_bwd_r<112>(rm, ra, stage, stream);
+            case 128: return launch_bwd_r<128>(rm, ra, stage, stream);
+            default: return cudaErrorInvalidValue;
+        }
+    };
+    {
+        ProfileScope scope(K_TC_BWD_R, stream);
+        if ((e = launch_r(0)) != cudaSuccess) return e;
     }
-    if (e != cudaSuccess) return e;
+    ProfileScope scope(K_TC_BWD_DQBAR, stream);
+    if ((e = launch_r(1)) != cudaSuccess) return e;
     const int64_t total = (int64_t)p.BH * p.N * (kD / 4);
     const int blocks = (int)((total + 255) / 256 < 148 * 32 ? (total + 255) / 256 : 148 * 32);
     tc_bwd_combine_kernel<<<blocks, 256, 0, stream>>>(w.dql, w.part, (__nv_bfloat16 *)dq, p, w.nmt,

@@ -115,7 +115,12 @@ enum KernelId {
     K_TC_QAGG = 8,        // S4 re-aggregated queries (tensor-core)
     K_BWD_L = 9,          // backward of the L-step and the output (generic)
     K_BWD_R = 10,         // backward of the R-step and the aggregation (generic)
-    K_COUNT = 11
+    K_TC_BWD_DELTA = 11,  // tensor-core backward: delta = sum L dP per query row
+    K_TC_BWD_DKZ = 12,    // tensor-core backward: dKtil, dZ, dH per key row
+    K_TC_BWD_DQ = 13,     // tensor-core backward: dq through the L-step
+    K_TC_BWD_R = 14,      // tensor-core backward: dk, dv and s*da per block
+    K_TC_BWD_DQBAR = 15,  // tensor-core backward: dq̄ partial sums and the final dq
+    K_COUNT = 16
 };
 
 // Brackets one kernel launch with CUDA events while profiling is enabled.
