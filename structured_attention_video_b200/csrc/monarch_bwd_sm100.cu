@@ -542,7 +542,14 @@ constexpr uint32_t kR = 4 * kTile;      // R as [row][key]
 constexpr uint32_t kKV = 5 * kTile;     // K then V of the block: 2 panels of B2P rows each
 constexpr uint32_t kBar = kKV + 4 * 128 * 128;
 constexpr uint32_t kSmem = kBar + 64 + 1024;
-constexpr uint32_t kSmemQ = 2 * kTile + 64 + 1024;   // tc_bwd_dqbar_kernel: da tile, K
+// tc_bwd_dqbar_kernel: a ring of stages, each one block's s*da tile and its K rows
+// (two 64-column panels of B2P rows)
+template <int B2P> struct Dq {
+    static constexpr uint32_t kStage = kTile + 2 * B2P * 128;
+    static constexpr int kNS = B2P <= 80 ? 4 : 3;
+    static constexpr uint32_t kBar = kNS * kStage;
+    static constexpr uint32_t kSmem = kBar + 128 + 1024;
+};
 }  // namespace rb
 
 struct RbArgs {
@@ -800,6 +807,8 @@ tc_bwd_r_kernel(const __grid_constant__ CUtensorMap tmQb, const __grid_constant_
 
 // dq̄ partial sums: unit (bh, row tile mt, chunk ch of upc blocks): sum over the
 // chunk's blocks of (s da) K, one tcgen05 product per block (K = the block's keys).
+// The blocks stream through a ring of three or four stages, so that the copies of
+// the next blocks are in flight while the tensor cores work on this one.
 template <int B2P>
 __global__ void __launch_bounds__(128, 1)
 tc_bwd_dqbar_kernel(const __grid_constant__ CUtensorMap tmDA, const __grid_constant__ CUtensorMap tmK,
@@ -807,21 +816,22 @@ tc_bwd_dqbar_kernel(const __grid_constant__ CUtensorMap tmDA, const __grid_const
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     const Problem &p = a.p;
-    uint64_t *ld_bar = reinterpret_cast<uint64_t *>(sm + 2 * kTile);
-    uint64_t *mma_bar = ld_bar + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ld_bar + 2);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(ld_bar + 3);
+    using C = rb::Dq<B2P>;
+    constexpr int NS = C::kNS;
+    uint64_t *ld_bar = reinterpret_cast<uint64_t *>(sm + C::kBar);   // [NS]: stage loaded
+    uint64_t *mma_bar = ld_bar + NS;                                  // [NS]: stage read
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ld_bar + 2 * NS);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(ld_bar + 2 * NS + 1);
     const int warp = threadIdx.x >> 5, r = threadIdx.x;
     int unit = blockIdx.x;
     const int ch = unit % a.nch;
     unit /= a.nch;
     const int mt = unit % a.nmt, bh = unit / a.nmt;
-    const int u_lo = ch * a.upc, u_hi = min(p.b1k, u_lo + a.upc);
+    const int u_lo = ch * a.upc, u_hi = min(p.b1k, u_lo + a.upc), nb = max(0, u_hi - u_lo);
     constexpr uint32_t kPanelKV = B2P * 128;
 
     if (threadIdx.x == 0) {
-        mbar_init(ld_bar, 1);
-        mbar_init(mma_bar, 1);
+        for (int i = 0; i < 2 * NS; i++) mbar_init(ld_bar + i, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -832,34 +842,53 @@ tc_bwd_dqbar_kernel(const __grid_constant__ CUtensorMap tmDA, const __grid_const
     const uint32_t tmem = *tmem_slot;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
     const WaitCtx w{a.limit, a.status, abort_flag};
-    uint32_t ld_issued = 0, ld_done = 0, mma_issued = 0, mma_done = 0;
-    const uint64_t dA = smem_desc_sw128(smem_u32(sm), 16, 1024);
-    const uint64_t dK = smem_desc_sw128(smem_u32(sm + kTile), kPanelKV, 1024);   // MN-major
+    uint32_t ld_issued[NS], ld_done[NS], mma_issued[NS], mma_done[NS];
+#pragma unroll
+    for (int st = 0; st < NS; st++) ld_issued[st] = ld_done[st] = mma_issued[st] = mma_done[st] = 0;
     constexpr uint32_t idO = idesc_bf16(128, 128, 0, 1);
-    bool ok = true;
-    for (int up = u_lo; ok && up < u_hi; up++) {
+    // block i of the chunk into stage i % NS (thread 0 issues the copies)
+    auto load = [&](int i) {
+        const int st = i % NS, up = u_lo + i;
         if (threadIdx.x == 0) {
+            uint8_t *base = sm + st * C::kStage;
             const int tok0 = up * p.b2, hh = bh % p.H, bb = bh / p.H;
-            mbar_expect_tx(ld_bar, 2 * kPanel + 2 * kPanelKV);
+            mbar_expect_tx(ld_bar + st, 2 * kPanel + 2 * kPanelKV);
             for (int pn = 0; pn < 2; pn++) {
-                tma_load_5d(sm + pn * kPanel, &tmDA, 0, mt * 128, pn, up, bh, ld_bar);
-                tma_load_4d(sm + kTile + pn * kPanelKV, &tmK, pn * 64, tok0, hh, bb, ld_bar);
+                tma_load_5d(base + pn * kPanel, &tmDA, 0, mt * 128, pn, up, bh, ld_bar + st);
+                tma_load_4d(base + kTile + pn * kPanelKV, &tmK, pn * 64, tok0, hh, bb, ld_bar + st);
             }
         }
-        ld_issued++;
-        if (!(ok = wait_block(ld_bar, ld_done & 1, w))) break;
-        ld_done++;
+        ld_issued[st]++;
+    };
+    for (int i = 0; i < NS && i < nb; i++) load(i);
+    bool ok = true;
+    for (int i = 0; ok && i < nb; i++) {
+        const int st = i % NS;
+        if (!(ok = wait_block(ld_bar + st, (i / NS) & 1, w))) break;
+        ld_done[st]++;
         if (warp == 0) {
             tc_fence_after();
+            const uint64_t dA = smem_desc_sw128(smem_u32(sm + st * C::kStage), 16, 1024);
+            const uint64_t dK = smem_desc_sw128(smem_u32(sm + st * C::kStage + kTile), kPanelKV, 1024);   // MN-major
 #pragma unroll
             for (int kk = 0; kk < B2P / 16; kk++)
                 mma_ss_warp(tmem, desc_plus(dA, (kk >> 2) * kPanel + (kk & 3) * 32),
-                            desc_plus(dK, kk * 2048), idO, (up > u_lo || kk > 0) ? 1u : 0u);
-            mma_commit_warp(mma_bar);
+                            desc_plus(dK, kk * 2048), idO, (i > 0 || kk > 0) ? 1u : 0u);
+            mma_commit_warp(mma_bar + st);
         }
-        mma_issued++;
-        if (!(ok = wait_block(mma_bar, mma_done & 1, w))) break;
-        mma_done++;
+        mma_issued[st]++;
+        // the previous block's products are done with its stage: refill it NS blocks on
+        // (block i's products keep the tensor cores busy meanwhile)
+        if (i >= 1 && i - 1 + NS < nb) {
+            const int sp = (i - 1) % NS;
+            if (!(ok = wait_block(mma_bar + sp, ((i - 1) / NS) & 1, w))) break;
+            mma_done[sp]++;
+            load(i - 1 + NS);
+        }
+    }
+    if (ok && nb > 0) {   // the last block's commit covers every product before it
+        const int sl = (nb - 1) % NS;
+        if ((ok = wait_block(mma_bar + sl, ((nb - 1) / NS) & 1, w))) mma_done[sl]++;
         tc_fence_after();
     }
     if (ok) {
@@ -879,10 +908,15 @@ tc_bwd_dqbar_kernel(const __grid_constant__ CUtensorMap tmDA, const __grid_const
             for (int e = 0; e < 8; e++) d4[e] = make_float4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
         }
     }
-    if (threadIdx.x == 0 && ld_issued > ld_done)
-        wait_phase_cleanup(ld_bar, (ld_issued - 1) & 1, kCleanupPolls);
-    if (warp == 0 && mma_issued > mma_done)
-        wait_phase_cleanup(mma_bar, (mma_issued - 1) & 1, kCleanupPolls);
+    // drain this CTA's own copies and products before its tensor memory is freed (a
+    // phase that completed unobserved satisfies its wait at once)
+#pragma unroll
+    for (int st = 0; st < NS; st++) {
+        if (threadIdx.x == 0 && ld_issued[st] > ld_done[st])
+            wait_phase_cleanup(ld_bar + st, (ld_issued[st] - 1) & 1, kCleanupPolls);
+        if (warp == 0 && mma_issued[st] > mma_done[st])
+            wait_phase_cleanup(mma_bar + st, (mma_issued[st] - 1) & 1, kCleanupPolls);
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -891,8 +925,25 @@ tc_bwd_dqbar_kernel(const __grid_constant__ CUtensorMap tmDA, const __grid_const
     }
 }
 
+// dq̄ = the sum of the chunks' partials, in a fixed order (chunk 0, 1, ...), written
+// over chunk 0: one thread per four elements of a (bh, row tile) stack, so every
+// row's sum is taken once rather than once per query of its tile.
+__global__ void tc_bwd_reduce_kernel(float *__restrict__ part, int64_t stacks, int nch) {
+    const int64_t per = 128 * 128 / 4, total = stacks * per;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        float4 *src = reinterpret_cast<float4 *>(part) + (idx / per) * nch * per + idx % per;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int c2 = 0; c2 < nch; c2++) {
+            const float4 x = src[(int64_t)c2 * per];
+            acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+        }
+        src[0] = acc;
+    }
+}
+
 // dq = dq_L + dq̄[g][v] / |T_g| (the aggregation's mean), bfloat16 output; dq̄ is
-// the sum of the chunks' partials, taken here in a fixed order.
+// chunk 0 of each stack after tc_bwd_reduce_kernel.
 __global__ void tc_bwd_combine_kernel(const float *__restrict__ dql, const float *__restrict__ part,
                                       __nv_bfloat16 *__restrict__ dq, Problem p, int nmt, int nch) {
     const int64_t total = (int64_t)p.BH * p.N * (kD / 4);
@@ -906,12 +957,8 @@ __global__ void tc_bwd_combine_kernel(const float *__restrict__ dql, const float
         while (g + 1 < p.tiles && tile_begin(g + 1, p.b1, p.tiles) <= u) g++;
         const float inv = 1.f / (float)(tile_begin(g + 1, p.b1, p.tiles) - tile_begin(g, p.b1, p.tiles));
         const int rgl = g * p.b2 + v, mt = rgl / 128, rl = rgl % 128;
-        const float *src = part + (((int64_t)bh * nmt + mt) * nch * 128 + rl) * 128 + j;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int c2 = 0; c2 < nch; c2++) {
-            const float4 x = *reinterpret_cast<const float4 *>(src + (int64_t)c2 * 128 * 128);
-            acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
-        }
+        const float4 acc =
+            *reinterpret_cast<const float4 *>(part + (((int64_t)bh * nmt + mt) * nch * 128 + rl) * 128 + j);
         const float4 l4 = *reinterpret_cast<const float4 *>(dql + tok * kD + j);
         uint2 o;
         o.x = pack_bf16(l4.x + acc.x * inv, l4.y + acc.y * inv);
@@ -984,10 +1031,10 @@ cudaError_t launch_bwd_r(const CUtensorMap *m, const RbArgs &a, int stage, cudaS
         tc_bwd_r_kernel<B2P><<<(unsigned)(a.p.BH * a.p.b1k), 256, rb::kSmem, s>>>(m[0], m[1], m[2],
                                                                                m[3], m[4], a);
     } else {
-        const cudaError_t e = set_smem(tc_bwd_dqbar_kernel<B2P>, rb::kSmemQ);
+        const cudaError_t e = set_smem(tc_bwd_dqbar_kernel<B2P>, rb::Dq<B2P>::kSmem);
         if (e != cudaSuccess) return e;
-        tc_bwd_dqbar_kernel<B2P><<<(unsigned)(a.p.BH * a.nmt * a.nch), 128, rb::kSmemQ, s>>>(m[5], m[1],
-                                                                                          a);
+        tc_bwd_dqbar_kernel<B2P><<<(unsigned)(a.p.BH * a.nmt * a.nch), 128, rb::Dq<B2P>::kSmem, s>>>(
+            m[5], m[1], a);
     }
     return cudaGetLastError();
 }
@@ -1072,6 +1119,9 @@ cudaError_t sm100_backward(const Problem &p, const void *q, const void *k, const
     }
     ProfileScope scope(K_TC_BWD_DQBAR, stream);
     if ((e = launch_r(1)) != cudaSuccess) return e;
+    const int64_t stacks = (int64_t)p.BH * w.nmt, rtotal = stacks * 128 * 128 / 4;
+    const int rblocks = (int)((rtotal + 255) / 256 < 148 * 32 ? (rtotal + 255) / 256 : 148 * 32);
+    tc_bwd_reduce_kernel<<<rblocks, 256, 0, stream>>>(w.part, stacks, w.nch);
     const int64_t total = (int64_t)p.BH * p.N * (kD / 4);
     const int blocks = (int)((total + 255) / 256 < 148 * 32 ? (total + 255) / 256 : 148 * 32);
     tc_bwd_combine_kernel<<<blocks, 256, 0, stream>>>(w.dql, w.part, (__nv_bfloat16 *)dq, p, w.nmt,
