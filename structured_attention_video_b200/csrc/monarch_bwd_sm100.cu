@@ -23,18 +23,20 @@ using namespace tcs;
 //   dS = L (dP - delta)  (the gradient of the natural logits s q.Ktil + H),
 //   dZ = L^T dy,  dKtil = s dS^T q,  dH = sum over the tile's queries of dS,
 //   dq (the L-step's part) = s dS Ktil.
-// Two kernels, one 128-thread CTA per unit, one MMA stage at a time: the two
-// logit products go to tensor memory, the threads overwrite them in place with
-// the bfloat16 pairs of L and dS, and the accumulating products read those as
-// their tensor-memory A operand.
+// Three kernels of 256 threads, two per TMEM lane group: the logit products go to
+// tensor memory, the threads overwrite them in place with the bfloat16 pairs of L
+// and dS, and the accumulating products read those as their tensor-memory A
+// operand.
 //   tc_bwd_dkz_kernel: unit (bh, g, v, 128-key block); the key block's Ktil and Z
 //     (M side) against each 128-query tile of the tile (N side): S^T, dP^T, then
-//     dZ += L^T dy and dKtil += dS^T q over the query tiles; dH per key row.
-//   tc_bwd_dq_kernel<0>: unit (bh, g, v, 128-query tile); the queries and dy (M
-//     side) against each 128-key block: S, dP, and delta = sum L dP per query row
-//     (= dy.y, from the same products that form dS, so that every dS row sums to
-//     zero up to rounding).
-//   tc_bwd_dq_kernel<1>: the same units, then dq += dS Ktil over the blocks.
+//     dZ += L^T dy and dKtil += dS^T q over the query tiles; dH per key row.  The
+//     two warps of a lane group split the query columns.
+//   tc_bwd_dq_kernel<0>: unit (bh, g, v, pair of 128-query tiles); the queries and
+//     dy of both tiles (M side) against each 64-key half: S, dP, and delta =
+//     sum L dP per query row (= dy.y, from the same products that form dS, so that
+//     every dS row sums to zero up to rounding).  Warps 0-3 take tile 0, warps 4-7
+//     tile 1.
+//   tc_bwd_dq_kernel<1>: the same units, then dq += dS Ktil over the halves.
 // Every wait is bounded; on a time-out the CTA records MONARCH_ERR_TIMEOUT,
 // drains its own copies and MMAs, frees its tensor memory and returns.
 // =====================================================================
@@ -288,6 +290,48 @@ tc_bwd_dkz_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     }
 }
 
+// The query side, two 128-query tiles of one problem per CTA: the keys stream in
+// 64-key halves of Ktil and Z through a ring of three stages, so that each pass
+// reads Ktil and Z once per pair of query tiles.  Tensor memory: per tile t, S at
+// columns t*128 + [0, 64) and dP at t*128 + [64, 128) (dS packed over S), and the
+// dq accumulators at 256 + t*128.
+namespace lq {
+constexpr uint32_t kHalf = 64 * 128 * 2;          // 64 key rows of 128 bfloat16: two 8 KB panels
+constexpr uint32_t kSlot = 2 * kHalf;             // a half of Ktil, then of Z
+constexpr int kNS = 3;
+constexpr uint32_t kRing = 4 * kTile;             // after q and dy of the two tiles
+constexpr uint32_t kHk = kRing + kNS * kSlot;     // [kNS][64] floats: H' of the half's keys
+constexpr uint32_t kBar = kHk + kNS * 64 * 4;
+constexpr uint32_t kSmem = kBar + 128 + 1024;     // + slack to align the base to 1024
+}  // namespace lq
+
+// Eight K-steps (K = 128) of D = A B^T, A a 128-row K-major SW128 tile (64-column
+// panels 16 KB apart), B a 64-row one (panels 8 KB apart): N = 64.  The offset
+// descriptors are formed inside the asm block; elect.sync picks the issuing lane.
+__device__ __forceinline__ void mma8_ss_k128_b64(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                                 uint32_t idesc) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        ".reg .b64 a1, a2, a3, a4, a5, a6, a7, b1, b2, b3, b4, b5, b6, b7;\n\t"
+        "add.s64 a1, %1, 2;\n\tadd.s64 a2, %1, 4;\n\tadd.s64 a3, %1, 6;\n\t"
+        "add.s64 a4, %1, 1024;\n\tadd.s64 a5, %1, 1026;\n\tadd.s64 a6, %1, 1028;\n\t"
+        "add.s64 a7, %1, 1030;\n\t"
+        "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
+        "add.s64 b4, %2, 512;\n\tadd.s64 b5, %2, 514;\n\tadd.s64 b6, %2, 516;\n\t"
+        "add.s64 b7, %2, 518;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a4, b4, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a5, b5, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a6, b6, %3, 1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a7, b7, %3, 1;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc)
+        : "memory");
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(256, 1)
 tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDy,
@@ -296,35 +340,40 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     const Problem &p = a.p;
-    uint64_t *q_bar = reinterpret_cast<uint64_t *>(sm + lb::kBar);
-    uint64_t *kb_bar = q_bar + 1;     // [2]: key block buffers
-    uint64_t *mma_bar = q_bar + 3;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(q_bar + 4);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(q_bar + 5);
-    float *hk = reinterpret_cast<float *>(sm + lb::kVec);   // [buffer][128]: H' of the block
-    float *ds_part = hk + 256;                               // [128]: the second half's delta
-    // two warps per group of 32 TMEM lanes: thread (j, half) takes query row j and the
-    // half's 64 key columns (chunks 2*half, 2*half + 1)
-    const int warp = threadIdx.x >> 5, j = (warp & 3) * 32 + (threadIdx.x & 31), half = warp >> 2;
+    constexpr int NS = lq::kNS;
+    uint64_t *q_bar = reinterpret_cast<uint64_t *>(sm + lq::kBar);
+    uint64_t *kz_bar = q_bar + 1;     // [NS]: a half of Ktil and Z in its stage
+    uint64_t *mma_bar = q_bar + 1 + NS;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_bar + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(mma_bar + 2);
+    float *hk = reinterpret_cast<float *>(sm + lq::kHk);
+    // warps 0-3 take tile 0 of the pair, warps 4-7 tile 1: thread j of a tile, query row j
+    const int warp = threadIdx.x >> 5, j = (warp & 3) * 32 + (threadIdx.x & 31), t = warp >> 2;
 
     int unit = blockIdx.x;
-    const int c = unit % a.nqt;
-    unit /= a.nqt;
+    const int npair = (a.nqt + 1) / 2;
+    const int pair = unit % npair;
+    unit /= npair;
     const int v = unit % p.b2;
     unit /= p.b2;
     const int g = unit % p.tiles, bh = unit / p.tiles;
     const int u_lo = tile_begin(g, p.b1, p.tiles), u_hi = tile_begin(g + 1, p.b1, p.tiles);
-    const int u0 = u_lo + 128 * c, nqc = min(128, u_hi - u0);
-    if (nqc <= 0) return;   // a tile shorter than the longest one: no query tile c (uniform)
+    const int u00 = u_lo + 256 * pair;                  // the pair's first query row
+    const int nq0 = min(128, u_hi - u00), nq1 = min(128, u_hi - u00 - 128);
+    if (nq0 <= 0) return;   // a tile shorter than the longest one: no such pair (uniform)
+    const int ntl = nq1 > 0 ? 2 : 1;                    // query tiles of the pair
+    const bool tile_ok = t < ntl;
+    const int u0 = u00 + 128 * t;
     const int64_t slab0 = (((int64_t)bh * p.tiles + g) * p.b2 + v) * p.b1k;
     const int64_t tok = (int64_t)bh * p.N + (int64_t)(u0 + j) * p.b2 + v;
-    const bool row_ok = j < nqc;
+    const bool row_ok = tile_ok && j < (t ? nq1 : nq0);
     const float lam = row_ok ? -pair_sum(a.lam[tok * 2].x) : 0.f;
     const float dlt = (MODE == 1 && row_ok) ? a.delta[tok] : 0.f;
+    const int nh = (p.b1k + 63) / 64;
     float dsum = 0.f;   // MODE 0: sum over the keys of L dP
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 4; i++) mbar_init(q_bar + i, 1);
+        for (int i = 0; i < 2 + NS; i++) mbar_init(q_bar + i, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -336,178 +385,153 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const WaitCtx w{a.limit, a.status, abort_flag};
     uint32_t q_issued = 0, q_done = 0, mma_issued = 0, mma_done = 0;
-    uint32_t kb_issued[2] = {0, 0}, kb_done[2] = {0, 0};
+    uint32_t kz_issued[NS], kz_done[NS];
+#pragma unroll
+    for (int st = 0; st < NS; st++) kz_issued[st] = kz_done[st] = 0;
+    bool uncommitted = false;   // warp 0 issued products after its last commit
 
-    // key block kk into buffer b: its Ktil and Z rows (thread 0) and its entropies
-    auto stage_k = [&](int kk, int b) {
+    // half h of the keys into stage h % NS: its Ktil and Z rows (thread 0; rows past b1k
+    // read zeros) and its entropies
+    auto stage = [&](int h) {
+        const int st = h % NS;
         if (threadIdx.x == 0) {
-            mbar_expect_tx(kb_bar + b, 2 * kTile);
+            uint8_t *base = sm + lq::kRing + st * lq::kSlot;
+            int r, u, b;
+            kz_coords(p, (int)(slab0 + 64 * h), r, u, b);
+            mbar_expect_tx(kz_bar + st, lq::kSlot);
             for (int pn = 0; pn < 2; pn++) {
-                ls_load_kz(sm + lb::tile(2 + 2 * b) + pn * kPanel, &tmKt, pn,
-                           (int)(slab0 + kk * 128), p, kb_bar + b);
-                ls_load_kz(sm + lb::tile(3 + 2 * b) + pn * kPanel, &tmZ, pn,
-                           (int)(slab0 + kk * 128), p, kb_bar + b);
+                tma_load_5d(base + pn * (lq::kHalf / 2), &tmKt, 0, r, pn, u, b, kz_bar + st);
+                tma_load_5d(base + lq::kHalf + pn * (lq::kHalf / 2), &tmZ, 0, r, pn, u, b, kz_bar + st);
             }
         }
-        kb_issued[b]++;
-        const int nkv = min(128, p.b1k - kk * 128), i = threadIdx.x;
-        if (i < 128) hk[b * 128 + i] = i < nkv ? pair_sum(a.hx[(slab0 + kk * 128 + i) * 2].x) : 0.f;
+        kz_issued[st]++;
+        const int i = threadIdx.x;
+        if (i < 64)
+            hk[st * 64 + i] = 64 * h + i < p.b1k ? pair_sum(a.hx[(slab0 + 64 * h + i) * 2].x) : 0.f;
     };
 
-    if (threadIdx.x == 0) {   // the query tile and its dy rows
-        mbar_expect_tx(q_bar, 2 * kTile);
-        for (int pn = 0; pn < 2; pn++) {
-            ls_load_q(sm + lb::tile(0) + pn * kPanel, &tmQ, pn * 64, v, u0, bh, p, q_bar);
-            ls_load_q(sm + lb::tile(1) + pn * kPanel, &tmDy, pn * 64, v, u0, bh, p, q_bar);
-        }
+    if (threadIdx.x == 0) {   // q and dy of the pair's tiles
+        mbar_expect_tx(q_bar, 2 * ntl * kTile);
+        for (int tt = 0; tt < ntl; tt++)
+            for (int pn = 0; pn < 2; pn++) {
+                ls_load_q(sm + lb::tile(2 * tt) + pn * kPanel, &tmQ, pn * 64, v, u00 + 128 * tt, bh, p, q_bar);
+                ls_load_q(sm + lb::tile(2 * tt + 1) + pn * kPanel, &tmDy, pn * 64, v, u00 + 128 * tt, bh, p,
+                          q_bar);
+            }
     }
     q_issued++;
-    stage_k(0, 0);
+    for (int h = 0; h < NS && h < nh; h++) stage(h);
     bool ok = wait_block(q_bar, 0, w);
     if (ok) q_done++;
 
-    const uint64_t dQk = smem_desc_sw128(smem_u32(sm + lb::tile(0)), 16, 1024);
-    const uint64_t dYk = smem_desc_sw128(smem_u32(sm + lb::tile(1)), 16, 1024);
-    constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0), idO = idesc_bf16(128, 128, 0, 1);
-    if constexpr (MODE == 0) {
-        // delta needs no accumulator: the products of block kb + 1 go to the other 256
-        // columns of tensor memory while the threads work on block kb
-        if (a.nkb > 1) stage_k(1, 1);
-        auto issue = [&](int kb) {   // warp 0
-            const int b = kb & 1;
-            const uint32_t tk = smem_u32(sm + lb::tile(2 + 2 * b)), tz = smem_u32(sm + lb::tile(3 + 2 * b));
-            tc_fence_after();
-            mma8_ss_k128(tmem + 256 * b, dQk, smem_desc_sw128(tk, 16, 1024), idS, 0u);         // S = q Ktil^T
-            mma8_ss_k128(tmem + 256 * b + 128, dYk, smem_desc_sw128(tz, 16, 1024), idS, 0u);   // dP = dy Z^T
-            mma_commit_warp(mma_bar);
-        };
-        if (ok && a.nkb > 0 && (ok = wait_block(kb_bar, 0, w))) {
-            kb_done[0]++;
-            if (warp == 0) issue(0);
-            mma_issued++;
-        }
-        for (int kb = 0; ok && kb < a.nkb; kb++) {
-            const int b = kb & 1, nkv = min(128, p.b1k - kb * 128);
-            if (!(ok = wait_block(mma_bar, mma_done & 1, w))) break;
-            mma_done++;
-            if (kb + 1 < a.nkb) {   // block kb + 1, loaded during the previous step
-                if (!(ok = wait_block(kb_bar + (b ^ 1), ((kb + 1) >> 1) & 1, w))) break;
-                kb_done[b ^ 1]++;
-                if (warp == 0) issue(kb + 1);
-                mma_issued++;
-            }
-            tc_fence_after();
-            const float *hkb = hk + b * 128;
-            const uint32_t tb = tl + 256 * b + 64 * half;
-            float sv[64], dv64[64];
-            tmem_ld32f(tb, sv);
-            tmem_ld32f(tb + 32, sv + 32);
-            tmem_ld32f(tb + 128, dv64);
-            tmem_ld32f(tb + 160, dv64 + 32);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 64; k++) {
-                const int key = 64 * half + k;
-                const float pr = (row_ok && key < nkv)
-                                     ? fast_exp2((sv[k] + hkb[key] - lam) * a.c_log2) : 0.f;
-                dsum = fmaf(pr, dv64[k], dsum);
-            }
-            // every thread is done with block kb's columns and entropies: the products
-            // of block kb + 2 may overwrite the columns, and buffer b takes its rows
-            tc_fence_before();
-            __syncthreads();
-            if (kb + 2 < a.nkb) stage_k(kb + 2, b);
-        }
-    } else {
-    for (int kb = 0; ok && kb < a.nkb; kb++) {
-        const int b = kb & 1, nkv = min(128, p.b1k - kb * 128);
-        // the next block into the other buffer: its last reader, block kb - 1, is done
-        if (kb + 1 < a.nkb) stage_k(kb + 1, b ^ 1);
-        const float *hkb = hk + b * 128;
-        const uint32_t tk = smem_u32(sm + lb::tile(2 + 2 * b)), tz = smem_u32(sm + lb::tile(3 + 2 * b));
-        if (!(ok = wait_block(kb_bar + b, (kb >> 1) & 1, w))) break;
-        kb_done[b]++;
+    constexpr uint32_t idS = idesc_bf16(128, 64, 0, 0), idO = idesc_bf16(128, 128, 0, 1);
+    for (int h = 0; ok && h < nh; h++) {
+        const int st = h % NS;
+        if (!(ok = wait_block(kz_bar + st, (h / NS) & 1, w))) break;
+        kz_done[st]++;
+        const uint32_t kt = smem_u32(sm + lq::kRing + st * lq::kSlot), zt = kt + lq::kHalf;
         if (warp == 0) {
             tc_fence_after();
-            mma8_ss_k128(tmem, dQk, smem_desc_sw128(tk, 16, 1024), idS, 0u);          // S = q Ktil^T
-            mma8_ss_k128(tmem + 128, dYk, smem_desc_sw128(tz, 16, 1024), idS, 0u);    // dP = dy Z^T
+            for (int tt = 0; tt < ntl; tt++) {
+                mma8_ss_k128_b64(tmem + tt * 128, smem_desc_sw128(smem_u32(sm + lb::tile(2 * tt)), 16, 1024),
+                                 smem_desc_sw128(kt, 16, 1024), idS);                          // S = q Ktil^T
+                mma8_ss_k128_b64(tmem + tt * 128 + 64,
+                                 smem_desc_sw128(smem_u32(sm + lb::tile(2 * tt + 1)), 16, 1024),
+                                 smem_desc_sw128(zt, 16, 1024), idS);                          // dP = dy Z^T
+            }
             mma_commit_warp(mma_bar);
+            uncommitted = false;
         }
         mma_issued++;
         if (!(ok = wait_block(mma_bar, mma_done & 1, w))) break;
         mma_done++;
+        // every product of half h - 1 is done too (the commit covers them): its stage
+        // takes half h + 2 (its entropies were last read before the previous barrier)
+        if (h >= 1 && h + 2 < nh) stage(h + 2);
         tc_fence_after();
-        // both halves read all of their S and dP columns before either writes dS over
-        // S (the upper half's packed pairs land on columns the lower half reads)
-        float sv[64], dv64[64];
-        tmem_ld32f(tl + 64 * half, sv);
-        tmem_ld32f(tl + 64 * half + 32, sv + 32);
-        tmem_ld32f(tl + 128 + 64 * half, dv64);
-        tmem_ld32f(tl + 128 + 64 * half + 32, dv64 + 32);
-        tmem_wait_ld();
-        __syncthreads();
+        if (tile_ok) {
+            const float *hkh = hk + st * 64;
+            const uint32_t ts = tl + t * 128;
+            float sv[64], dv[64];
+            tmem_ld32f(ts, sv);
+            tmem_ld32f(ts + 32, sv + 32);
+            tmem_ld32f(ts + 64, dv);
+            tmem_ld32f(ts + 96, dv + 32);
+            tmem_wait_ld();
+            if constexpr (MODE == 0) {
 #pragma unroll
-        for (int cc = 0; cc < 2; cc++) {
-            const int ch = 2 * half + cc;
-            const float *s = sv + 32 * cc, *d = dv64 + 32 * cc;
-            uint32_t dk[16];
-#pragma unroll
-            for (int k = 0; k < 32; k += 2) {
-                float dv[2];
-#pragma unroll
-                for (int e = 0; e < 2; e++) {
-                    const int key = ch * 32 + k + e;
-                    const float pr = (row_ok && key < nkv)
-                                         ? fast_exp2((s[k + e] + hkb[key] - lam) * a.c_log2) : 0.f;
-                    dv[e] = pr * (d[k + e] - dlt);
+                for (int k = 0; k < 64; k++) {
+                    const float pr = (row_ok && 64 * h + k < p.b1k)
+                                         ? fast_exp2((sv[k] + hkh[k] - lam) * a.c_log2) : 0.f;
+                    dsum = fmaf(pr, dv[k], dsum);
                 }
-                dk[k / 2] = pack_bf16(dv[0], dv[1]);
+            } else {
+                uint32_t dk[32];
+#pragma unroll
+                for (int k = 0; k < 64; k += 2) {
+                    float dd[2];
+#pragma unroll
+                    for (int e = 0; e < 2; e++) {
+                        const float pr = (row_ok && 64 * h + k + e < p.b1k)
+                                             ? fast_exp2((sv[k + e] + hkh[k + e] - lam) * a.c_log2) : 0.f;
+                        dd[e] = pr * (dv[k + e] - dlt);
+                    }
+                    dk[k / 2] = pack_bf16(dd[0], dd[1]);
+                }
+#pragma unroll
+                for (int q8 = 0; q8 < 4; q8++)
+                    tmem_st8(ts + q8 * 8, *reinterpret_cast<const uint32_t(*)[8]>(&dk[q8 * 8]));
+                tmem_wait_st();
             }
-            const uint32_t(&dk0)[8] = *reinterpret_cast<const uint32_t(*)[8]>(&dk[0]);
-            const uint32_t(&dk1)[8] = *reinterpret_cast<const uint32_t(*)[8]>(&dk[8]);
-            tmem_st8(tl + ch * 16, dk0);
-            tmem_st8(tl + ch * 16 + 8, dk1);
         }
-        tmem_wait_st();
+        // every thread is done with this half's columns (and in MODE 1 has stored dS)
         tc_fence_before();
         __syncthreads();
-        if (warp == 0) {
+        if (MODE == 1 && warp == 0) {
             tc_fence_after();
-            mma8_ts_mn128(tmem + 256, tmem, smem_desc_sw128(tk, kPanel, 1024), idO,
-                          kb > 0 ? 1u : 0u);   // dq' += dS Ktil
-            mma_commit_warp(mma_bar);
+            for (int tt = 0; tt < ntl; tt++)
+                mma4_ts_mn64(tmem + 256 + tt * 128, tmem + tt * 128, smem_desc_sw128(kt, lq::kHalf / 2, 1024),
+                             idO, h > 0 ? 1u : 0u);                                            // dq' += dS Ktil
+            uncommitted = true;
         }
-        mma_issued++;
-        if (!(ok = wait_block(mma_bar, mma_done & 1, w))) break;
-        mma_done++;
-        tc_fence_after();
-    }
     }
     if (MODE == 0) {
-        if (half == 1) ds_part[j] = dsum;
-        __syncthreads();
-        if (ok && row_ok && half == 0) a.delta[tok] = dsum + ds_part[j];
-    }
-    if (ok && MODE == 1) {
+        if (ok && row_ok) a.delta[tok] = dsum;
+    } else if (ok) {   // the last half's dq products, then dq' to memory
+        if (warp == 0) {
+            mma_commit_warp(mma_bar);
+            uncommitted = false;
+        }
+        mma_issued++;
+        if ((ok = wait_block(mma_bar, mma_done & 1, w))) mma_done++;
+        tc_fence_after();
+        if (ok && tile_ok) {
 #pragma unroll 1
-        for (int ch = 2 * half; ch < 2 * half + 2; ch++) {
-            float o[32];
-            tmem_ld32f(tl + 256 + ch * 32, o);
-            tmem_wait_ld();
-            if (row_ok) {
-                float4 *dst = reinterpret_cast<float4 *>(a.dql + tok * kD + ch * 32);
+            for (int ch = 0; ch < 4; ch++) {
+                float o[32];
+                tmem_ld32f(tl + 256 + t * 128 + ch * 32, o);
+                tmem_wait_ld();
+                if (row_ok) {
+                    float4 *dst = reinterpret_cast<float4 *>(a.dql + tok * kD + ch * 32);
 #pragma unroll
-                for (int e = 0; e < 8; e++)
-                    dst[e] = make_float4(o[4 * e] * p.scale, o[4 * e + 1] * p.scale,
-                                         o[4 * e + 2] * p.scale, o[4 * e + 3] * p.scale);
+                    for (int e = 0; e < 8; e++)
+                        dst[e] = make_float4(o[4 * e] * p.scale, o[4 * e + 1] * p.scale,
+                                             o[4 * e + 2] * p.scale, o[4 * e + 3] * p.scale);
+                }
             }
         }
+    }
+    // drain this CTA's own copies and products before its tensor memory is freed
+    if (warp == 0 && uncommitted) {
+        mma_commit_warp(mma_bar);
+        mma_issued++;
     }
     if (threadIdx.x == 0) {
         if (q_issued > q_done) wait_phase_cleanup(q_bar, 0, kCleanupPolls);
-        for (int b = 0; b < 2; b++)
-            if (kb_issued[b] > kb_done[b])
-                wait_phase_cleanup(kb_bar + b, (kb_issued[b] - 1) & 1, kCleanupPolls);
+#pragma unroll
+        for (int st = 0; st < NS; st++)
+            if (kz_issued[st] > kz_done[st])
+                wait_phase_cleanup(kz_bar + st, (kz_issued[st] - 1) & 1, kCleanupPolls);
     }
     if (warp == 0 && mma_issued > mma_done)
         wait_phase_cleanup(mma_bar, (mma_issued - 1) & 1, kCleanupPolls);
@@ -1064,10 +1088,12 @@ cudaError_t sm100_backward(const Problem &p, const void *q, const void *k, const
     const uint64_t dkz[5] = {64, rr, 2, slab, (uint64_t)p.BH};
     const uint64_t skz[4] = {128, rr * 128, 2 * rr * 128, slab * 2 * rr * 128};
     const uint32_t bkz[5] = {64, 1, 1, 128, 1};    // 128 blocks u' of one row r
+    const uint32_t bkz64[5] = {64, 1, 1, 64, 1};   // 64 blocks u' of one row r
     const uint32_t brow[5] = {64, 128, 1, 1, 1};   // 128 rows r of one block u'
-    CUtensorMap mq, mdy, mkt, mz;
+    CUtensorMap mq, mdy, mkt, mz, mkt64, mz64;
     if (!map_queries(&mq, q, p) || !map_queries(&mdy, dy, p) ||
-        !make_map(&mkt, ws.ktil, 5, dkz, skz, bkz) || !make_map(&mz, ws.z, 5, dkz, skz, bkz))
+        !make_map(&mkt, ws.ktil, 5, dkz, skz, bkz) || !make_map(&mz, ws.z, 5, dkz, skz, bkz) ||
+        !make_map(&mkt64, ws.ktil, 5, dkz, skz, bkz64) || !make_map(&mz64, ws.z, 5, dkz, skz, bkz64))
         return cudaErrorInvalidValue;
     CUtensorMap rm[6];
     const int mpad = qbar_tiles(p) * 128, b2p = b2_padded(p.b2);
@@ -1079,15 +1105,15 @@ cudaError_t sm100_backward(const Problem &p, const void *q, const void *k, const
         !make_map(&rm[4], w.dzb, 5, dkz, skz, brow) || !make_map(&rm[5], w.da, 5, dkz, skz, brow))
         return cudaErrorInvalidValue;
     if ((e = set_smem(tc_bwd_dkz_kernel, lb::kSmem)) != cudaSuccess ||
-        (e = set_smem(tc_bwd_dq_kernel<0>, lb::kSmem)) != cudaSuccess ||
-        (e = set_smem(tc_bwd_dq_kernel<1>, lb::kSmem)) != cudaSuccess)
+        (e = set_smem(tc_bwd_dq_kernel<0>, lq::kSmem)) != cudaSuccess ||
+        (e = set_smem(tc_bwd_dq_kernel<1>, lq::kSmem)) != cudaSuccess)
         return e;
     LbArgs la{p, ws.hx, ws.lam, w.delta, w.dktb, w.dzb, w.dhr, w.dql, c_log2, (p.b1k + 127) / 128,
               (tile_max_rows(p.b1, p.tiles) + 127) / 128, status, wait_limit};
-    const int64_t probs = (int64_t)p.BH * p.tiles * p.b2;
+    const int64_t probs = (int64_t)p.BH * p.tiles * p.b2, npair = (la.nqt + 1) / 2;
     {
         ProfileScope scope(K_TC_BWD_DELTA, stream);
-        tc_bwd_dq_kernel<0><<<(unsigned)(probs * la.nqt), 256, lb::kSmem, stream>>>(mq, mdy, mkt, mz, la);
+        tc_bwd_dq_kernel<0><<<(unsigned)(probs * npair), 256, lq::kSmem, stream>>>(mq, mdy, mkt64, mz64, la);
     }
     {
         ProfileScope scope(K_TC_BWD_DKZ, stream);
@@ -1095,7 +1121,7 @@ cudaError_t sm100_backward(const Problem &p, const void *q, const void *k, const
     }
     {
         ProfileScope scope(K_TC_BWD_DQ, stream);
-        tc_bwd_dq_kernel<1><<<(unsigned)(probs * la.nqt), 256, lb::kSmem, stream>>>(mq, mdy, mkt, mz, la);
+        tc_bwd_dq_kernel<1><<<(unsigned)(probs * npair), 256, lq::kSmem, stream>>>(mq, mdy, mkt64, mz64, la);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     RbArgs ra{p, mpad, w.dhr, w.da, (__nv_bfloat16 *)dk, (__nv_bfloat16 *)dv, w.part, w.nmt, w.nch,
