@@ -425,6 +425,64 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (ok) q_done++;
 
     constexpr uint32_t idS = idesc_bf16(128, 64, 0, 0), idO = idesc_bf16(128, 128, 0, 1);
+    if constexpr (MODE == 0) {
+        // delta needs no accumulator: the products of half h + 1 go to the other 256
+        // columns of tensor memory (buffer (h + 1) & 1) while the threads work on half h
+        auto issue = [&](int h) {   // warp 0
+            const uint32_t kt = smem_u32(sm + lq::kRing + (h % NS) * lq::kSlot), zt = kt + lq::kHalf;
+            const uint32_t tb = tmem + 256 * (h & 1);
+            tc_fence_after();
+            for (int tt = 0; tt < ntl; tt++) {
+                mma8_ss_k128_b64(tb + tt * 128, smem_desc_sw128(smem_u32(sm + lb::tile(2 * tt)), 16, 1024),
+                                 smem_desc_sw128(kt, 16, 1024), idS);                          // S = q Ktil^T
+                mma8_ss_k128_b64(tb + tt * 128 + 64,
+                                 smem_desc_sw128(smem_u32(sm + lb::tile(2 * tt + 1)), 16, 1024),
+                                 smem_desc_sw128(zt, 16, 1024), idS);                          // dP = dy Z^T
+            }
+            mma_commit_warp(mma_bar);
+        };
+        if (ok && nh > 0 && (ok = wait_block(kz_bar, 0, w))) {
+            kz_done[0]++;
+            if (warp == 0) issue(0);
+            mma_issued++;
+        }
+        for (int h = 0; ok && h < nh; h++) {
+            const int st = h % NS;
+            if (!(ok = wait_block(mma_bar, mma_done & 1, w))) break;
+            mma_done++;
+            if (h + 1 < nh) {   // half h + 1, loaded during an earlier step
+                const int s1 = (h + 1) % NS;
+                if (!(ok = wait_block(kz_bar + s1, ((h + 1) / NS) & 1, w))) break;
+                kz_done[s1]++;
+                if (warp == 0) issue(h + 1);
+                mma_issued++;
+            }
+            // the products of half h - 1 are done: its stage takes half h + 2 (its
+            // entropies were last read before the previous barrier)
+            if (h >= 1 && h + 2 < nh) stage(h + 2);
+            tc_fence_after();
+            if (tile_ok) {
+                const float *hkh = hk + st * 64;
+                const uint32_t ts = tl + 256 * (h & 1) + t * 128;
+                float sv[64], dv[64];
+                tmem_ld32f(ts, sv);
+                tmem_ld32f(ts + 32, sv + 32);
+                tmem_ld32f(ts + 64, dv);
+                tmem_ld32f(ts + 96, dv + 32);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 64; k++) {
+                    const float pr = (row_ok && 64 * h + k < p.b1k)
+                                         ? fast_exp2((sv[k] + hkh[k] - lam) * a.c_log2) : 0.f;
+                    dsum = fmaf(pr, dv[k], dsum);
+                }
+            }
+            // every thread is done with buffer h & 1: the products of half h + 2 may
+            // overwrite it
+            tc_fence_before();
+            __syncthreads();
+        }
+    } else {
     for (int h = 0; ok && h < nh; h++) {
         const int st = h % NS;
         if (!(ok = wait_block(kz_bar + st, (h / NS) & 1, w))) break;
@@ -458,14 +516,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tmem_ld32f(ts + 64, dv);
             tmem_ld32f(ts + 96, dv + 32);
             tmem_wait_ld();
-            if constexpr (MODE == 0) {
-#pragma unroll
-                for (int k = 0; k < 64; k++) {
-                    const float pr = (row_ok && 64 * h + k < p.b1k)
-                                         ? fast_exp2((sv[k] + hkh[k] - lam) * a.c_log2) : 0.f;
-                    dsum = fmaf(pr, dv[k], dsum);
-                }
-            } else {
+            {
                 uint32_t dk[32];
 #pragma unroll
                 for (int k = 0; k < 64; k += 2) {
@@ -487,13 +538,14 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         // every thread is done with this half's columns (and in MODE 1 has stored dS)
         tc_fence_before();
         __syncthreads();
-        if (MODE == 1 && warp == 0) {
+        if (warp == 0) {
             tc_fence_after();
             for (int tt = 0; tt < ntl; tt++)
                 mma4_ts_mn64(tmem + 256 + tt * 128, tmem + tt * 128, smem_desc_sw128(kt, lq::kHalf / 2, 1024),
                              idO, h > 0 ? 1u : 0u);                                            // dq' += dS Ktil
             uncommitted = true;
         }
+    }
     }
     if (MODE == 0) {
         if (ok && row_ok) a.delta[tok] = dsum;
