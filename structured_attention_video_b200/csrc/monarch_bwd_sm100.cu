@@ -483,69 +483,69 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             __syncthreads();
         }
     } else {
-    for (int h = 0; ok && h < nh; h++) {
-        const int st = h % NS;
-        if (!(ok = wait_block(kz_bar + st, (h / NS) & 1, w))) break;
-        kz_done[st]++;
-        const uint32_t kt = smem_u32(sm + lq::kRing + st * lq::kSlot), zt = kt + lq::kHalf;
-        if (warp == 0) {
-            tc_fence_after();
-            for (int tt = 0; tt < ntl; tt++) {
-                mma8_ss_k128_b64(tmem + tt * 128, smem_desc_sw128(smem_u32(sm + lb::tile(2 * tt)), 16, 1024),
-                                 smem_desc_sw128(kt, 16, 1024), idS);                          // S = q Ktil^T
-                mma8_ss_k128_b64(tmem + tt * 128 + 64,
-                                 smem_desc_sw128(smem_u32(sm + lb::tile(2 * tt + 1)), 16, 1024),
-                                 smem_desc_sw128(zt, 16, 1024), idS);                          // dP = dy Z^T
-            }
-            mma_commit_warp(mma_bar);
-            uncommitted = false;
-        }
-        mma_issued++;
-        if (!(ok = wait_block(mma_bar, mma_done & 1, w))) break;
-        mma_done++;
-        // every product of half h - 1 is done too (the commit covers them): its stage
-        // takes half h + 2 (its entropies were last read before the previous barrier)
-        if (h >= 1 && h + 2 < nh) stage(h + 2);
-        tc_fence_after();
-        if (tile_ok) {
-            const float *hkh = hk + st * 64;
-            const uint32_t ts = tl + t * 128;
-            float sv[64], dv[64];
-            tmem_ld32f(ts, sv);
-            tmem_ld32f(ts + 32, sv + 32);
-            tmem_ld32f(ts + 64, dv);
-            tmem_ld32f(ts + 96, dv + 32);
-            tmem_wait_ld();
-            {
-                uint32_t dk[32];
-#pragma unroll
-                for (int k = 0; k < 64; k += 2) {
-                    float dd[2];
-#pragma unroll
-                    for (int e = 0; e < 2; e++) {
-                        const float pr = (row_ok && 64 * h + k + e < p.b1k)
-                                             ? fast_exp2((sv[k + e] + hkh[k + e] - lam) * a.c_log2) : 0.f;
-                        dd[e] = pr * (dv[k + e] - dlt);
-                    }
-                    dk[k / 2] = pack_bf16(dd[0], dd[1]);
+        for (int h = 0; ok && h < nh; h++) {
+            const int st = h % NS;
+            if (!(ok = wait_block(kz_bar + st, (h / NS) & 1, w))) break;
+            kz_done[st]++;
+            const uint32_t kt = smem_u32(sm + lq::kRing + st * lq::kSlot), zt = kt + lq::kHalf;
+            if (warp == 0) {
+                tc_fence_after();
+                for (int tt = 0; tt < ntl; tt++) {
+                    mma8_ss_k128_b64(tmem + tt * 128, smem_desc_sw128(smem_u32(sm + lb::tile(2 * tt)), 16, 1024),
+                                     smem_desc_sw128(kt, 16, 1024), idS);                          // S = q Ktil^T
+                    mma8_ss_k128_b64(tmem + tt * 128 + 64,
+                                     smem_desc_sw128(smem_u32(sm + lb::tile(2 * tt + 1)), 16, 1024),
+                                     smem_desc_sw128(zt, 16, 1024), idS);                          // dP = dy Z^T
                 }
+                mma_commit_warp(mma_bar);
+                uncommitted = false;
+            }
+            mma_issued++;
+            if (!(ok = wait_block(mma_bar, mma_done & 1, w))) break;
+            mma_done++;
+            // every product of half h - 1 is done too (the commit covers them): its stage
+            // takes half h + 2 (its entropies were last read before the previous barrier)
+            if (h >= 1 && h + 2 < nh) stage(h + 2);
+            tc_fence_after();
+            if (tile_ok) {
+                const float *hkh = hk + st * 64;
+                const uint32_t ts = tl + t * 128;
+                float sv[64], dv[64];
+                tmem_ld32f(ts, sv);
+                tmem_ld32f(ts + 32, sv + 32);
+                tmem_ld32f(ts + 64, dv);
+                tmem_ld32f(ts + 96, dv + 32);
+                tmem_wait_ld();
+                {
+                    uint32_t dk[32];
 #pragma unroll
-                for (int q8 = 0; q8 < 4; q8++)
-                    tmem_st8(ts + q8 * 8, *reinterpret_cast<const uint32_t(*)[8]>(&dk[q8 * 8]));
-                tmem_wait_st();
+                    for (int k = 0; k < 64; k += 2) {
+                        float dd[2];
+#pragma unroll
+                        for (int e = 0; e < 2; e++) {
+                            const float pr = (row_ok && 64 * h + k + e < p.b1k)
+                                                 ? fast_exp2((sv[k + e] + hkh[k + e] - lam) * a.c_log2) : 0.f;
+                            dd[e] = pr * (dv[k + e] - dlt);
+                        }
+                        dk[k / 2] = pack_bf16(dd[0], dd[1]);
+                    }
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; q8++)
+                        tmem_st8(ts + q8 * 8, *reinterpret_cast<const uint32_t(*)[8]>(&dk[q8 * 8]));
+                    tmem_wait_st();
+                }
+            }
+            // every thread is done with this half's columns (and in MODE 1 has stored dS)
+            tc_fence_before();
+            __syncthreads();
+            if (warp == 0) {
+                tc_fence_after();
+                for (int tt = 0; tt < ntl; tt++)
+                    mma4_ts_mn64(tmem + 256 + tt * 128, tmem + tt * 128, smem_desc_sw128(kt, lq::kHalf / 2, 1024),
+                                 idO, h > 0 ? 1u : 0u);                                            // dq' += dS Ktil
+                uncommitted = true;
             }
         }
-        // every thread is done with this half's columns (and in MODE 1 has stored dS)
-        tc_fence_before();
-        __syncthreads();
-        if (warp == 0) {
-            tc_fence_after();
-            for (int tt = 0; tt < ntl; tt++)
-                mma4_ts_mn64(tmem + 256 + tt * 128, tmem + tt * 128, smem_desc_sw128(kt, lq::kHalf / 2, 1024),
-                             idO, h > 0 ? 1u : 0u);                                            // dq' += dS Ktil
-            uncommitted = true;
-        }
-    }
     }
     if (MODE == 0) {
         if (ok && row_ok) a.delta[tok] = dsum;
