@@ -81,6 +81,20 @@ def test_fwd_rejects_null_and_misaligned_pointers():
     assert _lib.monarch_attn_fwd_host(None, fake, fake, fake, *shape, 0, None) == 1
 
 
+def test_profile_kernel_names():
+    """Every kernel family has a distinct name, and out-of-range ids return NULL."""
+    names = []
+    k = 0
+    while _lib.monarch_profile_kernel_name(k) is not None:
+        names.append(_lib.monarch_profile_kernel_name(k))
+        k += 1
+    assert len(names) == len(set(names)) == 16
+    assert _lib.monarch_profile_kernel_name(-1) is None
+    for name in ("tc_lstep_kernel", "tc_rstep_kernel", "tc_qbar_kernel", "tc_bwd_dq_kernel<0>",
+                 "tc_bwd_dkz_kernel", "tc_bwd_dq_kernel<1>", "tc_bwd_r_kernel"):
+        assert name in names
+
+
 def test_status_strings():
     for code in range(8):
         assert len(_lib.monarch_status_string(code)) > 0
